@@ -1,0 +1,399 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each test checks the oracle against something other than itself: values the
+pages fix in a worked example (tests/golden/), a library routine (numpy,
+torch's float->bf16 cast), a closed form the input generator knows (the
+positions it changed), brute force on tiny inputs, or invariants of the
+method.  The comment on each test names the kind of mistake it would catch.
+"""
+from __future__ import annotations
+
+import ctypes
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests import _golden as G
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor -> uint16 numpy bits (host)."""
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16).reshape(-1)
+
+
+# ---------------------------------------------------------------- encode
+
+
+def test_encode_golden_worked_example():
+    # Off-by-one or 1-based indices, values taken from old instead of new,
+    # float instead of bit compare (+0/-0, NaN), wrong offsets with empty
+    # tensors: each changes the expected lists.
+    olds, news, offsets, indices, values = G.encode_example()
+    o, i, v = oracle.encode(olds, news)
+    np.testing.assert_array_equal(o, offsets)
+    np.testing.assert_array_equal(i, indices)
+    np.testing.assert_array_equal(v, values)
+
+
+def test_encode_matches_numpy_flatnonzero():
+    # Library pin: numpy's flatnonzero over the integer views, the same
+    # compare the verl snippet writes with torch (view(int) != view(int),
+    # nonzero).  Catches dropped tails, skipped elements, unstable order.
+    rng = np.random.default_rng(7)
+    sizes = [0, 1, 7, 8, 9, 4095, 4096, 4097, 100_003, 0, 65_536]
+    olds, news = [], []
+    for n in sizes:
+        a = rng.integers(0, 1 << 16, n, dtype=np.uint16)
+        b = a.copy()
+        flip = rng.random(n) < rng.choice([0.0, 0.01, 0.3, 1.0])
+        b[flip] ^= rng.integers(1, 1 << 16, int(flip.sum()), dtype=np.uint16)
+        olds.append(a)
+        news.append(b)
+    o, i, v = oracle.encode(olds, news)
+    exp_i, exp_v, exp_o = [], [], [0]
+    for a, b in zip(olds, news):
+        nz = np.flatnonzero(a != b)
+        exp_i.append(nz.astype(np.int32))
+        exp_v.append(b[nz])
+        exp_o.append(exp_o[-1] + nz.size)
+    np.testing.assert_array_equal(o, np.array(exp_o, dtype=np.int64))
+    np.testing.assert_array_equal(i, np.concatenate(exp_i))
+    np.testing.assert_array_equal(v, np.concatenate(exp_v))
+
+
+SPECIALS = [0x0000, 0x8000, 0x0001, 0x8001, 0x3F80, 0xBF80, 0x7F80, 0xFF80,
+            0x7FC0, 0x7FC1, 0x3F81, 0xBF81]
+
+
+def test_encode_bruteforce_tiny():
+    # Brute force over every pair of length-2 tensors drawn from 12 special
+    # bf16 patterns (signed zeros, subnormals, +-1, +-inf, two NaN payloads),
+    # against the set definition {i : old[i] != new[i]} on bits.
+    pairs = list(itertools.product(SPECIALS, repeat=2))
+    for a in pairs:
+        for b in pairs[::7]:
+            old = np.array(a, dtype=np.uint16)
+            new = np.array(b, dtype=np.uint16)
+            o, i, v = oracle.encode([old], [new])
+            want = [k for k in range(2) if a[k] != b[k]]
+            assert list(i) == want
+            assert list(v) == [b[k] for k in want]
+            assert list(o) == [0, len(want)]
+
+
+def test_encode_invariants_and_roundtrip():
+    # nnz equals the popcount of the change mask; indices strictly ascend in
+    # each segment; every value differs from old at its index; applying the
+    # delta to old gives new bit for bit; old == new gives an empty delta.
+    rng = np.random.default_rng(11)
+    olds = [rng.integers(0, 1 << 16, n, dtype=np.uint16) for n in (3000, 1, 0, 12345)]
+    news = []
+    for a in olds:
+        b = a.copy()
+        m = rng.random(a.size) < 0.05
+        b[m] = rng.integers(0, 1 << 16, int(m.sum()), dtype=np.uint16)
+        news.append(b)
+    o, i, v = oracle.encode(olds, news)
+    assert o[-1] == sum(int((a != b).sum()) for a, b in zip(olds, news))
+    for t, (a, b) in enumerate(zip(olds, news)):
+        seg = i[o[t]:o[t + 1]]
+        assert np.all(np.diff(seg) > 0)
+        assert np.all(a[seg] != v[o[t]:o[t + 1]])
+    snaps = [a.copy() for a in olds]
+    oracle.apply(snaps, o, i, v)
+    for s, b in zip(snaps, news):
+        np.testing.assert_array_equal(s, b)
+    o2, i2, v2 = oracle.encode(olds, [a.copy() for a in olds])
+    assert o2.tolist() == [0] * (len(olds) + 1) and i2.size == 0 and v2.size == 0
+
+
+def test_encode_capacity_counts_but_does_not_store():
+    olds, news, offsets, indices, values = G.encode_example()
+    o, i, v = oracle.encode(olds, news, capacity=2)
+    np.testing.assert_array_equal(o, offsets)          # still the full count
+    np.testing.assert_array_equal(i, indices[:2])
+    np.testing.assert_array_equal(v, values[:2])
+
+
+def test_encode_rejects_numel_at_int32_bound():
+    # int32 indices cannot address element 2^31 (the verl review lists the
+    # silent wrap-around of int32 positions as a risk): the oracle refuses.
+    lib = oracle._load()
+    numels = np.array([1 << 31], dtype=np.int64)
+    ptrs = (ctypes.c_void_p * 1)()
+    offs = np.zeros(2, dtype=np.int64)
+    rc = lib.ref_encode(1, numels.ctypes.data, ptrs, ptrs, offs.ctypes.data, None, None, 0)
+    assert rc == -1
+
+
+# ---------------------------------------------------------------- apply / chain
+
+
+def test_apply_leaves_unchanged_positions_and_empty_is_identity():
+    rng = np.random.default_rng(3)
+    old = rng.integers(0, 1 << 16, 5000, dtype=np.uint16)
+    new = old.copy()
+    pos = np.sort(rng.choice(5000, 40, replace=False))
+    new[pos] ^= 0x0101
+    o, i, v = oracle.encode([old], [new])
+    snap = old.copy()
+    oracle.apply([snap], o, i, v)
+    untouched = np.ones(5000, bool)
+    untouched[pos] = False
+    np.testing.assert_array_equal(snap[untouched], old[untouched])
+    np.testing.assert_array_equal(snap, new)
+    snap2 = old.copy()
+    oracle.apply([snap2], np.zeros(2, np.int64), np.zeros(0, np.int32), np.zeros(0, np.uint16))
+    np.testing.assert_array_equal(snap2, old)
+
+
+def test_apply_rejects_out_of_range_index():
+    snap = np.zeros(4, dtype=np.uint16)
+    with pytest.raises(ValueError):
+        oracle.apply([snap], np.array([0, 1], np.int64), np.array([4], np.int32),
+                     np.array([1], np.uint16))
+
+
+def test_chain_golden_later_delta_wins():
+    anchor, deltas, final = G.chain_example()
+    snaps = [a.copy() for a in anchor]
+    oracle.apply_chain(snaps, deltas)
+    for s, f in zip(snaps, final):
+        np.testing.assert_array_equal(s, f)
+
+
+def test_chain_replays_qwen_shaped_steps():
+    # Anchor + 10 deltas == the 10th step's weights, on the Qwen3-0.6B
+    # parameter list scaled down 32x (same 310 tensors).  Equal to applying
+    # the deltas one by one.
+    shapes = W.scaled_shapes(W.qwen3_0p6b_shapes(), 32)
+    s = W.SEEDS["qwen3_0p6b"]
+    w = W.init_set(shapes, s, "cpu", 0.02)
+    anchor = [bits(t) for t in w.tensors]
+    deltas = []
+    prev = anchor
+    for k in range(1, 11):
+        w = W.step_set(w, s, k, 3e-6, "cpu")
+        cur = [bits(t) for t in w.tensors]
+        deltas.append(oracle.encode(prev, cur))
+        prev = cur
+    snaps = [a.copy() for a in anchor]
+    oracle.apply_chain(snaps, deltas)
+    for a, b in zip(snaps, prev):
+        np.testing.assert_array_equal(a, b)
+    seq = [a.copy() for a in anchor]
+    for d in deltas:
+        oracle.apply(seq, *d)
+    for a, b in zip(seq, snaps):
+        np.testing.assert_array_equal(a, b)
+
+
+# ---------------------------------------------------------------- XOR
+
+
+def test_xor_golden():
+    old, new, mask = G.xor_example()
+    np.testing.assert_array_equal(oracle.xor_encode(old, new), mask)
+    buf = old.copy()
+    oracle.xor_apply(buf, mask)
+    np.testing.assert_array_equal(buf, new)
+
+
+def test_xor_closed_form_on_byte_layers():
+    # Closed form: the generator knows exactly which bytes it changed, so the
+    # mask's nonzero bytes must be exactly those positions; numpy's
+    # bitwise_xor gives the same mask (library pin); apply restores new.
+    old, new, pos = W.xor_layer(0, "cpu", nbytes=2_000_003, flips=1_700)
+    old, new, pos = old.numpy(), new.numpy(), pos.numpy()
+    mask = oracle.xor_encode(old, new)
+    np.testing.assert_array_equal(np.flatnonzero(mask), pos)
+    np.testing.assert_array_equal(mask, np.bitwise_xor(old, new))
+    buf = old.copy()
+    oracle.xor_apply(buf, mask)
+    np.testing.assert_array_equal(buf, new)
+    assert not oracle.xor_encode(old, old).any()
+
+
+def test_xor_agrees_with_sparse_encode_on_bf16():
+    # On bf16 data the byte mask is nonzero exactly at the bytes of the
+    # elements the sparse encode lists.
+    old, new = W.single("cpu")
+    a, b = bits(old.tensors[0]), bits(new.tensors[0])
+    mask = oracle.xor_encode(a.view(np.uint8), b.view(np.uint8)).view(np.uint16)
+    o, i, v = oracle.encode([a], [b])
+    np.testing.assert_array_equal(np.flatnonzero(mask), i)
+
+
+# ---------------------------------------------------------------- workload 5
+
+
+def test_stress_closed_form_positions():
+    # Closed form: every element the stress generator picks gets different
+    # low mantissa bits, so the encode lists exactly the picked positions.
+    sizes = W.stress_sizes(count=40, lo=16, hi=70_000)
+    clustered = W.stress_clustered(count=40)
+    w = W.stress_init(sizes, "cpu")
+    new, picks = W.stress_step(w, clustered, 1, "cpu")
+    o, i, v = oracle.encode([bits(t) for t in w.tensors], [bits(t) for t in new.tensors])
+    for t, p in enumerate(picks):
+        np.testing.assert_array_equal(i[o[t]:o[t + 1]], np.flatnonzero(p.numpy()))
+
+
+# ---------------------------------------------------------------- bf16 rounding
+
+
+def test_bf16_rne_golden_cases():
+    for f32, b16 in G.rounding_cases():
+        x = np.array([f32], dtype=np.uint32).view(np.float32)
+        assert int(oracle.bf16_rne(x)[0]) == b16, hex(f32)
+
+
+def test_bf16_rne_matches_torch_cast():
+    # Library pin: torch's float32 -> bfloat16 conversion rounds to nearest
+    # even.  Random bit patterns (no NaN) plus every tie pattern near 1.
+    rng = np.random.default_rng(5)
+    u = rng.integers(0, 1 << 32, 20000, dtype=np.uint64).astype(np.uint32)
+    u = u[(u & 0x7FFFFFFF) <= 0x7F800000]
+    ties = np.uint32(0x3F800000) + (np.arange(256, dtype=np.uint32) << 16) + np.uint32(0x8000)
+    u = np.concatenate([u, ties.astype(np.uint32)])
+    x = u.view(np.float32)
+    want = bits(torch.from_numpy(x.copy()).to(torch.bfloat16))
+    np.testing.assert_array_equal(oracle.bf16_rne(x), want)
+
+
+def test_update_step_matches_numpy_fp32():
+    # Library pin for the update model: numpy float32 ops (each rounded),
+    # then torch's cast.
+    rng = np.random.default_rng(9)
+    w = bits(torch.from_numpy(rng.normal(0, 0.03, 50000).astype(np.float32)).to(torch.bfloat16))
+    u = np.clip(rng.normal(0, 1, 50000).astype(np.float32), -10, 10)
+    lr = np.float32(3e-6)
+    x = w.astype(np.uint32) << 16
+    x = x.view(np.float32) - (lr * u)
+    want = bits(torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16))
+    np.testing.assert_array_equal(oracle.update_step(w, u, 3e-6), want)
+
+
+# ---------------------------------------------------------------- absorption
+
+
+def _neighbours(wbits):
+    """fp32 values at and around the two rounding midpoints of w."""
+    lib = oracle._load()
+    w = lib.ref_bf16_to_float(wbits)
+    out = []
+    for nb in ((wbits - 1) & 0xFFFF, (wbits + 1) & 0xFFFF):
+        m = (float(w) + float(lib.ref_bf16_to_float(nb))) / 2.0
+        m32 = np.float32(m)
+        out += [m32, np.nextafter(m32, np.float32(np.inf)), np.nextafter(m32, np.float32(-np.inf))]
+    return out
+
+
+def test_absorption_predictor_matches_integer_rounding():
+    # Two independent routes to "does the cast keep w's bits": exact
+    # midpoints in double vs the integer rounding of ref_bf16_rne (itself
+    # pinned to torch above).  Probes every midpoint and its fp32
+    # neighbours, so a tie rule or a power-of-two mistake shows up.
+    rng = np.random.default_rng(13)
+    ws = list(rng.integers(0x0080, 0x7F7F, 300)) + [0x3F80, 0x4000, 0x3C00, 0x0080, 0x0081,
+                                                   0x0001, 0x007F, 0x7F7E]
+    for wb in ws:
+        for sign in (0, 0x8000):
+            wbits = int(wb) | sign
+            for x in _neighbours(wbits):
+                want = int(oracle.bf16_rne(np.array([x], np.float32))[0] != wbits)
+                assert oracle.absorption_changed(wbits, x) == want, (hex(wbits), float(x))
+
+
+def test_absorption_power_of_two_is_asymmetric():
+    # At w = 1.0 the neighbour below is 2^-8 away and the one above 2^-7:
+    # a decrease of 0.75 * 2^-8 leaves the interval, an increase of the same
+    # size stays inside.
+    w = 0x3F80
+    assert oracle.absorption_changed(w, 1.0 - 0.75 * 2 ** -8) == 1
+    assert oracle.absorption_changed(w, 1.0 + 0.75 * 2 ** -8) == 0
+
+
+def _min_visible_step(wbits):
+    """Smallest |dw| (downwards) that changes w's bits, by bisection."""
+    w = float(oracle.bf16_to_float([wbits])[0])
+    lo, hi = 0.0, abs(w)
+    for _ in range(80):
+        mid = (lo + hi) / 2
+        x = np.float32(w - math.copysign(mid, w))
+        if oracle.absorption_changed(wbits, x):
+            hi = mid
+        else:
+            lo = mid
+    return hi
+
+
+def test_absorption_thresholds_from_the_pages():
+    # The pages' rule: an update below about |w|/256 is absorbed; at lr 3e-6
+    # and |w| in [1e-2, 1e-1] the update is always absorbed, and |w|/256 is
+    # about 4e-5 .. 4e-4.  The exact threshold lies within a factor of 2 of
+    # |w|/256 (the spacing is |w|*2^-7 only up to the position inside the
+    # binade).
+    d = G.keyed("absorption_thresholds.txt")
+    lr = float(d["lr"][0])
+    for wv in map(float, d["w"]):
+        wbits = int(oracle.bf16_rne(np.array([wv], np.float32))[0])
+        w = float(oracle.bf16_to_float([wbits])[0])
+        assert oracle.absorption_changed(wbits, np.float32(w) - np.float32(lr)) == 0
+        assert oracle.absorption_changed(wbits, np.float32(w) + np.float32(lr)) == 0
+        thr = _min_visible_step(wbits)
+        assert abs(w) / 512 <= thr <= abs(w) / 128 * 1.0001, (wv, thr)
+    assert round(0.01 / 256, 5) == float(d["threshold_at_1e-2"][0])
+    assert round(0.1 / 256, 4) == float(d["threshold_at_1e-1"][0])
+
+
+def test_workload1_absorption_predicts_encode_mask():
+    # Every element of workload 1: the generator's new weights equal the
+    # oracle's recomputation of the update, and the elements the absorption
+    # rule says change are exactly those the encode lists.
+    old, new = W.single("cpu")
+    a, b = bits(old.tensors[0]), bits(new.tensors[0])
+    u = W.update_noise(a.size, W.step_seed(W.SEEDS["single"], 1, 0), "cpu").numpy()
+    np.testing.assert_array_equal(oracle.update_step(a, u, 3e-6), b)
+    changed, count = oracle.absorption_predict(a, u, 3e-6)
+    o, i, v = oracle.encode([a], [b])
+    assert count == o[-1]
+    np.testing.assert_array_equal(np.flatnonzero(changed), i)
+    # The change rate the workload definition expects is "about 1%"; the
+    # stated update model gives about 2.3%.  Both are far from dense.
+    assert 0.005 < count / a.size < 0.05
+
+
+# ---------------------------------------------------------------- shapes and reported numbers
+
+
+def test_model_shapes_match_the_pages_sizes():
+    d = G.keyed("model_sizes.txt")
+    q = W.qwen3_0p6b_shapes()
+    nq = sum(W.numel(s) for _, s in q)
+    assert len(q) == 310 and nq == 596_049_920
+    assert round(nq * int(d["bytes_per_bf16"][0]) / 1e9, 1) == float(d["qwen3_0p6b_full_GB"][0])
+    assert 7e9 * 2 / 1e9 == float(d["seven_b_full_GB"][0])
+    ll = W.llama3_8b_shapes()
+    assert len(ll) == 291 and sum(W.numel(s) for _, s in ll) == 8_030_261_248
+    assert max(W.numel(s) for _, s in ll) < 2 ** 31
+
+
+def test_stress_sizes_are_log_uniform():
+    sizes = W.stress_sizes()
+    assert len(sizes) == 12000 and min(sizes) >= 256 and max(sizes) <= 4194304
+    expected = 12000 * (4194304 - 256) / math.log(4194304 / 256)
+    assert abs(sum(sizes) / expected - 1) < 0.05
+
+
+def test_sparsity_formula_reproduces_the_log_line():
+    d = G.keyed("sync_log.txt")
+    changed, total = int(d["changed"][0]), int(d["total"][0])
+    sparsity = 1 - changed / total
+    assert round(100 * sparsity, 2) == float(d["sparsity_percent"][0])
+    assert round(sparsity, 4) == float(d["sparsity_metadata"][0])
