@@ -1,0 +1,731 @@
+#!/usr/bin/env python
+"""Delta encode+apply throughput of bf16 weights on B200 (libdws).
+
+One step = dws_encode(old, new -> sparse delta) + dws_apply(delta -> snapshot)
+on the Llama-3-8B-shaped parameter set (291 tensors, 8,030,261,248 bf16
+elements, 16.06 GB per snapshot) after one simulated optimizer step at
+lr 3e-6.  Inputs (32 GB) are much larger than the 126 MB L2, so no flush is
+needed between steps.  value = weight bytes (2 B x elements, summed over
+ranks) / device time per step, max over ranks.
+
+Also reported on the same JSON line:
+  roofline      encode kernel: algorithmic bytes (4N + 6 nnz) / CUDA-event
+                time vs the measured HBM copy bandwidth;
+  cpu_baseline  the single-threaded CPU oracle on a bounded sample (rank 0, N=1);
+  e2e           the same metric with the new snapshot coming from pinned host
+                memory and the delta going device->host->device, copies timed;
+  rows          the other hot-path rows: encode at lr 1e-5, count-only,
+                XOR encode/apply and the double-buffered layer pipeline on 40
+                x 0.8 GB byte layers, chain replay of 10 deltas on the
+                Qwen3-0.6B-shaped set and on the 12000-tensor stress set.
+
+Multi-GPU: replicas only -- every rank runs the same workload on its own GPU
+(no data-path collective); NCCL is used for the barrier and the max-over-ranks
+timing reduction.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "delta encode+apply GB/s of bf16 weights (1 B200) and % of HBM peak"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--lr", type=float, default=3e-6)
+    ap.add_argument("--layers", type=int, default=None,
+                    help="only the first LAYERS decoder layers (a small case for profiling)")
+    ap.add_argument("--no-rows", action="store_true", help="skip the other hot-path rows")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle sample")
+    ap.add_argument("--rows-reps", type=int, default=5)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# plumbing
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def llama_shapes(layers):
+    import workloads as W
+    shapes = W.llama3_8b_shapes()
+    if layers is None:
+        return shapes
+    keep = [s for s in shapes if not s[0].startswith("model.layers.")]
+    lay = [s for s in shapes if s[0].startswith("model.layers.")
+           and int(s[0].split(".")[2]) < layers]
+    # a small case: decoder layers only (no embedding / lm_head)
+    return lay if layers > 0 else keep
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int, uuid: str | None):
+        self.dev = device_index
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        target = f"GPU-{self.uuid}" if self.uuid else str(self.dev)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", target, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < 10:  # wait for the first sample
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
+        with open(self.path) as f:
+            self.skip = len(f.read().splitlines())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        with open(self.path) as f:
+            lines = f.read().splitlines()[self.skip:]
+        os.unlink(self.path)
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < len(self.FIELDS):
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def encode_traffic_per_elem():
+    """DRAM bytes per element of the encode kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    summ = os.path.join(ROOT, "profiles", "encode_kernel_llama3_8b.md")
+    src = os.path.join(ROOT, "sparse_bf16_delta_b200", "csrc", "encode.cu")
+    if not os.path.exists(summ):
+        return None, None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for ln in open(summ):
+        if ln.startswith("- ") and ":" in ln:
+            k, _, v = ln[2:].partition(":")
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("encode.cu sha256[:16]") != h:
+        return None, None
+    try:
+        return float(vals["dram bytes per element"]), float(vals["nnz fraction"])
+    except (KeyError, ValueError):
+        return None, None
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle on a bounded sample (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+
+def host_tensor(shapes, s, lr, device, t):
+    """Tensor t of the workload (old and new bits on the host)."""
+    import numpy as np
+    import torch
+
+    import workloads as W
+
+    def bits(x):
+        return x.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+    name, shape = shapes[t]
+    n = W.numel(shape)
+    std_mean = (0.01, 1.0) if W.is_norm(name) else (0.02, 0.0)
+    w = W.init_tensor(n, W.weight_seed(s, t), device, *std_mean)
+    u = W.update_noise(n, W.step_seed(s, 1, t), device)
+    new = W.optimizer_step(w, u, lr)
+    return bits(w), bits(new)
+
+
+def layer_order(shapes):
+    order = [i for i, (nm, _) in enumerate(shapes) if nm.startswith("model.layers.")]
+    return order or list(range(len(shapes)))
+
+
+def time_oracle(pairs):
+    """Seconds the oracle spends on encode + apply over the (old, new) pairs."""
+    import oracle
+    tot = 0.0
+    for a, b in pairs:
+        snap = a.copy()
+        t0 = time.perf_counter()
+        o, i, v = oracle.encode([a], [b])
+        oracle.apply([snap], o, i, v)
+        tot += time.perf_counter() - t0
+    return tot
+
+
+def oracle_sample(shapes, s, lr, device, seconds):
+    """Time the oracle's encode + apply tensor by tensor (decoder layers in
+    order) until `seconds` of CPU time are spent.  Returns (bytes, secs,
+    elements, tensors)."""
+    tot_t, tot_n, count = 0.0, 0, 0
+    for t in layer_order(shapes):
+        a, b = host_tensor(shapes, s, lr, device, t)
+        tot_t += time_oracle([(a, b)])
+        tot_n += a.size
+        count += 1
+        if tot_t >= seconds:
+            break
+    return 2 * tot_n, tot_t, tot_n, count
+
+
+def cpu_model():
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ---------------------------------------------------------------------------
+# --impl reference: the oracle as it stands on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    import torch
+    import workloads as W
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    shapes = llama_shapes(args.layers)
+    s = W.SEEDS["llama3_8b"]
+    # Each step is a bounded sample of the workload, sized so that the whole
+    # run stays within about two minutes of oracle time.
+    per_step = min(5.0, max(0.3, 120.0 / max(1, args.steps + args.warmup)))
+    order = layer_order(shapes)
+    first = host_tensor(shapes, s, args.lr, dev, order[0])
+    rate = first[0].size / max(1e-6, time_oracle([first]))
+    pairs, n = [first], first[0].size
+    for t in order[1:]:
+        if n >= rate * per_step:
+            break
+        pairs.append(host_tensor(shapes, s, args.lr, dev, t))
+        n += pairs[-1][0].size
+    for _ in range(args.warmup):
+        time_oracle(pairs)
+    secs = [time_oracle(pairs) for _ in range(args.steps)]
+    tt = sum(secs)
+    value = 2 * n * args.steps / tt / 1e9
+    sample = (f"per step: the first {len(pairs)} decoder-layer tensors of the Llama-3-8B-shaped "
+              f"set ({n} bf16 elements, {2 * n / 1e9:.3f} GB of weights), oracle encode + apply, "
+              f"one thread")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tt / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u16", "data": "synthetic",
+        "config": {"workload": "llama3_8b-shaped bf16 parameter set (bounded sample per step)",
+                   "lr": args.lr, "parallelism": "replicas"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample, "cpu": cpu_model()},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# --impl ours
+# ---------------------------------------------------------------------------
+
+def events(n):
+    import torch
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def time_reps(fn, reps, warm=1):
+    """Median and min device time (ms) of fn() over reps, CUDA events."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a, b = events(2)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts), min(ts)
+
+
+def row(name, ms, alg_bytes, weight_bytes, peak, extra=None):
+    d = {"ms": round(ms, 4), "alg_GBps": round(alg_bytes / ms / 1e6, 1),
+         "weight_GBps": round(weight_bytes / ms / 1e6, 1),
+         "hbm_frac": round(alg_bytes / ms / 1e6 / peak, 4)}
+    if extra:
+        d.update(extra)
+    return name, d
+
+
+def run_rows(args, dev, peak):
+    """The other §(a) rows, each on its own workload, timed with events."""
+    import gc
+
+    import torch
+
+    import sparse_bf16_delta_b200 as dws
+    import workloads as W
+    out = {}
+
+    # --- Qwen3-0.6B-shaped chain of 10 deltas -------------------------------
+    t0 = time.time()
+    s = W.SEEDS["qwen3_0p6b"]
+    shapes = W.qwen3_0p6b_shapes()
+    sizes = [W.numel(sh) for _, sh in shapes]
+    std = [(0.01, 1.0) if W.is_norm(nm) else (0.02, 0.0) for nm, _ in shapes]
+    anchor_flat, anchor = W.pack_flat(sizes, lambda t, n: W.init_tensor(n, W.weight_seed(s, t), dev, *std[t]), dev)
+    plan = dws.DeltaPlan.for_tensors(anchor)
+    prev_flat, prev = W.pack_flat(sizes, lambda t, n: anchor[t], dev)
+    cur_flat, cur = W.pack_flat(sizes, lambda t, n: None, dev)
+    deltas, enc_ms, nnzs = [], [], []
+    for k in range(1, 11):
+        for t in range(len(sizes)):
+            u = W.update_noise(sizes[t], W.step_seed(s, k, t), dev)
+            cur[t].copy_(W.optimizer_step(prev[t], u, 3e-6))
+        ot, nt = dws.ptr_table(prev), dws.ptr_table(cur)
+        d = plan.encode_exact(ot, nt)
+        ms, _ = time_reps(lambda: plan.encode_into(ot, nt, d.offsets, d.indices, d.values), 3)
+        enc_ms.append(ms)
+        nnzs.append(d.nnz())
+        deltas.append(d)
+        prev_flat, cur_flat = cur_flat, prev_flat
+        prev, cur = cur, prev
+    snap_flat = anchor_flat.clone()
+    snap = [snap_flat[v.storage_offset() - anchor_flat.storage_offset():][:v.numel()] for v in anchor]
+    st = dws.ptr_table(snap)
+    ms, mn = time_reps(lambda: plan.apply_chain(st, deltas), args.rows_reps)
+    plan.raise_on_error("qwen chain")
+    ok = torch.equal(snap_flat, prev_flat)
+    N = sum(sizes)
+    tot = sum(nnzs)
+    out.update([row("apply_chain_qwen3_0p6b_k10", ms, 4 * N + 6 * tot, 2 * N, peak,
+                    {"min_ms": round(mn, 4), "nnz_total": tot, "exact": ok})])
+    mean_enc = statistics.mean(enc_ms)
+    out.update([row("encode_qwen3_0p6b", mean_enc, 4 * N + 6 * tot / 10, 2 * N, peak,
+                    {"nnz_mean": tot // 10, "sparsity_mean": round(1 - tot / 10 / N, 5)})])
+    del deltas, anchor_flat, prev_flat, cur_flat, snap_flat, anchor, prev, cur, snap, plan
+    gc.collect()
+    torch.cuda.empty_cache()
+    log(f"rows: qwen chain done in {time.time() - t0:.1f}s")
+
+    # --- XOR path: 40 layers x 0.8 GB ----------------------------------------
+    t0 = time.time()
+    L, B = 40, 800_000_000
+    olds, news, masks = [], [], []
+    for l in range(L):
+        o, n, _ = W.xor_layer(l, dev, nbytes=B)
+        olds.append(o)
+        news.append(n)
+        masks.append(torch.empty(B, dtype=torch.uint8, device=dev))
+    torch.cuda.synchronize()
+
+    def xor_enc():
+        for l in range(L):
+            dws.xor_encode(olds[l], news[l], masks[l])
+
+    ms, mn = time_reps(xor_enc, args.rows_reps)
+    ok = all(int(torch.count_nonzero(masks[l])) == 680_000 for l in (0, L - 1))
+    out.update([row("xor_encode_nvfp4_40x0.8GB", ms, 3 * L * B, L * B, peak,
+                    {"min_ms": round(mn, 4), "launches": L, "exact_flip_count": ok})])
+    # apply twice per rep so the buffers end where they started
+    bufs = olds
+
+    def xor_app2():
+        for l in range(L):
+            dws.xor_apply(bufs[l], masks[l])
+        for l in range(L):
+            dws.xor_apply(bufs[l], masks[l])
+
+    ms2, mn2 = time_reps(xor_app2, args.rows_reps)
+    out.update([row("xor_apply_nvfp4_40x0.8GB", ms2 / 2, 3 * L * B, L * B, peak,
+                    {"min_ms": round(mn2 / 2, 4)})])
+    # double-buffered layer pipeline, masks staged D2D (stand-in for the DE)
+    staging = [torch.empty(B, dtype=torch.uint8, device=dev) for _ in range(2)]
+    cs = torch.cuda.Stream()
+
+    def pipe2():
+        dws.xor_apply_layers(bufs, masks, staging[0], staging[1], copy_stream=cs)
+        dws.xor_apply_layers(bufs, masks, staging[0], staging[1], copy_stream=cs)
+
+    msp, mnp = time_reps(pipe2, max(2, args.rows_reps // 2))
+    dws.xor_apply(bufs[0], masks[0])
+    dws.xor_apply(bufs[L - 1], masks[L - 1])
+    torch.cuda.synchronize()
+    ok = torch.equal(bufs[0], news[0]) and torch.equal(bufs[L - 1], news[L - 1])
+    dws.xor_apply(bufs[0], masks[0])
+    dws.xor_apply(bufs[L - 1], masks[L - 1])
+    out.update([row("xor_apply_layers_double_buffered_40x0.8GB", msp / 2, 5 * L * B, L * B, peak,
+                    {"min_ms": round(mnp / 2, 4), "staging": "2 x 0.8 GB, D2D copy stream",
+                     "exact": ok})])
+    del olds, news, masks, bufs, staging
+    gc.collect()
+    torch.cuda.empty_cache()
+    log(f"rows: xor done in {time.time() - t0:.1f}s")
+
+    # --- stress: 12000 tensors, chain of 10 ----------------------------------
+    t0 = time.time()
+    s = W.SEEDS["stress"]
+    sizes = W.stress_sizes()
+    clustered = W.stress_clustered()
+    anchor_flat, anchor = W.pack_flat(sizes, lambda t, n: W.init_tensor(n, W.weight_seed(s, t), dev, 0.02), dev)
+    plan = dws.DeltaPlan.for_tensors(anchor)
+    prev_flat, prev = W.pack_flat(sizes, lambda t, n: anchor[t], dev)
+    cur_flat, cur = W.pack_flat(sizes, lambda t, n: None, dev)
+    deltas, nnzs, enc_ms, exp_nnz = [], [], [], []
+    for k in range(1, 11):
+        picked_total = 0
+        for t in range(len(sizes)):
+            nw, pk = W.stress_change(prev[t], clustered[t], W.step_seed(s, k, t), dev)
+            cur[t].copy_(nw)
+            picked_total += int(pk.sum())
+        ot, nt = dws.ptr_table(prev), dws.ptr_table(cur)
+        d = plan.encode_exact(ot, nt)
+        ms, _ = time_reps(lambda: plan.encode_into(ot, nt, d.offsets, d.indices, d.values), 3)
+        enc_ms.append(ms)
+        nnzs.append(d.nnz())
+        exp_nnz.append(picked_total)
+        deltas.append(d)
+        prev_flat, cur_flat = cur_flat, prev_flat
+        prev, cur = cur, prev
+    snap_flat = anchor_flat.clone()
+    snap = [snap_flat[v.storage_offset() - anchor_flat.storage_offset():][:v.numel()] for v in anchor]
+    st = dws.ptr_table(snap)
+    ms, mn = time_reps(lambda: plan.apply_chain(st, deltas), args.rows_reps)
+    plan.raise_on_error("stress chain")
+    ok = torch.equal(snap_flat, prev_flat) and nnzs == exp_nnz
+    N = sum(sizes)
+    tot = sum(nnzs)
+    out.update([row("apply_chain_stress_12000t_k10", ms, 4 * N + 6 * tot, 2 * N, peak,
+                    {"min_ms": round(mn, 4), "elements": N, "nnz_total": tot, "exact": ok})])
+    out.update([row("encode_stress_12000t", statistics.mean(enc_ms), 4 * N + 6 * tot / 10, 2 * N, peak,
+                    {"nnz_mean": tot // 10})])
+    del deltas, anchor_flat, prev_flat, cur_flat, snap_flat, anchor, prev, cur, snap, plan
+    gc.collect()
+    torch.cuda.empty_cache()
+    log(f"rows: stress chain done in {time.time() - t0:.1f}s")
+    return out
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_bf16_delta_b200 as dws
+    import workloads as W
+
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    peak, peak_kind = measured_peaks()
+
+    # ---- workload: Llama-3-8B-shaped set, one step -------------------------
+    t0 = time.time()
+    s = W.SEEDS["llama3_8b"]
+    shapes = llama_shapes(args.layers)
+    sizes = [W.numel(sh) for _, sh in shapes]
+    std = [(0.01, 1.0) if W.is_norm(nm) else (0.02, 0.0) for nm, _ in shapes]
+    T, N = len(sizes), sum(sizes)
+    old_flat, old = W.pack_flat(sizes, lambda t, n: W.init_tensor(n, W.weight_seed(s, t), dev, *std[t]), dev)
+
+    def make_new(lr):
+        def mk(t, n):
+            u = W.update_noise(n, W.step_seed(s, 1, t), dev)
+            return W.optimizer_step(old[t], u, lr)
+        return mk
+
+    new_flat, new = W.pack_flat(sizes, make_new(args.lr), dev)
+    torch.cuda.synchronize()
+    log(f"[rank {rank}] generated {T} tensors, {N} elements in {time.time() - t0:.1f}s")
+
+    plan = dws.DeltaPlan.for_tensors(old)
+    ot, nt = dws.ptr_table(old), dws.ptr_table(new)
+    offsets = plan.count(ot, nt)
+    plan.raise_on_error("dws_count")
+    nnz = int(offsets[-1].item())
+    indices = torch.empty(nnz, dtype=torch.int32, device=dev)
+    values = torch.empty(nnz, dtype=torch.int16, device=dev)
+    delta = dws.Delta(offsets, indices, values)
+    snap_flat = old_flat.clone()
+    snap = [snap_flat[v.storage_offset():][:v.numel()] for v in old]
+    st = dws.ptr_table(snap)
+
+    def encode():
+        plan.encode_into(ot, nt, offsets, indices, values)
+
+    def apply():
+        plan.apply(st, delta)
+
+    for _ in range(args.warmup):
+        encode()
+        apply()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    e_enc0, e_enc1, e_app1 = events(K), events(K), events(K)
+    start, end = events(2)
+    props = torch.cuda.get_device_properties(dev)
+    clocks = Clocks(local, str(getattr(props, "uuid", "")) or None)
+    clocks.start()
+    launches0 = dws.dws_launch_count()
+    start.record()
+    for k in range(K):
+        e_enc0[k].record()
+        encode()
+        e_enc1[k].record()
+        apply()
+        e_app1[k].record()
+    end.record()
+    torch.cuda.synchronize()
+    launches = dws.dws_launch_count() - launches0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    total_ms = start.elapsed_time(end)
+    enc_ms = statistics.mean(e_enc0[k].elapsed_time(e_enc1[k]) for k in range(K))
+    app_ms = statistics.mean(e_enc1[k].elapsed_time(e_app1[k]) for k in range(K))
+    if world > 1:
+        tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        total_ms = float(tmax.item())
+    ms_per_step = total_ms / K
+
+    # correctness of what was timed: the applied snapshot is the new snapshot
+    st_code, st_detail = plan.status()
+    exact = bool(torch.equal(snap_flat, new_flat)) and st_code == dws.DWS_OK
+    if not exact:
+        log(f"[rank {rank}] RESULT MISMATCH (status {st_code}, detail {st_detail})")
+
+    weight_bytes = 2 * N
+    value = world * weight_bytes / (ms_per_step / 1e3) / 1e9
+    enc_alg = 4 * N + 6 * nnz + 8 * (T + 1)
+    achieved = enc_alg / (enc_ms / 1e3) / 1e9
+    tpe, nnz_frac_prof = encode_traffic_per_elem()
+    traffic = None
+    if tpe is not None:
+        traffic = int(tpe * N)
+    app_alg = 8 * nnz
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u16",
+        "data": "synthetic (seeded random bf16 weights of the model's shapes; no trained weights)",
+        "config": {
+            "workload": (f"llama3_8b-shaped bf16 parameter set: {T} tensors, {N} elements "
+                         f"({weight_bytes / 1e9:.2f} GB per snapshot), one simulated optimizer step at lr {args.lr}"),
+            "step": "dws_encode(old,new -> delta) + dws_apply(delta -> snapshot), one launch each over all tensors",
+            "lr": args.lr, "nnz": nnz, "sparsity": round(1 - nnz / N, 6),
+            "delta_bytes": 6 * nnz + 8 * (T + 1),
+            "l2": "inputs (2 x 16 GB) >> 126 MB L2; no flush needed",
+            "parallelism": f"replicas x{world}",
+        },
+        "hbm_frac_step": round((enc_alg + app_alg) / (ms_per_step / 1e3) / 1e9 / peak, 4),
+        "kernels": {
+            "encode": {"ms": round(enc_ms, 4), "alg_bytes": enc_alg,
+                       "alg_GBps": round(achieved, 1), "weight_GBps": round(weight_bytes / enc_ms / 1e6, 1),
+                       "elems_per_s": round(N / enc_ms * 1e3, 1)},
+            "apply": {"ms": round(app_ms, 4), "alg_bytes": app_alg,
+                      "alg_GBps": round(app_alg / app_ms / 1e6, 1),
+                      "weight_GBps": round(weight_bytes / app_ms / 1e6, 1)},
+        },
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "encode (dws_encode: workspace reset + fused detect/scan/compact)",
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "exact": exact,
+    }
+
+    # ---- e2e: new snapshot from pinned host memory, delta through the host --
+    if not args.no_e2e:
+        host_new = torch.empty_like(new_flat, device="cpu").pin_memory()
+        host_new.copy_(new_flat)
+        h_off = torch.empty_like(offsets, device="cpu").pin_memory()
+        h_idx = torch.empty_like(indices, device="cpu").pin_memory()
+        h_val = torch.empty_like(values, device="cpu").pin_memory()
+        r_off, r_idx, r_val = torch.empty_like(offsets), torch.empty_like(indices), torch.empty_like(values)
+        rdelta = dws.Delta(r_off, r_idx, r_val)
+
+        def e2e_step():
+            new_flat.copy_(host_new, non_blocking=True)
+            plan.encode_into(ot, nt, offsets, indices, values)
+            h_off.copy_(offsets, non_blocking=True)
+            h_idx.copy_(indices, non_blocking=True)
+            h_val.copy_(values, non_blocking=True)
+            r_off.copy_(h_off, non_blocking=True)
+            r_idx.copy_(h_idx, non_blocking=True)
+            r_val.copy_(h_val, non_blocking=True)
+            plan.apply(st, rdelta)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = events(2)
+        a.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            tmax = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+            e_ms = float(tmax.item())
+        e_ms /= args.e2e_steps
+        dbytes = 8 * (T + 1) + 6 * nnz
+        ok = bool(torch.equal(snap_flat, new_flat)) and plan.status()[0] == dws.DWS_OK
+        line["e2e"] = {"value": round(world * weight_bytes / (e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+                       "h2d_bytes_per_step": 2 * new_flat.numel() + dbytes,
+                       "d2h_bytes_per_step": dbytes, "ms_per_step": round(e_ms, 3),
+                       "steps": args.e2e_steps, "exact": ok,
+                       "path": "pinned host new snapshot -> H2D -> dws_encode -> delta D2H -> H2D -> dws_apply"}
+        del host_new, h_off, h_idx, h_val, r_off, r_idx, r_val
+
+    # ---- encode / apply at lr 1e-5 and count-only ----------------------------
+    if not args.no_rows:
+        ms_c, _ = time_reps(lambda: plan.count(ot, nt, offsets), args.rows_reps)
+        rows = {}
+        rows.update([row("count_llama3_8b_lr%g" % args.lr, ms_c, 4 * N, weight_bytes, peak)])
+        lr2 = 1e-5
+        for t in range(T):
+            new[t].copy_(make_new(lr2)(t, sizes[t]))
+        offs2 = plan.count(ot, nt)
+        nnz2 = int(offs2[-1].item())
+        del indices, values, delta
+        idx2 = torch.empty(nnz2, dtype=torch.int32, device=dev)
+        val2 = torch.empty(nnz2, dtype=torch.int16, device=dev)
+        d2 = dws.Delta(offs2, idx2, val2)
+        ms_e, mn_e = time_reps(lambda: plan.encode_into(ot, nt, offs2, idx2, val2), args.rows_reps)
+        snap_flat.copy_(old_flat)
+        ms_a, mn_a = time_reps(lambda: plan.apply(st, d2), args.rows_reps)
+        ok = bool(torch.equal(snap_flat, new_flat)) and plan.status()[0] == dws.DWS_OK
+        rows.update([row("encode_llama3_8b_lr1e-5", ms_e, 4 * N + 6 * nnz2, weight_bytes, peak,
+                         {"min_ms": round(mn_e, 4), "nnz": nnz2, "sparsity": round(1 - nnz2 / N, 6)})])
+        rows.update([row("apply_llama3_8b_lr1e-5", ms_a, 8 * nnz2, weight_bytes, peak,
+                         {"min_ms": round(mn_a, 4), "exact": ok})])
+        del old_flat, new_flat, snap_flat, old, new, snap, idx2, val2, d2, offs2
+        import gc
+        gc.collect()
+        torch.cuda.empty_cache()
+        if args.layers is None:
+            rows.update(run_rows(args, dev, peak))
+        line["rows"] = rows
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1) ---------
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        b, sec, n, c = oracle_sample(llama_shapes(args.layers), s, args.lr, dev, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": round(b / sec / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": (f"the first {c} decoder-layer tensors of the same Llama-3-8B-shaped set "
+                       f"({n} elements, {2 * n / 1e9:.2f} GB of weights), oracle encode + apply "
+                       f"in {sec:.1f} s on one thread"),
+            "cpu": cpu_model(), "host_threads": os.cpu_count()}
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0 if exact else 3
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

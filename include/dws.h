@@ -1,0 +1,266 @@
+/*
+ * dws.h -- libdws: delta weight sync kernels for NVIDIA B200 (sm_100a).
+ *
+ * The data-parallel hot path of delta weight sync for asynchronous RL:
+ * bitwise change detection between the pre-step and post-step bf16 weight
+ * snapshots, stream compaction of the changed elements into a sparse delta
+ * (per tensor: ascending int32 element indices and the bf16 values there),
+ * the receiver-side scatter of one delta or of a chain of deltas onto an
+ * anchor snapshot, and the dense XOR-mask variant for packed low-precision
+ * weights.  Everything is integer work on raw bits and bit-exact.
+ *
+ * Sources, by page title and section:
+ *   [TRL]  "Shipping a Trillion Parameters With a Hub Bucket: Delta Weight
+ *          Sync in TRL" (Hugging Face blog, Korean translation) -- §2 why
+ *          bf16 RL updates leave ~99% of weights bit-identical, §4.1 the
+ *          delta format and anchor/delta cadence, §4.2 the trainer's
+ *          snapshot/step/diff, §4.3 the receiver's snap[indices] = values.
+ *   [verl] review of verl PR #6974 (delta_sharded engine), key source
+ *          snippets: sparse_gather.py (shard_delta_indices,
+ *          gather_v_batched_to_rank0), encode.py; risks list (int32
+ *          position overflow).
+ *   [XOR]  humans& weight-sync summary ("... کمتر از ۰.۲۳ ثانیه توقف"),
+ *          paragraphs 1-3: XOR mask delta, per-layer double buffering.
+ *
+ * Conventions for every entry point
+ *   - All device buffers are allocated and owned by the caller.  libdws never
+ *     allocates device memory; a plan owns a little host memory only.
+ *   - Every call enqueues work on the caller's stream and returns without
+ *     waiting for it (except dws_status, which synchronises).  `stream` is a
+ *     cudaStream_t; NULL means the legacy default stream.
+ *   - The return value covers errors the host can see (bad sizes, null
+ *     pointers, a workspace that is too small, a failed launch).  Errors only
+ *     the device can see (output capacity exceeded, an index out of range in
+ *     a delta, a bounded wait that ran out) are recorded in the workspace's
+ *     status word and read with dws_status().
+ *   - "device array" means an array in device memory; "host array" an array
+ *     in host memory that may be freed as soon as the call returns.
+ *   - Calls that share one workspace must be ordered on one stream (or by
+ *     events): the workspace holds per-call scratch.
+ *   - Element indices are local to their tensor, 0-based, row-major flat,
+ *     and int32: a tensor must have fewer than 2^31 elements ([verl] lists
+ *     silent int32 wrap-around of positions as a risk; here it is rejected).
+ */
+#ifndef DWS_H
+#define DWS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DWS_API __attribute__((visibility("default")))
+#else
+#define DWS_API
+#endif
+
+/* Layout-compatible with cudaStream_t; declared here so that this header does
+ * not need the CUDA headers. */
+typedef struct CUstream_st *dws_stream_t;
+
+typedef enum dws_status {
+    DWS_OK = 0,
+    DWS_ERR_INVALID = 1,     /* bad argument (host), or bad pointer/table seen on the device */
+    DWS_ERR_UNSUPPORTED = 2, /* element size other than 2 bytes for encode/apply */
+    DWS_ERR_CAPACITY = 3,    /* device: more changed elements than the output capacity */
+    DWS_ERR_BAD_DELTA = 4,   /* device: delta index out of range, not ascending, bad offsets */
+    DWS_ERR_TIMEOUT = 5,     /* device: a bounded wait in the encode scan ran out */
+    DWS_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+    DWS_ERR_WORKSPACE = 7    /* workspace too small, or not prepared for this plan */
+} dws_status_t;
+
+/* Opaque host-side description of a list of tensors (a model's parameters). */
+typedef struct dws_plan dws_plan_t;
+
+/* ------------------------------------------------------------------------
+ * Plan: the multi-tensor descriptor table.
+ * One launch of any kernel below covers every tensor of the plan ([verl]
+ * sparse_gather.py batches K parameters into one collective round and the
+ * review records replacing per-parameter .item() loops by one transfer; here
+ * the same idea makes one kernel launch cover a whole model).
+ * ------------------------------------------------------------------------ */
+
+/* Create a plan for `num_tensors` tensors with `numels[t]` elements each
+ * (host array) of `elem_size` bytes.  0 <= numels[t] < 2^31; empty tensors are
+ * allowed.  The sparse path compares 16-bit patterns, so elem_size must be 2
+ * (bf16); any other size returns DWS_ERR_UNSUPPORTED, as the verl helper
+ * refuses element sizes it has no integer view for.
+ * Errors: DWS_ERR_INVALID for num_tensors <= 0, a null pointer or a numel out
+ * of range; DWS_ERR_UNSUPPORTED for elem_size != 2.  On success *plan_out owns
+ * host memory; free it with dws_plan_destroy. */
+DWS_API dws_status_t dws_plan_create(const int64_t *numels, int32_t num_tensors, int32_t elem_size,
+                             dws_plan_t **plan_out);
+DWS_API void dws_plan_destroy(dws_plan_t *plan);
+
+DWS_API int32_t dws_plan_num_tensors(const dws_plan_t *plan);
+DWS_API int64_t dws_plan_num_elements(const dws_plan_t *plan);
+/* Encode/apply-chain work units: tensors are cut into tiles of
+ * dws_tile_elems() elements; a tile never straddles two tensors and an empty
+ * tensor still has one (empty) tile. */
+DWS_API int64_t dws_plan_num_tiles(const dws_plan_t *plan);
+DWS_API int64_t dws_tile_elems(void);
+
+/* Bytes of device workspace the plan needs (a few bytes per tile plus the
+ * tensor table).  The caller allocates it (256-byte alignment or better). */
+DWS_API size_t dws_plan_workspace_bytes(const dws_plan_t *plan);
+
+/* Write the plan's tables into `workspace` (enqueued on `stream`).  Call once
+ * per workspace before the first dws_count/encode/apply/apply_chain that uses
+ * it, and again if the workspace was used for another plan.  Kernels check a
+ * fingerprint of the plan in the workspace and record DWS_ERR_WORKSPACE
+ * (doing nothing else) when it does not match.
+ * Errors: DWS_ERR_INVALID (null), DWS_ERR_WORKSPACE (too small), DWS_ERR_CUDA. */
+DWS_API dws_status_t dws_plan_upload(const dws_plan_t *plan, void *workspace,
+                             size_t workspace_bytes, dws_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Encode: change detection + scan + compaction, one fused kernel.
+ * [verl] sparse_gather.py shard_delta_indices: mask = new.view(int) !=
+ * snap.view(int); local_idx = mask.nonzero(); values = new[local_idx].
+ * [TRL] §4.1: a delta stores, per changed parameter, int32 element indices
+ * and the bf16 values at those indices; §4.2: the mask comes from comparing
+ * bf16 snapshots taken before and after the optimizer step.
+ * ------------------------------------------------------------------------ */
+
+/* old_ptrs, new_ptrs: device arrays of num_tensors device pointers; tensor t
+ *   is a contiguous array of numels[t] bf16 values (2-byte aligned; 16-byte
+ *   alignment takes the fast path).  An element is changed iff its 16-bit
+ *   pattern differs (so +0/-0 differ and identical NaN bits do not).
+ * offsets: device array [num_tensors + 1] (int64), written: offsets[0] = 0,
+ *   tensor t's entries are [offsets[t], offsets[t+1]), offsets[T] = nnz.
+ * indices, values: device arrays of `capacity` entries; entry j holds the
+ *   tensor-local index (ascending within a tensor) and the new bf16 bits.
+ *   Tensors appear in plan order.
+ * If nnz > capacity, the first `capacity` entries are written, offsets are
+ *   still complete, and DWS_ERR_CAPACITY is recorded with detail = nnz.
+ * workspace: prepared by dws_plan_upload.  Old and new snapshots are only
+ *   read. */
+DWS_API dws_status_t dws_encode(const dws_plan_t *plan,
+                        const void *const *old_ptrs, const void *const *new_ptrs,
+                        int64_t *offsets, int32_t *indices, uint16_t *values,
+                        int64_t capacity,
+                        void *workspace, size_t workspace_bytes, dws_stream_t stream);
+
+/* dws_encode with explicit controls of the scan's bounded wait.
+ * wait_limit_ns: how long a tile waits for its predecessor's count before it
+ *   records DWS_ERR_TIMEOUT and every waiting tile gives up (<= 0: 2 s).
+ * debug_withhold_tile: -1 normally.  A tile number >= 0 makes that tile never
+ *   publish its count, so that its successors' wait runs out: a host-driven
+ *   way to test the timeout path without faulting anything. */
+DWS_API dws_status_t dws_encode_ex(const dws_plan_t *plan,
+                           const void *const *old_ptrs, const void *const *new_ptrs,
+                           int64_t *offsets, int32_t *indices, uint16_t *values,
+                           int64_t capacity,
+                           void *workspace, size_t workspace_bytes, dws_stream_t stream,
+                           int64_t wait_limit_ns, int64_t debug_withhold_tile);
+
+/* Detect + scan only: writes offsets[num_tensors + 1] (per-tensor change
+ * counts as a prefix, offsets[T] = nnz) and no entries.  Lets a caller size
+ * the index/value buffers before dws_encode.  Same arguments as dws_encode. */
+DWS_API dws_status_t dws_count(const dws_plan_t *plan,
+                       const void *const *old_ptrs, const void *const *new_ptrs,
+                       int64_t *offsets,
+                       void *workspace, size_t workspace_bytes, dws_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Apply: [TRL] §4.3 receive_weights -- for each changed parameter,
+ * snap.flatten()[indices] = values, in place on the receiver's snapshot
+ * (the vLLM PR it cites applies with index_copy_ in place; [verl]'s SGLang
+ * loader does an in-place masked copy).
+ * ------------------------------------------------------------------------ */
+
+/* snap_ptrs: device array of num_tensors device pointers to the bf16
+ *   snapshots, modified in place.
+ * offsets, indices, values: one delta in the dws_encode layout (device).
+ * count: number of entries the index/value arrays hold (host value, usually
+ *   nnz).  Entries j >= min(count, offsets[T]) are never read.
+ * Every index is range-checked against its tensor's numel and required to be
+ * ascending within its tensor; a violating entry is skipped and
+ * DWS_ERR_BAD_DELTA recorded (detail = entry number).  offsets must start at
+ * 0, be non-decreasing and end at <= count, else DWS_ERR_BAD_DELTA and
+ * nothing is written. */
+DWS_API dws_status_t dws_apply(const dws_plan_t *plan, void *const *snap_ptrs,
+                       const int64_t *offsets, const int32_t *indices,
+                       const uint16_t *values, int64_t count,
+                       void *workspace, size_t workspace_bytes, dws_stream_t stream);
+
+/* One delta of a chain (device pointers; count as in dws_apply). */
+typedef struct dws_delta {
+    const int64_t *offsets;
+    const int32_t *indices;
+    const uint16_t *values;
+    int64_t count;
+} dws_delta_t;
+
+#define DWS_MAX_CHAIN 64
+
+/* Anchor + delta chain ([TRL] §4.1: an anchor every N syncs, sparse deltas in
+ * between; a new replica takes the latest anchor and replays the deltas after
+ * it).  Applies deltas[0..K-1] in order onto snap_ptrs in ONE launch: each
+ * block owns a range of elements and replays all K deltas over it, so where
+ * deltas touch the same element the later one wins, exactly as K sequential
+ * dws_apply calls.  deltas: host array of K (1 <= K <= DWS_MAX_CHAIN).
+ * Indices are range-checked (DWS_ERR_BAD_DELTA, entry skipped). */
+DWS_API dws_status_t dws_apply_chain(const dws_plan_t *plan, void *const *snap_ptrs,
+                             const dws_delta_t *deltas, int32_t K,
+                             void *workspace, size_t workspace_bytes, dws_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * XOR-mask variant, [XOR] paragraph 1: mask = old ^ new bit by bit, the same
+ * size as the model; the receiver gets new = old ^ mask with no
+ * floating-point arithmetic.  Works on any bytes (e.g. packed NVFP4).
+ * ------------------------------------------------------------------------ */
+
+/* mask[b] = old[b] ^ new[b] for b < nbytes (device pointers, any alignment;
+ * equal alignment mod 16 takes the vector path).  nbytes >= 0. */
+DWS_API dws_status_t dws_xor_encode(const void *old_bytes, const void *new_bytes, void *mask,
+                            int64_t nbytes, dws_stream_t stream);
+
+/* buf[b] ^= mask[b] for b < nbytes, in place (device pointers). */
+DWS_API dws_status_t dws_xor_apply(void *buf, const void *mask, int64_t nbytes, dws_stream_t stream);
+
+/* Per-layer double-buffered XOR apply ([XOR] paragraph 3: one engine fills a
+ * buffer with the next layer's mask while the XOR kernel applies the other;
+ * the two buffers hold two layers, so the KV cache does not have to go).
+ * For each layer l: bufs[l] ^= masks[l] over nbytes[l] bytes.  The mask is
+ * first copied (cudaMemcpyAsync, any source the runtime can read: device
+ * memory or pinned host memory) into staging buffer (u % 2) on copy_stream
+ * while the previous unit is applied on apply_stream; a layer larger than
+ * staging_bytes is split into staging-sized units.  Events order the two
+ * streams; copy_stream first waits for work already queued on apply_stream,
+ * and when the call's work on apply_stream is done, all of it is done.
+ * bufs, masks, nbytes: host arrays of L entries (device/host pointers).
+ * staging0/1: device buffers of staging_bytes each (caller-owned). */
+DWS_API dws_status_t dws_xor_apply_layers(void *const *bufs, const void *const *masks,
+                                  const int64_t *nbytes, int32_t L,
+                                  void *staging0, void *staging1, int64_t staging_bytes,
+                                  dws_stream_t apply_stream, dws_stream_t copy_stream);
+
+/* ------------------------------------------------------------------------
+ * Status
+ * ------------------------------------------------------------------------ */
+
+/* Wait for `stream`, read the workspace's status word, clear it, and return
+ * it (DWS_OK if no device error since the last read).  *detail (nullable)
+ * receives the error's detail value (required nnz for DWS_ERR_CAPACITY,
+ * entry number for DWS_ERR_BAD_DELTA, tile number for DWS_ERR_TIMEOUT). */
+DWS_API dws_status_t dws_status(void *workspace, int64_t *detail, dws_stream_t stream);
+
+DWS_API const char *dws_strerror(dws_status_t status);
+
+/* Number of kernels libdws has launched in this process so far (all devices,
+ * all entry points).  A diagnostic: the difference across a region of calls is
+ * the number of libdws kernels that region enqueued. */
+DWS_API uint64_t dws_launch_count(void);
+
+/* Library version, e.g. "libdws 0.1 sm_100a". */
+DWS_API const char *dws_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DWS_H */

@@ -1,0 +1,385 @@
+"""Python binding of libdws, the B200 (sm_100a) delta weight sync library.
+
+Two layers, both argument marshalling only -- every step of the hot path runs
+in libdws's CUDA kernels:
+
+* ``dws_*`` functions with the C ABI's names and arguments (pointers as
+  Python ints, streams as ``torch.cuda.Stream.cuda_stream`` ints).
+* ``DeltaPlan`` and a few helpers that take torch CUDA tensors, allocate
+  outputs / workspace with torch and call the ``dws_*`` functions.
+
+Importing this package loads ``libdws.so`` from the package directory and
+raises ``ImportError`` if it is missing: there is no CPU fallback.  Build it
+with ``python -m sparse_bf16_delta_b200._build`` (or ``__graft_entry__.build()``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdws.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libdws.so not found at {LIB_PATH}; build it with "
+        "`python -m sparse_bf16_delta_b200._build` (needs nvcc for sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# Status codes (include/dws.h)
+DWS_OK = 0
+DWS_ERR_INVALID = 1
+DWS_ERR_UNSUPPORTED = 2
+DWS_ERR_CAPACITY = 3
+DWS_ERR_BAD_DELTA = 4
+DWS_ERR_TIMEOUT = 5
+DWS_ERR_CUDA = 6
+DWS_ERR_WORKSPACE = 7
+DWS_MAX_CHAIN = 64
+
+_i32, _i64, _sz, _vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
+
+
+class dws_delta_t(ctypes.Structure):
+    _fields_ = [("offsets", _vp), ("indices", _vp), ("values", _vp), ("count", _i64)]
+
+
+def _sig(name, restype, argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = argtypes
+    return f
+
+
+_sig("dws_plan_create", _i32, [_vp, _i32, _i32, ctypes.POINTER(_vp)])
+_sig("dws_plan_destroy", None, [_vp])
+_sig("dws_plan_num_tensors", _i32, [_vp])
+_sig("dws_plan_num_elements", _i64, [_vp])
+_sig("dws_plan_num_tiles", _i64, [_vp])
+_sig("dws_tile_elems", _i64, [])
+_sig("dws_plan_workspace_bytes", _sz, [_vp])
+_sig("dws_plan_upload", _i32, [_vp, _vp, _sz, _vp])
+_sig("dws_encode", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
+_sig("dws_encode_ex", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _i64, _i64])
+_sig("dws_count", _i32, [_vp, _vp, _vp, _vp, _vp, _sz, _vp])
+_sig("dws_apply", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
+_sig("dws_apply_chain", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _vp, _sz, _vp])
+_sig("dws_xor_encode", _i32, [_vp, _vp, _vp, _i64, _vp])
+_sig("dws_xor_apply", _i32, [_vp, _vp, _i64, _vp])
+_sig("dws_xor_apply_layers", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i64, _vp, _vp])
+_sig("dws_status", _i32, [_vp, ctypes.POINTER(_i64), _vp])
+_sig("dws_strerror", ctypes.c_char_p, [_i32])
+_sig("dws_version", ctypes.c_char_p, [])
+_sig("dws_launch_count", ctypes.c_uint64, [])
+
+
+class DwsError(RuntimeError):
+    def __init__(self, code: int, where: str, detail: int | None = None):
+        self.code = int(code)
+        self.detail = detail
+        msg = f"{where}: {dws_strerror(code)} (status {code})"
+        if detail is not None:
+            msg += f", detail {detail}"
+        super().__init__(msg)
+
+
+def _check(code: int, where: str) -> None:
+    if code != DWS_OK:
+        raise DwsError(code, where)
+
+
+# ---------------------------------------------------------------------------
+# C-ABI names (pointers and streams as ints)
+# ---------------------------------------------------------------------------
+
+def dws_plan_create(numels, elem_size: int = 2) -> int:
+    arr = (ctypes.c_int64 * max(1, len(numels)))(*[int(n) for n in numels])
+    out = _vp()
+    _check(_lib.dws_plan_create(arr, len(numels), int(elem_size), ctypes.byref(out)),
+           "dws_plan_create")
+    return out.value
+
+
+def dws_plan_destroy(plan: int) -> None:
+    _lib.dws_plan_destroy(plan)
+
+
+def dws_plan_num_tensors(plan: int) -> int:
+    return _lib.dws_plan_num_tensors(plan)
+
+
+def dws_plan_num_elements(plan: int) -> int:
+    return _lib.dws_plan_num_elements(plan)
+
+
+def dws_plan_num_tiles(plan: int) -> int:
+    return _lib.dws_plan_num_tiles(plan)
+
+
+def dws_tile_elems() -> int:
+    return _lib.dws_tile_elems()
+
+
+def dws_plan_workspace_bytes(plan: int) -> int:
+    return _lib.dws_plan_workspace_bytes(plan)
+
+
+def dws_plan_upload(plan, workspace, workspace_bytes, stream) -> int:
+    return _lib.dws_plan_upload(plan, workspace, workspace_bytes, stream)
+
+
+def dws_encode(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, workspace,
+               workspace_bytes, stream) -> int:
+    return _lib.dws_encode(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
+                           workspace, workspace_bytes, stream)
+
+
+def dws_encode_ex(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, workspace,
+                  workspace_bytes, stream, wait_limit_ns, debug_withhold_tile) -> int:
+    return _lib.dws_encode_ex(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
+                              workspace, workspace_bytes, stream, wait_limit_ns,
+                              debug_withhold_tile)
+
+
+def dws_count(plan, old_ptrs, new_ptrs, offsets, workspace, workspace_bytes, stream) -> int:
+    return _lib.dws_count(plan, old_ptrs, new_ptrs, offsets, workspace, workspace_bytes, stream)
+
+
+def dws_apply(plan, snap_ptrs, offsets, indices, values, count, workspace, workspace_bytes,
+              stream) -> int:
+    return _lib.dws_apply(plan, snap_ptrs, offsets, indices, values, count, workspace,
+                          workspace_bytes, stream)
+
+
+def dws_apply_chain(plan, snap_ptrs, deltas, K, workspace, workspace_bytes, stream) -> int:
+    """``deltas``: a ctypes array of dws_delta_t (see ``make_delta_array``)."""
+    return _lib.dws_apply_chain(plan, snap_ptrs, deltas, K, workspace, workspace_bytes, stream)
+
+
+def dws_xor_encode(old_bytes, new_bytes, mask, nbytes, stream) -> int:
+    return _lib.dws_xor_encode(old_bytes, new_bytes, mask, nbytes, stream)
+
+
+def dws_xor_apply(buf, mask, nbytes, stream) -> int:
+    return _lib.dws_xor_apply(buf, mask, nbytes, stream)
+
+
+def dws_xor_apply_layers(bufs, masks, nbytes, L, staging0, staging1, staging_bytes,
+                         apply_stream, copy_stream) -> int:
+    """``bufs``, ``masks``: ctypes void* arrays; ``nbytes``: ctypes int64 array."""
+    return _lib.dws_xor_apply_layers(bufs, masks, nbytes, L, staging0, staging1, staging_bytes,
+                                     apply_stream, copy_stream)
+
+
+def dws_status(workspace, stream):
+    """Returns (status, detail) and clears the workspace's status word."""
+    detail = ctypes.c_int64(0)
+    st = _lib.dws_status(workspace, ctypes.byref(detail), stream)
+    return int(st), int(detail.value)
+
+
+def dws_strerror(code: int) -> str:
+    return _lib.dws_strerror(int(code)).decode()
+
+
+def dws_version() -> str:
+    return _lib.dws_version().decode()
+
+
+def dws_launch_count() -> int:
+    return int(_lib.dws_launch_count())
+
+
+def make_delta_array(deltas):
+    """[(offsets_ptr, indices_ptr, values_ptr, count), ...] -> ctypes array."""
+    arr = (dws_delta_t * max(1, len(deltas)))()
+    for k, (o, i, v, c) in enumerate(deltas):
+        arr[k] = dws_delta_t(o, i, v, c)
+    return arr
+
+
+def make_ptr_array(ptrs):
+    arr = (ctypes.c_void_p * max(1, len(ptrs)))()
+    for k, p in enumerate(ptrs):
+        arr[k] = p
+    return arr
+
+
+# ---------------------------------------------------------------------------
+# torch convenience layer (allocation + marshalling)
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream=None) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def ptr_table(tensors, device=None):
+    """Device int64 array of the tensors' data pointers (the per-call
+    pointer arrays the C ABI takes)."""
+    torch = _torch()
+    dev = device if device is not None else tensors[0].device
+    ptrs = [int(t.data_ptr()) if t.numel() > 0 else 0 for t in tensors]
+    return torch.tensor(ptrs, dtype=torch.int64).to(dev, non_blocking=False)
+
+
+class Delta:
+    """One sparse delta on the device: offsets int64[T+1], indices int32[n],
+    values as bf16 bits (int16 storage) [n]."""
+
+    def __init__(self, offsets, indices, values):
+        self.offsets = offsets
+        self.indices = indices
+        self.values = values
+
+    @property
+    def count(self) -> int:
+        return int(self.indices.numel())
+
+    def nnz(self) -> int:
+        return int(self.offsets[-1].item())
+
+    def as_ref(self):
+        return (self.offsets.data_ptr(), self.indices.data_ptr() if self.count else 0,
+                self.values.data_ptr() if self.count else 0, self.count)
+
+
+class DeltaPlan:
+    """A plan (multi-tensor descriptor table) for a list of bf16 tensors with a
+    torch-allocated, uploaded workspace."""
+
+    def __init__(self, numels, device="cuda", elem_size: int = 2, stream=None):
+        torch = _torch()
+        self.numels = [int(n) for n in numels]
+        self.handle = dws_plan_create(self.numels, elem_size)
+        self.device = torch.device(device)
+        self.workspace_bytes = dws_plan_workspace_bytes(self.handle)
+        self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)
+        _check(dws_plan_upload(self.handle, self.workspace.data_ptr(), self.workspace_bytes,
+                               _stream_handle(stream)), "dws_plan_upload")
+
+    @classmethod
+    def for_tensors(cls, tensors, **kw):
+        return cls([t.numel() for t in tensors], device=tensors[0].device, **kw)
+
+    @property
+    def num_tensors(self) -> int:
+        return len(self.numels)
+
+    @property
+    def num_elements(self) -> int:
+        return dws_plan_num_elements(self.handle)
+
+    @property
+    def num_tiles(self) -> int:
+        return dws_plan_num_tiles(self.handle)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            dws_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- status --
+    def status(self, stream=None):
+        return dws_status(self.workspace.data_ptr(), _stream_handle(stream))
+
+    def raise_on_error(self, where="libdws", stream=None):
+        st, detail = self.status(stream)
+        if st != DWS_OK:
+            raise DwsError(st, where, detail)
+
+    # -- encode --
+    def count(self, old_table, new_table, offsets=None, stream=None):
+        torch = _torch()
+        if offsets is None:
+            offsets = torch.empty(self.num_tensors + 1, dtype=torch.int64, device=self.device)
+        _check(dws_count(self.handle, old_table.data_ptr(), new_table.data_ptr(),
+                         offsets.data_ptr(), self.workspace.data_ptr(), self.workspace_bytes,
+                         _stream_handle(stream)), "dws_count")
+        return offsets
+
+    def encode_into(self, old_table, new_table, offsets, indices, values, stream=None):
+        _check(dws_encode(self.handle, old_table.data_ptr(), new_table.data_ptr(),
+                          offsets.data_ptr(), indices.data_ptr() if indices.numel() else 0,
+                          values.data_ptr() if values.numel() else 0, int(indices.numel()),
+                          self.workspace.data_ptr(), self.workspace_bytes,
+                          _stream_handle(stream)), "dws_encode")
+
+    def encode(self, old_table, new_table, capacity: int, stream=None) -> Delta:
+        """One-pass encode into buffers of `capacity` entries (trimmed to nnz;
+        raises DwsError(DWS_ERR_CAPACITY) if nnz > capacity)."""
+        torch = _torch()
+        offsets = torch.empty(self.num_tensors + 1, dtype=torch.int64, device=self.device)
+        indices = torch.empty(max(0, capacity), dtype=torch.int32, device=self.device)
+        values = torch.empty(max(0, capacity), dtype=torch.int16, device=self.device)
+        self.encode_into(old_table, new_table, offsets, indices, values, stream)
+        self.raise_on_error("dws_encode", stream)
+        nnz = int(offsets[-1].item())
+        return Delta(offsets, indices[:nnz], values[:nnz])
+
+    def encode_exact(self, old_table, new_table, stream=None) -> Delta:
+        """Count first, then encode into exactly-sized buffers (two passes)."""
+        offsets = self.count(old_table, new_table, stream=stream)
+        self.raise_on_error("dws_count", stream)
+        return self.encode(old_table, new_table, int(offsets[-1].item()), stream)
+
+    # -- apply --
+    def apply(self, snap_table, delta: Delta, stream=None):
+        o, i, v, c = delta.as_ref()
+        _check(dws_apply(self.handle, snap_table.data_ptr(), o, i, v, c,
+                         self.workspace.data_ptr(), self.workspace_bytes,
+                         _stream_handle(stream)), "dws_apply")
+
+    def apply_chain(self, snap_table, deltas, stream=None):
+        arr = make_delta_array([d.as_ref() for d in deltas])
+        _check(dws_apply_chain(self.handle, snap_table.data_ptr(), arr, len(deltas),
+                               self.workspace.data_ptr(), self.workspace_bytes,
+                               _stream_handle(stream)), "dws_apply_chain")
+
+
+def xor_encode(old, new, mask=None, stream=None):
+    """mask = old ^ new over the tensors' bytes (device tensors)."""
+    torch = _torch()
+    nbytes = old.numel() * old.element_size()
+    if new.numel() * new.element_size() != nbytes:
+        raise ValueError("size mismatch")
+    if mask is None:
+        mask = torch.empty(nbytes, dtype=torch.uint8, device=old.device)
+    _check(dws_xor_encode(old.data_ptr(), new.data_ptr(), mask.data_ptr(), nbytes,
+                          _stream_handle(stream)), "dws_xor_encode")
+    return mask
+
+
+def xor_apply(buf, mask, stream=None):
+    """buf ^= mask in place over buf's bytes."""
+    nbytes = buf.numel() * buf.element_size()
+    if mask.numel() * mask.element_size() != nbytes:
+        raise ValueError("size mismatch")
+    _check(dws_xor_apply(buf.data_ptr(), mask.data_ptr(), nbytes, _stream_handle(stream)),
+           "dws_xor_apply")
+
+
+def xor_apply_layers(bufs, masks, staging0, staging1, apply_stream=None, copy_stream=None):
+    """Double-buffered per-layer XOR apply (see dws_xor_apply_layers)."""
+    L = len(bufs)
+    nb = (ctypes.c_int64 * max(1, L))(*[b.numel() * b.element_size() for b in bufs])
+    sb = min(staging0.numel() * staging0.element_size(),
+             staging1.numel() * staging1.element_size())
+    _check(dws_xor_apply_layers(make_ptr_array([b.data_ptr() for b in bufs]),
+                                make_ptr_array([m.data_ptr() for m in masks]), nb, L,
+                                staging0.data_ptr(), staging1.data_ptr(), sb,
+                                _stream_handle(apply_stream), _stream_handle(copy_stream)),
+           "dws_xor_apply_layers")

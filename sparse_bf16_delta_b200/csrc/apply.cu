@@ -1,0 +1,470 @@
+// apply.cu -- receiver side: scatter one delta, or replay a chain of deltas
+// onto an anchor, in place.
+//
+// What it computes ("Delta Weight Sync in TRL" §4.3 receive_weights): for
+// each tensor t and entry j of its segment, snap_t[indices[j]] = values[j];
+// for a chain (§4.1: anchor every N syncs, a new replica replays the deltas
+// after the latest anchor) the deltas in order, the later one winning.
+//
+// dws_apply -- one delta, direct scatter.  Each CTA takes 2048 consecutive
+//   entries (coalesced index/value reads), finds their tensors by binary
+//   search over offsets, range-checks every index and stores the 2-byte
+//   values.  DRAM traffic is the touched 32-byte sectors (read-modify-write)
+//   plus 6 bytes per entry, which is less than streaming the snapshot through
+//   at the densities the workloads have.
+//
+// dws_apply_chain -- K deltas, one launch, merge mode.  Each CTA owns a
+//   contiguous range of snapshot tiles (8192 elements).  Per tile: a 1-D bulk
+//   async copy brings the snapshot tile into shared memory while the CTA reads
+//   every delta's entries for the tile (one cursor per delta, advanced tile
+//   by tile, so each delta is binary-searched only once per CTA) and tags them
+//   into a shared array with atomicMax on ((k+1) << 16 | value): the highest k,
+//   i.e. the latest delta, wins regardless of thread order.  The merged tile
+//   goes back with a bulk store.  Traffic: the snapshot read and written once
+//   plus 6 bytes per entry, instead of K read-modify-write scatters.
+#include <cuda_runtime.h>
+
+#include "dws_internal.cuh"
+
+namespace dws {
+namespace {
+
+constexpr unsigned long long kLoadWaitLimitNs = 4000000000ull;  // 4 s
+
+// ---------------------------------------------------------------------------
+// Validation of the deltas' offsets (one CTA per delta), before any write.
+// ---------------------------------------------------------------------------
+struct CheckParams {
+    WsView ws;
+    DeltaRef d[DWS_MAX_CHAIN];
+    int K;
+};
+
+__global__ void delta_check_kernel(CheckParams p) {
+    if (!ws_matches(p.ws)) return;
+    const DeltaRef d = p.d[blockIdx.x];
+    const int T = p.ws.num_tensors;
+    int bad = 0;
+    if (threadIdx.x == 0) {
+        bad |= (d.offsets[0] != 0);
+        bad |= (d.offsets[T] > d.count);
+    }
+    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+        bad |= (d.offsets[t] > d.offsets[t + 1]);
+    }
+    bad = __syncthreads_or(bad);
+    if (threadIdx.x == 0) {
+        if (bad) {
+            atomicOr(&p.ws.hdr->delta_bad, 1u);
+            record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, -1 - static_cast<long long>(blockIdx.x));
+        }
+    }
+}
+
+__global__ void delta_flag_clear_kernel(WsView ws) { ws.hdr->delta_bad = 0u; }
+
+// Largest t in [lo, hi] with offsets[t] <= j (offsets validated non-decreasing).
+__device__ __forceinline__ int tensor_of_entry(const long long *offsets, int lo, int hi,
+                                               long long j) {
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offsets[mid] <= j) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// ---------------------------------------------------------------------------
+// Single delta: direct scatter
+// ---------------------------------------------------------------------------
+constexpr int kApplyThreads = 256;
+constexpr int kApplyPerThread = 8;
+constexpr int kApplyEntries = kApplyThreads * kApplyPerThread;
+
+struct ApplyParams {
+    WsView ws;
+    uint16_t *const *snap_ptrs;
+    DeltaRef d;
+};
+
+__global__ void __launch_bounds__(kApplyThreads) apply_kernel(ApplyParams p) {
+    __shared__ int s_t0, s_t1, s_go;
+    __shared__ long long s_end;
+    if (!ws_matches(p.ws)) return;
+    const int T = p.ws.num_tensors;
+    const long long base = static_cast<long long>(blockIdx.x) * kApplyEntries;
+    if (threadIdx.x == 0) {
+        const long long nnz = p.d.offsets[T];
+        const long long total = nnz < p.d.count ? nnz : p.d.count;
+        long long end = base + kApplyEntries;
+        if (end > total) end = total;
+        s_end = end;
+        s_go = (ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) == 0u) && base < end;
+        if (s_go) {
+            s_t0 = tensor_of_entry(p.d.offsets, 0, T - 1, base);
+            s_t1 = tensor_of_entry(p.d.offsets, s_t0, T - 1, end - 1);
+        }
+    }
+    __syncthreads();
+    if (!s_go) return;
+    const long long end = s_end;
+    const int t0 = s_t0, t1 = s_t1;
+
+    int idx[kApplyPerThread];
+    uint16_t val[kApplyPerThread];
+#pragma unroll
+    for (int r = 0; r < kApplyPerThread; ++r) {
+        const long long j = base + threadIdx.x + r * kApplyThreads;
+        if (j < end) {
+            idx[r] = __ldg(p.d.indices + j);
+            val[r] = __ldg(p.d.values + j);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kApplyPerThread; ++r) {
+        const long long j = base + threadIdx.x + r * kApplyThreads;
+        if (j >= end) continue;
+        const int t = (t0 == t1) ? t0 : tensor_of_entry(p.d.offsets, t0, t1, j);
+        const long long n = p.ws.numel[t];
+        const long long seg = p.d.offsets[t];
+        const int i = idx[r];
+        bool ok = (i >= 0) && (static_cast<long long>(i) < n);
+        if (ok && j > seg) ok = (__ldg(p.d.indices + j - 1) < i);
+        uint16_t *dst = p.snap_ptrs[t];
+        if (ok && dst != nullptr && (reinterpret_cast<uintptr_t>(dst) & 1u) == 0) {
+            dst[i] = val[r];
+        } else {
+            record_error(p.ws.hdr, ok ? DWS_ERR_INVALID : DWS_ERR_BAD_DELTA, j);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Chain replay: tile merge
+// ---------------------------------------------------------------------------
+constexpr int kChainThreads = 256;
+constexpr int kChainMaxSlots = 4096;  // K * block_len entries read per round
+
+struct ChainParams {
+    WsView ws;
+    uint16_t *const *snap_ptrs;
+    long long tiles_per_cta;
+    int K;
+    int block_len;  // entries read per delta per round
+    DeltaRef d[DWS_MAX_CHAIN];
+};
+
+struct TileMeta {
+    uint16_t *ptr;  // tile start in the snapshot
+    int tensor;
+    int local_start;
+    int count;
+    int bulk;  // leading elements moved by bulk copies (multiple of 8)
+};
+
+struct ChainSmem {
+    uint16_t tile[2][kTileElems];
+    uint32_t tag[kTileElems];
+    long long cur[DWS_MAX_CHAIN];
+    long long end[DWS_MAX_CHAIN];
+    int consumed[DWS_MAX_CHAIN];
+    int active[DWS_MAX_CHAIN];
+    unsigned long long bar[2];
+    TileMeta meta[2];
+};
+
+// Thread 0: describe tile i and start its load into buffer b.
+__device__ void chain_issue(const ChainParams &p, ChainSmem &sm, long long i, int b,
+                            unsigned long long policy) {
+    TileMeta m;
+    m.ptr = nullptr;
+    m.tensor = 0;
+    m.local_start = 0;
+    m.count = 0;
+    m.bulk = 0;
+    const int t = p.ws.tile_tensor[i];
+    if (t >= 0 && t < p.ws.num_tensors) {
+        const long long ls = (i - p.ws.first_tile[t]) << kTileShift;
+        const long long n = p.ws.numel[t];
+        if (ls >= 0 && ls <= n) {
+            const long long rest = n - ls;
+            m.tensor = t;
+            m.local_start = static_cast<int>(ls);
+            m.count = static_cast<int>(rest < kTileElems ? rest : kTileElems);
+            uint16_t *sp = p.snap_ptrs[t];
+            const uintptr_t ua = reinterpret_cast<uintptr_t>(sp);
+            if (m.count > 0 && (sp == nullptr || (ua & 1u))) {
+                record_error(p.ws.hdr, DWS_ERR_INVALID, t);
+                m.count = 0;
+            } else if (m.count > 0) {
+                m.ptr = sp + ls;
+                m.bulk = (ua & 15u) == 0 ? (m.count & ~7) : 0;
+            }
+        } else {
+            record_error(p.ws.hdr, DWS_ERR_WORKSPACE, i);
+        }
+    } else {
+        record_error(p.ws.hdr, DWS_ERR_WORKSPACE, i);
+    }
+    mbar_arrive_expect_tx(&sm.bar[b], static_cast<uint32_t>(m.bulk) * 2u);
+    if (m.bulk > 0) bulk_load(sm.tile[b], m.ptr, static_cast<uint32_t>(m.bulk) * 2u, &sm.bar[b], policy);
+    sm.meta[b] = m;
+}
+
+// Warp-cooperative lower bound: first position in [lo, hi) whose index is
+// >= key (indices ascending within the segment).
+__device__ long long warp_lower_bound(const int *indices, long long lo, long long hi, int key) {
+    const int lane = threadIdx.x & 31;
+    while (hi - lo > 32) {
+        const long long step = (hi - lo) / 32;
+        const long long pos = lo + lane * step;
+        const int v = indices[pos];
+        const unsigned int below = __ballot_sync(0xffffffffu, v < key);
+        const int c = __popc(below);
+        if (c == 0) return lo;  // indices[lo] >= key
+        const long long new_lo = lo + (c - 1) * step + 1;
+        if (c < 32) hi = lo + c * step;
+        lo = new_lo;
+    }
+    const long long pos = lo + lane;
+    const int v = (pos < hi) ? indices[pos] : 0x7fffffff;
+    const unsigned int below = __ballot_sync(0xffffffffu, v < key);
+    return lo + __popc(below);
+}
+
+__global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    ChainSmem &sm = *reinterpret_cast<ChainSmem *>(smem_raw);
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    constexpr int kWarps = kChainThreads / 32;
+
+    if (!ws_matches(p.ws)) return;
+    if (ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) != 0u) return;
+
+    const long long tb = static_cast<long long>(blockIdx.x) * p.tiles_per_cta;
+    long long te = tb + p.tiles_per_cta;
+    if (te > p.ws.num_tiles) te = p.ws.num_tiles;
+    if (tb >= te) return;
+
+    unsigned long long policy = 0;
+    for (int e = tid; e < kTileElems; e += kChainThreads) sm.tag[e] = 0u;
+    if (tid == 0) {
+        policy = l2_evict_first_policy();
+        mbar_init(&sm.bar[0], 1);
+        mbar_init(&sm.bar[1], 1);
+        mbar_fence_init();
+        chain_issue(p, sm, tb, 0, policy);
+    }
+    __syncthreads();
+
+    // Cursors at the CTA's first tile: one binary search per delta.
+    {
+        const TileMeta m0 = sm.meta[0];
+        for (int k = warp; k < p.K; k += kWarps) {
+            const DeltaRef d = p.d[k];
+            const long long lo = d.offsets[m0.tensor];
+            const long long hi = d.offsets[m0.tensor + 1];
+            // At a tensor's first tile start at the segment head, so that a
+            // negative index is seen (and flagged) rather than skipped.
+            const long long c = (m0.local_start == 0)
+                                    ? lo
+                                    : warp_lower_bound(d.indices, lo, hi, m0.local_start);
+            if (lane == 0) {
+                sm.cur[k] = c;
+                sm.end[k] = hi;
+                sm.consumed[k] = 0;
+            }
+        }
+    }
+    __syncthreads();
+
+    uint32_t phase_bits = 0;
+    for (long long i = tb; i < te; ++i) {
+        const int b = static_cast<int>((i - tb) & 1);
+        if (tid == 0 && i + 1 < te) {
+            bulk_wait_read_all();  // the store from the other buffer has read it
+            chain_issue(p, sm, i + 1, b ^ 1, policy);
+        }
+        const TileMeta m = sm.meta[b];
+        const int ls = m.local_start;
+
+        // New tensor inside the CTA's range: the previous tensor's entries
+        // must all have been consumed (else some index was >= numel).
+        if (i != tb && ls == 0) {
+            if (tid < p.K) {
+                const DeltaRef d = p.d[tid];
+                if (sm.cur[tid] != sm.end[tid]) record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, sm.cur[tid]);
+                sm.cur[tid] = d.offsets[m.tensor];
+                sm.end[tid] = d.offsets[m.tensor + 1];
+            }
+            __syncthreads();
+        }
+
+        // ---- entry phase: tag this tile's entries of every delta ----------
+        if (tid < p.K) sm.active[tid] = (sm.cur[tid] < sm.end[tid]);
+        __syncthreads();
+        const int L = p.block_len;
+        const int slots = p.K * L;
+        for (;;) {
+            for (int sidx = tid; sidx < slots; sidx += kChainThreads) {
+                const int k = sidx / L;
+                const int r = sidx - k * L;
+                if (!sm.active[k]) continue;
+                const long long j = sm.cur[k] + r;
+                if (j >= sm.end[k]) continue;
+                const DeltaRef &d = p.d[k];
+                const int idx = __ldg(d.indices + j);
+                if (idx < ls) {
+                    // Not ascending (or negative): skip, but consume it.
+                    record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, j);
+                    atomicMax(&sm.consumed[k], r + 1);
+                } else if (idx - ls < m.count) {
+                    const uint32_t key = (static_cast<uint32_t>(k + 1) << 16) | __ldg(d.values + j);
+                    atomicMax(&sm.tag[idx - ls], key);
+                    atomicMax(&sm.consumed[k], r + 1);
+                }
+            }
+            __syncthreads();
+            int again = 0;
+            if (tid < p.K) {
+                const int c = sm.consumed[tid];
+                sm.consumed[tid] = 0;
+                if (sm.active[tid]) {
+                    sm.cur[tid] += c;
+                    again = (c == L) && (sm.cur[tid] < sm.end[tid]);
+                    sm.active[tid] = again;
+                }
+            }
+            if (!__syncthreads_or(again)) break;
+        }
+
+        // ---- merge: tags over the snapshot tile ----------------------------
+        const uint32_t parity = (phase_bits >> b) & 1u;
+        phase_bits ^= (1u << b);
+        const bool loaded = mbar_wait(&sm.bar[b], parity, kLoadWaitLimitNs);
+        if (!__syncthreads_and(loaded)) {  // leave together, before any write
+            if (tid == 0) record_error(p.ws.hdr, DWS_ERR_TIMEOUT, i);
+            return;
+        }
+        int touched = 0;
+        for (int c = tid; c * 8 < m.count; c += kChainThreads) {
+            const int e0 = c * 8;
+            uint4 t0 = *reinterpret_cast<const uint4 *>(&sm.tag[e0]);
+            uint4 t1 = *reinterpret_cast<const uint4 *>(&sm.tag[e0 + 4]);
+            const uint32_t any = t0.x | t0.y | t0.z | t0.w | t1.x | t1.y | t1.z | t1.w;
+            if (any == 0u) continue;
+            touched = 1;
+            const uint32_t tg[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            *reinterpret_cast<uint4 *>(&sm.tag[e0]) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(&sm.tag[e0 + 4]) = make_uint4(0, 0, 0, 0);
+            if (e0 + 8 <= m.bulk) {
+                uint16_t *v = &sm.tile[b][e0];
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (tg[q]) v[q] = static_cast<uint16_t>(tg[q] & 0xffffu);
+            } else {
+                // Outside the bulk-copied part: write straight to the snapshot.
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (tg[q] && e0 + q < m.count) m.ptr[e0 + q] = static_cast<uint16_t>(tg[q] & 0xffffu);
+            }
+        }
+        if (m.bulk > 0) fence_proxy_async_smem();
+        touched = __syncthreads_or(touched);
+        if (tid == 0 && touched && m.bulk > 0) {
+            bulk_store(m.ptr, sm.tile[b], static_cast<uint32_t>(m.bulk) * 2u);
+            bulk_commit();
+        }
+    }
+
+    // The CTA's range ends at the end of a tensor: all of its entries must
+    // have been consumed.
+    {
+        const long long last = te - 1;
+        const int t = p.ws.tile_tensor[last];
+        const bool tensor_ends = (last + 1 == p.ws.num_tiles) || (p.ws.tile_tensor[last + 1] != t);
+        if (tensor_ends && tid < p.K && sm.cur[tid] != sm.end[tid])
+            record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, sm.cur[tid]);
+    }
+    if (tid == 0) bulk_wait_all();
+}
+
+}  // namespace
+
+size_t chain_smem_bytes() { return sizeof(ChainSmem); }
+
+cudaError_t chain_set_attributes() {
+    return cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sizeof(ChainSmem)));
+}
+
+cudaError_t chain_occupancy(int *ctas_per_sm) {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, chain_kernel, kChainThreads,
+                                                         sizeof(ChainSmem));
+}
+
+cudaError_t launch_delta_check(const WsView &ws, const DeltaRef *deltas, int K, cudaStream_t s) {
+    delta_flag_clear_kernel<<<1, 1, 0, s>>>(ws);
+    cudaError_t e = launched();
+    if (e != cudaSuccess) return e;
+    CheckParams p;
+    p.ws = ws;
+    p.K = K;
+    for (int k = 0; k < K; ++k) p.d[k] = deltas[k];
+    delta_check_kernel<<<K, 256, 0, s>>>(p);
+    return launched();
+}
+
+cudaError_t launch_apply(const WsView &ws, uint16_t *const *snap_ptrs, const DeltaRef &d,
+                         cudaStream_t s) {
+    cudaError_t e = launch_delta_check(ws, &d, 1, s);
+    if (e != cudaSuccess) return e;
+    if (d.count <= 0) return cudaSuccess;
+    ApplyParams p;
+    p.ws = ws;
+    p.snap_ptrs = snap_ptrs;
+    p.d = d;
+    const long long blocks = (d.count + kApplyEntries - 1) / kApplyEntries;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    apply_kernel<<<static_cast<unsigned int>(blocks), kApplyThreads, 0, s>>>(p);
+    return launched();
+}
+
+cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs,
+                               const DeltaRef *deltas, int K, long long total_entries,
+                               long long total_elems, cudaStream_t s) {
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    e = launch_delta_check(ws, deltas, K, s);
+    if (e != cudaSuccess) return e;
+
+    ChainParams p;
+    p.ws = ws;
+    p.snap_ptrs = snap_ptrs;
+    p.K = K;
+    for (int k = 0; k < K; ++k) p.d[k] = deltas[k];
+    // Entries read per delta per round: the mean per full tile with margin.
+    const double per_tile = total_elems > 0
+                                ? double(total_entries) / K * kTileElems / double(total_elems)
+                                : 0.0;
+    long long L = static_cast<long long>(per_tile * 1.25) + 32;
+    L = (L + 31) & ~31LL;
+    long long cap = kChainMaxSlots / K;
+    if (cap < 32) cap = 32;
+    if (L > cap) L = cap;
+    if (L < 32) L = 32;
+    p.block_len = static_cast<int>(L);
+
+    long long grid = static_cast<long long>(di.sm_count) * di.chain_ctas_per_sm;
+    if (grid > ws.num_tiles) grid = ws.num_tiles;
+    if (grid < 1) grid = 1;
+    p.tiles_per_cta = (ws.num_tiles + grid - 1) / grid;
+    grid = (ws.num_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
+    chain_kernel<<<static_cast<unsigned int>(grid), kChainThreads, sizeof(ChainSmem), s>>>(p);
+    return launched();
+}
+
+}  // namespace dws

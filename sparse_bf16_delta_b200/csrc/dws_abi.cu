@@ -1,0 +1,398 @@
+// dws_abi.cu -- the libdws C ABI (declared in include/dws.h): host-side
+// validation, the plan (multi-tensor descriptor table), workspace upload,
+// kernel launches, the two-stream XOR layer pipeline and status readback.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "dws_internal.cuh"
+
+namespace dws {
+size_t encode_smem_bytes();
+cudaError_t encode_set_attributes();
+cudaError_t encode_occupancy(int *ctas_per_sm);
+size_t chain_smem_bytes();
+cudaError_t chain_set_attributes();
+cudaError_t chain_occupancy(int *ctas_per_sm);
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::once_flag g_once[kMaxDevices];
+DeviceInfo g_info[kMaxDevices];
+cudaError_t g_err[kMaxDevices];
+
+void init_device(int dev) {
+    DeviceInfo di{};
+    cudaError_t e = cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = encode_set_attributes();
+    if (e == cudaSuccess) e = chain_set_attributes();
+    if (e == cudaSuccess) e = encode_occupancy(&di.encode_ctas_per_sm);
+    if (e == cudaSuccess) e = chain_occupancy(&di.chain_ctas_per_sm);
+    if (e == cudaSuccess) {
+        if (di.encode_ctas_per_sm < 1) di.encode_ctas_per_sm = 1;
+        if (di.chain_ctas_per_sm < 1) di.chain_ctas_per_sm = 1;
+    }
+    g_info[dev] = di;
+    g_err[dev] = e;
+}
+}  // namespace
+
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}
+
+cudaError_t launched() {
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+    return e;
+}
+
+cudaError_t device_info(DeviceInfo *out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::call_once(g_once[dev], init_device, dev);
+    if (g_err[dev] != cudaSuccess) return g_err[dev];
+    *out = g_info[dev];
+    return cudaSuccess;
+}
+
+}  // namespace dws
+
+using dws::WsHeader;
+using dws::WsLayout;
+using dws::WsView;
+
+struct dws_plan {
+    int32_t T;
+    int64_t N;
+    int64_t ntiles;
+    uint64_t fingerprint;
+    WsLayout layout;
+    std::vector<unsigned char> image;  // header + numel + first_tile, as uploaded
+};
+
+namespace {
+
+uint64_t fnv1a(uint64_t h, uint64_t v) {
+    for (int i = 0; i < 8; ++i) {
+        h ^= (v >> (8 * i)) & 0xffu;
+        h *= 0x100000001b3ull;
+    }
+    return h;
+}
+
+WsView view_of(const dws_plan *p, void *ws) {
+    unsigned char *base = static_cast<unsigned char *>(ws);
+    WsView v;
+    v.hdr = reinterpret_cast<WsHeader *>(base);
+    v.numel = reinterpret_cast<const long long *>(base + p->layout.numel_off);
+    v.first_tile = reinterpret_cast<const long long *>(base + p->layout.first_tile_off);
+    v.tile_tensor = reinterpret_cast<const int *>(base + p->layout.tile_tensor_off);
+    v.tile_status = reinterpret_cast<unsigned long long *>(base + p->layout.tile_status_off);
+    v.num_tiles = p->ntiles;
+    v.num_tensors = p->T;
+    v.fingerprint = p->fingerprint;
+    return v;
+}
+
+dws_status_t check_ws(const dws_plan *p, const void *ws, size_t ws_bytes) {
+    if (p == nullptr || ws == nullptr) return DWS_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DWS_ERR_WORKSPACE;
+    if (ws_bytes < p->layout.total) return DWS_ERR_WORKSPACE;
+    return DWS_OK;
+}
+
+dws_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? DWS_OK : DWS_ERR_CUDA; }
+
+dws_status_t encode_common(const dws_plan_t *plan, const void *const *old_ptrs,
+                           const void *const *new_ptrs, int64_t *offsets, int32_t *indices,
+                           uint16_t *values, int64_t capacity, void *workspace,
+                           size_t workspace_bytes, dws_stream_t stream, bool compact,
+                           int64_t wait_limit_ns, int64_t withhold) {
+    dws_status_t st = check_ws(plan, workspace, workspace_bytes);
+    if (st != DWS_OK) return st;
+    if (old_ptrs == nullptr || new_ptrs == nullptr || offsets == nullptr) return DWS_ERR_INVALID;
+    if (compact) {
+        if (capacity < 0) return DWS_ERR_INVALID;
+        if (capacity > 0 && (indices == nullptr || values == nullptr)) return DWS_ERR_INVALID;
+    }
+    const WsView v = view_of(plan, workspace);
+    return from_cuda(dws::launch_encode(
+        v, reinterpret_cast<const uint16_t *const *>(old_ptrs),
+        reinterpret_cast<const uint16_t *const *>(new_ptrs), reinterpret_cast<long long *>(offsets),
+        reinterpret_cast<int *>(indices), values, compact ? capacity : 0, compact,
+        wait_limit_ns, withhold, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+dws_status_t dws_plan_create(const int64_t *numels, int32_t num_tensors, int32_t elem_size,
+                             dws_plan_t **plan_out) {
+    if (plan_out == nullptr) return DWS_ERR_INVALID;
+    *plan_out = nullptr;
+    if (numels == nullptr || num_tensors <= 0) return DWS_ERR_INVALID;
+    if (elem_size != 2) return DWS_ERR_UNSUPPORTED;
+    int64_t N = 0, ntiles = 0;
+    for (int32_t t = 0; t < num_tensors; ++t) {
+        const int64_t n = numels[t];
+        if (n < 0 || n > INT32_MAX) return DWS_ERR_INVALID;
+        N += n;
+        ntiles += (n == 0) ? 1 : (n + dws::kTileElems - 1) / dws::kTileElems;
+    }
+    dws_plan *p = new (std::nothrow) dws_plan;
+    if (p == nullptr) return DWS_ERR_INVALID;
+    p->T = num_tensors;
+    p->N = N;
+    p->ntiles = ntiles;
+    p->layout = dws::ws_layout(num_tensors, ntiles);
+
+    uint64_t h = 0xcbf29ce484222325ull;
+    h = fnv1a(h, static_cast<uint64_t>(num_tensors));
+    for (int32_t t = 0; t < num_tensors; ++t) h = fnv1a(h, static_cast<uint64_t>(numels[t]));
+    p->fingerprint = h;
+
+    // Static image: header, numel[T], first_tile[T+1] at their layout offsets.
+    const size_t image_bytes = p->layout.tile_tensor_off;
+    try {
+        p->image.assign(image_bytes, 0);
+    } catch (...) {
+        delete p;
+        return DWS_ERR_INVALID;
+    }
+    WsHeader hdr;
+    std::memset(&hdr, 0, sizeof hdr);
+    hdr.magic = dws::kWsMagic;
+    hdr.fingerprint = p->fingerprint;
+    hdr.num_tiles = ntiles;
+    hdr.num_tensors = num_tensors;
+    std::memcpy(p->image.data(), &hdr, sizeof hdr);
+    long long *numel_img = reinterpret_cast<long long *>(p->image.data() + p->layout.numel_off);
+    long long *first_img = reinterpret_cast<long long *>(p->image.data() + p->layout.first_tile_off);
+    long long acc = 0;
+    for (int32_t t = 0; t < num_tensors; ++t) {
+        numel_img[t] = numels[t];
+        first_img[t] = acc;
+        acc += (numels[t] == 0) ? 1 : (numels[t] + dws::kTileElems - 1) / dws::kTileElems;
+    }
+    first_img[num_tensors] = acc;
+    *plan_out = p;
+    return DWS_OK;
+}
+
+void dws_plan_destroy(dws_plan_t *plan) { delete plan; }
+
+int32_t dws_plan_num_tensors(const dws_plan_t *plan) { return plan ? plan->T : 0; }
+int64_t dws_plan_num_elements(const dws_plan_t *plan) { return plan ? plan->N : 0; }
+int64_t dws_plan_num_tiles(const dws_plan_t *plan) { return plan ? plan->ntiles : 0; }
+int64_t dws_tile_elems(void) { return dws::kTileElems; }
+
+size_t dws_plan_workspace_bytes(const dws_plan_t *plan) { return plan ? plan->layout.total : 0; }
+
+dws_status_t dws_plan_upload(const dws_plan_t *plan, void *workspace, size_t workspace_bytes,
+                             dws_stream_t stream) {
+    dws_status_t st = check_ws(plan, workspace, workspace_bytes);
+    if (st != DWS_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(workspace, plan->image.data(), plan->image.size(),
+                                    cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return DWS_ERR_CUDA;
+    return from_cuda(dws::launch_fill_tile_map(view_of(plan, workspace), s));
+}
+
+dws_status_t dws_encode(const dws_plan_t *plan, const void *const *old_ptrs,
+                        const void *const *new_ptrs, int64_t *offsets, int32_t *indices,
+                        uint16_t *values, int64_t capacity, void *workspace,
+                        size_t workspace_bytes, dws_stream_t stream) {
+    return encode_common(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, workspace,
+                         workspace_bytes, stream, true, 0, -1);
+}
+
+dws_status_t dws_encode_ex(const dws_plan_t *plan, const void *const *old_ptrs,
+                           const void *const *new_ptrs, int64_t *offsets, int32_t *indices,
+                           uint16_t *values, int64_t capacity, void *workspace,
+                           size_t workspace_bytes, dws_stream_t stream, int64_t wait_limit_ns,
+                           int64_t debug_withhold_tile) {
+    return encode_common(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, workspace,
+                         workspace_bytes, stream, true, wait_limit_ns, debug_withhold_tile);
+}
+
+dws_status_t dws_count(const dws_plan_t *plan, const void *const *old_ptrs,
+                       const void *const *new_ptrs, int64_t *offsets, void *workspace,
+                       size_t workspace_bytes, dws_stream_t stream) {
+    return encode_common(plan, old_ptrs, new_ptrs, offsets, nullptr, nullptr, 0, workspace,
+                         workspace_bytes, stream, false, 0, -1);
+}
+
+dws_status_t dws_apply(const dws_plan_t *plan, void *const *snap_ptrs, const int64_t *offsets,
+                       const int32_t *indices, const uint16_t *values, int64_t count,
+                       void *workspace, size_t workspace_bytes, dws_stream_t stream) {
+    dws_status_t st = check_ws(plan, workspace, workspace_bytes);
+    if (st != DWS_OK) return st;
+    if (snap_ptrs == nullptr || offsets == nullptr || count < 0) return DWS_ERR_INVALID;
+    if (count > 0 && (indices == nullptr || values == nullptr)) return DWS_ERR_INVALID;
+    dws::DeltaRef d{reinterpret_cast<const long long *>(offsets),
+                    reinterpret_cast<const int *>(indices), values, count};
+    return from_cuda(dws::launch_apply(view_of(plan, workspace),
+                                       reinterpret_cast<uint16_t *const *>(snap_ptrs), d,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dws_status_t dws_apply_chain(const dws_plan_t *plan, void *const *snap_ptrs,
+                             const dws_delta_t *deltas, int32_t K, void *workspace,
+                             size_t workspace_bytes, dws_stream_t stream) {
+    dws_status_t st = check_ws(plan, workspace, workspace_bytes);
+    if (st != DWS_OK) return st;
+    if (snap_ptrs == nullptr || deltas == nullptr || K < 1 || K > DWS_MAX_CHAIN)
+        return DWS_ERR_INVALID;
+    dws::DeltaRef d[DWS_MAX_CHAIN];
+    long long total = 0;
+    for (int32_t k = 0; k < K; ++k) {
+        if (deltas[k].offsets == nullptr || deltas[k].count < 0) return DWS_ERR_INVALID;
+        if (deltas[k].count > 0 && (deltas[k].indices == nullptr || deltas[k].values == nullptr))
+            return DWS_ERR_INVALID;
+        d[k] = dws::DeltaRef{reinterpret_cast<const long long *>(deltas[k].offsets),
+                             reinterpret_cast<const int *>(deltas[k].indices), deltas[k].values,
+                             deltas[k].count};
+        total += deltas[k].count;
+    }
+    return from_cuda(dws::launch_apply_chain(view_of(plan, workspace),
+                                             reinterpret_cast<uint16_t *const *>(snap_ptrs), d, K,
+                                             total, plan->N,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dws_status_t dws_xor_encode(const void *old_bytes, const void *new_bytes, void *mask,
+                            int64_t nbytes, dws_stream_t stream) {
+    if (nbytes < 0) return DWS_ERR_INVALID;
+    if (nbytes == 0) return DWS_OK;
+    if (old_bytes == nullptr || new_bytes == nullptr || mask == nullptr) return DWS_ERR_INVALID;
+    return from_cuda(dws::launch_xor(static_cast<const uint8_t *>(old_bytes),
+                                     static_cast<const uint8_t *>(new_bytes),
+                                     static_cast<uint8_t *>(mask), nbytes,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dws_status_t dws_xor_apply(void *buf, const void *mask, int64_t nbytes, dws_stream_t stream) {
+    if (nbytes < 0) return DWS_ERR_INVALID;
+    if (nbytes == 0) return DWS_OK;
+    if (buf == nullptr || mask == nullptr) return DWS_ERR_INVALID;
+    return from_cuda(dws::launch_xor(static_cast<const uint8_t *>(buf),
+                                     static_cast<const uint8_t *>(mask),
+                                     static_cast<uint8_t *>(buf), nbytes,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dws_status_t dws_xor_apply_layers(void *const *bufs, const void *const *masks,
+                                  const int64_t *nbytes, int32_t L, void *staging0,
+                                  void *staging1, int64_t staging_bytes,
+                                  dws_stream_t apply_stream, dws_stream_t copy_stream) {
+    if (bufs == nullptr || masks == nullptr || nbytes == nullptr || L < 0) return DWS_ERR_INVALID;
+    if (staging0 == nullptr || staging1 == nullptr || staging_bytes <= 0) return DWS_ERR_INVALID;
+    for (int32_t l = 0; l < L; ++l) {
+        if (nbytes[l] < 0) return DWS_ERR_INVALID;
+        if (nbytes[l] > 0 && (bufs[l] == nullptr || masks[l] == nullptr)) return DWS_ERR_INVALID;
+    }
+    if (L == 0) return DWS_OK;
+    cudaStream_t as = reinterpret_cast<cudaStream_t>(apply_stream);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
+    void *staging[2] = {staging0, staging1};
+
+    cudaEvent_t start, copied[2], applied[2];
+    cudaError_t e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming);
+    if (e != cudaSuccess) return DWS_ERR_CUDA;
+    int made = 0;
+    for (int b = 0; b < 2 && e == cudaSuccess; ++b) {
+        e = cudaEventCreateWithFlags(&copied[b], cudaEventDisableTiming);
+        if (e == cudaSuccess) {
+            e = cudaEventCreateWithFlags(&applied[b], cudaEventDisableTiming);
+            if (e == cudaSuccess) ++made;
+            else cudaEventDestroy(copied[b]);
+        }
+    }
+    // The copy stream starts after what is already queued on the apply stream.
+    if (e == cudaSuccess) e = cudaEventRecord(start, as);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, start, 0);
+
+    bool used[2] = {false, false};
+    long long unit = 0;
+    for (int32_t l = 0; l < L && e == cudaSuccess; ++l) {
+        for (int64_t off = 0; off < nbytes[l] && e == cudaSuccess; off += staging_bytes) {
+            const int64_t len = (nbytes[l] - off < staging_bytes) ? (nbytes[l] - off) : staging_bytes;
+            const int b = static_cast<int>(unit & 1);
+            // Staging buffer b is free once the apply that read it is done.
+            if (used[b]) e = cudaStreamWaitEvent(cs, applied[b], 0);
+            if (e == cudaSuccess)
+                e = cudaMemcpyAsync(staging[b], static_cast<const uint8_t *>(masks[l]) + off,
+                                    static_cast<size_t>(len), cudaMemcpyDefault, cs);
+            if (e == cudaSuccess) e = cudaEventRecord(copied[b], cs);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(as, copied[b], 0);
+            if (e == cudaSuccess)
+                e = dws::launch_xor(static_cast<const uint8_t *>(bufs[l]) + off,
+                                    static_cast<const uint8_t *>(staging[b]),
+                                    static_cast<uint8_t *>(bufs[l]) + off, len, as);
+            if (e == cudaSuccess) e = cudaEventRecord(applied[b], as);
+            used[b] = true;
+            ++unit;
+        }
+    }
+    // Events are released once their pending work completes.
+    cudaEventDestroy(start);
+    for (int b = 0; b < made; ++b) {
+        cudaEventDestroy(copied[b]);
+        cudaEventDestroy(applied[b]);
+    }
+    return from_cuda(e);
+}
+
+dws_status_t dws_status(void *workspace, int64_t *detail, dws_stream_t stream) {
+    if (workspace == nullptr) return DWS_ERR_INVALID;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    WsHeader *hdr = static_cast<WsHeader *>(workspace);
+    struct {
+        unsigned int status;
+        unsigned int pad;
+        long long detail;
+    } host{};
+    cudaError_t e = cudaMemcpyAsync(&host.status, &hdr->status, sizeof(unsigned int),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(&host.detail, &hdr->detail, sizeof(long long), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return DWS_ERR_CUDA;
+    if (detail) *detail = host.detail;
+    if (host.status != 0u) {
+        e = cudaMemsetAsync(&hdr->status, 0, sizeof(unsigned int), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(&hdr->detail, 0, sizeof(long long), s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return DWS_ERR_CUDA;
+    }
+    return static_cast<dws_status_t>(host.status);
+}
+
+const char *dws_strerror(dws_status_t status) {
+    switch (status) {
+        case DWS_OK: return "ok";
+        case DWS_ERR_INVALID: return "invalid argument";
+        case DWS_ERR_UNSUPPORTED: return "unsupported element size";
+        case DWS_ERR_CAPACITY: return "output capacity exceeded";
+        case DWS_ERR_BAD_DELTA: return "bad delta (index out of range, not ascending, or bad offsets)";
+        case DWS_ERR_TIMEOUT: return "bounded wait ran out";
+        case DWS_ERR_CUDA: return "CUDA runtime error";
+        case DWS_ERR_WORKSPACE: return "workspace too small or not prepared for this plan";
+    }
+    return "unknown status";
+}
+
+uint64_t dws_launch_count(void) { return dws::g_launches.load(std::memory_order_relaxed); }
+
+const char *dws_version(void) { return "libdws 0.1 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,295 @@
+// dws_internal.cuh -- shared definitions of libdws's kernels and host code:
+// the workspace layout, the device status word, and thin inline-PTX wrappers
+// for the sm_100a features the kernels use (mbarrier transaction counts,
+// 1-D bulk async copies between global and shared memory, L2 eviction
+// hints, gpu-scope relaxed loads/stores, the global nanosecond timer).
+//
+// No cluster multicast is used anywhere in libdws: every bulk copy moves data
+// between this GPU's global memory and the issuing CTA's own shared memory.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/dws.h"
+
+namespace dws {
+
+// ---------------------------------------------------------------------------
+// Tiling shared by the encode scan and the chain replay: a tensor is cut into
+// tiles of kTileElems elements (16 KiB of bf16 per snapshot); a tile never
+// straddles two tensors and an empty tensor owns one empty tile.
+// ---------------------------------------------------------------------------
+constexpr int kTileElems = 8192;
+constexpr int kTileShift = 13;
+static_assert((1 << kTileShift) == kTileElems, "tile size must be a power of two");
+
+// ---------------------------------------------------------------------------
+// Workspace layout (device memory owned by the caller)
+//
+//   [0, 256)          WsHeader
+//   numel             int64[T]           tensor sizes          (static)
+//   first_tile        int64[T+1]         first tile of tensor  (static)
+//   tile_tensor       int32[ntiles]      tensor of each tile   (static)
+//   tile_status       uint64[ntiles]     encode scan state     (per call)
+//
+// Every region starts on a 256-byte boundary.  The static regions are written
+// by dws_plan_upload; the header's magic + fingerprint tie the workspace to
+// the plan that wrote it.
+// ---------------------------------------------------------------------------
+constexpr unsigned long long kWsMagic = 0x3130305357534457ull;  // "DWSWS001"
+
+struct WsHeader {
+    unsigned long long magic;        // 0
+    unsigned long long fingerprint;  // 8
+    long long num_tiles;             // 16
+    int num_tensors;                 // 24
+    unsigned int status;             // 28  first device error (dws_status_t), 0 = none
+    long long detail;                // 32  detail of that error
+    unsigned long long ticket;       // 40  encode: next tile ticket
+    unsigned int abort;              // 48  encode: a bounded wait ran out, all waiters leave
+    unsigned int delta_bad;          // 52  apply/chain: offsets of some delta failed validation
+    unsigned char pad[256 - 56];
+};
+static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
+
+struct WsLayout {
+    size_t numel_off, first_tile_off, tile_tensor_off, tile_status_off, total;
+};
+
+inline size_t round_up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout ws_layout(int T, long long ntiles) {
+    WsLayout L;
+    L.numel_off = 256;
+    L.first_tile_off = round_up256(L.numel_off + sizeof(long long) * size_t(T));
+    L.tile_tensor_off = round_up256(L.first_tile_off + sizeof(long long) * size_t(T + 1));
+    L.tile_status_off = round_up256(L.tile_tensor_off + sizeof(int) * size_t(ntiles));
+    L.total = round_up256(L.tile_status_off + sizeof(unsigned long long) * size_t(ntiles));
+    return L;
+}
+
+// Device view of a prepared workspace, passed by value to every kernel.
+struct WsView {
+    WsHeader *hdr;
+    const long long *numel;
+    const long long *first_tile;
+    const int *tile_tensor;
+    unsigned long long *tile_status;
+    long long num_tiles;
+    int num_tensors;
+    unsigned long long fingerprint;
+};
+
+// Encode scan state per tile: 2 flag bits + a 62-bit count.
+constexpr unsigned long long kFlagShift = 62;
+constexpr unsigned long long kFlagAggregate = 1ull << kFlagShift;  // tile's own count
+constexpr unsigned long long kFlagPrefix = 2ull << kFlagShift;     // inclusive prefix
+constexpr unsigned long long kValueMask = (1ull << kFlagShift) - 1;
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+#if defined(__CUDACC__)
+
+__device__ __forceinline__ void record_error(WsHeader *hdr, unsigned int code, long long detail) {
+    if (atomicCAS(&hdr->status, 0u, code) == 0u) {
+        atomicExch(reinterpret_cast<unsigned long long *>(&hdr->detail),
+                   static_cast<unsigned long long>(detail));
+    }
+}
+
+// One thread per CTA checks that the workspace belongs to the plan of this
+// launch; returns the verdict to every thread of the CTA.
+__device__ __forceinline__ bool ws_matches(const WsView &ws) {
+    __shared__ int ok;
+    if (threadIdx.x == 0) {
+        const WsHeader *h = ws.hdr;
+        ok = (h->magic == kWsMagic && h->fingerprint == ws.fingerprint &&
+              h->num_tiles == ws.num_tiles && h->num_tensors == ws.num_tensors);
+        if (!ok) record_error(ws.hdr, DWS_ERR_WORKSPACE, 0);
+    }
+    __syncthreads();
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned int ld_relaxed_gpu_u32(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// L2 policy: data read once (snapshots, masks) is evicted first.
+__device__ __forceinline__ unsigned long long l2_evict_first_policy() {
+    unsigned long long pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// --- mbarrier (shared::cta) -------------------------------------------------
+__device__ __forceinline__ void mbar_init(unsigned long long *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete.  Bulk copies of valid memory
+// always complete; the limit only keeps a broken invariant from spinning
+// forever.  Returns false if the limit was reached.
+__device__ __forceinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity,
+                                          unsigned long long limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
+// --- 1-D bulk async copies (no tensor map, no multicast) --------------------
+// global -> this CTA's shared memory, completion counted on `bar`.
+// dst and src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gmem_src, uint32_t bytes,
+                                          unsigned long long *bar, unsigned long long policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(smem_dst)),
+        "l"(gmem_src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// this CTA's shared memory -> global, tracked by the issuing thread's bulk group.
+__device__ __forceinline__ void bulk_store(void *gmem_dst, const void *smem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gmem_dst),
+                 "r"(smem_addr(smem_src)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// The issuing thread's committed bulk stores have finished READING shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// The issuing thread's committed bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (a later bulk store reads them).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// --- cache-hinted global accesses -------------------------------------------
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_stream_v4(void *p, uint4 v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_stream_u32(void *p, uint32_t v) {
+    asm volatile("st.global.cs.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_stream_u16(void *p, uint16_t v) {
+    asm volatile("st.global.cs.u16 [%0], %1;" ::"l"(p), "h"(v) : "memory");
+}
+
+#endif  // __CUDACC__
+
+// ---------------------------------------------------------------------------
+// Kernel launchers (defined in the .cu files, called by the C ABI)
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+    int sm_count;
+    int encode_ctas_per_sm;
+    int chain_ctas_per_sm;
+};
+
+// Per-device constants and one-time kernel attribute setup (thread-safe).
+cudaError_t device_info(DeviceInfo *out);
+
+// Count one kernel launch (dws_launch_count); returns cudaGetLastError().
+cudaError_t launched();
+
+cudaError_t launch_fill_tile_map(const WsView &ws, cudaStream_t s);
+cudaError_t launch_ws_reset(const WsView &ws, cudaStream_t s);
+cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
+                          const uint16_t *const *new_ptrs, long long *offsets, int *indices,
+                          uint16_t *values, long long capacity, bool compact,
+                          long long wait_limit_ns, long long withhold_tile, cudaStream_t s);
+
+struct DeltaRef {
+    const long long *offsets;
+    const int *indices;
+    const uint16_t *values;
+    long long count;
+};
+
+cudaError_t launch_delta_check(const WsView &ws, const DeltaRef *deltas, int K, cudaStream_t s);
+cudaError_t launch_apply(const WsView &ws, uint16_t *const *snap_ptrs, const DeltaRef &d,
+                         cudaStream_t s);
+cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs,
+                               const DeltaRef *deltas, int K, long long total_entries,
+                               long long total_elems, cudaStream_t s);
+
+cudaError_t launch_xor(const uint8_t *a, const uint8_t *b, uint8_t *out, long long nbytes,
+                       cudaStream_t s);
+
+}  // namespace dws

@@ -1,0 +1,33 @@
+"""Helpers shared by the GPU tests: moving bits between torch and numpy and
+comparing libdws outputs with the CPU oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    """Any 2-byte tensor -> its uint16 bits on the host."""
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1)
+
+
+def host_bytes(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().view(torch.uint8).cpu().numpy().reshape(-1)
+
+
+def dev_bits(a: np.ndarray, device="cuda") -> torch.Tensor:
+    """uint16 numpy -> bf16 device tensor with those bits."""
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16).copy()).to(device).view(torch.bfloat16)
+
+
+def delta_to_host(delta):
+    return (delta.offsets.cpu().numpy(), delta.indices.cpu().numpy(),
+            delta.values.cpu().numpy().view(np.uint16))
+
+
+def assert_delta_equal(got, want):
+    go, gi, gv = got
+    wo, wi, wv = want
+    np.testing.assert_array_equal(go, wo)
+    np.testing.assert_array_equal(gi, wi)
+    np.testing.assert_array_equal(gv, wv)

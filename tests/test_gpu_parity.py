@@ -1,0 +1,422 @@
+"""libdws on the GPU against the CPU oracle, element by element.
+
+Sizes span several 8192-element tiles with ragged tails, empty tensors,
+unaligned views, thousands of tiny tensors, capacity overflow, bad deltas and
+the scan's bounded wait.  Every comparison is exact (integer work)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests import _golden as G
+from tests._dev import assert_delta_equal, delta_to_host, dev_bits, host_bits, host_bytes
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dws():
+    import sparse_bf16_delta_b200 as m
+    return m
+
+
+def _random_pair(rng, n, rate):
+    a = rng.integers(0, 1 << 16, n, dtype=np.uint16)
+    b = a.copy()
+    if n:
+        m = rng.random(n) < rate
+        b[m] ^= rng.integers(1, 1 << 16, int(m.sum()), dtype=np.uint16)
+    return a, b
+
+
+def _gpu_encode(dws, olds, news, capacity=None):
+    plan = dws.DeltaPlan.for_tensors(olds)
+    ot, nt = dws.ptr_table(olds), dws.ptr_table(news)
+    if capacity is None:
+        d = plan.encode_exact(ot, nt)
+    else:
+        d = plan.encode(ot, nt, capacity)
+    return plan, d
+
+
+# ---------------------------------------------------------------- encode
+
+
+def test_encode_golden_worked_example(dws):
+    olds, news, offsets, indices, values = G.encode_example()
+    _, d = _gpu_encode(dws, [dev_bits(a) for a in olds], [dev_bits(b) for b in news])
+    assert_delta_equal(delta_to_host(d), (offsets, indices, values))
+
+
+def test_encode_workload1_matches_oracle(dws):
+    old, new = W.single("cuda")
+    plan, d = _gpu_encode(dws, old.tensors, new.tensors)
+    want = oracle.encode([host_bits(old.tensors[0])], [host_bits(new.tensors[0])])
+    assert_delta_equal(delta_to_host(d), want)
+    assert 0 < want[0][-1] < old.total
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_encode_ragged_sizes_and_rates(dws, seed):
+    rng = np.random.default_rng(100 + seed)
+    sizes = [0, 1, 7, 8, 9, 8191, 8192, 8193, 3 * 8192 + 5, 100_003, 0, 65_536, 2, 40_000]
+    rates = [0.0, 0.01, 0.3, 1.0, 0.035]
+    pairs = [_random_pair(rng, n, rates[i % len(rates)]) for i, n in enumerate(sizes)]
+    olds = [dev_bits(a) for a, _ in pairs]
+    news = [dev_bits(b) for _, b in pairs]
+    plan, d = _gpu_encode(dws, olds, news)
+    want = oracle.encode([a for a, _ in pairs], [b for _, b in pairs])
+    assert_delta_equal(delta_to_host(d), want)
+    # dws_count alone gives the same offsets
+    offs = plan.count(dws.ptr_table(olds), dws.ptr_table(news))
+    plan.raise_on_error()
+    np.testing.assert_array_equal(offs.cpu().numpy(), want[0])
+
+
+def test_encode_unaligned_views(dws):
+    # Views starting 1, 3, 5 elements into a buffer (2-byte but not 16-byte
+    # aligned), with old and new misaligned differently: the plain-load path.
+    rng = np.random.default_rng(5)
+    olds, news, ha, hb = [], [], [], []
+    for k, (n, oa, ob) in enumerate([(20_000, 1, 3), (8192 * 2 + 3, 5, 5), (17, 2, 0), (9000, 0, 7)]):
+        a, b = _random_pair(rng, n, 0.05 * (k + 1))
+        base_a = torch.zeros(n + 16, dtype=torch.bfloat16, device="cuda")
+        base_b = torch.zeros(n + 16, dtype=torch.bfloat16, device="cuda")
+        va, vb = base_a[oa:oa + n], base_b[ob:ob + n]
+        va.copy_(dev_bits(a))
+        vb.copy_(dev_bits(b))
+        olds.append(va)
+        news.append(vb)
+        ha.append(a)
+        hb.append(b)
+    _, d = _gpu_encode(dws, olds, news)
+    assert_delta_equal(delta_to_host(d), oracle.encode(ha, hb))
+
+
+def test_encode_many_tiny_tensors(dws):
+    # 3000 tensors, most of them a single short tile: thousands of tickets
+    # and look-backs across tiles with counts of 0..40.
+    rng = np.random.default_rng(17)
+    sizes = rng.integers(0, 41, 3000)
+    pairs = [_random_pair(rng, int(n), 0.2) for n in sizes]
+    olds = [dev_bits(a) for a, _ in pairs]
+    news = [dev_bits(b) for _, b in pairs]
+    _, d = _gpu_encode(dws, olds, news)
+    assert_delta_equal(delta_to_host(d), oracle.encode([a for a, _ in pairs], [b for _, b in pairs]))
+
+
+def test_encode_capacity_overflow_reports_required_nnz(dws):
+    rng = np.random.default_rng(23)
+    pairs = [_random_pair(rng, n, 0.1) for n in (50_000, 30_001, 0, 8192)]
+    olds = [dev_bits(a) for a, _ in pairs]
+    news = [dev_bits(b) for _, b in pairs]
+    want = oracle.encode([a for a, _ in pairs], [b for _, b in pairs])
+    nnz = int(want[0][-1])
+    cap = nnz // 2
+    plan = dws.DeltaPlan.for_tensors(olds)
+    offsets = torch.empty(len(olds) + 1, dtype=torch.int64, device="cuda")
+    idx = torch.full((cap + 64,), -7, dtype=torch.int32, device="cuda")
+    val = torch.full((cap + 64,), -7, dtype=torch.int16, device="cuda")
+    code = dws.dws_encode(plan.handle, dws.ptr_table(olds).data_ptr(), dws.ptr_table(news).data_ptr(),
+                          offsets.data_ptr(), idx.data_ptr(), val.data_ptr(), cap,
+                          plan.workspace.data_ptr(), plan.workspace_bytes,
+                          torch.cuda.current_stream().cuda_stream)
+    assert code == dws.DWS_OK
+    st, detail = plan.status()
+    assert st == dws.DWS_ERR_CAPACITY and detail == nnz
+    np.testing.assert_array_equal(offsets.cpu().numpy(), want[0])
+    np.testing.assert_array_equal(idx[:cap].cpu().numpy(), want[1][:cap])
+    np.testing.assert_array_equal(val[:cap].cpu().numpy().view(np.uint16), want[2][:cap])
+    assert (idx[cap:].cpu().numpy() == -7).all() and (val[cap:].cpu().numpy() == -7).all()
+
+
+def test_encode_identical_and_all_changed(dws):
+    rng = np.random.default_rng(29)
+    a = rng.integers(0, 1 << 16, 1_000_003, dtype=np.uint16)
+    t = dev_bits(a)
+    _, d = _gpu_encode(dws, [t], [t.clone()])
+    assert d.nnz() == 0 and d.count == 0
+    b = a ^ np.uint16(0x0001)
+    _, d = _gpu_encode(dws, [t], [dev_bits(b)])
+    assert_delta_equal(delta_to_host(d), oracle.encode([a], [b]))
+    assert d.nnz() == a.size
+
+
+def test_encode_reuses_workspace_across_calls(dws):
+    rng = np.random.default_rng(31)
+    a1, b1 = _random_pair(rng, 70_000, 0.02)
+    a2, b2 = _random_pair(rng, 70_000, 0.4)
+    plan = dws.DeltaPlan([70_000])
+    for a, b in ((a1, b1), (a2, b2), (a1, b1)):
+        ot, nt = dws.ptr_table([dev_bits(a)]), dws.ptr_table([dev_bits(b)])
+        d = plan.encode_exact(ot, nt)
+        assert_delta_equal(delta_to_host(d), oracle.encode([a], [b]))
+
+
+def test_encode_timeout_is_reported_and_context_survives(dws):
+    # Tile 1 never publishes its count; tile 2's bounded wait runs out after
+    # 50 ms, the kernel records DWS_ERR_TIMEOUT, every waiter leaves, and the
+    # context stays usable for the next call.
+    rng = np.random.default_rng(37)
+    a, b = _random_pair(rng, 8192 * 6 + 100, 0.05)
+    olds, news = [dev_bits(a)], [dev_bits(b)]
+    plan = dws.DeltaPlan.for_tensors(olds)
+    cap = a.size
+    offsets = torch.zeros(2, dtype=torch.int64, device="cuda")
+    idx = torch.empty(cap, dtype=torch.int32, device="cuda")
+    val = torch.empty(cap, dtype=torch.int16, device="cuda")
+    ot, nt = dws.ptr_table(olds), dws.ptr_table(news)
+    code = dws.dws_encode_ex(plan.handle, ot.data_ptr(), nt.data_ptr(), offsets.data_ptr(),
+                             idx.data_ptr(), val.data_ptr(), cap, plan.workspace.data_ptr(),
+                             plan.workspace_bytes, torch.cuda.current_stream().cuda_stream,
+                             50_000_000, 1)
+    assert code == dws.DWS_OK
+    st, detail = plan.status()
+    assert st == dws.DWS_ERR_TIMEOUT and detail >= 2
+    d = plan.encode_exact(ot, nt)
+    assert_delta_equal(delta_to_host(d), oracle.encode([a], [b]))
+
+
+def test_workspace_of_another_plan_is_refused(dws):
+    rng = np.random.default_rng(41)
+    a, b = _random_pair(rng, 1000, 0.5)
+    plan_a = dws.DeltaPlan([1000])
+    plan_b = dws.DeltaPlan([999, 1])
+    ot, nt = dws.ptr_table([dev_bits(a)]), dws.ptr_table([dev_bits(b)])
+    offsets = torch.full((2,), -3, dtype=torch.int64, device="cuda")
+    idx = torch.full((1000,), -3, dtype=torch.int32, device="cuda")
+    val = torch.full((1000,), -3, dtype=torch.int16, device="cuda")
+    # plan_a's call with plan_b's (large enough) workspace
+    assert plan_b.workspace_bytes >= plan_a.workspace_bytes
+    code = dws.dws_encode(plan_a.handle, ot.data_ptr(), nt.data_ptr(), offsets.data_ptr(),
+                          idx.data_ptr(), val.data_ptr(), 1000, plan_b.workspace.data_ptr(),
+                          plan_b.workspace_bytes, torch.cuda.current_stream().cuda_stream)
+    assert code == dws.DWS_OK
+    st, _ = plan_b.status()
+    assert st == dws.DWS_ERR_WORKSPACE
+    assert (offsets.cpu().numpy() == -3).all() and (idx.cpu().numpy() == -3).all()
+
+
+# ---------------------------------------------------------------- apply
+
+
+def _guarded(a: np.ndarray, guard=64):
+    """Device copy of a with guard elements (0x5a5a) on both sides."""
+    base = torch.full((a.size + 2 * guard,), 0x5a5a, dtype=torch.int16, device="cuda")
+    base[guard:guard + a.size] = torch.from_numpy(a.view(np.int16).copy()).cuda()
+    return base, base[guard:guard + a.size].view(torch.bfloat16)
+
+
+def _guards_intact(base, n, guard=64):
+    h = base.cpu().numpy()
+    return (h[:guard] == 0x5a5a).all() and (h[guard + n:] == 0x5a5a).all()
+
+
+def test_apply_roundtrip_leaves_unchanged_positions(dws):
+    rng = np.random.default_rng(43)
+    sizes = [30_000, 0, 8192 * 3 + 1, 5, 100_000]
+    pairs = [_random_pair(rng, n, 0.03) for n in sizes]
+    olds = [dev_bits(a) for a, _ in pairs]
+    news = [dev_bits(b) for _, b in pairs]
+    plan, d = _gpu_encode(dws, olds, news)
+    snaps = [_guarded(a) for a, _ in pairs]
+    plan.apply(dws.ptr_table([s for _, s in snaps]), d)
+    plan.raise_on_error("apply")
+    for (base, s), (a, b) in zip(snaps, pairs):
+        np.testing.assert_array_equal(host_bits(s), b)
+        assert _guards_intact(base, a.size)
+
+
+def test_apply_empty_delta_is_identity(dws):
+    a = np.arange(5000, dtype=np.uint16)
+    t = dev_bits(a)
+    plan, d = _gpu_encode(dws, [t], [t.clone()])
+    snap = t.clone()
+    plan.apply(dws.ptr_table([snap]), d)
+    plan.raise_on_error()
+    np.testing.assert_array_equal(host_bits(snap), a)
+
+
+def test_apply_rejects_out_of_range_and_unsorted_entries(dws):
+    n = 1000
+    plan = dws.DeltaPlan([n])
+    base, snap = _guarded(np.zeros(n, np.uint16))
+    for idx in ([5, n], [5, -1], [7, 7], [9, 3]):
+        offsets = torch.tensor([0, 2], dtype=torch.int64, device="cuda")
+        indices = torch.tensor(idx, dtype=torch.int32, device="cuda")
+        values = torch.tensor([0x1111, 0x2222], dtype=torch.int16, device="cuda")
+        plan.apply(dws.ptr_table([snap]), dws.Delta(offsets, indices, values))
+        st, detail = plan.status()
+        assert st == dws.DWS_ERR_BAD_DELTA and detail == 1, idx
+        assert _guards_intact(base, n)
+
+
+def test_apply_with_bad_offsets_writes_nothing(dws):
+    n = 1000
+    plan = dws.DeltaPlan([n, n])
+    snaps = [dev_bits(np.zeros(n, np.uint16)) for _ in range(2)]
+    for offs in ([0, 3, 2], [1, 2, 3], [0, 2, 9]):
+        offsets = torch.tensor(offs, dtype=torch.int64, device="cuda")
+        indices = torch.tensor([1, 2, 3], dtype=torch.int32, device="cuda")
+        values = torch.tensor([1, 1, 1], dtype=torch.int16, device="cuda")
+        plan.apply(dws.ptr_table(snaps), dws.Delta(offsets, indices, values))
+        st, _ = plan.status()
+        assert st == dws.DWS_ERR_BAD_DELTA, offs
+        assert all(int(s.view(torch.int16).abs().sum()) == 0 for s in snaps)
+
+
+# ---------------------------------------------------------------- chain
+
+
+def test_chain_golden_later_delta_wins(dws):
+    anchor, deltas, final = G.chain_example()
+    snaps = [dev_bits(a) for a in anchor]
+    plan = dws.DeltaPlan.for_tensors(snaps)
+    dd = [dws.Delta(torch.from_numpy(o).cuda(), torch.from_numpy(i).cuda(),
+                    torch.from_numpy(v.view(np.int16)).cuda()) for o, i, v in deltas]
+    plan.apply_chain(dws.ptr_table(snaps), dd)
+    plan.raise_on_error()
+    for s, f in zip(snaps, final):
+        np.testing.assert_array_equal(host_bits(s), f)
+
+
+def _chain_case(dws, shapes_or_sizes, steps, stepper, anchor_set):
+    """Encode `steps` steps on the GPU (each delta checked against the oracle),
+    replay them in one chain launch onto a copy of the anchor."""
+    prev = anchor_set
+    plan = dws.DeltaPlan.for_tensors(prev.tensors)
+    deltas, host_deltas = [], []
+    prev_h = [host_bits(t) for t in prev.tensors]
+    for k in range(1, steps + 1):
+        cur = stepper(prev, k)
+        d = plan.encode_exact(dws.ptr_table(prev.tensors), dws.ptr_table(cur.tensors))
+        cur_h = [host_bits(t) for t in cur.tensors]
+        want = oracle.encode(prev_h, cur_h)
+        assert_delta_equal(delta_to_host(d), want)
+        deltas.append(d)
+        host_deltas.append(want)
+        prev, prev_h = cur, cur_h
+    snaps = [t.clone() for t in anchor_set.tensors]
+    plan.apply_chain(dws.ptr_table(snaps), deltas)
+    plan.raise_on_error("apply_chain")
+    ref = [host_bits(t) for t in anchor_set.tensors]
+    oracle.apply_chain(ref, host_deltas)
+    for s, r, f in zip(snaps, ref, prev_h):
+        np.testing.assert_array_equal(host_bits(s), r)
+        np.testing.assert_array_equal(r, f)
+
+
+def test_chain_qwen_shaped_scaled_ten_steps(dws):
+    s = W.SEEDS["qwen3_0p6b"]
+    shapes = W.scaled_shapes(W.qwen3_0p6b_shapes(), 8)
+    w0 = W.init_set(shapes, s, "cuda", 0.02)
+    _chain_case(dws, shapes, 10, lambda w, k: W.step_set(w, s, k, 3e-6, "cuda"), w0)
+
+
+def test_chain_stress_scaled_ten_steps(dws):
+    sizes = W.stress_sizes(count=300, lo=16, hi=300_000)
+    clustered = W.stress_clustered(count=300)
+    w0 = W.stress_init(sizes, "cuda")
+    _chain_case(dws, sizes, 10, lambda w, k: W.stress_step(w, clustered, k, "cuda")[0], w0)
+
+
+def test_chain_on_unaligned_snapshots(dws):
+    # Snapshot views that are not 16-byte aligned take the direct-store path.
+    rng = np.random.default_rng(47)
+    n = 8192 * 2 + 77
+    anchor = rng.integers(0, 1 << 16, n, dtype=np.uint16)
+    cur = anchor.copy()
+    host_deltas = []
+    for k in range(4):
+        nxt = cur.copy()
+        m = rng.random(n) < 0.2
+        nxt[m] ^= np.uint16(0x0101 + k)
+        host_deltas.append(oracle.encode([cur], [nxt]))
+        cur = nxt
+    base = torch.zeros(n + 8, dtype=torch.bfloat16, device="cuda")
+    snap = base[3:3 + n]
+    snap.copy_(dev_bits(anchor))
+    plan = dws.DeltaPlan([n])
+    dd = [dws.Delta(torch.from_numpy(o).cuda(), torch.from_numpy(i).cuda(),
+                    torch.from_numpy(v.view(np.int16)).cuda()) for o, i, v in host_deltas]
+    plan.apply_chain(dws.ptr_table([snap]), dd)
+    plan.raise_on_error()
+    np.testing.assert_array_equal(host_bits(snap), cur)
+
+
+def test_chain_rejects_index_beyond_numel(dws):
+    n = 9000
+    plan = dws.DeltaPlan([n])
+    snap = dev_bits(np.zeros(n, np.uint16))
+    d = dws.Delta(torch.tensor([0, 2], dtype=torch.int64, device="cuda"),
+                  torch.tensor([3, n + 5], dtype=torch.int32, device="cuda"),
+                  torch.tensor([7, 7], dtype=torch.int16, device="cuda"))
+    plan.apply_chain(dws.ptr_table([snap]), [d])
+    st, _ = plan.status()
+    assert st == dws.DWS_ERR_BAD_DELTA
+    h = host_bits(snap)
+    assert h[3] == 7 and h.sum() == 7
+
+
+# ---------------------------------------------------------------- XOR
+
+
+@pytest.mark.parametrize("n,oa,ob,oc", [(0, 0, 0, 0), (1, 0, 0, 0), (15, 3, 3, 3), (16, 0, 0, 0),
+                                        (17, 1, 1, 1), (1_000_003, 5, 5, 5), (100_001, 1, 2, 3),
+                                        (4096 * 64 + 9, 0, 8, 0)])
+def test_xor_encode_apply_alignments(dws, n, oa, ob, oc):
+    rng = np.random.default_rng(n + oa)
+    a = rng.integers(0, 256, n, dtype=np.uint8)
+    b = a.copy()
+    if n:
+        m = rng.random(n) < 0.3
+        b[m] = rng.integers(0, 256, int(m.sum()), dtype=np.uint8)
+    ba = torch.zeros(n + 32, dtype=torch.uint8, device="cuda")
+    bb = torch.zeros(n + 32, dtype=torch.uint8, device="cuda")
+    bc = torch.full((n + 32,), 0xAB, dtype=torch.uint8, device="cuda")
+    va, vb, vc = ba[oa:oa + n], bb[ob:ob + n], bc[oc:oc + n]
+    va.copy_(torch.from_numpy(a))
+    vb.copy_(torch.from_numpy(b))
+    dws.xor_encode(va, vb, vc)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_bytes(vc), oracle.xor_encode(a, b))
+    h = bc.cpu().numpy()
+    assert (h[:oc] == 0xAB).all() and (h[oc + n:] == 0xAB).all()
+    dws.xor_apply(va, vc)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_bytes(va), b)
+
+
+def test_xor_layer_closed_form(dws):
+    old, new, pos = W.xor_layer(2, "cuda", nbytes=3_000_017, flips=2_550)
+    mask = dws.xor_encode(old, new)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(np.flatnonzero(host_bytes(mask)), pos.cpu().numpy())
+    buf = old.clone()
+    dws.xor_apply(buf, mask)
+    torch.cuda.synchronize()
+    assert torch.equal(buf, new)
+
+
+@pytest.mark.parametrize("pinned_masks", [False, True])
+def test_xor_apply_layers_double_buffered(dws, pinned_masks):
+    sizes = [1_000_000, 333_333, 2_500_001, 16, 0, 777_777]
+    olds, news, masks = [], [], []
+    for l, n in enumerate(sizes):
+        o, nw, _ = W.xor_layer(l, "cuda", nbytes=max(n, 1), flips=max(1, n // 1000))
+        o, nw = o[:n], nw[:n]
+        olds.append(o.clone())
+        news.append(nw)
+        m = dws.xor_encode(o, nw) if n else torch.empty(0, dtype=torch.uint8, device="cuda")
+        masks.append(m.cpu().pin_memory() if pinned_masks else m)
+    torch.cuda.synchronize()
+    staging = [torch.empty(600_000, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    copy_stream = torch.cuda.Stream()
+    dws.xor_apply_layers(olds, masks, staging[0], staging[1],
+                         apply_stream=torch.cuda.current_stream(), copy_stream=copy_stream)
+    torch.cuda.current_stream().synchronize()
+    for o, nw in zip(olds, news):
+        assert torch.equal(o, nw)

@@ -190,6 +190,27 @@ class BF16Set:
         return sum(self.numels)
 
 
+def pack_flat(sizes, make, device, align: int = 128):
+    """Lay tensors out back to back in one zero-filled bf16 buffer, each
+    starting on a multiple of ``align`` elements (as separate allocations
+    would be aligned).  ``make(t, n)`` returns tensor t's values (or None to
+    leave zeros).  Returns (flat buffer, list of views)."""
+    offs, off = [], 0
+    for n in sizes:
+        offs.append(off)
+        off += (int(n) + align - 1) // align * align
+    flat = torch.zeros(max(off, 1), dtype=torch.bfloat16, device=device)
+    views = []
+    for t, (o, n) in enumerate(zip(offs, sizes)):
+        v = flat[o:o + int(n)]
+        x = make(t, int(n))
+        if x is not None:
+            v.copy_(x)
+            del x
+        views.append(v)
+    return flat, views
+
+
 def init_set(shapes, s: int, device, std: float) -> BF16Set:
     names, ts = [], []
     for t, (name, shape) in enumerate(shapes):
