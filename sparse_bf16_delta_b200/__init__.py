@@ -227,7 +227,11 @@ def ptr_table(tensors, device=None):
     torch = _torch()
     dev = device if device is not None else tensors[0].device
     ptrs = [int(t.data_ptr()) if t.numel() > 0 else 0 for t in tensors]
-    return torch.tensor(ptrs, dtype=torch.int64).to(dev, non_blocking=False)
+    table = torch.tensor(ptrs, dtype=torch.int64).to(dev, non_blocking=False)
+    # The table holds references to its tensors, so their memory cannot be
+    # freed (and reused) while a kernel may still read through the table.
+    table._dws_tensors = list(tensors)
+    return table
 
 
 class Delta:

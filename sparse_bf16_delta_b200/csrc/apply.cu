@@ -144,18 +144,21 @@ __global__ void __launch_bounds__(kApplyThreads) apply_kernel(ApplyParams p) {
 // ---------------------------------------------------------------------------
 constexpr int kChainThreads = 256;
 constexpr int kChainMaxSlots = 4096;  // K * block_len entries read per round
+constexpr int kChainSlotsPerThread = kChainMaxSlots / kChainThreads;
 
 struct ChainParams {
     WsView ws;
     uint16_t *const *snap_ptrs;
     long long tiles_per_cta;
     int K;
-    int block_len;  // entries read per delta per round
+    int block_len;  // entries read per delta per round (multiple of 32)
     DeltaRef d[DWS_MAX_CHAIN];
 };
 
-struct TileMeta {
-    uint16_t *ptr;  // tile start in the snapshot
+// A unit: up to kChainUnitTiles consecutive plan tiles of one tensor.
+struct UnitMeta {
+    uint16_t *ptr;   // unit start in the snapshot
+    long long next;  // first plan tile after the unit
     int tensor;
     int local_start;
     int count;
@@ -163,34 +166,42 @@ struct TileMeta {
 };
 
 struct ChainSmem {
-    uint16_t tile[2][kTileElems];
-    uint32_t tag[kTileElems];
+    uint16_t tile[2][kChainUnitElems];
+    uint32_t tag[kChainUnitElems];
     long long cur[DWS_MAX_CHAIN];
     long long end[DWS_MAX_CHAIN];
     int consumed[DWS_MAX_CHAIN];
     int active[DWS_MAX_CHAIN];
     unsigned long long bar[2];
-    TileMeta meta[2];
+    UnitMeta meta[2];
 };
 
-// Thread 0: describe tile i and start its load into buffer b.
-__device__ void chain_issue(const ChainParams &p, ChainSmem &sm, long long i, int b,
+// Thread 0: describe the unit starting at plan tile i (ending before `te`)
+// and start its load into buffer b.
+__device__ void chain_issue(const ChainParams &p, ChainSmem &sm, long long i, long long te, int b,
                             unsigned long long policy) {
-    TileMeta m;
+    UnitMeta m;
     m.ptr = nullptr;
+    m.next = i + 1;
     m.tensor = 0;
     m.local_start = 0;
     m.count = 0;
     m.bulk = 0;
     const int t = p.ws.tile_tensor[i];
     if (t >= 0 && t < p.ws.num_tensors) {
-        const long long ls = (i - p.ws.first_tile[t]) << kTileShift;
+        const long long first = p.ws.first_tile[t];
+        long long j = p.ws.first_tile[t + 1];
+        if (j > i + kChainUnitTiles) j = i + kChainUnitTiles;
+        if (j > te) j = te;
+        const long long ls = (i - first) << kTileShift;
         const long long n = p.ws.numel[t];
-        if (ls >= 0 && ls <= n) {
+        if (ls >= 0 && ls <= n && j > i) {
             const long long rest = n - ls;
+            const long long span = (j - i) << kTileShift;
+            m.next = j;
             m.tensor = t;
             m.local_start = static_cast<int>(ls);
-            m.count = static_cast<int>(rest < kTileElems ? rest : kTileElems);
+            m.count = static_cast<int>(rest < span ? rest : span);
             uint16_t *sp = p.snap_ptrs[t];
             const uintptr_t ua = reinterpret_cast<uintptr_t>(sp);
             if (m.count > 0 && (sp == nullptr || (ua & 1u))) {
@@ -249,19 +260,19 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
     if (tb >= te) return;
 
     unsigned long long policy = 0;
-    for (int e = tid; e < kTileElems; e += kChainThreads) sm.tag[e] = 0u;
+    for (int e = tid; e < kChainUnitElems; e += kChainThreads) sm.tag[e] = 0u;
     if (tid == 0) {
         policy = l2_evict_first_policy();
         mbar_init(&sm.bar[0], 1);
         mbar_init(&sm.bar[1], 1);
         mbar_fence_init();
-        chain_issue(p, sm, tb, 0, policy);
+        chain_issue(p, sm, tb, te, 0, policy);
     }
     __syncthreads();
 
-    // Cursors at the CTA's first tile: one binary search per delta.
+    // Cursors at the CTA's first unit: one binary search per delta.
     {
-        const TileMeta m0 = sm.meta[0];
+        const UnitMeta m0 = sm.meta[0];
         for (int k = warp; k < p.K; k += kWarps) {
             const DeltaRef d = p.d[k];
             const long long lo = d.offsets[m0.tensor];
@@ -280,51 +291,73 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
     }
     __syncthreads();
 
+    const int L = p.block_len;
+    const int slots = p.K * L;
     uint32_t phase_bits = 0;
-    for (long long i = tb; i < te; ++i) {
-        const int b = static_cast<int>((i - tb) & 1);
-        if (tid == 0 && i + 1 < te) {
+    int b = 0;
+    bool first_unit = true;
+    for (long long i = tb; i < te;) {
+        const UnitMeta m = sm.meta[b];
+        if (tid == 0 && m.next < te) {
             bulk_wait_read_all();  // the store from the other buffer has read it
-            chain_issue(p, sm, i + 1, b ^ 1, policy);
+            chain_issue(p, sm, m.next, te, b ^ 1, policy);
         }
-        const TileMeta m = sm.meta[b];
         const int ls = m.local_start;
 
         // New tensor inside the CTA's range: the previous tensor's entries
         // must all have been consumed (else some index was >= numel).
-        if (i != tb && ls == 0) {
+        if (!first_unit && ls == 0) {
             if (tid < p.K) {
                 const DeltaRef d = p.d[tid];
                 if (sm.cur[tid] != sm.end[tid]) record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, sm.cur[tid]);
                 sm.cur[tid] = d.offsets[m.tensor];
                 sm.end[tid] = d.offsets[m.tensor + 1];
             }
-            __syncthreads();
         }
-
-        // ---- entry phase: tag this tile's entries of every delta ----------
         if (tid < p.K) sm.active[tid] = (sm.cur[tid] < sm.end[tid]);
         __syncthreads();
-        const int L = p.block_len;
-        const int slots = p.K * L;
+
+        // ---- entry phase: tag this unit's entries of every delta ----------
         for (;;) {
-            for (int sidx = tid; sidx < slots; sidx += kChainThreads) {
-                const int k = sidx / L;
-                const int r = sidx - k * L;
-                if (!sm.active[k]) continue;
-                const long long j = sm.cur[k] + r;
-                if (j >= sm.end[k]) continue;
-                const DeltaRef &d = p.d[k];
-                const int idx = __ldg(d.indices + j);
-                if (idx < ls) {
-                    // Not ascending (or negative): skip, but consume it.
-                    record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, j);
-                    atomicMax(&sm.consumed[k], r + 1);
-                } else if (idx - ls < m.count) {
-                    const uint32_t key = (static_cast<uint32_t>(k + 1) << 16) | __ldg(d.values + j);
-                    atomicMax(&sm.tag[idx - ls], key);
-                    atomicMax(&sm.consumed[k], r + 1);
+            int idx[kChainSlotsPerThread];
+            uint16_t val[kChainSlotsPerThread];
+            bool valid[kChainSlotsPerThread];
+#pragma unroll
+            for (int q = 0; q < kChainSlotsPerThread; ++q) {
+                const int sidx = tid + q * kChainThreads;
+                valid[q] = false;
+                if (sidx < slots) {
+                    const int k = sidx / L;
+                    const long long j = sm.cur[k] + (sidx - k * L);
+                    if (sm.active[k] && j < sm.end[k]) {
+                        valid[q] = true;
+                        idx[q] = __ldg(p.d[k].indices + j);
+                        val[q] = __ldg(p.d[k].values + j);
+                    }
                 }
+            }
+#pragma unroll
+            for (int q = 0; q < kChainSlotsPerThread; ++q) {
+                const int sidx = tid + q * kChainThreads;
+                if (q * kChainThreads >= slots) break;  // uniform across the CTA
+                bool take = false;
+                if (valid[q]) {
+                    const int k = sidx / L;
+                    if (idx[q] < ls) {
+                        // Not ascending (or negative): skip, but consume it.
+                        record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, sm.cur[k] + (sidx - k * L));
+                        take = true;
+                    } else if (idx[q] - ls < m.count) {
+                        const uint32_t key = (static_cast<uint32_t>(k + 1) << 16) | val[q];
+                        atomicMax(&sm.tag[idx[q] - ls], key);
+                        take = true;
+                    }
+                }
+                // 32 consecutive slots of a warp belong to one delta (L is a
+                // multiple of 32): count them with one shared atomic.
+                const unsigned int ballot = __ballot_sync(0xffffffffu, take);
+                if (lane == 0 && ballot != 0u && sidx < slots)
+                    atomicAdd(&sm.consumed[sidx / L], __popc(ballot));
             }
             __syncthreads();
             int again = 0;
@@ -340,7 +373,7 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
             if (!__syncthreads_or(again)) break;
         }
 
-        // ---- merge: tags over the snapshot tile ----------------------------
+        // ---- merge: tags over the snapshot unit ----------------------------
         const uint32_t parity = (phase_bits >> b) & 1u;
         phase_bits ^= (1u << b);
         const bool loaded = mbar_wait(&sm.bar[b], parity, kLoadWaitLimitNs);
@@ -377,6 +410,9 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
             bulk_store(m.ptr, sm.tile[b], static_cast<uint32_t>(m.bulk) * 2u);
             bulk_commit();
         }
+        i = m.next;
+        b ^= 1;
+        first_unit = false;
     }
 
     // The CTA's range ends at the end of a tensor: all of its entries must
@@ -446,16 +482,16 @@ cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs,
     p.snap_ptrs = snap_ptrs;
     p.K = K;
     for (int k = 0; k < K; ++k) p.d[k] = deltas[k];
-    // Entries read per delta per round: the mean per full tile with margin.
-    const double per_tile = total_elems > 0
-                                ? double(total_entries) / K * kTileElems / double(total_elems)
+    // Entries read per delta per round: the mean per full unit with margin,
+    // a multiple of 32 (one warp's slots always belong to one delta) and
+    // K * L <= kChainMaxSlots (K <= 64 keeps L >= 64).
+    const double per_unit = total_elems > 0
+                                ? double(total_entries) / K * kChainUnitElems / double(total_elems)
                                 : 0.0;
-    long long L = static_cast<long long>(per_tile * 1.25) + 32;
+    long long L = static_cast<long long>(per_unit * 1.25) + 32;
     L = (L + 31) & ~31LL;
-    long long cap = kChainMaxSlots / K;
-    if (cap < 32) cap = 32;
+    const long long cap = (kChainMaxSlots / K) & ~31LL;
     if (L > cap) L = cap;
-    if (L < 32) L = 32;
     p.block_len = static_cast<int>(L);
 
     long long grid = static_cast<long long>(di.sm_count) * di.chain_ctas_per_sm;

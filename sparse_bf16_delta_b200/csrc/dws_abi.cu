@@ -95,6 +95,7 @@ WsView view_of(const dws_plan *p, void *ws) {
     v.first_tile = reinterpret_cast<const long long *>(base + p->layout.first_tile_off);
     v.tile_tensor = reinterpret_cast<const int *>(base + p->layout.tile_tensor_off);
     v.tile_status = reinterpret_cast<unsigned long long *>(base + p->layout.tile_status_off);
+    v.tile_desc = reinterpret_cast<dws::TileDesc *>(base + p->layout.tile_desc_off);
     v.num_tiles = p->ntiles;
     v.num_tensors = p->T;
     v.fingerprint = p->fingerprint;

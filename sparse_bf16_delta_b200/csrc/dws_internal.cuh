@@ -20,11 +20,15 @@ namespace dws {
 // ---------------------------------------------------------------------------
 // Tiling shared by the encode scan and the chain replay: a tensor is cut into
 // tiles of kTileElems elements (16 KiB of bf16 per snapshot); a tile never
-// straddles two tensors and an empty tensor owns one empty tile.
+// straddles two tensors and an empty tensor owns one empty tile.  The chain
+// replay works on units of up to kChainUnitTiles consecutive tiles of one
+// tensor.
 // ---------------------------------------------------------------------------
 constexpr int kTileElems = 8192;
 constexpr int kTileShift = 13;
 static_assert((1 << kTileShift) == kTileElems, "tile size must be a power of two");
+constexpr int kChainUnitTiles = 1;
+constexpr int kChainUnitElems = kChainUnitTiles * kTileElems;
 
 // ---------------------------------------------------------------------------
 // Workspace layout (device memory owned by the caller)
@@ -34,6 +38,7 @@ static_assert((1 << kTileShift) == kTileElems, "tile size must be a power of two
 //   first_tile        int64[T+1]         first tile of tensor  (static)
 //   tile_tensor       int32[ntiles]      tensor of each tile   (static)
 //   tile_status       uint64[ntiles]     encode scan state     (per call)
+//   tile_desc         TileDesc[ntiles]   encode tile pointers  (per call)
 //
 // Every region starts on a 256-byte boundary.  The static regions are written
 // by dws_plan_upload; the header's magic + fingerprint tie the workspace to
@@ -55,8 +60,20 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
 
+// Per-call description of an encode tile, written by the prepare pass so the
+// encode kernel needs one 32-byte load per ticket.
+struct TileDesc {
+    const uint16_t *old_p;  // tile start in the old snapshot (null if count == 0)
+    const uint16_t *new_p;  // tile start in the new snapshot
+    int tensor;
+    int local_start;  // first element of the tile within its tensor
+    int count;        // elements in the tile (0 .. kTileElems)
+    int bulk;         // leading elements that can move by bulk copy (multiple of 8)
+};
+static_assert(sizeof(TileDesc) == 32, "tile descriptor is 32 bytes");
+
 struct WsLayout {
-    size_t numel_off, first_tile_off, tile_tensor_off, tile_status_off, total;
+    size_t numel_off, first_tile_off, tile_tensor_off, tile_status_off, tile_desc_off, total;
 };
 
 inline size_t round_up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -67,7 +84,8 @@ inline WsLayout ws_layout(int T, long long ntiles) {
     L.first_tile_off = round_up256(L.numel_off + sizeof(long long) * size_t(T));
     L.tile_tensor_off = round_up256(L.first_tile_off + sizeof(long long) * size_t(T + 1));
     L.tile_status_off = round_up256(L.tile_tensor_off + sizeof(int) * size_t(ntiles));
-    L.total = round_up256(L.tile_status_off + sizeof(unsigned long long) * size_t(ntiles));
+    L.tile_desc_off = round_up256(L.tile_status_off + sizeof(unsigned long long) * size_t(ntiles));
+    L.total = round_up256(L.tile_desc_off + sizeof(TileDesc) * size_t(ntiles));
     return L;
 }
 
@@ -78,6 +96,7 @@ struct WsView {
     const long long *first_tile;
     const int *tile_tensor;
     unsigned long long *tile_status;
+    TileDesc *tile_desc;
     long long num_tiles;
     int num_tensors;
     unsigned long long fingerprint;
@@ -269,7 +288,6 @@ cudaError_t device_info(DeviceInfo *out);
 cudaError_t launched();
 
 cudaError_t launch_fill_tile_map(const WsView &ws, cudaStream_t s);
-cudaError_t launch_ws_reset(const WsView &ws, cudaStream_t s);
 cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
                           const uint16_t *const *new_ptrs, long long *offsets, int *indices,
                           uint16_t *values, long long capacity, bool compact,

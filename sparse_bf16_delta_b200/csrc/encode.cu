@@ -7,19 +7,32 @@
 // plan order with a per-tensor offsets[] prefix.
 //
 // How (single pass over both snapshots, 4 bytes read per element):
-//   * Persistent CTAs take tiles (8192 elements) by atomic ticket, so a tile's
-//     predecessors are always resident or finished (forward progress of the
-//     scan below).
-//   * Each CTA keeps kStages tiles in flight: thread 0 issues 1-D bulk async
-//     copies (cp.async.bulk, global -> own shared memory, mbarrier
-//     transaction counts, L2 evict-first) of both snapshots for the next
-//     tickets while the CTA works on the current one.
+//   * A prepare pass (one thread per tile) clears the scan state and writes a
+//     32-byte descriptor per tile: pointers to the tile in both snapshots,
+//     tensor, local start, element count.
+//   * Persistent CTAs (256 threads, 2 per SM) take tiles of 8192 elements by
+//     atomic ticket, so a tile's predecessors are always resident or finished
+//     (forward progress of the scan below).  Each CTA owns kStages stages,
+//     each holding both snapshots' 16 KiB of a tile, filled by two 1-D bulk
+//     async copies (cp.async.bulk, global -> own shared memory, mbarrier
+//     transaction count, L2 evict-first).
+//   * The CTA runs an event loop that never blocks on the scan.  Each turn it
+//     (a) counts the oldest loaded stage if its data has arrived --
+//     detect, block scan, publish the tile's count, stage the changed offsets
+//     -- and (b) takes one non-blocking look-back step for the oldest counted
+//     tile; when that tile's prefix is known it writes the tile's entries,
+//     and the freed stage is refilled with a new ticket.  A tile's count thus
+//     depends only on its own data arriving, never on another tile's
+//     look-back: a ticket that is held while its CTA waits on a look-back
+//     makes every later tile wait on it in turn (convoys).
 //   * detect: 16-byte shared-memory reads in a bank-conflict-free order, a
 //     32-bit change mask per thread, popc; block scan of the counts.
 //   * scan: decoupled look-back over the tile status words (flag + 62-bit
-//     count), a warp probing 32 predecessors at a time; bounded by a wall-clock
-//     limit after which the kernel records DWS_ERR_TIMEOUT and all waiters
-//     leave.
+//     count); warp 0 reads 256 predecessors per round trip (8 per lane) and,
+//     while waiting, re-reads only the words still unpublished (re-reading
+//     whole windows from every waiting warp floods the L2 with requests to
+//     the hottest lines).  Bounded by a wall-clock limit after which the
+//     kernel records DWS_ERR_TIMEOUT and every CTA leaves.
 //   * compact: the tile's changed offsets are staged in shared memory (over
 //     the old snapshot's slot, no longer needed), then written out with
 //     consecutive threads storing consecutive entries (coalesced).
@@ -36,22 +49,22 @@ constexpr int kStages = 3;
 constexpr int kChunks = kTileElems / 8;  // 16-byte chunks of bf16 per tile
 static_assert(kChunks == 4 * kThreads, "each thread owns 4 chunks (32 elements)");
 
-constexpr unsigned long long kLoadWaitLimitNs = 4000000000ull;  // 4 s
+// Stage states.
+constexpr int kEmptyDone = 0;  // no more tickets for this stage
+constexpr int kLoading = 1;    // ticket taken, bulk copies in flight
+constexpr int kCounted = 2;    // count published, waiting for its prefix
+
+// Look-back step results.
+constexpr long long kNotReady = -2;
+constexpr long long kGaveUp = -1;
 
 struct StageMeta {
-    long long ticket;      // >= num_tiles: no more work
-    const uint16_t *old_p;  // tile start in the old snapshot
-    const uint16_t *new_p;  // tile start in the new snapshot
-    int tensor;
-    int local_start;  // first element of the tile within its tensor
-    int count;        // elements in the tile (0 .. kTileElems)
-    int bulk;         // leading elements delivered by bulk copy (multiple of 8)
+    long long ticket;
+    TileDesc d;
 };
 
 struct EncodeParams {
     WsView ws;
-    const uint16_t *const *old_ptrs;
-    const uint16_t *const *new_ptrs;
     long long *offsets;
     int *indices;
     uint16_t *values;
@@ -64,108 +77,119 @@ struct EncodeSmem {
     uint16_t buf[kStages][2][kTileElems];  // [stage][0 = old | staging, 1 = new]
     unsigned long long bar[kStages];
     StageMeta meta[kStages];
+    int state[kStages];
+    int total[kStages];
     int warp_sum[kWarps];
-    long long tile_prefix;
+    long long step_result;
 };
 
-// Thread 0: take the next ticket and start loading it into stage s.
-__device__ void issue_tile(const EncodeParams &p, EncodeSmem &sm, int s,
-                           unsigned long long policy) {
+// Thread 0: take the next ticket, read its descriptor, start loading it into
+// stage s (or mark the stage done).
+__device__ void refill(const EncodeParams &p, EncodeSmem &sm, int s) {
     StageMeta m;
     m.ticket = static_cast<long long>(atomicAdd(&p.ws.hdr->ticket, 1ull));
-    m.old_p = nullptr;
-    m.new_p = nullptr;
-    m.tensor = 0;
-    m.local_start = 0;
-    m.count = 0;
-    m.bulk = 0;
     if (m.ticket < p.ws.num_tiles) {
-        const int t = p.ws.tile_tensor[m.ticket];
-        bool ok = (t >= 0 && t < p.ws.num_tensors);
-        if (ok) {
-            const long long first = p.ws.first_tile[t];
-            const long long n = p.ws.numel[t];
-            const long long ls = (m.ticket - first) << kTileShift;
-            ok = (ls >= 0 && ls <= n);
-            if (ok) {
-                const long long rest = n - ls;
-                m.tensor = t;
-                m.local_start = static_cast<int>(ls);
-                m.count = static_cast<int>(rest < kTileElems ? rest : kTileElems);
-                if (m.count > 0) {
-                    const uint16_t *op = p.old_ptrs[t];
-                    const uint16_t *np = p.new_ptrs[t];
-                    const uintptr_t ua = reinterpret_cast<uintptr_t>(op);
-                    const uintptr_t ub = reinterpret_cast<uintptr_t>(np);
-                    if (op == nullptr || np == nullptr || ((ua | ub) & 1u)) {
-                        record_error(p.ws.hdr, DWS_ERR_INVALID, t);
-                        m.count = 0;
-                    } else {
-                        m.old_p = op + ls;
-                        m.new_p = np + ls;
-                        m.bulk = ((ua | ub) & 15u) == 0 ? (m.count & ~7) : 0;
-                    }
-                }
-            }
+        m.d = p.ws.tile_desc[m.ticket];
+        const uint32_t bulk = static_cast<uint32_t>(m.d.bulk);
+        mbar_arrive_expect_tx(&sm.bar[s], bulk * 4u);
+        if (bulk > 0) {
+            const unsigned long long policy = l2_evict_first_policy();
+            bulk_load(sm.buf[s][0], m.d.old_p, bulk * 2u, &sm.bar[s], policy);
+            bulk_load(sm.buf[s][1], m.d.new_p, bulk * 2u, &sm.bar[s], policy);
         }
-        if (!ok) {
-            record_error(p.ws.hdr, DWS_ERR_WORKSPACE, m.ticket);
-            m.count = 0;
-        }
-        mbar_arrive_expect_tx(&sm.bar[s], static_cast<uint32_t>(m.bulk) * 4u);
-        if (m.bulk > 0) {
-            const uint32_t bytes = static_cast<uint32_t>(m.bulk) * 2u;
-            bulk_load(sm.buf[s][0], m.old_p, bytes, &sm.bar[s], policy);
-            bulk_load(sm.buf[s][1], m.new_p, bytes, &sm.bar[s], policy);
-        }
+        sm.state[s] = kLoading;
+    } else {
+        sm.state[s] = kEmptyDone;
     }
     sm.meta[s] = m;
 }
 
-// Warp 0: exclusive prefix of tile `ticket` by decoupled look-back.
-// Returns -1 if the bounded wait ran out or another tile gave up.
-__device__ long long look_back(const EncodeParams &p, long long ticket) {
+// Resumable decoupled look-back, run by warp 0 (state in its registers).
+// Lane l holds predecessors base - 8l - q (q = 0..7, newest first).
+constexpr int kProbePerLane = 8;
+constexpr int kWindow = 32 * kProbePerLane;
+
+struct LookBack {
+    long long ticket;
+    long long base;
+    unsigned long long acc;
+    unsigned long long t0;
+    unsigned long long w[kProbePerLane];
+};
+
+__device__ __forceinline__ void lb_load_window(LookBack &lb, const unsigned long long *status) {
     const int lane = threadIdx.x & 31;
-    unsigned long long *status = p.ws.tile_status;
-    long long base = ticket - 1;
-    unsigned long long acc = 0;
-    unsigned long long t0 = 0;
-    unsigned int backoff = 32;
-    while (true) {
-        const long long j = base - lane;
-        const unsigned long long st = (j >= 0) ? ld_relaxed_gpu(status + j) : kFlagPrefix;
-        const unsigned int flag = static_cast<unsigned int>(st >> kFlagShift);
-        const unsigned int pmask = __ballot_sync(0xffffffffu, flag == 2u);
-        const unsigned int xmask = __ballot_sync(0xffffffffu, flag == 0u);
-        const int first_p = pmask ? (__ffs(pmask) - 1) : 32;
-        const unsigned int needed = (first_p >= 31) ? 0xffffffffu : ((2u << first_p) - 1u);
-        if (xmask & needed) {
-            // Some predecessor has not published yet: wait, boundedly.
-            int give_up = 0;
-            if (lane == 0) {
-                const unsigned long long now = global_timer_ns();
-                if (t0 == 0) t0 = now;
-                if (now - t0 > static_cast<unsigned long long>(p.wait_limit_ns)) {
-                    atomicExch(&p.ws.hdr->abort, 1u);
-                    record_error(p.ws.hdr, DWS_ERR_TIMEOUT, ticket);
-                    give_up = 1;
-                } else if (ld_relaxed_gpu_u32(&p.ws.hdr->abort) != 0u) {
-                    give_up = 1;
+#pragma unroll
+    for (int q = 0; q < kProbePerLane; ++q) {
+        const long long j = lb.base - kProbePerLane * lane - q;
+        lb.w[q] = (j >= 0) ? ld_relaxed_gpu(status + j) : kFlagPrefix;
+    }
+}
+
+__device__ __forceinline__ void lb_start(LookBack &lb, const EncodeParams &p, long long ticket) {
+    lb.ticket = ticket;
+    lb.base = ticket - 1;
+    lb.acc = 0;
+    lb.t0 = 0;
+    lb_load_window(lb, p.ws.tile_status);
+}
+
+// One step: evaluate the window loaded by the previous step.  Returns the
+// exclusive prefix, kNotReady (loads for the next step issued), or kGaveUp.
+__device__ long long lb_step(LookBack &lb, const EncodeParams &p) {
+    const int lane = threadIdx.x & 31;
+    int first_p = kProbePerLane;
+    bool unready = false;
+    unsigned long long sum = 0;
+#pragma unroll
+    for (int q = 0; q < kProbePerLane; ++q) {
+        if (first_p == kProbePerLane) {
+            const unsigned int flag = static_cast<unsigned int>(lb.w[q] >> kFlagShift);
+            if (flag == 0u) {
+                unready = true;
+            } else {
+                sum += lb.w[q] & kValueMask;
+                if (flag == 2u) first_p = q;
+            }
+        }
+    }
+    const unsigned int pmask = __ballot_sync(0xffffffffu, first_p < kProbePerLane);
+    const int p_lane = pmask ? (__ffs(pmask) - 1) : 32;
+    const bool blocks = (lane <= p_lane) && unready;
+    if (__any_sync(0xffffffffu, blocks)) {
+        int give_up = 0;
+        if (lane == 0) {
+            const unsigned long long now = global_timer_ns();
+            if (lb.t0 == 0) lb.t0 = now;
+            if (now - lb.t0 > static_cast<unsigned long long>(p.wait_limit_ns)) {
+                atomicExch(&p.ws.hdr->abort, 1u);
+                record_error(p.ws.hdr, DWS_ERR_TIMEOUT, lb.ticket);
+                give_up = 1;
+            } else if (ld_relaxed_gpu_u32(&p.ws.hdr->abort) != 0u) {
+                give_up = 1;
+            }
+        }
+        if (__shfl_sync(0xffffffffu, give_up, 0)) return kGaveUp;
+        // Re-read only the unpublished words that are needed.
+        if (blocks) {
+#pragma unroll
+            for (int q = 0; q < kProbePerLane; ++q) {
+                if ((lb.w[q] >> kFlagShift) == 0ull) {
+                    const long long j = lb.base - kProbePerLane * lane - q;
+                    lb.w[q] = ld_relaxed_gpu(p.ws.tile_status + j);
                 }
             }
-            give_up = __shfl_sync(0xffffffffu, give_up, 0);
-            if (give_up) return -1;
-            __nanosleep(backoff);
-            if (backoff < 1024) backoff <<= 1;
-            continue;
         }
-        unsigned long long v = (lane <= first_p) ? (st & kValueMask) : 0ull;
-#pragma unroll
-        for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
-        acc += v;
-        if (first_p < 32) return static_cast<long long>(acc);
-        base -= 32;
+        return kNotReady;
     }
+    unsigned long long v = (lane <= p_lane) ? sum : 0ull;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+    lb.acc += v;
+    if (p_lane < 32) return static_cast<long long>(lb.acc);
+    lb.base -= kWindow;
+    lb_load_window(lb, p.ws.tile_status);
+    return kNotReady;
 }
 
 template <bool kCompact>
@@ -178,179 +202,237 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(EncodeParams p) {
 
     if (!ws_matches(p.ws)) return;
 
-    unsigned long long policy = 0;
     if (tid == 0) {
-        policy = l2_evict_first_policy();
         for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
         mbar_fence_init();
-        for (int s = 0; s < kStages; ++s) issue_tile(p, sm, s, policy);
+        for (int s = 0; s < kStages; ++s) refill(p, sm, s);
     }
     __syncthreads();
 
     uint32_t phase_bits = 0;
+    int next_count = 0;   // oldest stage still to be counted (ring order)
+    int next_finish = 0;  // oldest counted stage waiting for its prefix
+    bool lb_active = false;
+    LookBack lb;
     bool stop = false;
-    int s = 0;
+
     for (;;) {
-        const StageMeta m = sm.meta[s];
-        if (m.ticket >= p.ws.num_tiles) break;
+        const int fs = next_finish;
+        const int f_state = sm.state[fs];
+        if (f_state == kEmptyDone) break;  // every stage after it is done too
+        bool progress = false;
 
-        // ---- wait for the tile's bulk copies -------------------------------
-        const uint32_t parity = (phase_bits >> s) & 1u;
-        phase_bits ^= (1u << s);
-        const bool loaded = mbar_wait(&sm.bar[s], parity, kLoadWaitLimitNs);
-
-        uint16_t *old_s = sm.buf[s][0];
-        uint16_t *new_s = sm.buf[s][1];
-
-        // ---- detect: 32 elements per thread, 4 chunks of 8 ----------------
-        uint32_t mask = 0;
+        // ---- (a) count the oldest loaded stage once its data is there ------
+        const int c = next_count;
+        if (sm.state[c] == kLoading) {
+            const uint32_t parity = (phase_bits >> c) & 1u;
+            const bool ready = __syncthreads_and(mbar_try_wait(&sm.bar[c], parity));
+            if (ready) {
+                phase_bits ^= (1u << c);
+                const StageMeta m = sm.meta[c];
+                const TileDesc &d = m.d;
+                uint16_t *old_s = sm.buf[c][0];
+                uint16_t *new_s = sm.buf[c][1];
+                uint32_t mask = 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int slot = ((tid >> 1) + j) & 3;  // conflict-free 16-byte reads
-            const int c = 4 * tid + slot;
-            const int e0 = c * 8;
-            uint4 a, b;
-            if (e0 + 8 <= m.bulk) {
-                a = *reinterpret_cast<const uint4 *>(old_s + e0);
-                b = *reinterpret_cast<const uint4 *>(new_s + e0);
-            } else {
-                uint16_t av[8], bv[8];
+                for (int j = 0; j < 4; ++j) {
+                    const int slot = ((tid >> 1) + j) & 3;  // conflict-free 16-byte reads
+                    const int e0 = (4 * tid + slot) * 8;
+                    uint4 a, b;
+                    if (e0 + 8 <= d.bulk) {
+                        a = *reinterpret_cast<const uint4 *>(old_s + e0);
+                        b = *reinterpret_cast<const uint4 *>(new_s + e0);
+                    } else {
+                        uint16_t av[8], bv[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int e = e0 + q;
-                    av[q] = (e < m.count) ? m.old_p[e] : uint16_t(0);
-                    bv[q] = (e < m.count) ? m.new_p[e] : uint16_t(0);
-                    if (kCompact && e < m.count) new_s[e] = bv[q];
+                        for (int q = 0; q < 8; ++q) {
+                            const int e = e0 + q;
+                            av[q] = (e < d.count) ? d.old_p[e] : uint16_t(0);
+                            bv[q] = (e < d.count) ? d.new_p[e] : uint16_t(0);
+                            if (kCompact && e < d.count) new_s[e] = bv[q];
+                        }
+                        a.x = av[0] | (uint32_t(av[1]) << 16);
+                        a.y = av[2] | (uint32_t(av[3]) << 16);
+                        a.z = av[4] | (uint32_t(av[5]) << 16);
+                        a.w = av[6] | (uint32_t(av[7]) << 16);
+                        b.x = bv[0] | (uint32_t(bv[1]) << 16);
+                        b.y = bv[2] | (uint32_t(bv[3]) << 16);
+                        b.z = bv[4] | (uint32_t(bv[5]) << 16);
+                        b.w = bv[6] | (uint32_t(bv[7]) << 16);
+                    }
+                    const uint32_t x0 = a.x ^ b.x, x1 = a.y ^ b.y, x2 = a.z ^ b.z, x3 = a.w ^ b.w;
+                    const uint32_t bits8 =
+                        ((x0 & 0xffffu) != 0) | (((x0 >> 16) != 0) << 1) |
+                        (((x1 & 0xffffu) != 0) << 2) | (((x1 >> 16) != 0) << 3) |
+                        (((x2 & 0xffffu) != 0) << 4) | (((x2 >> 16) != 0) << 5) |
+                        (((x3 & 0xffffu) != 0) << 6) | (((x3 >> 16) != 0) << 7);
+                    mask |= bits8 << (8 * slot);
                 }
-                a.x = av[0] | (uint32_t(av[1]) << 16);
-                a.y = av[2] | (uint32_t(av[3]) << 16);
-                a.z = av[4] | (uint32_t(av[5]) << 16);
-                a.w = av[6] | (uint32_t(av[7]) << 16);
-                b.x = bv[0] | (uint32_t(bv[1]) << 16);
-                b.y = bv[2] | (uint32_t(bv[3]) << 16);
-                b.z = bv[4] | (uint32_t(bv[5]) << 16);
-                b.w = bv[6] | (uint32_t(bv[7]) << 16);
-            }
-            const uint32_t x0 = a.x ^ b.x, x1 = a.y ^ b.y, x2 = a.z ^ b.z, x3 = a.w ^ b.w;
-            uint32_t bits8 = ((x0 & 0xffffu) != 0) | (((x0 >> 16) != 0) << 1) |
-                             (((x1 & 0xffffu) != 0) << 2) | (((x1 >> 16) != 0) << 3) |
-                             (((x2 & 0xffffu) != 0) << 4) | (((x2 >> 16) != 0) << 5) |
-                             (((x3 & 0xffffu) != 0) << 6) | (((x3 >> 16) != 0) << 7);
-            mask |= bits8 << (8 * slot);
-        }
-        const int cnt = __popc(mask);
-
-        // ---- block scan of the per-thread counts --------------------------
-        int incl = cnt;
+                const int cnt = __popc(mask);
+                int incl = cnt;
 #pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d) incl += v;
-        }
-        if (lane == 31) sm.warp_sum[warp] = incl;
-        // (1) counts published; everyone is done reading old_s.  The load wait
-        // is bounded; if it ran out anywhere, the whole CTA leaves together
-        // before anything is published or written.
-        if (!__syncthreads_and(loaded)) {
-            if (tid == 0) record_error(p.ws.hdr, DWS_ERR_TIMEOUT, m.ticket);
-            return;
-        }
-        int warp_off = 0, total = 0;
+                for (int dd = 1; dd < 32; dd <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, dd);
+                    if (lane >= dd) incl += v;
+                }
+                if (lane == 31) sm.warp_sum[warp] = incl;
+                __syncthreads();  // warp sums visible; old_s no longer read
+                int warp_off = 0, total = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const int v = sm.warp_sum[w];
-            warp_off += (w < warp) ? v : 0;
-            total += v;
-        }
-        const int excl = warp_off + incl - cnt;
-
-        // Warp 0 publishes the tile's aggregate before anything else.
-        const bool withheld = (m.ticket == p.withhold);
-        if (tid == 0 && !withheld) {
-            const unsigned long long flag = (m.ticket == 0) ? kFlagPrefix : kFlagAggregate;
-            st_relaxed_gpu(p.ws.tile_status + m.ticket,
-                           flag | static_cast<unsigned long long>(total));
-        }
-
-        // ---- stage the changed offsets (in ascending order) ---------------
-        if (kCompact) {
-            uint16_t *stage = old_s;
-            uint32_t mm = mask;
-            int r = excl;
-            while (mm) {
-                const int bit = __ffs(mm) - 1;
-                mm &= mm - 1;
-                stage[r++] = static_cast<uint16_t>(32 * tid + bit);
-            }
-        }
-
-        // ---- scan: exclusive prefix of this tile --------------------------
-        if (warp == 0) {
-            long long prefix;
-            if (withheld) {
-                prefix = -1;
-            } else if (m.ticket == 0) {
-                prefix = 0;
-            } else {
-                prefix = look_back(p, m.ticket);
-                if (lane == 0 && prefix >= 0) {
-                    st_relaxed_gpu(p.ws.tile_status + m.ticket,
-                                   kFlagPrefix | static_cast<unsigned long long>(prefix + total));
+                for (int w = 0; w < kWarps; ++w) {
+                    const int v = sm.warp_sum[w];
+                    warp_off += (w < warp) ? v : 0;
+                    total += v;
                 }
-            }
-            if (lane == 0) sm.tile_prefix = prefix;
-        }
-        __syncthreads();  // (2) staging complete, prefix known
-        const long long prefix = sm.tile_prefix;
-
-        if (prefix >= 0) {
-            if (tid == 0) {
-                if (m.local_start == 0) p.offsets[m.tensor] = prefix;
-                if (m.ticket == p.ws.num_tiles - 1) {
-                    const long long nnz = prefix + total;
-                    p.offsets[p.ws.num_tensors] = nnz;
-                    if (kCompact && nnz > p.capacity) record_error(p.ws.hdr, DWS_ERR_CAPACITY, nnz);
+                if (tid == 0) {
+                    if (m.ticket != p.withhold) {
+                        const unsigned long long flag =
+                            (m.ticket == 0) ? kFlagPrefix : kFlagAggregate;
+                        st_relaxed_gpu(p.ws.tile_status + m.ticket,
+                                       flag | static_cast<unsigned long long>(total));
+                    }
+                    sm.total[c] = total;
+                    sm.state[c] = kCounted;
                 }
-            }
-            // ---- compact: coalesced writes of the staged entries ----------
-            if (kCompact) {
-                const uint16_t *stage = old_s;
-                for (int i = tid; i < total; i += kThreads) {
-                    const long long pos = prefix + i;
-                    if (pos < p.capacity) {
-                        const int o = stage[i];
-                        st_stream_u32(p.indices + pos, static_cast<uint32_t>(m.local_start + o));
-                        st_stream_u16(p.values + pos, new_s[o]);
+                if (kCompact) {
+                    uint16_t *stage = old_s;
+                    uint32_t mm = mask;
+                    int rr = warp_off + incl - cnt;
+                    while (mm) {
+                        const int bit = __ffs(mm) - 1;
+                        mm &= mm - 1;
+                        stage[rr++] = static_cast<uint16_t>(32 * tid + bit);
                     }
                 }
+                next_count = (c + 1 == kStages) ? 0 : c + 1;
+                progress = true;
+                __syncthreads();  // staging, state and total visible
             }
-        } else if (!withheld) {
-            stop = true;  // the scan gave up: nothing after this tile is valid
         }
-        __syncthreads();  // (3) stage s fully consumed
 
-        if (stop) break;
-        if (tid == 0) issue_tile(p, sm, s, policy);
-        s = (s + 1 == kStages) ? 0 : s + 1;
+        // ---- (b) one look-back step for the oldest counted tile ------------
+        if (sm.state[fs] == kCounted) {
+            const StageMeta m = sm.meta[fs];
+            if (warp == 0) {
+                long long r;
+                if (m.ticket == p.withhold) {
+                    r = kGaveUp;
+                } else if (m.ticket == 0) {
+                    r = 0;
+                } else {
+                    if (!lb_active) {
+                        lb_start(lb, p, m.ticket);
+                        lb_active = true;
+                    }
+                    r = lb_step(lb, p);
+                }
+                if (lane == 0) {
+                    if (r >= 0 && m.ticket != 0) {
+                        st_relaxed_gpu(p.ws.tile_status + m.ticket,
+                                       kFlagPrefix |
+                                           static_cast<unsigned long long>(r + sm.total[fs]));
+                    }
+                    sm.step_result = r;
+                }
+                if (r != kNotReady) lb_active = false;
+            }
+            __syncthreads();
+            const long long prefix = sm.step_result;
+            if (prefix != kNotReady) {
+                const TileDesc &d = m.d;
+                const int total = sm.total[fs];
+                if (prefix >= 0) {
+                    if (tid == 0) {
+                        if (d.local_start == 0) p.offsets[d.tensor] = prefix;
+                        if (m.ticket == p.ws.num_tiles - 1) {
+                            const long long nnz = prefix + total;
+                            p.offsets[p.ws.num_tensors] = nnz;
+                            if (kCompact && nnz > p.capacity)
+                                record_error(p.ws.hdr, DWS_ERR_CAPACITY, nnz);
+                        }
+                    }
+                    if (kCompact) {
+                        const uint16_t *stage = sm.buf[fs][0];
+                        const uint16_t *new_s = sm.buf[fs][1];
+                        for (int i = tid; i < total; i += kThreads) {
+                            const long long pos = prefix + i;
+                            if (pos < p.capacity) {
+                                const int o = stage[i];
+                                st_stream_u32(p.indices + pos,
+                                              static_cast<uint32_t>(d.local_start + o));
+                                st_stream_u16(p.values + pos, new_s[o]);
+                            }
+                        }
+                    }
+                } else if (m.ticket != p.withhold) {
+                    stop = true;  // the scan gave up: nothing after this tile is valid
+                }
+                __syncthreads();  // stage fs fully consumed
+                if (stop) break;
+                if (tid == 0) refill(p, sm, fs);
+                next_finish = (fs + 1 == kStages) ? 0 : fs + 1;
+                progress = true;
+                __syncthreads();  // refilled state visible
+            }
+        }
+        if (!progress) __nanosleep(64);
     }
 
-    // Leaving early: wait for the loads still in flight into our buffers.
+    // Leaving early: wait for the loads still in flight into our stages.
     if (stop) {
-        for (int k = 1; k < kStages; ++k) {
-            const int t = (s + k) % kStages;
-            if (sm.meta[t].ticket < p.ws.num_tiles) {
-                const uint32_t parity = (phase_bits >> t) & 1u;
-                mbar_wait(&sm.bar[t], parity, kLoadWaitLimitNs);
+        for (int s = 0; s < kStages; ++s) {
+            if (sm.state[s] == kLoading) {
+                const uint32_t parity = (phase_bits >> s) & 1u;
+                mbar_wait(&sm.bar[s], parity, 4000000000ull);
             }
         }
     }
 }
 
-__global__ void ws_reset_kernel(WsView ws) {
+// Per call: clear the scan state and describe every tile (pointers into both
+// snapshots, count, bulk-copyable prefix), checking the pointer tables.
+__global__ void prepare_kernel(WsView ws, const uint16_t *const *old_ptrs,
+                               const uint16_t *const *new_ptrs) {
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
          i < ws.num_tiles; i += stride) {
         ws.tile_status[i] = 0ull;
+        TileDesc d;
+        d.old_p = nullptr;
+        d.new_p = nullptr;
+        d.tensor = 0;
+        d.local_start = 0;
+        d.count = 0;
+        d.bulk = 0;
+        const int t = ws.tile_tensor[i];
+        bool ok = (t >= 0 && t < ws.num_tensors);
+        if (ok) {
+            const long long n = ws.numel[t];
+            const long long ls = (i - ws.first_tile[t]) << kTileShift;
+            ok = (ls >= 0 && ls <= n);
+            if (ok) {
+                const long long rest = n - ls;
+                d.tensor = t;
+                d.local_start = static_cast<int>(ls);
+                d.count = static_cast<int>(rest < kTileElems ? rest : kTileElems);
+                if (d.count > 0) {
+                    const uint16_t *op = old_ptrs[t];
+                    const uint16_t *np = new_ptrs[t];
+                    const uintptr_t ua = reinterpret_cast<uintptr_t>(op);
+                    const uintptr_t ub = reinterpret_cast<uintptr_t>(np);
+                    if (op == nullptr || np == nullptr || ((ua | ub) & 1u)) {
+                        record_error(ws.hdr, DWS_ERR_INVALID, t);
+                        d.count = 0;
+                    } else {
+                        d.old_p = op + ls;
+                        d.new_p = np + ls;
+                        d.bulk = ((ua | ub) & 15u) == 0 ? (d.count & ~7) : 0;
+                    }
+                }
+            }
+        }
+        if (!ok) record_error(ws.hdr, DWS_ERR_WORKSPACE, i);
+        ws.tile_desc[i] = d;
     }
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         ws.hdr->ticket = 0ull;
@@ -392,17 +474,6 @@ cudaError_t encode_occupancy(int *ctas_per_sm) {
                                                          kThreads, sizeof(EncodeSmem));
 }
 
-cudaError_t launch_ws_reset(const WsView &ws, cudaStream_t s) {
-    DeviceInfo di;
-    cudaError_t e = device_info(&di);
-    if (e != cudaSuccess) return e;
-    long long blocks = (ws.num_tiles + 255) / 256;
-    if (blocks > 4LL * di.sm_count) blocks = 4LL * di.sm_count;
-    if (blocks < 1) blocks = 1;
-    ws_reset_kernel<<<static_cast<unsigned int>(blocks), 256, 0, s>>>(ws);
-    return launched();
-}
-
 cudaError_t launch_fill_tile_map(const WsView &ws, cudaStream_t s) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
@@ -421,13 +492,15 @@ cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
-    e = launch_ws_reset(ws, s);
+    long long pblocks = (ws.num_tiles + 255) / 256;
+    if (pblocks > 8LL * di.sm_count) pblocks = 8LL * di.sm_count;
+    if (pblocks < 1) pblocks = 1;
+    prepare_kernel<<<static_cast<unsigned int>(pblocks), 256, 0, s>>>(ws, old_ptrs, new_ptrs);
+    e = launched();
     if (e != cudaSuccess) return e;
 
     EncodeParams p;
     p.ws = ws;
-    p.old_ptrs = old_ptrs;
-    p.new_ptrs = new_ptrs;
     p.offsets = offsets;
     p.indices = indices;
     p.values = values;

@@ -120,7 +120,9 @@ def test_encode_capacity_overflow_reports_required_nnz(dws):
     offsets = torch.empty(len(olds) + 1, dtype=torch.int64, device="cuda")
     idx = torch.full((cap + 64,), -7, dtype=torch.int32, device="cuda")
     val = torch.full((cap + 64,), -7, dtype=torch.int16, device="cuda")
-    code = dws.dws_encode(plan.handle, dws.ptr_table(olds).data_ptr(), dws.ptr_table(news).data_ptr(),
+    # keep the pointer tables alive until the kernel has run
+    ot, nt = dws.ptr_table(olds), dws.ptr_table(news)
+    code = dws.dws_encode(plan.handle, ot.data_ptr(), nt.data_ptr(),
                           offsets.data_ptr(), idx.data_ptr(), val.data_ptr(), cap,
                           plan.workspace.data_ptr(), plan.workspace_bytes,
                           torch.cuda.current_stream().cuda_stream)
