@@ -10,21 +10,25 @@
 //   * A prepare pass (one thread per tile) clears the scan state and writes a
 //     32-byte descriptor per tile: pointers to the tile in both snapshots,
 //     tensor, local start, element count.
-//   * Persistent CTAs (256 threads, 2 per SM) take tiles of 8192 elements by
-//     atomic ticket, so a tile's predecessors are always resident or finished
-//     (forward progress of the scan below).  Each CTA owns kStages stages,
-//     each holding both snapshots' 16 KiB of a tile, filled by two 1-D bulk
-//     async copies (cp.async.bulk, global -> own shared memory, mbarrier
-//     transaction count, L2 evict-first).
-//   * The CTA runs an event loop that never blocks on the scan.  Each turn it
-//     (a) counts the oldest loaded stage if its data has arrived --
-//     detect, block scan, publish the tile's count, stage the changed offsets
-//     -- and (b) takes one non-blocking look-back step for the oldest counted
-//     tile; when that tile's prefix is known it writes the tile's entries,
-//     and the freed stage is refilled with a new ticket.  A tile's count thus
-//     depends only on its own data arriving, never on another tile's
-//     look-back: a ticket that is held while its CTA waits on a look-back
-//     makes every later tile wait on it in turn (convoys).
+//   * One persistent CTA per SM, warp-specialised.  Tiles of 8192 elements
+//     are taken by atomic ticket, so a tile's predecessors are always
+//     resident or finished (forward progress of the scan below).
+//   * Producer (one thread): takes tickets and reads tile descriptors two
+//     tiles ahead, and refills each of the kStages stages as soon as it is
+//     released: two 1-D bulk async copies (cp.async.bulk, global -> own
+//     shared memory, mbarrier transaction count, L2 evict-first) bring both
+//     snapshots' 16 KiB of the tile.
+//   * Counting group (8 warps): for each stage in ticket order: detect,
+//     block scan, publish the tile's count, move the changed (offset, value)
+//     pairs into a shared ring, queue the tile, release the stage.  A stage
+//     is busy only from its refill to its count, and a tile's count never
+//     waits on any look-back: a ticket held while its CTA waits on a
+//     look-back makes every later tile wait on it in turn (convoys), and a
+//     stage held through a look-back caps the data in flight.
+//   * Look-back group (7 warps): each takes queued tiles in turn, resolves
+//     the tile's exclusive prefix, publishes it, writes the tile's entries
+//     from the ring with consecutive lanes storing consecutive entries
+//     (coalesced), and releases its ring space.
 //   * detect: 16-byte shared-memory reads in a bank-conflict-free order, a
 //     32-bit change mask per thread, popc; block scan of the counts.
 //   * scan: decoupled look-back over the tile status words (flag + 62-bit
@@ -33,9 +37,6 @@
 //     whole windows from every waiting warp floods the L2 with requests to
 //     the hottest lines).  Bounded by a wall-clock limit after which the
 //     kernel records DWS_ERR_TIMEOUT and every CTA leaves.
-//   * compact: the tile's changed offsets are staged in shared memory (over
-//     the old snapshot's slot, no longer needed), then written out with
-//     consecutive threads storing consecutive entries (coalesced).
 #include <cuda_runtime.h>
 
 #include "dws_internal.cuh"
@@ -43,24 +44,33 @@
 namespace dws {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-constexpr int kStages = 3;
+constexpr int kCountWarps = 8;
+constexpr int kCountThreads = 32 * kCountWarps;  // the counting group
+constexpr int kLookWarps = 7;                     // the look-back group
+constexpr int kProducerWarp = kCountWarps + kLookWarps;
+constexpr int kPublishThread = 64;  // publishes tile counts (thread 0 keeps the queue)
+constexpr int kThreads = 32 * (kProducerWarp + 1);
+constexpr int kStages = 4;
+constexpr int kRing = 16384;  // pending (offset | value << 16) entries
+constexpr int kQueue = 64;    // pending tiles
+constexpr int kCountBar = 1;  // named barrier of the counting group
 constexpr int kChunks = kTileElems / 8;  // 16-byte chunks of bf16 per tile
-static_assert(kChunks == 4 * kThreads, "each thread owns 4 chunks (32 elements)");
+static_assert(kChunks == 4 * kCountThreads, "each counting thread owns 4 chunks (32 elements)");
+static_assert((kRing & (kRing - 1)) == 0 && kRing >= kTileElems, "ring holds any tile");
 
-// Stage states.
-constexpr int kEmptyDone = 0;  // no more tickets for this stage
-constexpr int kLoading = 1;    // ticket taken, bulk copies in flight
-constexpr int kCounted = 2;    // count published, waiting for its prefix
-
-// Look-back step results.
-constexpr long long kNotReady = -2;
-constexpr long long kGaveUp = -1;
+constexpr unsigned long long kLoadWaitLimitNs = 4000000000ull;  // 4 s
 
 struct StageMeta {
-    long long ticket;
+    long long ticket;  // >= num_tiles: no more work for this stage
     TileDesc d;
+};
+
+struct Pending {
+    long long ticket;
+    int tensor;
+    int local_start;
+    int pos;    // first ring entry
+    int total;  // changed elements (ring entries when compacting)
 };
 
 struct EncodeParams {
@@ -74,318 +84,457 @@ struct EncodeParams {
 };
 
 struct EncodeSmem {
-    uint16_t buf[kStages][2][kTileElems];  // [stage][0 = old | staging, 1 = new]
-    unsigned long long bar[kStages];
+    uint16_t buf[kStages][2][kTileElems];  // [stage][old | new]
+    uint32_t ring[kRing];
+    unsigned long long bar[kStages];        // stage filled (transaction count)
+    unsigned long long empty_bar[kStages];  // stage released by the counting group
+    int fills[kStages];                     // fills issued per stage
+    int producer_done;
     StageMeta meta[kStages];
-    int state[kStages];
-    int total[kStages];
-    int warp_sum[kWarps];
-    long long step_result;
+    Pending q[kQueue];
+    int q_done[kQueue];  // i + 1 once queue entry i is written out
+    int q_tail;          // entries queued (release)
+    int q_final;         // total entries once counting has finished, else -1
+    int stop;            // a look-back gave up: everyone leaves
+    int alloc_pos;       // ring position of the tile being queued, -1 = leave
+    int warp_sum[kCountWarps];
 };
 
-// Thread 0: take the next ticket, read its descriptor, start loading it into
-// stage s (or mark the stage done).
-__device__ void refill(const EncodeParams &p, EncodeSmem &sm, int s) {
+// Thread 0, in two steps: take a ticket (early, so its latency hides behind
+// a tile's work), then read its descriptor and start the stage's loads.
+__device__ __forceinline__ long long take_ticket(const EncodeParams &p) {
+    return static_cast<long long>(atomicAdd(&p.ws.hdr->ticket, 1ull));
+}
+
+__device__ __forceinline__ TileDesc load_desc(const EncodeParams &p, long long ticket) {
+    TileDesc d;
+    if (ticket < p.ws.num_tiles) {
+        d = p.ws.tile_desc[ticket];
+    } else {
+        d.old_p = nullptr;
+        d.new_p = nullptr;
+        d.tensor = 0;
+        d.local_start = 0;
+        d.count = 0;
+        d.bulk = 0;
+    }
+    return d;
+}
+
+__device__ void issue_stage(const EncodeParams &p, EncodeSmem &sm, int s, long long ticket,
+                            const TileDesc &desc) {
     StageMeta m;
-    m.ticket = static_cast<long long>(atomicAdd(&p.ws.hdr->ticket, 1ull));
-    if (m.ticket < p.ws.num_tiles) {
-        m.d = p.ws.tile_desc[m.ticket];
+    m.ticket = ticket;
+    m.d = desc;
+    sm.meta[s] = m;
+    sm.fills[s] += 1;
+    if (ticket < p.ws.num_tiles) {
         const uint32_t bulk = static_cast<uint32_t>(m.d.bulk);
-        mbar_arrive_expect_tx(&sm.bar[s], bulk * 4u);
+        mbar_arrive_expect_tx(&sm.bar[s], bulk * 4u);  // release: meta is visible
         if (bulk > 0) {
             const unsigned long long policy = l2_evict_first_policy();
             bulk_load(sm.buf[s][0], m.d.old_p, bulk * 2u, &sm.bar[s], policy);
             bulk_load(sm.buf[s][1], m.d.new_p, bulk * 2u, &sm.bar[s], policy);
         }
-        sm.state[s] = kLoading;
     } else {
-        sm.state[s] = kEmptyDone;
+        mbar_arrive(&sm.bar[s]);  // no more work: wake the counting group
     }
-    sm.meta[s] = m;
 }
 
-// Resumable decoupled look-back, run by warp 0 (state in its registers).
-// Lane l holds predecessors base - 8l - q (q = 0..7, newest first).
+// Decoupled look-back, run by one warp.  Lane l reads predecessors
+// base - 8l - q (q = 0..7, newest first), 256 per round trip.  While some
+// needed predecessor is unpublished, only those words are read again (with
+// backoff): an aggregate stays valid even after it turns into a prefix, and
+// re-reading whole windows from every waiting warp floods the L2 with
+// requests to the hottest lines.  Returns -1 if the bounded wait ran out or
+// another tile gave up.
 constexpr int kProbePerLane = 8;
 constexpr int kWindow = 32 * kProbePerLane;
 
-struct LookBack {
-    long long ticket;
-    long long base;
-    unsigned long long acc;
-    unsigned long long t0;
-    unsigned long long w[kProbePerLane];
-};
-
-__device__ __forceinline__ void lb_load_window(LookBack &lb, const unsigned long long *status) {
+__device__ long long look_back(const EncodeParams &p, const EncodeSmem &sm, long long ticket) {
     const int lane = threadIdx.x & 31;
+    const unsigned long long *status = p.ws.tile_status;
+    long long base = ticket - 1;
+    unsigned long long acc = 0;
+    unsigned long long t0 = 0;
+    unsigned int backoff = 32;
+    while (true) {
+        unsigned long long w[kProbePerLane];
 #pragma unroll
-    for (int q = 0; q < kProbePerLane; ++q) {
-        const long long j = lb.base - kProbePerLane * lane - q;
-        lb.w[q] = (j >= 0) ? ld_relaxed_gpu(status + j) : kFlagPrefix;
-    }
-}
-
-__device__ __forceinline__ void lb_start(LookBack &lb, const EncodeParams &p, long long ticket) {
-    lb.ticket = ticket;
-    lb.base = ticket - 1;
-    lb.acc = 0;
-    lb.t0 = 0;
-    lb_load_window(lb, p.ws.tile_status);
-}
-
-// One step: evaluate the window loaded by the previous step.  Returns the
-// exclusive prefix, kNotReady (loads for the next step issued), or kGaveUp.
-__device__ long long lb_step(LookBack &lb, const EncodeParams &p) {
-    const int lane = threadIdx.x & 31;
-    int first_p = kProbePerLane;
-    bool unready = false;
-    unsigned long long sum = 0;
-#pragma unroll
-    for (int q = 0; q < kProbePerLane; ++q) {
-        if (first_p == kProbePerLane) {
-            const unsigned int flag = static_cast<unsigned int>(lb.w[q] >> kFlagShift);
-            if (flag == 0u) {
-                unready = true;
-            } else {
-                sum += lb.w[q] & kValueMask;
-                if (flag == 2u) first_p = q;
-            }
+        for (int q = 0; q < kProbePerLane; ++q) {
+            const long long j = base - kProbePerLane * lane - q;
+            w[q] = (j >= 0) ? ld_relaxed_gpu(status + j) : kFlagPrefix;
         }
-    }
-    const unsigned int pmask = __ballot_sync(0xffffffffu, first_p < kProbePerLane);
-    const int p_lane = pmask ? (__ffs(pmask) - 1) : 32;
-    const bool blocks = (lane <= p_lane) && unready;
-    if (__any_sync(0xffffffffu, blocks)) {
-        int give_up = 0;
-        if (lane == 0) {
-            const unsigned long long now = global_timer_ns();
-            if (lb.t0 == 0) lb.t0 = now;
-            if (now - lb.t0 > static_cast<unsigned long long>(p.wait_limit_ns)) {
-                atomicExch(&p.ws.hdr->abort, 1u);
-                record_error(p.ws.hdr, DWS_ERR_TIMEOUT, lb.ticket);
-                give_up = 1;
-            } else if (ld_relaxed_gpu_u32(&p.ws.hdr->abort) != 0u) {
-                give_up = 1;
-            }
-        }
-        if (__shfl_sync(0xffffffffu, give_up, 0)) return kGaveUp;
-        // Re-read only the unpublished words that are needed.
-        if (blocks) {
+        int p_lane;
+        unsigned long long sum;
+        while (true) {
+            int first_p = kProbePerLane;
+            bool unready = false;
+            sum = 0;
 #pragma unroll
             for (int q = 0; q < kProbePerLane; ++q) {
-                if ((lb.w[q] >> kFlagShift) == 0ull) {
-                    const long long j = lb.base - kProbePerLane * lane - q;
-                    lb.w[q] = ld_relaxed_gpu(p.ws.tile_status + j);
+                if (first_p == kProbePerLane) {
+                    const unsigned int flag = static_cast<unsigned int>(w[q] >> kFlagShift);
+                    if (flag == 0u) {
+                        unready = true;
+                    } else {
+                        sum += w[q] & kValueMask;
+                        if (flag == 2u) first_p = q;
+                    }
+                }
+            }
+            const unsigned int pmask = __ballot_sync(0xffffffffu, first_p < kProbePerLane);
+            p_lane = pmask ? (__ffs(pmask) - 1) : 32;
+            const bool blocks = (lane <= p_lane) && unready;
+            if (!__any_sync(0xffffffffu, blocks)) break;
+
+            int give_up = 0;
+            if (lane == 0) {
+                const unsigned long long now = global_timer_ns();
+                if (t0 == 0) t0 = now;
+                if (now - t0 > static_cast<unsigned long long>(p.wait_limit_ns)) {
+                    atomicExch(&p.ws.hdr->abort, 1u);
+                    record_error(p.ws.hdr, DWS_ERR_TIMEOUT, ticket);
+                    give_up = 1;
+                } else if (ld_relaxed_gpu_u32(&p.ws.hdr->abort) != 0u ||
+                           *reinterpret_cast<const volatile int *>(&sm.stop) != 0) {
+                    give_up = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, give_up, 0)) return -1;
+            __nanosleep(backoff);
+            if (backoff < 256) backoff <<= 1;
+            if (blocks) {
+#pragma unroll
+                for (int q = 0; q < kProbePerLane; ++q) {
+                    if ((w[q] >> kFlagShift) == 0ull) {
+                        const long long j = base - kProbePerLane * lane - q;
+                        w[q] = ld_relaxed_gpu(status + j);
+                    }
                 }
             }
         }
-        return kNotReady;
-    }
-    unsigned long long v = (lane <= p_lane) ? sum : 0ull;
+        unsigned long long v = (lane <= p_lane) ? sum : 0ull;
 #pragma unroll
-    for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
-    lb.acc += v;
-    if (p_lane < 32) return static_cast<long long>(lb.acc);
-    lb.base -= kWindow;
-    lb_load_window(lb, p.ws.tile_status);
-    return kNotReady;
+        for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+        acc += v;
+        if (p_lane < 32) return static_cast<long long>(acc);
+        base -= kWindow;
+    }
 }
 
+// ---------------------------------------------------------------------------
+// Counting group: threads 0 .. kCountThreads-1
+// ---------------------------------------------------------------------------
+// ---------------------------------------------------------------------------
+// Producer: lane 0 of warp kProducerWarp
+// ---------------------------------------------------------------------------
+__device__ void produce(const EncodeParams &p, EncodeSmem &sm) {
+    // Lookahead: right after fill k is issued, the ticket of fill k+4 is taken
+    // and the descriptor of fill k+2 read (its ticket taken two fills
+    // earlier), so neither latency is waited on.
+    long long tk0 = take_ticket(p);
+    long long tk1 = take_ticket(p);
+    long long tk2 = take_ticket(p);
+    long long tk3 = take_ticket(p);
+    TileDesc dk0 = load_desc(p, tk0);
+    TileDesc dk1 = load_desc(p, tk1);
+    for (long long k = 0;; ++k) {
+        const int s = static_cast<int>(k % kStages);
+        if (k >= kStages) {
+            const uint32_t parity = static_cast<uint32_t>((k / kStages - 1) & 1);
+            unsigned int backoff = 32;
+            while (!mbar_try_wait(&sm.empty_bar[s], parity)) {
+                if (*reinterpret_cast<volatile int *>(&sm.stop) != 0 ||
+                    ld_relaxed_gpu_u32(&p.ws.hdr->abort) != 0u) {
+                    st_release_cta(&sm.producer_done, 1);
+                    return;
+                }
+                __nanosleep(backoff);
+                if (backoff < 256) backoff <<= 1;
+            }
+        }
+        if (*reinterpret_cast<volatile int *>(&sm.stop) != 0) break;
+        // Issue first: the arrive has release semantics and would otherwise
+        // wait for the lookahead loads below to come back.
+        issue_stage(p, sm, s, tk0, dk0);
+        if (tk0 >= p.ws.num_tiles) break;
+        tk0 = tk1;
+        tk1 = tk2;
+        tk2 = tk3;
+        dk0 = dk1;
+        dk1 = load_desc(p, tk1);
+        tk3 = take_ticket(p);
+    }
+    st_release_cta(&sm.producer_done, 1);
+}
+
+// ---------------------------------------------------------------------------
+// Counting group: threads 0 .. kCountThreads-1
+// ---------------------------------------------------------------------------
 template <bool kCompact>
-__global__ void __launch_bounds__(kThreads, 2) encode_kernel(EncodeParams p) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    EncodeSmem &sm = *reinterpret_cast<EncodeSmem *>(smem_raw);
+__device__ void count_group(const EncodeParams &p, EncodeSmem &sm) {
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
 
+    // Thread 0's bookkeeping of the queue and the ring.
+    int q_tail = 0, q_head = 0;
+    int ring_tail = 0, ring_head = 0;
+
+    long long waits = 0;  // stage fills consumed so far
+    bool failed = false;
+    for (;; ++waits) {
+        const int s = static_cast<int>(waits % kStages);
+        const uint32_t parity = static_cast<uint32_t>((waits / kStages) & 1);
+        const bool loaded = mbar_wait(&sm.bar[s], parity, kLoadWaitLimitNs);
+        const StageMeta m = sm.meta[s];      // written before the fill's arrive
+        const bool done = m.ticket >= p.ws.num_tiles;
+        const bool work = loaded && !done;
+        const TileDesc &d = m.d;
+        if (tid == 0 && work) {
+            // Room for a whole tile in the ring and one queue slot, so the
+            // writes below need no further check (freed in order by the
+            // look-back group).
+            unsigned int backoff = 32;
+            bool ok = true;
+            for (;;) {
+                // Plain volatile polling: an acquire would also wait for this
+                // thread's outstanding global accesses.  The ring is only
+                // rewritten after the flag is seen, and a look-back warp sets
+                // its flag after all its ring reads have returned.
+                while (q_head < q_tail &&
+                       *reinterpret_cast<volatile int *>(&sm.q_done[q_head % kQueue]) == q_head + 1) {
+                    ring_head += kCompact ? sm.q[q_head % kQueue].total : 0;
+                    ++q_head;
+                }
+                if (q_tail - q_head < kQueue && ring_tail + kTileElems - ring_head <= kRing) break;
+                if (*reinterpret_cast<volatile int *>(&sm.stop) != 0 ||
+                    ld_relaxed_gpu_u32(&p.ws.hdr->abort) != 0u) {
+                    ok = false;
+                    break;
+                }
+                __nanosleep(backoff);
+                if (backoff < 1024) backoff <<= 1;
+            }
+            sm.alloc_pos = ok ? ring_tail : -1;
+        }
+
+        uint16_t *old_s = sm.buf[s][0];
+        uint16_t *new_s = sm.buf[s][1];
+        uint32_t mask = 0;
+        if (work) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int slot = ((tid >> 1) + j) & 3;  // conflict-free 16-byte reads
+                const int e0 = (4 * tid + slot) * 8;
+                uint4 a, b;
+                if (e0 + 8 <= d.bulk) {
+                    a = *reinterpret_cast<const uint4 *>(old_s + e0);
+                    b = *reinterpret_cast<const uint4 *>(new_s + e0);
+                } else {
+                    uint16_t av[8], bv[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int e = e0 + q;
+                        av[q] = (e < d.count) ? d.old_p[e] : uint16_t(0);
+                        bv[q] = (e < d.count) ? d.new_p[e] : uint16_t(0);
+                        if (kCompact && e < d.count) new_s[e] = bv[q];
+                    }
+                    a.x = av[0] | (uint32_t(av[1]) << 16);
+                    a.y = av[2] | (uint32_t(av[3]) << 16);
+                    a.z = av[4] | (uint32_t(av[5]) << 16);
+                    a.w = av[6] | (uint32_t(av[7]) << 16);
+                    b.x = bv[0] | (uint32_t(bv[1]) << 16);
+                    b.y = bv[2] | (uint32_t(bv[3]) << 16);
+                    b.z = bv[4] | (uint32_t(bv[5]) << 16);
+                    b.w = bv[6] | (uint32_t(bv[7]) << 16);
+                }
+                const uint32_t x0 = a.x ^ b.x, x1 = a.y ^ b.y, x2 = a.z ^ b.z, x3 = a.w ^ b.w;
+                const uint32_t bits8 = ((x0 & 0xffffu) != 0) | (((x0 >> 16) != 0) << 1) |
+                                       (((x1 & 0xffffu) != 0) << 2) | (((x1 >> 16) != 0) << 3) |
+                                       (((x2 & 0xffffu) != 0) << 4) | (((x2 >> 16) != 0) << 5) |
+                                       (((x3 & 0xffffu) != 0) << 6) | (((x3 >> 16) != 0) << 7);
+                mask |= bits8 << (8 * slot);
+            }
+        }
+        const int cnt = __popc(mask);
+        int incl = cnt;
+#pragma unroll
+        for (int dd = 1; dd < 32; dd <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, dd);
+            if (lane >= dd) incl += v;
+        }
+        if (lane == 31) sm.warp_sum[warp] = incl;
+        // (A) warp sums and ring position visible.  If a load wait ran out
+        // anywhere, or a look-back gave up, the group leaves together; a fill
+        // whose wait ran out is still pending and is drained below.
+        const bool go = loaded && (*reinterpret_cast<volatile int *>(&sm.stop) == 0);
+        if (!named_bar_and(kCountBar, kCountThreads, go)) {
+            if (!loaded) record_error(p.ws.hdr, DWS_ERR_TIMEOUT, waits);
+            if (loaded) ++waits;
+            failed = true;
+            break;
+        }
+        if (done) {  // every thread saw the same loaded meta
+            ++waits;
+            break;
+        }
+        const int pos = sm.alloc_pos;
+        if (pos < 0) {
+            ++waits;
+            failed = true;
+            break;
+        }
+        int warp_off = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < kCountWarps; ++w) {
+            const int v = sm.warp_sum[w];
+            warp_off += (w < warp) ? v : 0;
+            total += v;
+        }
+        // The count is published by a thread that does no shared-memory
+        // release afterwards (a release would wait for this global store).
+        if (tid == kPublishThread && m.ticket != p.withhold) {
+            const unsigned long long flag = (m.ticket == 0) ? kFlagPrefix : kFlagAggregate;
+            st_relaxed_gpu(p.ws.tile_status + m.ticket, flag | static_cast<unsigned long long>(total));
+        }
+        if (kCompact) {
+            uint32_t mm = mask;
+            int rr = pos + warp_off + incl - cnt;
+            while (mm) {
+                const int bit = __ffs(mm) - 1;
+                mm &= mm - 1;
+                const int o = 32 * tid + bit;
+                sm.ring[rr & (kRing - 1)] = static_cast<uint32_t>(o) | (static_cast<uint32_t>(new_s[o]) << 16);
+                ++rr;
+            }
+        }
+        named_bar(kCountBar, kCountThreads);  // (C) entries in the ring, stage s consumed
+        if (tid == 0) {
+            Pending &e = sm.q[q_tail % kQueue];
+            e.ticket = m.ticket;
+            e.tensor = d.tensor;
+            e.local_start = d.local_start;
+            e.pos = pos;
+            e.total = total;
+            ring_tail += kCompact ? total : 0;
+            ++q_tail;
+            st_release_cta(&sm.q_tail, q_tail);
+            mbar_arrive(&sm.empty_bar[s]);  // the producer may refill stage s
+        }
+    }
+
+    // Counting is over: the look-back group stops after the last entry.
+    if (tid == 0) st_release_cta(&sm.q_final, q_tail);
+    if (failed) {
+        // Leaving on an error: stop the producer, then wait for every fill it
+        // issued that has not been consumed.  (A ticket taken but never
+        // loaded only happens here, after the global abort flag was set.)
+        if (tid == 0) *reinterpret_cast<volatile int *>(&sm.stop) = 1;
+        unsigned long long t0 = global_timer_ns();
+        while (ld_acquire_cta(&sm.producer_done) == 0 && global_timer_ns() - t0 < kLoadWaitLimitNs) {
+            __nanosleep(256);
+        }
+        named_bar(kCountBar, kCountThreads);
+        for (int k = 0; k < kStages; ++k) {
+            // fills of stage k consumed so far (waits counted above)
+            const long long consumed = (waits + kStages - 1 - k) / kStages;
+            if (sm.fills[k] > consumed) {
+                mbar_wait(&sm.bar[k], static_cast<uint32_t>(consumed & 1), kLoadWaitLimitNs);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Look-back group: warps kCountWarps .. kCountWarps + kLookWarps - 1
+// ---------------------------------------------------------------------------
+template <bool kCompact>
+__device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
+    const int lane = threadIdx.x & 31;
+    const int j = (threadIdx.x >> 5) - kCountWarps;
+    for (int i = j;; i += kLookWarps) {
+        // Wait for queue entry i, or for the end.
+        unsigned int backoff = 32;
+        for (;;) {
+            if (ld_acquire_cta(&sm.q_tail) > i) break;
+            const int fin = ld_acquire_cta(&sm.q_final);
+            if ((fin >= 0 && i >= fin) || *reinterpret_cast<volatile int *>(&sm.stop) != 0) return;
+            __nanosleep(backoff);
+            if (backoff < 512) backoff <<= 1;
+        }
+        const Pending e = sm.q[i % kQueue];
+        long long prefix;
+        if (e.ticket == p.withhold) {
+            prefix = -1;
+        } else if (e.ticket == 0) {
+            prefix = 0;
+        } else {
+            prefix = look_back(p, sm, e.ticket);
+        }
+        if (prefix >= 0) {
+            if (lane == 0) {
+                if (e.ticket != 0)
+                    st_relaxed_gpu(p.ws.tile_status + e.ticket,
+                                   kFlagPrefix | static_cast<unsigned long long>(prefix + e.total));
+                if (e.local_start == 0) p.offsets[e.tensor] = prefix;
+                if (e.ticket == p.ws.num_tiles - 1) {
+                    const long long nnz = prefix + e.total;
+                    p.offsets[p.ws.num_tensors] = nnz;
+                    if (kCompact && nnz > p.capacity) record_error(p.ws.hdr, DWS_ERR_CAPACITY, nnz);
+                }
+            }
+            if (kCompact) {
+                for (int k = lane; k < e.total; k += 32) {
+                    const long long out = prefix + k;
+                    if (out < p.capacity) {
+                        const uint32_t v = sm.ring[(e.pos + k) & (kRing - 1)];
+                        st_stream_u32(p.indices + out, static_cast<uint32_t>(e.local_start) + (v & 0xffffu));
+                        st_stream_u16(p.values + out, static_cast<uint16_t>(v >> 16));
+                    }
+                }
+            }
+        } else if (e.ticket != p.withhold) {
+            if (lane == 0) *reinterpret_cast<volatile int *>(&sm.stop) = 1;
+        }
+        // Every lane's ring reads have returned (their values were stored), so
+        // a plain store lets the counting group reuse the ring space.
+        __syncwarp();
+        if (lane == 0) *reinterpret_cast<volatile int *>(&sm.q_done[i % kQueue]) = i + 1;
+    }
+}
+
+template <bool kCompact>
+__global__ void __launch_bounds__(kThreads, 1) encode_kernel(EncodeParams p) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    EncodeSmem &sm = *reinterpret_cast<EncodeSmem *>(smem_raw);
+    const int tid = threadIdx.x;
+
     if (!ws_matches(p.ws)) return;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[s], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.bar[s], 1);
+            mbar_init(&sm.empty_bar[s], 1);
+            sm.fills[s] = 0;
+        }
         mbar_fence_init();
-        for (int s = 0; s < kStages; ++s) refill(p, sm, s);
+        sm.q_tail = 0;
+        sm.q_final = -1;
+        sm.stop = 0;
+        sm.producer_done = 0;
+        for (int k = 0; k < kQueue; ++k) sm.q_done[k] = 0;
     }
     __syncthreads();
 
-    uint32_t phase_bits = 0;
-    int next_count = 0;   // oldest stage still to be counted (ring order)
-    int next_finish = 0;  // oldest counted stage waiting for its prefix
-    bool lb_active = false;
-    LookBack lb;
-    bool stop = false;
-
-    for (;;) {
-        const int fs = next_finish;
-        const int f_state = sm.state[fs];
-        if (f_state == kEmptyDone) break;  // every stage after it is done too
-        bool progress = false;
-
-        // ---- (a) count the oldest loaded stage once its data is there ------
-        const int c = next_count;
-        if (sm.state[c] == kLoading) {
-            const uint32_t parity = (phase_bits >> c) & 1u;
-            const bool ready = __syncthreads_and(mbar_try_wait(&sm.bar[c], parity));
-            if (ready) {
-                phase_bits ^= (1u << c);
-                const StageMeta m = sm.meta[c];
-                const TileDesc &d = m.d;
-                uint16_t *old_s = sm.buf[c][0];
-                uint16_t *new_s = sm.buf[c][1];
-                uint32_t mask = 0;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int slot = ((tid >> 1) + j) & 3;  // conflict-free 16-byte reads
-                    const int e0 = (4 * tid + slot) * 8;
-                    uint4 a, b;
-                    if (e0 + 8 <= d.bulk) {
-                        a = *reinterpret_cast<const uint4 *>(old_s + e0);
-                        b = *reinterpret_cast<const uint4 *>(new_s + e0);
-                    } else {
-                        uint16_t av[8], bv[8];
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const int e = e0 + q;
-                            av[q] = (e < d.count) ? d.old_p[e] : uint16_t(0);
-                            bv[q] = (e < d.count) ? d.new_p[e] : uint16_t(0);
-                            if (kCompact && e < d.count) new_s[e] = bv[q];
-                        }
-                        a.x = av[0] | (uint32_t(av[1]) << 16);
-                        a.y = av[2] | (uint32_t(av[3]) << 16);
-                        a.z = av[4] | (uint32_t(av[5]) << 16);
-                        a.w = av[6] | (uint32_t(av[7]) << 16);
-                        b.x = bv[0] | (uint32_t(bv[1]) << 16);
-                        b.y = bv[2] | (uint32_t(bv[3]) << 16);
-                        b.z = bv[4] | (uint32_t(bv[5]) << 16);
-                        b.w = bv[6] | (uint32_t(bv[7]) << 16);
-                    }
-                    const uint32_t x0 = a.x ^ b.x, x1 = a.y ^ b.y, x2 = a.z ^ b.z, x3 = a.w ^ b.w;
-                    const uint32_t bits8 =
-                        ((x0 & 0xffffu) != 0) | (((x0 >> 16) != 0) << 1) |
-                        (((x1 & 0xffffu) != 0) << 2) | (((x1 >> 16) != 0) << 3) |
-                        (((x2 & 0xffffu) != 0) << 4) | (((x2 >> 16) != 0) << 5) |
-                        (((x3 & 0xffffu) != 0) << 6) | (((x3 >> 16) != 0) << 7);
-                    mask |= bits8 << (8 * slot);
-                }
-                const int cnt = __popc(mask);
-                int incl = cnt;
-#pragma unroll
-                for (int dd = 1; dd < 32; dd <<= 1) {
-                    const int v = __shfl_up_sync(0xffffffffu, incl, dd);
-                    if (lane >= dd) incl += v;
-                }
-                if (lane == 31) sm.warp_sum[warp] = incl;
-                __syncthreads();  // warp sums visible; old_s no longer read
-                int warp_off = 0, total = 0;
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) {
-                    const int v = sm.warp_sum[w];
-                    warp_off += (w < warp) ? v : 0;
-                    total += v;
-                }
-                if (tid == 0) {
-                    if (m.ticket != p.withhold) {
-                        const unsigned long long flag =
-                            (m.ticket == 0) ? kFlagPrefix : kFlagAggregate;
-                        st_relaxed_gpu(p.ws.tile_status + m.ticket,
-                                       flag | static_cast<unsigned long long>(total));
-                    }
-                    sm.total[c] = total;
-                    sm.state[c] = kCounted;
-                }
-                if (kCompact) {
-                    uint16_t *stage = old_s;
-                    uint32_t mm = mask;
-                    int rr = warp_off + incl - cnt;
-                    while (mm) {
-                        const int bit = __ffs(mm) - 1;
-                        mm &= mm - 1;
-                        stage[rr++] = static_cast<uint16_t>(32 * tid + bit);
-                    }
-                }
-                next_count = (c + 1 == kStages) ? 0 : c + 1;
-                progress = true;
-                __syncthreads();  // staging, state and total visible
-            }
-        }
-
-        // ---- (b) one look-back step for the oldest counted tile ------------
-        if (sm.state[fs] == kCounted) {
-            const StageMeta m = sm.meta[fs];
-            if (warp == 0) {
-                long long r;
-                if (m.ticket == p.withhold) {
-                    r = kGaveUp;
-                } else if (m.ticket == 0) {
-                    r = 0;
-                } else {
-                    if (!lb_active) {
-                        lb_start(lb, p, m.ticket);
-                        lb_active = true;
-                    }
-                    r = lb_step(lb, p);
-                }
-                if (lane == 0) {
-                    if (r >= 0 && m.ticket != 0) {
-                        st_relaxed_gpu(p.ws.tile_status + m.ticket,
-                                       kFlagPrefix |
-                                           static_cast<unsigned long long>(r + sm.total[fs]));
-                    }
-                    sm.step_result = r;
-                }
-                if (r != kNotReady) lb_active = false;
-            }
-            __syncthreads();
-            const long long prefix = sm.step_result;
-            if (prefix != kNotReady) {
-                const TileDesc &d = m.d;
-                const int total = sm.total[fs];
-                if (prefix >= 0) {
-                    if (tid == 0) {
-                        if (d.local_start == 0) p.offsets[d.tensor] = prefix;
-                        if (m.ticket == p.ws.num_tiles - 1) {
-                            const long long nnz = prefix + total;
-                            p.offsets[p.ws.num_tensors] = nnz;
-                            if (kCompact && nnz > p.capacity)
-                                record_error(p.ws.hdr, DWS_ERR_CAPACITY, nnz);
-                        }
-                    }
-                    if (kCompact) {
-                        const uint16_t *stage = sm.buf[fs][0];
-                        const uint16_t *new_s = sm.buf[fs][1];
-                        for (int i = tid; i < total; i += kThreads) {
-                            const long long pos = prefix + i;
-                            if (pos < p.capacity) {
-                                const int o = stage[i];
-                                st_stream_u32(p.indices + pos,
-                                              static_cast<uint32_t>(d.local_start + o));
-                                st_stream_u16(p.values + pos, new_s[o]);
-                            }
-                        }
-                    }
-                } else if (m.ticket != p.withhold) {
-                    stop = true;  // the scan gave up: nothing after this tile is valid
-                }
-                __syncthreads();  // stage fs fully consumed
-                if (stop) break;
-                if (tid == 0) refill(p, sm, fs);
-                next_finish = (fs + 1 == kStages) ? 0 : fs + 1;
-                progress = true;
-                __syncthreads();  // refilled state visible
-            }
-        }
-        if (!progress) __nanosleep(64);
-    }
-
-    // Leaving early: wait for the loads still in flight into our stages.
-    if (stop) {
-        for (int s = 0; s < kStages; ++s) {
-            if (sm.state[s] == kLoading) {
-                const uint32_t parity = (phase_bits >> s) & 1u;
-                mbar_wait(&sm.bar[s], parity, 4000000000ull);
-            }
-        }
+    const int warp = tid >> 5;
+    if (warp < kCountWarps) {
+        count_group<kCompact>(p, sm);
+    } else if (warp < kProducerWarp) {
+        look_group<kCompact>(p, sm);
+    } else if ((tid & 31) == 0) {
+        produce(p, sm);
     }
 }
 
