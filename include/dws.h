@@ -165,6 +165,32 @@ DWS_API dws_status_t dws_count(const dws_plan_t *plan,
                        int64_t *offsets,
                        void *workspace, size_t workspace_bytes, dws_stream_t stream);
 
+/* Allocation-free variant of dws_encode, for callers that cannot allocate
+ * device memory: code running inside another framework's memory pool, where
+ * every device allocation must go through an allocator the caller does not
+ * control (or is not allowed at all), and latency-critical paths that cannot
+ * afford a cudaMalloc and the device-wide synchronisation it implies.  The
+ * source pages have no counterpart to this entry point; it computes exactly
+ * what dws_encode computes.
+ * The scan's scratch lives in a fixed 3 MiB array in device memory that every
+ * GPU loading libdws holds until the process exits; nothing is allocated.
+ * numels: host array [num_tensors] of bf16 element counts (0 <= n < 2^31).
+ * old_ptrs, new_ptrs, offsets, indices, values, capacity: as in dws_encode.
+ * status_out: device array [2] (nullable) that receives the call's device
+ *   status (a dws_status_t) and its detail, as dws_status() would report them.
+ * Limits: at most 256 tensors and 65,536 tiles of 8192 elements
+ *   (536,870,912 elements); larger requests return DWS_ERR_WORKSPACE and
+ *   enqueue nothing.
+ * Every call shares the one array of its device and leaves its contents
+ *   behind; each call re-initialises what it reads.  Calls that overlap on the
+ *   same GPU race: order them on one stream or with events.
+ * The first call on a device looks up the array's address there; make it
+ *   before capturing any stream on that device. */
+DWS_API dws_status_t dws_encode_noalloc(const int64_t *numels, int32_t num_tensors,
+                                        const void *const *old_ptrs, const void *const *new_ptrs,
+                                        int64_t *offsets, int32_t *indices, uint16_t *values,
+                                        int64_t capacity, int64_t *status_out, dws_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Apply: [TRL] §4.3 receive_weights -- for each changed parameter,
  * snap.flatten()[indices] = values, in place on the receiver's snapshot

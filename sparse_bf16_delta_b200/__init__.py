@@ -63,6 +63,7 @@ _sig("dws_plan_upload", _i32, [_vp, _vp, _sz, _vp])
 _sig("dws_encode", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_encode_ex", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _i64, _i64])
 _sig("dws_count", _i32, [_vp, _vp, _vp, _vp, _vp, _sz, _vp])
+_sig("dws_encode_noalloc", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp])
 _sig("dws_apply", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_apply_chain", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _vp, _sz, _vp])
 _sig("dws_xor_encode", _i32, [_vp, _vp, _vp, _i64, _vp])
@@ -140,6 +141,15 @@ def dws_encode_ex(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, 
     return _lib.dws_encode_ex(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
                               workspace, workspace_bytes, stream, wait_limit_ns,
                               debug_withhold_tile)
+
+
+def dws_encode_noalloc(numels, old_ptrs, new_ptrs, offsets, indices, values, capacity,
+                       status_out, stream) -> int:
+    """Encode without a caller-provided workspace (see include/dws.h): the
+    scratch is a fixed device array inside libdws.  ``numels`` is a list."""
+    arr = (ctypes.c_int64 * max(1, len(numels)))(*[int(n) for n in numels])
+    return _lib.dws_encode_noalloc(arr, len(numels), old_ptrs, new_ptrs, offsets, indices, values,
+                                   capacity, status_out, stream)
 
 
 def dws_count(plan, old_ptrs, new_ptrs, offsets, workspace, workspace_bytes, stream) -> int:
