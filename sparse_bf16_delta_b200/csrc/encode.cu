@@ -295,10 +295,11 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm) {
         if (tid == 0 && work) {
             // Room for a whole tile in the ring and one queue slot, so the
             // writes below need no further check (freed in order by the
-            // look-back group).
+            // look-back group).  The cached head only lags, so the flags are
+            // polled only when the cached view says the ring or queue is full.
             unsigned int backoff = 32;
             bool ok = true;
-            for (;;) {
+            while (!(q_tail - q_head < kQueue && ring_tail + kTileElems - ring_head <= kRing)) {
                 // Plain volatile polling: an acquire would also wait for this
                 // thread's outstanding global accesses.  The ring is only
                 // rewritten after the flag is seen, and a look-back warp sets
