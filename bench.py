@@ -62,6 +62,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--rows-reps", type=int, default=5)
+    ap.add_argument("--rows-only", default=None,
+                    help="comma list of qwen_chain, xor, stress_chain: time only these rows "
+                         "(no Llama-3-8B step; a small case for profiling)")
     return ap.parse_args()
 
 
@@ -338,8 +341,25 @@ def row(name, ms, alg_bytes, weight_bytes, peak, extra=None):
     return name, d
 
 
-def run_rows(args, dev, peak):
-    """The other §(a) rows, each on its own workload, timed with events."""
+ROW_GROUPS = ("qwen_chain", "xor", "stress_chain")
+# (dws_apply_chain_ex mode, row-name suffix); 0 = the library's default
+CHAIN_MODES = ((0, ""), (1, "_tile_merge"), (2, "_scatter"))
+
+
+def run_rows(args, dev, peak, groups=ROW_GROUPS):
+    """The other hot-path rows, each on its own workload, timed with events."""
+    out = {}
+    if "qwen_chain" in groups:
+        out.update(rows_qwen_chain(args, dev, peak))
+    if "xor" in groups:
+        out.update(rows_xor(args, dev, peak))
+    if "stress_chain" in groups:
+        out.update(rows_stress_chain(args, dev, peak))
+    return out
+
+
+def rows_qwen_chain(args, dev, peak):
+    """Qwen3-0.6B-shaped chain of 10 deltas: replay, and encode of each step."""
     import gc
 
     import torch
@@ -347,8 +367,6 @@ def run_rows(args, dev, peak):
     import sparse_bf16_delta_b200 as dws
     import workloads as W
     out = {}
-
-    # --- Qwen3-0.6B-shaped chain of 10 deltas -------------------------------
     t0 = time.time()
     s = W.SEEDS["qwen3_0p6b"]
     shapes = W.qwen3_0p6b_shapes()
@@ -371,25 +389,39 @@ def run_rows(args, dev, peak):
         deltas.append(d)
         prev_flat, cur_flat = cur_flat, prev_flat
         prev, cur = cur, prev
-    snap_flat = anchor_flat.clone()
-    snap = [snap_flat[v.storage_offset() - anchor_flat.storage_offset():][:v.numel()] for v in anchor]
-    st = dws.ptr_table(snap)
-    ms, mn = time_reps(lambda: plan.apply_chain(st, deltas), args.rows_reps)
-    plan.raise_on_error("qwen chain")
-    ok = torch.equal(snap_flat, prev_flat)
     N = sum(sizes)
     tot = sum(nnzs)
-    out.update([row("apply_chain_qwen3_0p6b_k10", ms, 4 * N + 6 * tot, 2 * N, peak,
-                    {"min_ms": round(mn, 4), "nnz_total": tot, "exact": ok})])
+    for mode, suffix in CHAIN_MODES:
+        snap_flat = anchor_flat.clone()
+        snap = [snap_flat[v.storage_offset() - anchor_flat.storage_offset():][:v.numel()] for v in anchor]
+        st = dws.ptr_table(snap)
+        # every rep replays onto the result of the previous one: the same
+        # writes, and the snapshot stays the final one
+        ms, mn = time_reps(lambda: plan.apply_chain(st, deltas, mode=mode), args.rows_reps)
+        plan.raise_on_error("qwen chain")
+        ok = torch.equal(snap_flat, prev_flat)
+        out.update([row("apply_chain_qwen3_0p6b_k10" + suffix, ms, 4 * N + 6 * tot, 2 * N, peak,
+                        {"min_ms": round(mn, 4), "nnz_total": tot, "exact": ok})])
+        del snap_flat, snap, st
     mean_enc = statistics.mean(enc_ms)
     out.update([row("encode_qwen3_0p6b", mean_enc, 4 * N + 6 * tot / 10, 2 * N, peak,
                     {"nnz_mean": tot // 10, "sparsity_mean": round(1 - tot / 10 / N, 5)})])
-    del deltas, anchor_flat, prev_flat, cur_flat, snap_flat, anchor, prev, cur, snap, plan
+    del deltas, anchor_flat, prev_flat, cur_flat, anchor, prev, cur, plan
     gc.collect()
     torch.cuda.empty_cache()
     log(f"rows: qwen chain done in {time.time() - t0:.1f}s")
+    return out
 
-    # --- XOR path: 40 layers x 0.8 GB ----------------------------------------
+
+def rows_xor(args, dev, peak):
+    """XOR path: 40 layers x 0.8 GB, encode, apply, double-buffered apply."""
+    import gc
+
+    import torch
+
+    import sparse_bf16_delta_b200 as dws
+    import workloads as W
+    out = {}
     t0 = time.time()
     L, B = 40, 800_000_000
     olds, news, masks = [], [], []
@@ -442,8 +474,18 @@ def run_rows(args, dev, peak):
     gc.collect()
     torch.cuda.empty_cache()
     log(f"rows: xor done in {time.time() - t0:.1f}s")
+    return out
 
-    # --- stress: 12000 tensors, chain of 10 ----------------------------------
+
+def rows_stress_chain(args, dev, peak):
+    """12000 log-uniform tensors, half with clustered changes: chain of 10."""
+    import gc
+
+    import torch
+
+    import sparse_bf16_delta_b200 as dws
+    import workloads as W
+    out = {}
     t0 = time.time()
     s = W.SEEDS["stress"]
     sizes = W.stress_sizes()
@@ -468,19 +510,21 @@ def run_rows(args, dev, peak):
         deltas.append(d)
         prev_flat, cur_flat = cur_flat, prev_flat
         prev, cur = cur, prev
-    snap_flat = anchor_flat.clone()
-    snap = [snap_flat[v.storage_offset() - anchor_flat.storage_offset():][:v.numel()] for v in anchor]
-    st = dws.ptr_table(snap)
-    ms, mn = time_reps(lambda: plan.apply_chain(st, deltas), args.rows_reps)
-    plan.raise_on_error("stress chain")
-    ok = torch.equal(snap_flat, prev_flat) and nnzs == exp_nnz
     N = sum(sizes)
     tot = sum(nnzs)
-    out.update([row("apply_chain_stress_12000t_k10", ms, 4 * N + 6 * tot, 2 * N, peak,
-                    {"min_ms": round(mn, 4), "elements": N, "nnz_total": tot, "exact": ok})])
+    for mode, suffix in CHAIN_MODES:
+        snap_flat = anchor_flat.clone()
+        snap = [snap_flat[v.storage_offset() - anchor_flat.storage_offset():][:v.numel()] for v in anchor]
+        st = dws.ptr_table(snap)
+        ms, mn = time_reps(lambda: plan.apply_chain(st, deltas, mode=mode), args.rows_reps)
+        plan.raise_on_error("stress chain")
+        ok = torch.equal(snap_flat, prev_flat) and nnzs == exp_nnz
+        out.update([row("apply_chain_stress_12000t_k10" + suffix, ms, 4 * N + 6 * tot, 2 * N, peak,
+                        {"min_ms": round(mn, 4), "elements": N, "nnz_total": tot, "exact": ok})])
+        del snap_flat, snap, st
     out.update([row("encode_stress_12000t", statistics.mean(enc_ms), 4 * N + 6 * tot / 10, 2 * N, peak,
                     {"nnz_mean": tot // 10})])
-    del deltas, anchor_flat, prev_flat, cur_flat, snap_flat, anchor, prev, cur, snap, plan
+    del deltas, anchor_flat, prev_flat, cur_flat, anchor, prev, cur, plan
     gc.collect()
     torch.cuda.empty_cache()
     log(f"rows: stress chain done in {time.time() - t0:.1f}s")
@@ -501,6 +545,20 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
     peak, peak_kind = measured_peaks()
+
+    if args.rows_only:
+        groups = [g.strip() for g in args.rows_only.split(",") if g.strip()]
+        bad = [g for g in groups if g not in ROW_GROUPS]
+        if bad:
+            raise SystemExit(f"unknown row group(s) {bad}; choose from {ROW_GROUPS}")
+        rows = run_rows(args, dev, peak, groups)
+        exact = all(v.get("exact", True) and v.get("exact_flip_count", True) for v in rows.values())
+        if rank == 0:
+            print(json.dumps({"rows": rows, "rows_only": groups}), flush=True)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0 if exact else 3
 
     # ---- workload: Llama-3-8B-shaped set, one step -------------------------
     t0 = time.time()

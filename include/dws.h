@@ -234,6 +234,26 @@ DWS_API dws_status_t dws_apply_chain(const dws_plan_t *plan, void *const *snap_p
                              const dws_delta_t *deltas, int32_t K,
                              void *workspace, size_t workspace_bytes, dws_stream_t stream);
 
+/* How dws_apply_chain_ex replays the chain; both give the same snapshot.
+ * DWS_CHAIN_AUTO: the library's choice (what dws_apply_chain does).
+ * DWS_CHAIN_TILE_MERGE: every snapshot tile is read into shared memory, the
+ *   entries of all K deltas are merged into it (the latest delta wins per
+ *   element) and the whole tile is written back: 4 bytes per element of the
+ *   snapshot plus 6 per entry, whatever the deltas touch.
+ * DWS_CHAIN_SCATTER: per window of tiles, the deltas are replayed from the last
+ *   to the first and an element is stored only by the latest delta that
+ *   touches it (a written-bit per element in shared memory); untouched parts of
+ *   the snapshot are neither read nor written. */
+#define DWS_CHAIN_AUTO 0
+#define DWS_CHAIN_TILE_MERGE 1
+#define DWS_CHAIN_SCATTER 2
+
+/* dws_apply_chain with an explicit replay mode (one of DWS_CHAIN_*; anything
+ * else is DWS_ERR_INVALID).  Same arguments, results and errors otherwise. */
+DWS_API dws_status_t dws_apply_chain_ex(const dws_plan_t *plan, void *const *snap_ptrs,
+                                const dws_delta_t *deltas, int32_t K, int32_t mode,
+                                void *workspace, size_t workspace_bytes, dws_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * XOR-mask variant, [XOR] paragraph 1: mask = old ^ new bit by bit, the same
  * size as the model; the receiver gets new = old ^ mask with no

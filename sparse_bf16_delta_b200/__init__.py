@@ -37,6 +37,9 @@ DWS_ERR_TIMEOUT = 5
 DWS_ERR_CUDA = 6
 DWS_ERR_WORKSPACE = 7
 DWS_MAX_CHAIN = 64
+DWS_CHAIN_AUTO = 0
+DWS_CHAIN_TILE_MERGE = 1
+DWS_CHAIN_SCATTER = 2
 
 _i32, _i64, _sz, _vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
 
@@ -66,6 +69,7 @@ _sig("dws_count", _i32, [_vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _sig("dws_encode_noalloc", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp])
 _sig("dws_apply", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_apply_chain", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _vp, _sz, _vp])
+_sig("dws_apply_chain_ex", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _i32, _vp, _sz, _vp])
 _sig("dws_xor_encode", _i32, [_vp, _vp, _vp, _i64, _vp])
 _sig("dws_xor_apply", _i32, [_vp, _vp, _i64, _vp])
 _sig("dws_xor_apply_layers", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i64, _vp, _vp])
@@ -165,6 +169,13 @@ def dws_apply(plan, snap_ptrs, offsets, indices, values, count, workspace, works
 def dws_apply_chain(plan, snap_ptrs, deltas, K, workspace, workspace_bytes, stream) -> int:
     """``deltas``: a ctypes array of dws_delta_t (see ``make_delta_array``)."""
     return _lib.dws_apply_chain(plan, snap_ptrs, deltas, K, workspace, workspace_bytes, stream)
+
+
+def dws_apply_chain_ex(plan, snap_ptrs, deltas, K, mode, workspace, workspace_bytes,
+                       stream) -> int:
+    """dws_apply_chain with an explicit replay mode (DWS_CHAIN_*)."""
+    return _lib.dws_apply_chain_ex(plan, snap_ptrs, deltas, K, mode, workspace, workspace_bytes,
+                                   stream)
 
 
 def dws_xor_encode(old_bytes, new_bytes, mask, nbytes, stream) -> int:
@@ -357,11 +368,16 @@ class DeltaPlan:
                          self.workspace.data_ptr(), self.workspace_bytes,
                          _stream_handle(stream)), "dws_apply")
 
-    def apply_chain(self, snap_table, deltas, stream=None):
+    def apply_chain(self, snap_table, deltas, stream=None, mode=DWS_CHAIN_AUTO):
         arr = make_delta_array([d.as_ref() for d in deltas])
-        _check(dws_apply_chain(self.handle, snap_table.data_ptr(), arr, len(deltas),
-                               self.workspace.data_ptr(), self.workspace_bytes,
-                               _stream_handle(stream)), "dws_apply_chain")
+        if mode == DWS_CHAIN_AUTO:
+            _check(dws_apply_chain(self.handle, snap_table.data_ptr(), arr, len(deltas),
+                                   self.workspace.data_ptr(), self.workspace_bytes,
+                                   _stream_handle(stream)), "dws_apply_chain")
+        else:
+            _check(dws_apply_chain_ex(self.handle, snap_table.data_ptr(), arr, len(deltas), mode,
+                                      self.workspace.data_ptr(), self.workspace_bytes,
+                                      _stream_handle(stream)), "dws_apply_chain_ex")
 
 
 def xor_encode(old, new, mask=None, stream=None):

@@ -427,6 +427,224 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
     if (tid == 0) bulk_wait_all();
 }
 
+// ---------------------------------------------------------------------------
+// Chain replay: reverse-order scatter over windows, with a written-bitmap
+// ---------------------------------------------------------------------------
+// Each CTA owns a contiguous range of plan tiles and walks it in windows of
+// kWinTiles tiles.  Per window the deltas are replayed from the LAST to the
+// first: an entry is stored only if no later delta has stored that element
+// (one bit per element of the window in shared memory), which leaves exactly
+// what the forward replay leaves, and every element is written at most once.
+// The snapshot is never read by the SM; partial 32-byte sectors are merged in
+// L2.  Per delta, the window's entries are one contiguous stretch of the
+// delta (entries are ordered by tensor, then index): the CTA's warps stream
+// it in chunks of 32 entries, kScatDepth chunks in flight per warp, and the
+// stretch ends at the first entry past the window, which is where the next
+// window's stretch starts.
+constexpr int kScatThreads = 256;
+constexpr int kScatWarps = kScatThreads / 32;
+constexpr int kWinTiles = 32;
+constexpr int kWinElems = kWinTiles * kTileElems;
+constexpr int kScatDepth = 4;
+
+struct ScatParams {
+    WsView ws;
+    uint16_t *const *snap_ptrs;
+    long long tiles_per_cta;
+    int K;
+    DeltaRef d[DWS_MAX_CHAIN];
+};
+
+struct ScatSmem {
+    uint32_t written[kWinElems / 32];
+    long long cur[DWS_MAX_CHAIN];          // per delta: first entry not yet consumed
+    long long base[kWinTiles];             // per window tensor: (first_tile - window start) * tile
+    long long numel[kWinTiles];
+    uint16_t *ptr[kWinTiles];
+    long long offs[kWinTiles + 1];         // current delta's offsets of the window tensors
+    unsigned long long next;               // first entry past the window (min over warps)
+};
+
+__global__ void __launch_bounds__(kScatThreads, 4) chain_scatter_kernel(ScatParams p) {
+    __shared__ __align__(16) ScatSmem sm;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+
+    if (!ws_matches(p.ws)) return;
+    if (ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) != 0u) return;
+
+    const long long tb = static_cast<long long>(blockIdx.x) * p.tiles_per_cta;
+    long long te = tb + p.tiles_per_cta;
+    if (te > p.ws.num_tiles) te = p.ws.num_tiles;
+    if (tb >= te) return;
+
+    // Cursors at the CTA's first tile: one warp-cooperative search per delta.
+    {
+        const int t0 = p.ws.tile_tensor[tb];
+        const long long ls = (tb - p.ws.first_tile[t0]) << kTileShift;
+        for (int k = warp; k < p.K; k += kScatWarps) {
+            const DeltaRef d = p.d[k];
+            const long long lo = d.offsets[t0];
+            const long long hi = d.offsets[t0 + 1];
+            // At a tensor's first tile start at the segment head, so that a
+            // negative index is seen (and flagged) rather than skipped.
+            const long long c = (ls == 0) ? lo : warp_lower_bound(d.indices, lo, hi, static_cast<int>(ls));
+            if (lane == 0) sm.cur[k] = c;
+        }
+    }
+
+    for (long long a = tb; a < te; a += kWinTiles) {
+        const long long b = (a + kWinTiles < te) ? a + kWinTiles : te;
+        const int win_words = static_cast<int>(b - a) * (kTileElems / 32);
+        const int t_lo = p.ws.tile_tensor[a];
+        const int nt = p.ws.tile_tensor[b - 1] - t_lo + 1;  // <= b - a: every tensor owns a tile
+        if (t_lo < 0 || nt < 1 || nt > kWinTiles || t_lo + nt > p.ws.num_tensors) {
+            if (tid == 0) record_error(p.ws.hdr, DWS_ERR_WORKSPACE, a);
+            return;  // uniform: every thread read the same table entries
+        }
+        __syncthreads();  // previous window (and the cursor set-up) complete
+        for (int w = tid; w < win_words; w += kScatThreads) sm.written[w] = 0u;
+        if (tid < nt) {
+            const int t = t_lo + tid;
+            const long long n = p.ws.numel[t];
+            uint16_t *ptr = p.snap_ptrs[t];
+            if (n > 0 && (ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 1u))) {
+                record_error(p.ws.hdr, DWS_ERR_INVALID, t);
+                ptr = nullptr;
+            }
+            sm.base[tid] = (p.ws.first_tile[t] - a) << kTileShift;
+            sm.numel[tid] = n;
+            sm.ptr[tid] = ptr;
+        }
+        const long long win_len = (b - a) << kTileShift;
+
+        for (int k = p.K - 1; k >= 0; --k) {
+            const DeltaRef d = p.d[k];
+            if (tid <= nt) sm.offs[tid] = d.offsets[t_lo + tid];
+            if (tid == 0) sm.next = ~0ull;
+            __syncthreads();
+            const long long jmax = sm.offs[nt];
+            constexpr long long kStride = 32LL * kScatWarps;
+            long long j = sm.cur[k] + 32 * warp + lane;  // this lane's entry of the current chunk
+            const int *pi = d.indices + j;
+            const uint16_t *pv = d.values + j;
+
+            int ix[kScatDepth];
+            uint16_t vx[kScatDepth];
+#pragma unroll
+            for (int q = 0; q < kScatDepth; ++q) {
+                if (j + q * kStride < jmax) {
+                    ix[q] = __ldg(pi + q * kStride);
+                    vx[q] = __ldg(pv + q * kStride);
+                }
+            }
+            // The warp's current tensor (its chunks only move forward) and
+            // that tensor's constants: segment, window offset, size, pointer.
+            int tw = 0;
+            long long seg_lo = sm.offs[0], seg_hi = sm.offs[1];
+            int off_c = static_cast<int>(-sm.base[0]);  // window start - tensor start (elements)
+            uint32_t numel_c = static_cast<uint32_t>(sm.numel[0]);
+            uint16_t *ptr_c = sm.ptr[0];
+            bool stop = false;
+            for (;;) {
+#pragma unroll
+                for (int q = 0; q < kScatDepth; ++q) {
+                    const long long cstart = j - lane;
+                    if (cstart >= jmax) {  // whole chunk past the stretch (uniform)
+                        stop = true;
+                        break;
+                    }
+                    const int idx = ix[q];
+                    const uint16_t val = vx[q];
+                    if (j + kScatDepth * kStride < jmax) {
+                        ix[q] = __ldg(pi + kScatDepth * kStride);
+                        vx[q] = __ldg(pv + kScatDepth * kStride);
+                    }
+                    const bool valid = j < jmax;
+                    if (cstart >= seg_hi) {  // uniform: move to the chunk's first tensor
+                        while (tw + 1 < nt && sm.offs[tw + 1] <= cstart) ++tw;
+                        seg_lo = sm.offs[tw];
+                        seg_hi = sm.offs[tw + 1];
+                        off_c = static_cast<int>(-sm.base[tw]);
+                        numel_c = static_cast<uint32_t>(sm.numel[tw]);
+                        ptr_c = sm.ptr[tw];
+                    }
+                    const long long clast = (cstart + 31 < jmax) ? cstart + 31 : jmax - 1;
+                    // 0: nothing, 1: store, 2: bad entry (consumed), 3: past the window
+                    int cls = 0;
+                    uint32_t rel = 0;  // element within the window (when cls == 1)
+                    uint16_t *dst = ptr_c;
+                    if (cstart >= seg_lo && clast < seg_hi) {
+                        // Common case, all 32-bit: the chunk lies in one tensor.
+                        // (off_c < numel <= 2^31 - 1; rel wraps for indices
+                        // below the window, which `before` catches.)
+                        const bool ok = static_cast<uint32_t>(idx) < numel_c;
+                        const bool before = idx < off_c;
+                        rel = static_cast<uint32_t>(idx) - static_cast<uint32_t>(off_c);
+                        if (valid) cls = (!ok || before) ? 2 : (rel >= static_cast<uint32_t>(win_len) ? 3 : 1);
+                    } else if (valid) {
+                        // The chunk crosses a tensor boundary: per-lane tensor.
+                        int tl = tw;
+                        while (tl + 1 < nt && sm.offs[tl + 1] <= j) ++tl;
+                        if (j < sm.offs[tl] || idx < 0 || static_cast<long long>(idx) >= sm.numel[tl]) {
+                            cls = 2;
+                        } else {
+                            const long long r = sm.base[tl] + idx;
+                            cls = (r >= win_len) ? 3 : (r < 0 ? 2 : 1);
+                            rel = static_cast<uint32_t>(r);
+                            dst = sm.ptr[tl];
+                        }
+                    }
+                    const unsigned int past = __ballot_sync(0xffffffffu, cls == 3);
+                    if (past != 0u) {
+                        const int first = __ffs(past) - 1;
+                        if (lane == first) atomicMin(&sm.next, static_cast<unsigned long long>(j));
+                        if (lane > first) cls = 0;
+                        stop = true;
+                    }
+                    const bool ins = (cls == 1);
+                    bool store = ins;
+                    if (p.K > 1) {  // uniform: a single delta needs no written-bits
+                        const uint32_t word = rel >> 5;
+                        const uint32_t bit = 1u << (rel & 31u);
+                        if (ins) store = (sm.written[word] & bit) == 0u;
+                        // Mark this delta's elements: one OR per lane, or two
+                        // for a run of 32 consecutive elements (a clustered
+                        // change), where per-lane ORs would all hit one word.
+                        const uint32_t prev = __shfl_up_sync(0xffffffffu, rel, 1);
+                        const unsigned int run = __ballot_sync(0xffffffffu, ins && (lane == 0 || rel > prev));
+                        const uint32_t r0 = __shfl_sync(0xffffffffu, rel, 0);
+                        const uint32_t r31 = __shfl_sync(0xffffffffu, rel, 31);
+                        if (run == 0xffffffffu && r31 - r0 == 31u) {
+                            if (lane == 0) atomicOr(&sm.written[r0 >> 5], ~0u << (r0 & 31u));
+                            if (lane == 31 && (r31 & 31u) != 31u)
+                                atomicOr(&sm.written[r31 >> 5], (2u << (r31 & 31u)) - 1u);
+                        } else if (ins) {
+                            atomicOr(&sm.written[word], bit);
+                        }
+                    }
+                    if (store) {
+                        if (dst != nullptr) dst[idx] = val;
+                    } else if (cls == 2) {
+                        record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, j);
+                    }
+                    if (stop) break;
+                    j += kStride;
+                    pi += kStride;
+                    pv += kStride;
+                }
+                if (stop) break;
+            }
+            __syncthreads();  // every entry of this delta stored before the next (earlier) one
+            if (tid == 0) {
+                const unsigned long long nx = sm.next;
+                sm.cur[k] = (nx < static_cast<unsigned long long>(jmax)) ? static_cast<long long>(nx) : jmax;
+            }
+        }
+    }
+}
+
 }  // namespace
 
 size_t chain_smem_bytes() { return sizeof(ChainSmem); }
@@ -434,6 +652,11 @@ size_t chain_smem_bytes() { return sizeof(ChainSmem); }
 cudaError_t chain_set_attributes() {
     return cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(sizeof(ChainSmem)));
+}
+
+cudaError_t scatter_occupancy(int *ctas_per_sm) {
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, chain_scatter_kernel,
+                                                         kScatThreads, 0);
 }
 
 cudaError_t chain_occupancy(int *ctas_per_sm) {
@@ -500,6 +723,30 @@ cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs,
     p.tiles_per_cta = (ws.num_tiles + grid - 1) / grid;
     grid = (ws.num_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
     chain_kernel<<<static_cast<unsigned int>(grid), kChainThreads, sizeof(ChainSmem), s>>>(p);
+    return launched();
+}
+
+cudaError_t launch_apply_chain_scatter(const WsView &ws, uint16_t *const *snap_ptrs,
+                                       const DeltaRef *deltas, int K, cudaStream_t s) {
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    e = launch_delta_check(ws, deltas, K, s);
+    if (e != cudaSuccess) return e;
+    ScatParams p;
+    p.ws = ws;
+    p.snap_ptrs = snap_ptrs;
+    p.K = K;
+    for (int k = 0; k < K; ++k) p.d[k] = deltas[k];
+    long long grid = static_cast<long long>(di.sm_count) * di.scatter_ctas_per_sm;
+    const long long windows = (ws.num_tiles + kWinTiles - 1) / kWinTiles;
+    if (grid > windows) grid = windows;
+    if (grid < 1) grid = 1;
+    // whole windows per CTA, so that only the last window of the plan is short
+    const long long win_per_cta = (windows + grid - 1) / grid;
+    p.tiles_per_cta = win_per_cta * kWinTiles;
+    grid = (ws.num_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
+    chain_scatter_kernel<<<static_cast<unsigned int>(grid), kScatThreads, 0, s>>>(p);
     return launched();
 }
 

@@ -18,6 +18,7 @@ cudaError_t encode_occupancy(int *ctas_per_sm);
 size_t chain_smem_bytes();
 cudaError_t chain_set_attributes();
 cudaError_t chain_occupancy(int *ctas_per_sm);
+cudaError_t scatter_occupancy(int *ctas_per_sm);
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -32,9 +33,11 @@ void init_device(int dev) {
     if (e == cudaSuccess) e = chain_set_attributes();
     if (e == cudaSuccess) e = encode_occupancy(&di.encode_ctas_per_sm);
     if (e == cudaSuccess) e = chain_occupancy(&di.chain_ctas_per_sm);
+    if (e == cudaSuccess) e = scatter_occupancy(&di.scatter_ctas_per_sm);
     if (e == cudaSuccess) {
         if (di.encode_ctas_per_sm < 1) di.encode_ctas_per_sm = 1;
         if (di.chain_ctas_per_sm < 1) di.chain_ctas_per_sm = 1;
+        if (di.scatter_ctas_per_sm < 1) di.scatter_ctas_per_sm = 1;
     }
     g_info[dev] = di;
     g_err[dev] = e;
@@ -249,9 +252,18 @@ dws_status_t dws_apply(const dws_plan_t *plan, void *const *snap_ptrs, const int
 dws_status_t dws_apply_chain(const dws_plan_t *plan, void *const *snap_ptrs,
                              const dws_delta_t *deltas, int32_t K, void *workspace,
                              size_t workspace_bytes, dws_stream_t stream) {
+    return dws_apply_chain_ex(plan, snap_ptrs, deltas, K, DWS_CHAIN_AUTO, workspace,
+                              workspace_bytes, stream);
+}
+
+dws_status_t dws_apply_chain_ex(const dws_plan_t *plan, void *const *snap_ptrs,
+                                const dws_delta_t *deltas, int32_t K, int32_t mode,
+                                void *workspace, size_t workspace_bytes, dws_stream_t stream) {
     dws_status_t st = check_ws(plan, workspace, workspace_bytes);
     if (st != DWS_OK) return st;
     if (snap_ptrs == nullptr || deltas == nullptr || K < 1 || K > DWS_MAX_CHAIN)
+        return DWS_ERR_INVALID;
+    if (mode != DWS_CHAIN_AUTO && mode != DWS_CHAIN_TILE_MERGE && mode != DWS_CHAIN_SCATTER)
         return DWS_ERR_INVALID;
     dws::DeltaRef d[DWS_MAX_CHAIN];
     long long total = 0;
@@ -264,6 +276,11 @@ dws_status_t dws_apply_chain(const dws_plan_t *plan, void *const *snap_ptrs,
                              deltas[k].count};
         total += deltas[k].count;
     }
+    if (mode == DWS_CHAIN_AUTO) mode = DWS_CHAIN_SCATTER;
+    if (mode == DWS_CHAIN_SCATTER)
+        return from_cuda(dws::launch_apply_chain_scatter(
+            view_of(plan, workspace), reinterpret_cast<uint16_t *const *>(snap_ptrs), d, K,
+            reinterpret_cast<cudaStream_t>(stream)));
     return from_cuda(dws::launch_apply_chain(view_of(plan, workspace),
                                              reinterpret_cast<uint16_t *const *>(snap_ptrs), d, K,
                                              total, plan->N,

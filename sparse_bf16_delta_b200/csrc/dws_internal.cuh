@@ -313,6 +313,7 @@ struct DeviceInfo {
     int sm_count;
     int encode_ctas_per_sm;
     int chain_ctas_per_sm;
+    int scatter_ctas_per_sm;
 };
 
 // Per-device constants and one-time kernel attribute setup (thread-safe).
@@ -340,6 +341,8 @@ cudaError_t launch_apply(const WsView &ws, uint16_t *const *snap_ptrs, const Del
 cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs,
                                const DeltaRef *deltas, int K, long long total_entries,
                                long long total_elems, cudaStream_t s);
+cudaError_t launch_apply_chain_scatter(const WsView &ws, uint16_t *const *snap_ptrs,
+                                       const DeltaRef *deltas, int K, cudaStream_t s);
 
 cudaError_t launch_xor(const uint8_t *a, const uint8_t *b, uint8_t *out, long long nbytes,
                        cudaStream_t s);

@@ -28,7 +28,7 @@ def lib():
 def test_header_declares_the_boundary():
     syms = _declared_symbols()
     for name in ["dws_plan_create", "dws_plan_upload", "dws_encode", "dws_count", "dws_apply",
-                 "dws_apply_chain", "dws_xor_encode", "dws_xor_apply", "dws_xor_apply_layers",
+                 "dws_apply_chain", "dws_apply_chain_ex", "dws_xor_encode", "dws_xor_apply", "dws_xor_apply_layers",
                  "dws_status", "dws_strerror"]:
         assert name in syms
 
@@ -93,6 +93,9 @@ def test_host_side_argument_errors_need_no_device():
         arr = dws.make_delta_array([(1, 1, 1, 0)])
         assert dws.dws_apply_chain(p, 1, arr, 0, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_apply_chain(p, 1, arr, 65, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_apply_chain_ex(p, 1, arr, 1, 3, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_apply_chain_ex(p, 1, arr, 1, -1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_apply_chain_ex(p, 1, arr, 0, 2, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
     finally:
         dws.dws_plan_destroy(p)
     assert dws.dws_xor_encode(1, 1, 1, -1, None) == dws.DWS_ERR_INVALID

@@ -117,13 +117,15 @@ def test_qwen3_0p6b_chain_full(dws):
         deltas.append(d)
         prev_flat, cur_flat = cur_flat, prev_flat
         prev, cur = cur, prev
-    # one apply of the first delta, then the fused 10-delta replay
-    snap_flat = anchor_flat.clone()
-    snap = [snap_flat[v.storage_offset():][:v.numel()] for v in anchor]
-    plan.apply_chain(dws.ptr_table(snap), deltas)
-    plan.raise_on_error("apply_chain")
-    assert torch.equal(snap_flat, prev_flat)
-    del anchor_flat, prev_flat, cur_flat, snap_flat, deltas, plan
+    # the fused 10-delta replay, in both modes
+    for mode in (dws.DWS_CHAIN_TILE_MERGE, dws.DWS_CHAIN_SCATTER):
+        snap_flat = anchor_flat.clone()
+        snap = [snap_flat[v.storage_offset():][:v.numel()] for v in anchor]
+        plan.apply_chain(dws.ptr_table(snap), deltas, mode=mode)
+        plan.raise_on_error("apply_chain")
+        assert torch.equal(snap_flat, prev_flat), mode
+        del snap_flat, snap
+    del anchor_flat, prev_flat, cur_flat, deltas, plan
     _free()
 
 
@@ -185,12 +187,14 @@ def test_stress_12000_tensors_chain_full(dws):
         deltas.append(d)
         prev_flat, cur_flat = cur_flat, prev_flat
         prev, cur = cur, prev
-    snap_flat = anchor_flat.clone()
-    snap = [snap_flat[v.storage_offset() - anchor_flat.storage_offset():][:v.numel()] for v in anchor]
-    plan.apply_chain(dws.ptr_table(snap), deltas)
-    plan.raise_on_error("apply_chain")
-    assert torch.equal(snap_flat, prev_flat)
-    del anchor_flat, prev_flat, cur_flat, snap_flat, deltas, plan
+    for mode in (dws.DWS_CHAIN_TILE_MERGE, dws.DWS_CHAIN_SCATTER):
+        snap_flat = anchor_flat.clone()
+        snap = [snap_flat[v.storage_offset() - anchor_flat.storage_offset():][:v.numel()] for v in anchor]
+        plan.apply_chain(dws.ptr_table(snap), deltas, mode=mode)
+        plan.raise_on_error("apply_chain")
+        assert torch.equal(snap_flat, prev_flat), mode
+        del snap_flat, snap
+    del anchor_flat, prev_flat, cur_flat, deltas, plan
     _free()
 
 

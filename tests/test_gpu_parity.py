@@ -272,20 +272,24 @@ def test_apply_with_bad_offsets_writes_nothing(dws):
 
 # ---------------------------------------------------------------- chain
 
+# Both replay modes of dws_apply_chain_ex must give the sequential replay.
+CHAIN_MODES = pytest.mark.parametrize("mode", [1, 2], ids=["tile_merge", "scatter"])
 
-def test_chain_golden_later_delta_wins(dws):
+
+@CHAIN_MODES
+def test_chain_golden_later_delta_wins(dws, mode):
     anchor, deltas, final = G.chain_example()
     snaps = [dev_bits(a) for a in anchor]
     plan = dws.DeltaPlan.for_tensors(snaps)
     dd = [dws.Delta(torch.from_numpy(o).cuda(), torch.from_numpy(i).cuda(),
                     torch.from_numpy(v.view(np.int16)).cuda()) for o, i, v in deltas]
-    plan.apply_chain(dws.ptr_table(snaps), dd)
+    plan.apply_chain(dws.ptr_table(snaps), dd, mode=mode)
     plan.raise_on_error()
     for s, f in zip(snaps, final):
         np.testing.assert_array_equal(host_bits(s), f)
 
 
-def _chain_case(dws, shapes_or_sizes, steps, stepper, anchor_set):
+def _chain_case(dws, shapes_or_sizes, steps, stepper, anchor_set, modes=(1, 2)):
     """Encode `steps` steps on the GPU (each delta checked against the oracle),
     replay them in one chain launch onto a copy of the anchor."""
     prev = anchor_set
@@ -301,14 +305,15 @@ def _chain_case(dws, shapes_or_sizes, steps, stepper, anchor_set):
         deltas.append(d)
         host_deltas.append(want)
         prev, prev_h = cur, cur_h
-    snaps = [t.clone() for t in anchor_set.tensors]
-    plan.apply_chain(dws.ptr_table(snaps), deltas)
-    plan.raise_on_error("apply_chain")
     ref = [host_bits(t) for t in anchor_set.tensors]
     oracle.apply_chain(ref, host_deltas)
-    for s, r, f in zip(snaps, ref, prev_h):
-        np.testing.assert_array_equal(host_bits(s), r)
-        np.testing.assert_array_equal(r, f)
+    for mode in modes:
+        snaps = [t.clone() for t in anchor_set.tensors]
+        plan.apply_chain(dws.ptr_table(snaps), deltas, mode=mode)
+        plan.raise_on_error("apply_chain")
+        for s, r, f in zip(snaps, ref, prev_h):
+            np.testing.assert_array_equal(host_bits(s), r)
+            np.testing.assert_array_equal(r, f)
 
 
 def test_chain_qwen_shaped_scaled_ten_steps(dws):
@@ -325,7 +330,8 @@ def test_chain_stress_scaled_ten_steps(dws):
     _chain_case(dws, sizes, 10, lambda w, k: W.stress_step(w, clustered, k, "cuda")[0], w0)
 
 
-def test_chain_on_unaligned_snapshots(dws):
+@CHAIN_MODES
+def test_chain_on_unaligned_snapshots(dws, mode):
     # Snapshot views that are not 16-byte aligned take the direct-store path.
     rng = np.random.default_rng(47)
     n = 8192 * 2 + 77
@@ -344,23 +350,97 @@ def test_chain_on_unaligned_snapshots(dws):
     plan = dws.DeltaPlan([n])
     dd = [dws.Delta(torch.from_numpy(o).cuda(), torch.from_numpy(i).cuda(),
                     torch.from_numpy(v.view(np.int16)).cuda()) for o, i, v in host_deltas]
-    plan.apply_chain(dws.ptr_table([snap]), dd)
+    plan.apply_chain(dws.ptr_table([snap]), dd, mode=mode)
     plan.raise_on_error()
     np.testing.assert_array_equal(host_bits(snap), cur)
 
 
-def test_chain_rejects_index_beyond_numel(dws):
+@CHAIN_MODES
+def test_chain_max_length_tiny_and_empty_tensors(dws, mode):
+    # 64 deltas (the maximum) of mixed densities, one of them empty, over a
+    # plan of many tiny tensors, empty tensors and a few multi-tile ones, so
+    # that windows and CTA ranges cut through tensors and hold many of them.
+    rng = np.random.default_rng(64)
+    sizes = [0, 1, 5, 0, 8191, 8192, 8193, 3] + [int(x) for x in rng.integers(1, 600, 120)] + \
+            [3 * 8192 + 17, 0, 300_001, 2, 70_000]
+    anchor = [rng.integers(0, 1 << 16, n, dtype=np.uint16) for n in sizes]
+    cur = [a.copy() for a in anchor]
+    host_deltas = []
+    for k in range(64):
+        rate = [0.0, 0.001, 0.02, 0.3, 0.9][k % 5]
+        nxt = []
+        for c in cur:
+            x = c.copy()
+            if c.size:
+                m = rng.random(c.size) < rate
+                x[m] ^= rng.integers(1, 1 << 16, int(m.sum()), dtype=np.uint16)
+            nxt.append(x)
+        host_deltas.append(oracle.encode(cur, nxt))
+        cur = nxt
+    ref = [a.copy() for a in anchor]
+    oracle.apply_chain(ref, host_deltas)
+    for r, c in zip(ref, cur):
+        np.testing.assert_array_equal(r, c)
+    snaps = [dev_bits(a) for a in anchor]
+    plan = dws.DeltaPlan(sizes)
+    dd = [dws.Delta(torch.from_numpy(o).cuda(), torch.from_numpy(i).cuda(),
+                    torch.from_numpy(v.view(np.int16)).cuda()) for o, i, v in host_deltas]
+    plan.apply_chain(dws.ptr_table(snaps), dd, mode=mode)
+    plan.raise_on_error()
+    for s, c in zip(snaps, cur):
+        np.testing.assert_array_equal(host_bits(s), c)
+
+
+@CHAIN_MODES
+def test_chain_single_delta_equals_apply(dws, mode):
+    rng = np.random.default_rng(65)
+    sizes = [40_000, 8192 * 40 + 3, 1]
+    a = [rng.integers(0, 1 << 16, n, dtype=np.uint16) for n in sizes]
+    b = []
+    for x in a:
+        y = x.copy()
+        m = rng.random(x.size) < 0.05
+        y[m] ^= np.uint16(0x8001)
+        b.append(y)
+    o, i, v = oracle.encode(a, b)
+    d = dws.Delta(torch.from_numpy(o).cuda(), torch.from_numpy(i).cuda(),
+                  torch.from_numpy(v.view(np.int16)).cuda())
+    plan = dws.DeltaPlan(sizes)
+    snaps = [dev_bits(x) for x in a]
+    plan.apply_chain(dws.ptr_table(snaps), [d], mode=mode)
+    plan.raise_on_error()
+    for s, y in zip(snaps, b):
+        np.testing.assert_array_equal(host_bits(s), y)
+
+
+@CHAIN_MODES
+def test_chain_rejects_index_beyond_numel(dws, mode):
     n = 9000
     plan = dws.DeltaPlan([n])
     snap = dev_bits(np.zeros(n, np.uint16))
     d = dws.Delta(torch.tensor([0, 2], dtype=torch.int64, device="cuda"),
                   torch.tensor([3, n + 5], dtype=torch.int32, device="cuda"),
                   torch.tensor([7, 7], dtype=torch.int16, device="cuda"))
-    plan.apply_chain(dws.ptr_table([snap]), [d])
+    plan.apply_chain(dws.ptr_table([snap]), [d], mode=mode)
     st, _ = plan.status()
     assert st == dws.DWS_ERR_BAD_DELTA
     h = host_bits(snap)
     assert h[3] == 7 and h.sum() == 7
+
+
+@CHAIN_MODES
+def test_chain_rejects_negative_index(dws, mode):
+    n = 9000
+    plan = dws.DeltaPlan([n])
+    snap = dev_bits(np.zeros(n, np.uint16))
+    d = dws.Delta(torch.tensor([0, 2], dtype=torch.int64, device="cuda"),
+                  torch.tensor([-4, 11], dtype=torch.int32, device="cuda"),
+                  torch.tensor([7, 7], dtype=torch.int16, device="cuda"))
+    plan.apply_chain(dws.ptr_table([snap]), [d], mode=mode)
+    st, _ = plan.status()
+    assert st == dws.DWS_ERR_BAD_DELTA
+    h = host_bits(snap)
+    assert h[11] == 7 and h.sum() == 7
 
 
 # ---------------------------------------------------------------- XOR
