@@ -83,6 +83,23 @@ def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time (all ranks take part; world 1: ms itself)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replicas_value(world, bytes_per_rank, ms_per_step):
+    """Whole-job GB/s: every replica moves bytes_per_rank per step, the step
+    taking the slowest rank's time."""
+    return world * bytes_per_rank / (ms_per_step / 1e3) / 1e9
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -630,10 +647,7 @@ def run_ours(args):
     total_ms = start.elapsed_time(end)
     enc_ms = statistics.mean(e_enc0[k].elapsed_time(e_enc1[k]) for k in range(K))
     app_ms = statistics.mean(e_enc1[k].elapsed_time(e_app1[k]) for k in range(K))
-    if world > 1:
-        tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-        total_ms = float(tmax.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / K
 
     # correctness of what was timed: the applied snapshot is the new snapshot
@@ -643,7 +657,7 @@ def run_ours(args):
         log(f"[rank {rank}] RESULT MISMATCH (status {st_code}, detail {st_detail})")
 
     weight_bytes = 2 * N
-    value = world * weight_bytes / (ms_per_step / 1e3) / 1e9
+    value = replicas_value(world, weight_bytes, ms_per_step)
     enc_alg = 4 * N + 6 * nnz + 8 * (T + 1)
     achieved = enc_alg / (enc_ms / 1e3) / 1e9
     tpe, nnz_frac_prof = encode_traffic_per_elem()
@@ -715,15 +729,10 @@ def run_ours(args):
             e2e_step()
         b.record()
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
-        if world > 1:
-            tmax = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-            e_ms = float(tmax.item())
-        e_ms /= args.e2e_steps
+        e_ms = max_over_ranks(a.elapsed_time(b), world, dev) / args.e2e_steps
         dbytes = 8 * (T + 1) + 6 * nnz
         ok = bool(torch.equal(snap_flat, new_flat)) and plan.status()[0] == dws.DWS_OK
-        line["e2e"] = {"value": round(world * weight_bytes / (e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+        line["e2e"] = {"value": round(replicas_value(world, weight_bytes, e_ms), 2), "unit": "GB/s",
                        "h2d_bytes_per_step": 2 * new_flat.numel() + dbytes,
                        "d2h_bytes_per_step": dbytes, "ms_per_step": round(e_ms, 3),
                        "steps": args.e2e_steps, "exact": ok,

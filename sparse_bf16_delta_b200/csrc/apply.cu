@@ -87,49 +87,89 @@ struct ApplyParams {
     DeltaRef d;
 };
 
+// Warp-cooperative: the largest t in [0, T-1] with offsets[t] <= j (offsets
+// non-decreasing, offsets[0] = 0 <= j).  Each round probes 32 evenly spaced
+// tensors, so T = 291 takes two dependent loads and T = 12000 three.
+__device__ int warp_tensor_of_entry(const long long *offsets, int T, long long j) {
+    const int lane = threadIdx.x & 31;
+    int lo = 0, hi = T - 1;  // the answer lies in [lo, hi]
+    while (true) {
+        const int span = hi - lo + 1;
+        const int step = (span + 31) / 32;
+        const int t = lo + lane * step;
+        const bool le = (t <= hi) && (__ldg(offsets + t) <= j);
+        const unsigned int b = __ballot_sync(0xffffffffu, le);  // a prefix of lanes; lane 0 set
+        const int c = __popc(b);
+        if (step == 1) return lo + c - 1;
+        const int nlo = lo + (c - 1) * step;
+        const int nhi = lo + c * step - 1;
+        lo = nlo;
+        hi = nhi < hi ? nhi : hi;
+    }
+}
+
 __global__ void __launch_bounds__(kApplyThreads) apply_kernel(ApplyParams p) {
-    __shared__ int s_t0, s_t1, s_go;
+    __shared__ int s_t[2];
+    __shared__ int s_go;
     __shared__ long long s_end;
-    if (!ws_matches(p.ws)) return;
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
     const int T = p.ws.num_tensors;
     const long long base = static_cast<long long>(blockIdx.x) * kApplyEntries;
-    if (threadIdx.x == 0) {
-        const long long nnz = p.d.offsets[T];
-        const long long total = nnz < p.d.count ? nnz : p.d.count;
-        long long end = base + kApplyEntries;
-        if (end > total) end = total;
-        s_end = end;
-        s_go = (ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) == 0u) && base < end;
-        if (s_go) {
-            s_t0 = tensor_of_entry(p.d.offsets, 0, T - 1, base);
-            s_t1 = tensor_of_entry(p.d.offsets, s_t0, T - 1, end - 1);
-        }
-    }
-    __syncthreads();
-    if (!s_go) return;
-    const long long end = s_end;
-    const int t0 = s_t0, t1 = s_t1;
+    const long long cap = p.d.count;  // entries the arrays hold
+    if (base >= cap) return;          // uniform
 
+    // Everything below is read before any check, so that the latencies
+    // overlap: the entries (the caller's arrays, bounded by count), the
+    // workspace header and the delta's offsets.  Nothing is written until
+    // the checks have passed.
     int idx[kApplyPerThread];
     uint16_t val[kApplyPerThread];
 #pragma unroll
     for (int r = 0; r < kApplyPerThread; ++r) {
-        const long long j = base + threadIdx.x + r * kApplyThreads;
-        if (j < end) {
+        const long long j = base + tid + r * kApplyThreads;
+        if (j < cap) {
             idx[r] = __ldg(p.d.indices + j);
             val[r] = __ldg(p.d.values + j);
         }
     }
+    if (warp < 2) {  // tensors of the block's first and last entries
+        const long long last = (base + kApplyEntries < cap ? base + kApplyEntries : cap) - 1;
+        const int t = warp_tensor_of_entry(p.d.offsets, T, warp == 0 ? base : last);
+        if (lane == 0) s_t[warp] = t;
+    }
+    if (tid == 64) {
+        const WsHeader *h = p.ws.hdr;
+        const bool ok = (h->magic == kWsMagic && h->fingerprint == p.ws.fingerprint &&
+                         h->num_tiles == p.ws.num_tiles && h->num_tensors == T);
+        if (!ok) record_error(p.ws.hdr, DWS_ERR_WORKSPACE, 0);
+        const long long nnz = p.d.offsets[T];
+        const long long total = nnz < cap ? nnz : cap;
+        const long long end = (base + kApplyEntries < total) ? base + kApplyEntries : total;
+        s_end = end;
+        s_go = ok && (ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) == 0u) && base < end;
+    }
+    __syncthreads();
+    if (!s_go) return;
+    const long long end = s_end;
+    const int t0 = s_t[0], t1 = s_t[1];
+
 #pragma unroll
     for (int r = 0; r < kApplyPerThread; ++r) {
-        const long long j = base + threadIdx.x + r * kApplyThreads;
+        const long long j = base + tid + r * kApplyThreads;
+        // entry j - 1 is the previous lane's (lane 0: read it)
+        int prev = __shfl_up_sync(0xffffffffu, idx[r], 1);
         if (j >= end) continue;
         const int t = (t0 == t1) ? t0 : tensor_of_entry(p.d.offsets, t0, t1, j);
         const long long n = p.ws.numel[t];
         const long long seg = p.d.offsets[t];
         const int i = idx[r];
         bool ok = (i >= 0) && (static_cast<long long>(i) < n);
-        if (ok && j > seg) ok = (__ldg(p.d.indices + j - 1) < i);
+        if (ok && j > seg) {
+            if (lane == 0) prev = __ldg(p.d.indices + j - 1);
+            ok = prev < i;
+        }
         uint16_t *dst = p.snap_ptrs[t];
         if (ok && dst != nullptr && (reinterpret_cast<uintptr_t>(dst) & 1u) == 0) {
             dst[i] = val[r];
@@ -441,7 +481,7 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
 // it in chunks of 32 entries, kScatDepth chunks in flight per warp, and the
 // stretch ends at the first entry past the window, which is where the next
 // window's stretch starts.
-constexpr int kScatThreads = 256;
+constexpr int kScatThreads = 512;
 constexpr int kScatWarps = kScatThreads / 32;
 constexpr int kWinTiles = 32;
 constexpr int kWinElems = kWinTiles * kTileElems;
@@ -461,11 +501,11 @@ struct ScatSmem {
     long long base[kWinTiles];             // per window tensor: (first_tile - window start) * tile
     long long numel[kWinTiles];
     uint16_t *ptr[kWinTiles];
-    long long offs[kWinTiles + 1];         // current delta's offsets of the window tensors
-    unsigned long long next;               // first entry past the window (min over warps)
+    long long offs[2][kWinTiles + 1];      // a delta's offsets of the window tensors (by phase parity)
+    unsigned long long next[2];            // first entry past the window (min over warps)
 };
 
-__global__ void __launch_bounds__(kScatThreads, 4) chain_scatter_kernel(ScatParams p) {
+__global__ void __launch_bounds__(kScatThreads, 2) chain_scatter_kernel(ScatParams p) {
     __shared__ __align__(16) ScatSmem sm;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -518,31 +558,35 @@ __global__ void __launch_bounds__(kScatThreads, 4) chain_scatter_kernel(ScatPara
             sm.ptr[tid] = ptr;
         }
         const long long win_len = (b - a) << kTileShift;
+        constexpr long long kStride = 32LL * kScatWarps;
+        if (tid <= nt) sm.offs[(p.K - 1) & 1][tid] = p.d[p.K - 1].offsets[t_lo + tid];
+        if (tid == 0) sm.next[(p.K - 1) & 1] = ~0ull;
 
+        int ix[kScatDepth];
+        uint16_t vx[kScatDepth];
+        bool prefetched = false;  // the phase's first chunks already requested (uniform)
         for (int k = p.K - 1; k >= 0; --k) {
             const DeltaRef d = p.d[k];
-            if (tid <= nt) sm.offs[tid] = d.offsets[t_lo + tid];
-            if (tid == 0) sm.next = ~0ull;
-            __syncthreads();
-            const long long jmax = sm.offs[nt];
-            constexpr long long kStride = 32LL * kScatWarps;
+            const int ph = k & 1;
+            const long long *offs = sm.offs[ph];
+            if (k == p.K - 1) __syncthreads();  // the window's set-up visible (later phases: below)
+            const long long jmax = offs[nt];
             long long j = sm.cur[k] + 32 * warp + lane;  // this lane's entry of the current chunk
             const int *pi = d.indices + j;
             const uint16_t *pv = d.values + j;
-
-            int ix[kScatDepth];
-            uint16_t vx[kScatDepth];
+            if (!prefetched) {
 #pragma unroll
-            for (int q = 0; q < kScatDepth; ++q) {
-                if (j + q * kStride < jmax) {
-                    ix[q] = __ldg(pi + q * kStride);
-                    vx[q] = __ldg(pv + q * kStride);
+                for (int q = 0; q < kScatDepth; ++q) {
+                    if (j + q * kStride < jmax) {
+                        ix[q] = __ldg(pi + q * kStride);
+                        vx[q] = __ldg(pv + q * kStride);
+                    }
                 }
             }
             // The warp's current tensor (its chunks only move forward) and
             // that tensor's constants: segment, window offset, size, pointer.
             int tw = 0;
-            long long seg_lo = sm.offs[0], seg_hi = sm.offs[1];
+            long long seg_lo = offs[0], seg_hi = offs[1];
             int off_c = static_cast<int>(-sm.base[0]);  // window start - tensor start (elements)
             uint32_t numel_c = static_cast<uint32_t>(sm.numel[0]);
             uint16_t *ptr_c = sm.ptr[0];
@@ -563,9 +607,9 @@ __global__ void __launch_bounds__(kScatThreads, 4) chain_scatter_kernel(ScatPara
                     }
                     const bool valid = j < jmax;
                     if (cstart >= seg_hi) {  // uniform: move to the chunk's first tensor
-                        while (tw + 1 < nt && sm.offs[tw + 1] <= cstart) ++tw;
-                        seg_lo = sm.offs[tw];
-                        seg_hi = sm.offs[tw + 1];
+                        while (tw + 1 < nt && offs[tw + 1] <= cstart) ++tw;
+                        seg_lo = offs[tw];
+                        seg_hi = offs[tw + 1];
                         off_c = static_cast<int>(-sm.base[tw]);
                         numel_c = static_cast<uint32_t>(sm.numel[tw]);
                         ptr_c = sm.ptr[tw];
@@ -586,8 +630,8 @@ __global__ void __launch_bounds__(kScatThreads, 4) chain_scatter_kernel(ScatPara
                     } else if (valid) {
                         // The chunk crosses a tensor boundary: per-lane tensor.
                         int tl = tw;
-                        while (tl + 1 < nt && sm.offs[tl + 1] <= j) ++tl;
-                        if (j < sm.offs[tl] || idx < 0 || static_cast<long long>(idx) >= sm.numel[tl]) {
+                        while (tl + 1 < nt && offs[tl + 1] <= j) ++tl;
+                        if (j < offs[tl] || idx < 0 || static_cast<long long>(idx) >= sm.numel[tl]) {
                             cls = 2;
                         } else {
                             const long long r = sm.base[tl] + idx;
@@ -599,7 +643,7 @@ __global__ void __launch_bounds__(kScatThreads, 4) chain_scatter_kernel(ScatPara
                     const unsigned int past = __ballot_sync(0xffffffffu, cls == 3);
                     if (past != 0u) {
                         const int first = __ffs(past) - 1;
-                        if (lane == first) atomicMin(&sm.next, static_cast<unsigned long long>(j));
+                        if (lane == first) atomicMin(&sm.next[ph], static_cast<unsigned long long>(j));
                         if (lane > first) cls = 0;
                         stop = true;
                     }
@@ -636,9 +680,28 @@ __global__ void __launch_bounds__(kScatThreads, 4) chain_scatter_kernel(ScatPara
                 }
                 if (stop) break;
             }
+            // This warp is done with delta k.  While the others finish,
+            // request the next (earlier) delta's offsets and first chunks:
+            // its stretch starts at its cursor, and reading up to its count
+            // stays inside its arrays.
+            prefetched = false;
+            if (k > 0) {
+                const DeltaRef dn = p.d[k - 1];
+                if (tid <= nt) sm.offs[ph ^ 1][tid] = dn.offsets[t_lo + tid];
+                if (tid == 0) sm.next[ph ^ 1] = ~0ull;
+                const long long jn = sm.cur[k - 1] + 32 * warp + lane;
+#pragma unroll
+                for (int q = 0; q < kScatDepth; ++q) {
+                    if (jn + q * kStride < dn.count) {
+                        ix[q] = __ldg(dn.indices + jn + q * kStride);
+                        vx[q] = __ldg(dn.values + jn + q * kStride);
+                    }
+                }
+                prefetched = true;
+            }
             __syncthreads();  // every entry of this delta stored before the next (earlier) one
             if (tid == 0) {
-                const unsigned long long nx = sm.next;
+                const unsigned long long nx = sm.next[ph];
                 sm.cur[k] = (nx < static_cast<unsigned long long>(jmax)) ? static_cast<long long>(nx) : jmax;
             }
         }

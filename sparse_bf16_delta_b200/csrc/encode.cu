@@ -18,19 +18,22 @@
 //     released: two 1-D bulk async copies (cp.async.bulk, global -> own
 //     shared memory, mbarrier transaction count, L2 evict-first) bring both
 //     snapshots' 16 KiB of the tile.
-//   * Counting group (8 warps): for each stage in ticket order: detect,
-//     block scan, publish the tile's count, move the changed (offset, value)
-//     pairs into a shared ring, queue the tile, release the stage.  A stage
-//     is busy only from its refill to its count, and a tile's count never
-//     waits on any look-back: a ticket held while its CTA waits on a
-//     look-back makes every later tile wait on it in turn (convoys), and a
-//     stage held through a look-back caps the data in flight.
-//   * Look-back group (7 warps): each takes queued tiles in turn, resolves
+//   * Two counting groups of 4 warps take the stage fills in turn (group g
+//     the fills g, g + 2, ...), so two tiles are counted at once and one
+//     group's barriers and latencies overlap the other's work.  Per tile:
+//     detect, block scan, publish the tile's count, move the changed
+//     (offset, value) pairs into the group's shared ring, queue the tile,
+//     release the stage.  A stage is busy only from its refill to its
+//     count, and a tile's count never waits on any look-back: a ticket held
+//     while its CTA waits on a look-back makes every later tile wait on it
+//     in turn (convoys), and a stage held through a look-back caps the data
+//     in flight.
+//   * Look-back group (5 warps): each takes queued tiles in turn, resolves
 //     the tile's exclusive prefix, publishes it, writes the tile's entries
 //     from the ring with consecutive lanes storing consecutive entries
 //     (coalesced), and releases its ring space.
 //   * detect: 16-byte shared-memory reads in a bank-conflict-free order, a
-//     32-bit change mask per thread, popc; block scan of the counts.
+//     64-bit change mask per thread, popc; block scan of the counts.
 //   * scan: decoupled look-back over the tile status words (flag + 62-bit
 //     count); warp 0 reads 256 predecessors per round trip (8 per lane) and,
 //     while waiting, re-reads only the words still unpublished (re-reading
@@ -44,18 +47,21 @@
 namespace dws {
 namespace {
 
-constexpr int kCountWarps = 8;
-constexpr int kCountThreads = 32 * kCountWarps;  // the counting group
-constexpr int kLookWarps = 7;                     // the look-back group
+constexpr int kGroups = 2;      // counting groups; group g counts stage fills g, g + 2, ...
+constexpr int kGroupWarps = 4;  // warps per counting group
+constexpr int kGroupThreads = 32 * kGroupWarps;
+constexpr int kCountWarps = kGroups * kGroupWarps;
+constexpr int kElemsPerThread = kTileElems / kGroupThreads;  // 64
+constexpr int kLookWarps = 5;                     // the look-back group
 constexpr int kProducerWarp = kCountWarps + kLookWarps;
-constexpr int kPublishThread = 64;  // publishes tile counts (thread 0 keeps the queue)
+constexpr int kPublishThread = 64;  // of a group: publishes tile counts (its thread 0 keeps the queue)
 constexpr int kThreads = 32 * (kProducerWarp + 1);
 constexpr int kStages = 4;
-constexpr int kRing = 16384;  // pending (offset | value << 16) entries
-constexpr int kQueue = 64;    // pending tiles
-constexpr int kCountBar = 1;  // named barrier of the counting group
-constexpr int kChunks = kTileElems / 8;  // 16-byte chunks of bf16 per tile
-static_assert(kChunks == 4 * kCountThreads, "each counting thread owns 4 chunks (32 elements)");
+constexpr int kRing = 8192;  // per group: pending (offset | value << 16) entries
+constexpr int kQueue = 64;   // pending tiles
+constexpr int kCountBar = 1;  // named barrier of group g: kCountBar + g
+static_assert(kElemsPerThread == 64, "each counting thread owns 8 chunks of 8 elements");
+static_assert(kStages % kGroups == 0, "a stage always serves the same group");
 static_assert((kRing & (kRing - 1)) == 0 && kRing >= kTileElems, "ring holds any tile");
 
 constexpr unsigned long long kLoadWaitLimitNs = 4000000000ull;  // 4 s
@@ -69,6 +75,7 @@ struct Pending {
     long long ticket;
     int tensor;
     int local_start;
+    int group;  // whose ring holds the entries
     int pos;    // first ring entry
     int total;  // changed elements (ring entries when compacting)
 };
@@ -85,19 +92,20 @@ struct EncodeParams {
 
 struct EncodeSmem {
     uint16_t buf[kStages][2][kTileElems];  // [stage][old | new]
-    uint32_t ring[kRing];
+    uint32_t ring[kGroups][kRing];
     unsigned long long bar[kStages];        // stage filled (transaction count)
     unsigned long long empty_bar[kStages];  // stage released by the counting group
     int fills[kStages];                     // fills issued per stage
     int producer_done;
     StageMeta meta[kStages];
     Pending q[kQueue];
-    int q_done[kQueue];  // i + 1 once queue entry i is written out
-    int q_tail;          // entries queued (release)
-    int q_final;         // total entries once counting has finished, else -1
-    int stop;            // a look-back gave up: everyone leaves
-    int alloc_pos;       // ring position of the tile being queued, -1 = leave
-    int warp_sum[kCountWarps];
+    int q_ready[kQueue];  // i + 1 once queue entry i is complete (release)
+    int q_done[kQueue];   // i + 1 once queue entry i is written out
+    int q_final;          // number of tiles once counting has finished, else INT_MAX
+    int stop;             // a look-back gave up: everyone leaves
+    int alloc_pos[kGroups];  // ring position of the group's tile, -1 = leave
+    int ring_free[kGroups];  // ring entries known to be free when the tile was taken
+    int warp_sum[kGroups][kGroupWarps];
 };
 
 // Thread 0, in two steps: take a ticket (early, so its latency hides behind
@@ -203,7 +211,7 @@ __device__ long long look_back(const EncodeParams &p, const EncodeSmem &sm, long
             }
             if (__shfl_sync(0xffffffffu, give_up, 0)) return -1;
             __nanosleep(backoff);
-            if (backoff < 256) backoff <<= 1;
+            if (backoff < 1024) backoff <<= 1;
             if (blocks) {
 #pragma unroll
                 for (int q = 0; q < kProbePerLane; ++q) {
@@ -224,9 +232,6 @@ __device__ long long look_back(const EncodeParams &p, const EncodeSmem &sm, long
 }
 
 // ---------------------------------------------------------------------------
-// Counting group: threads 0 .. kCountThreads-1
-// ---------------------------------------------------------------------------
-// ---------------------------------------------------------------------------
 // Producer: lane 0 of warp kProducerWarp
 // ---------------------------------------------------------------------------
 __device__ void produce(const EncodeParams &p, EncodeSmem &sm) {
@@ -239,6 +244,7 @@ __device__ void produce(const EncodeParams &p, EncodeSmem &sm) {
     long long tk3 = take_ticket(p);
     TileDesc dk0 = load_desc(p, tk0);
     TileDesc dk1 = load_desc(p, tk1);
+    int markers = 0;
     for (long long k = 0;; ++k) {
         const int s = static_cast<int>(k % kStages);
         if (k >= kStages) {
@@ -258,7 +264,7 @@ __device__ void produce(const EncodeParams &p, EncodeSmem &sm) {
         // Issue first: the arrive has release semantics and would otherwise
         // wait for the lookahead loads below to come back.
         issue_stage(p, sm, s, tk0, dk0);
-        if (tk0 >= p.ws.num_tiles) break;
+        if (tk0 >= p.ws.num_tiles && ++markers == kGroups) break;  // one end marker per group
         tk0 = tk1;
         tk1 = tk2;
         tk2 = tk3;
@@ -270,21 +276,24 @@ __device__ void produce(const EncodeParams &p, EncodeSmem &sm) {
 }
 
 // ---------------------------------------------------------------------------
-// Counting group: threads 0 .. kCountThreads-1
+// Counting groups: group g is threads g * kGroupThreads .. + kGroupThreads - 1
 // ---------------------------------------------------------------------------
 template <bool kCompact>
-__device__ void count_group(const EncodeParams &p, EncodeSmem &sm) {
-    const int tid = threadIdx.x;
+__device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) {
+    const int tid = threadIdx.x - g * kGroupThreads;  // thread within the group
     const int lane = tid & 31;
     const int warp = tid >> 5;
+    const int bar = kCountBar + g;
+    uint32_t *ring = sm.ring[g];
 
-    // Thread 0's bookkeeping of the queue and the ring.
-    int q_tail = 0, q_head = 0;
+    // The group's thread 0 keeps the group's queue entries (g, g + kGroups,
+    // ...) and ring.
+    int q_head = g;
     int ring_tail = 0, ring_head = 0;
 
-    long long waits = 0;  // stage fills consumed so far
+    long long waits = g;  // the group's next stage fill (fills g, g + kGroups, ...)
     bool failed = false;
-    for (;; ++waits) {
+    for (;; waits += kGroups) {
         const int s = static_cast<int>(waits % kStages);
         const uint32_t parity = static_cast<uint32_t>((waits / kStages) & 1);
         const bool loaded = mbar_wait(&sm.bar[s], parity, kLoadWaitLimitNs);
@@ -293,23 +302,23 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm) {
         const bool work = loaded && !done;
         const TileDesc &d = m.d;
         if (tid == 0 && work) {
-            // Room for a whole tile in the ring and one queue slot, so the
-            // writes below need no further check (freed in order by the
-            // look-back group).  The cached head only lags, so the flags are
-            // polled only when the cached view says the ring or queue is full.
+            // A queue slot for this tile (freed in order by the look-back
+            // group).  The cached head only lags, so the flags are polled only
+            // when the cached view says the queue is full.  Ring space is
+            // reserved after the count, for the tile's actual entries.
             unsigned int backoff = 32;
             bool ok = true;
-            while (!(q_tail - q_head < kQueue && ring_tail + kTileElems - ring_head <= kRing)) {
+            while (!(waits - q_head < kQueue)) {
                 // Plain volatile polling: an acquire would also wait for this
                 // thread's outstanding global accesses.  The ring is only
                 // rewritten after the flag is seen, and a look-back warp sets
                 // its flag after all its ring reads have returned.
-                while (q_head < q_tail &&
+                while (q_head < waits &&
                        *reinterpret_cast<volatile int *>(&sm.q_done[q_head % kQueue]) == q_head + 1) {
                     ring_head += kCompact ? sm.q[q_head % kQueue].total : 0;
-                    ++q_head;
+                    q_head += kGroups;
                 }
-                if (q_tail - q_head < kQueue && ring_tail + kTileElems - ring_head <= kRing) break;
+                if (waits - q_head < kQueue) break;
                 if (*reinterpret_cast<volatile int *>(&sm.stop) != 0 ||
                     ld_relaxed_gpu_u32(&p.ws.hdr->abort) != 0u) {
                     ok = false;
@@ -318,17 +327,18 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm) {
                 __nanosleep(backoff);
                 if (backoff < 1024) backoff <<= 1;
             }
-            sm.alloc_pos = ok ? ring_tail : -1;
+            sm.alloc_pos[g] = ok ? ring_tail : -1;
+            sm.ring_free[g] = kRing - (ring_tail - ring_head);
         }
 
         uint16_t *old_s = sm.buf[s][0];
         uint16_t *new_s = sm.buf[s][1];
-        uint32_t mask = 0;
+        uint32_t mask_lo = 0, mask_hi = 0;  // elements 64 tid + [0, 32) and + [32, 64)
         if (work) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int slot = ((tid >> 1) + j) & 3;  // conflict-free 16-byte reads
-                const int e0 = (4 * tid + slot) * 8;
+            for (int j = 0; j < 8; ++j) {
+                const int slot = (tid + j) & 7;  // conflict-free 16-byte reads
+                const int e0 = (8 * tid + slot) * 8;
                 uint4 a, b;
                 if (e0 + 8 <= d.bulk) {
                     a = *reinterpret_cast<const uint4 *>(old_s + e0);
@@ -356,43 +366,73 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm) {
                                        (((x1 & 0xffffu) != 0) << 2) | (((x1 >> 16) != 0) << 3) |
                                        (((x2 & 0xffffu) != 0) << 4) | (((x2 >> 16) != 0) << 5) |
                                        (((x3 & 0xffffu) != 0) << 6) | (((x3 >> 16) != 0) << 7);
-                mask |= bits8 << (8 * slot);
+                if (slot < 4) mask_lo |= bits8 << (8 * slot);
+                else mask_hi |= bits8 << (8 * (slot - 4));
             }
         }
-        const int cnt = __popc(mask);
+        const int cnt = __popc(mask_lo) + __popc(mask_hi);
         int incl = cnt;
 #pragma unroll
         for (int dd = 1; dd < 32; dd <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, incl, dd);
             if (lane >= dd) incl += v;
         }
-        if (lane == 31) sm.warp_sum[warp] = incl;
+        if (lane == 31) sm.warp_sum[g][warp] = incl;
         // (A) warp sums and ring position visible.  If a load wait ran out
         // anywhere, or a look-back gave up, the group leaves together; a fill
         // whose wait ran out is still pending and is drained below.
         const bool go = loaded && (*reinterpret_cast<volatile int *>(&sm.stop) == 0);
-        if (!named_bar_and(kCountBar, kCountThreads, go)) {
+        if (!named_bar_and(bar, kGroupThreads, go)) {
             if (!loaded) record_error(p.ws.hdr, DWS_ERR_TIMEOUT, waits);
-            if (loaded) ++waits;
+            if (loaded) waits += kGroups;
             failed = true;
             break;
         }
         if (done) {  // every thread saw the same loaded meta
-            ++waits;
+            waits += kGroups;
             break;
         }
-        const int pos = sm.alloc_pos;
+        const int pos = sm.alloc_pos[g];
         if (pos < 0) {
-            ++waits;
+            waits += kGroups;
             failed = true;
             break;
         }
         int warp_off = 0, total = 0;
 #pragma unroll
-        for (int w = 0; w < kCountWarps; ++w) {
-            const int v = sm.warp_sum[w];
+        for (int w = 0; w < kGroupWarps; ++w) {
+            const int v = sm.warp_sum[g][w];
             warp_off += (w < warp) ? v : 0;
             total += v;
+        }
+        // Room in the ring for this tile's entries: known free space first,
+        // else thread 0 polls the flags until the look-back group has
+        // written out enough older tiles.
+        if (kCompact && total > sm.ring_free[g]) {  // uniform: all read the same words
+            if (tid == 0) {
+                unsigned int backoff = 32;
+                while (kRing - (ring_tail - ring_head) < total) {
+                    while (q_head < waits &&
+                           *reinterpret_cast<volatile int *>(&sm.q_done[q_head % kQueue]) == q_head + 1) {
+                        ring_head += sm.q[q_head % kQueue].total;
+                        q_head += kGroups;
+                    }
+                    if (kRing - (ring_tail - ring_head) >= total) break;
+                    if (*reinterpret_cast<volatile int *>(&sm.stop) != 0 ||
+                        ld_relaxed_gpu_u32(&p.ws.hdr->abort) != 0u) {
+                        sm.alloc_pos[g] = -1;
+                        break;
+                    }
+                    __nanosleep(backoff);
+                    if (backoff < 1024) backoff <<= 1;
+                }
+            }
+            named_bar(bar, kGroupThreads);  // (B) ring space for this tile
+            if (sm.alloc_pos[g] < 0) {
+                waits += kGroups;
+                failed = true;
+                break;
+            }
         }
         // The count is published by a thread that does no shared-memory
         // release afterwards (a release would wait for this global store).
@@ -401,33 +441,38 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm) {
             st_relaxed_gpu(p.ws.tile_status + m.ticket, flag | static_cast<unsigned long long>(total));
         }
         if (kCompact) {
-            uint32_t mm = mask;
             int rr = pos + warp_off + incl - cnt;
-            while (mm) {
-                const int bit = __ffs(mm) - 1;
-                mm &= mm - 1;
-                const int o = 32 * tid + bit;
-                sm.ring[rr & (kRing - 1)] = static_cast<uint32_t>(o) | (static_cast<uint32_t>(new_s[o]) << 16);
-                ++rr;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t mm = h ? mask_hi : mask_lo;
+                while (mm) {
+                    const int bit = __ffs(mm) - 1;
+                    mm &= mm - 1;
+                    const int o = kElemsPerThread * tid + 32 * h + bit;
+                    ring[rr & (kRing - 1)] = static_cast<uint32_t>(o) | (static_cast<uint32_t>(new_s[o]) << 16);
+                    ++rr;
+                }
             }
         }
-        named_bar(kCountBar, kCountThreads);  // (C) entries in the ring, stage s consumed
+        named_bar(bar, kGroupThreads);  // (C) entries in the ring, stage s consumed
         if (tid == 0) {
-            Pending &e = sm.q[q_tail % kQueue];
+            const int slot = static_cast<int>(waits % kQueue);
+            Pending &e = sm.q[slot];
             e.ticket = m.ticket;
             e.tensor = d.tensor;
             e.local_start = d.local_start;
+            e.group = g;
             e.pos = pos;
             e.total = total;
             ring_tail += kCompact ? total : 0;
-            ++q_tail;
-            st_release_cta(&sm.q_tail, q_tail);
+            st_release_cta(&sm.q_ready[slot], static_cast<int>(waits) + 1);
             mbar_arrive(&sm.empty_bar[s]);  // the producer may refill stage s
         }
     }
 
-    // Counting is over: the look-back group stops after the last entry.
-    if (tid == 0) st_release_cta(&sm.q_final, q_tail);
+    // Counting is over: the look-back group stops after the last tile.  The
+    // end markers are fills N and N + 1 (one per group), N tiles.
+    if (tid == 0 && !failed) atomicMin(&sm.q_final, static_cast<int>(waits - kGroups));
     if (failed) {
         // Leaving on an error: stop the producer, then wait for every fill it
         // issued that has not been consumed.  (A ticket taken but never
@@ -437,9 +482,9 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm) {
         while (ld_acquire_cta(&sm.producer_done) == 0 && global_timer_ns() - t0 < kLoadWaitLimitNs) {
             __nanosleep(256);
         }
-        named_bar(kCountBar, kCountThreads);
-        for (int k = 0; k < kStages; ++k) {
-            // fills of stage k consumed so far (waits counted above)
+        named_bar(bar, kGroupThreads);
+        for (int k = g; k < kStages; k += kGroups) {  // the group's stages
+            // fills of stage k consumed so far (fills before `waits`)
             const long long consumed = (waits + kStages - 1 - k) / kStages;
             if (sm.fills[k] > consumed) {
                 mbar_wait(&sm.bar[k], static_cast<uint32_t>(consumed & 1), kLoadWaitLimitNs);
@@ -459,9 +504,9 @@ __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
         // Wait for queue entry i, or for the end.
         unsigned int backoff = 32;
         for (;;) {
-            if (ld_acquire_cta(&sm.q_tail) > i) break;
+            if (ld_acquire_cta(&sm.q_ready[i % kQueue]) == i + 1) break;
             const int fin = ld_acquire_cta(&sm.q_final);
-            if ((fin >= 0 && i >= fin) || *reinterpret_cast<volatile int *>(&sm.stop) != 0) return;
+            if (i >= fin || *reinterpret_cast<volatile int *>(&sm.stop) != 0) return;
             __nanosleep(backoff);
             if (backoff < 512) backoff <<= 1;
         }
@@ -490,7 +535,7 @@ __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
                 for (int k = lane; k < e.total; k += 32) {
                     const long long out = prefix + k;
                     if (out < p.capacity) {
-                        const uint32_t v = sm.ring[(e.pos + k) & (kRing - 1)];
+                        const uint32_t v = sm.ring[e.group][(e.pos + k) & (kRing - 1)];
                         st_stream_u32(p.indices + out, static_cast<uint32_t>(e.local_start) + (v & 0xffffu));
                         st_stream_u16(p.values + out, static_cast<uint16_t>(v >> 16));
                     }
@@ -521,17 +566,19 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(EncodeParams p) {
             sm.fills[s] = 0;
         }
         mbar_fence_init();
-        sm.q_tail = 0;
-        sm.q_final = -1;
+        sm.q_final = 0x7fffffff;
         sm.stop = 0;
         sm.producer_done = 0;
-        for (int k = 0; k < kQueue; ++k) sm.q_done[k] = 0;
+        for (int k = 0; k < kQueue; ++k) {
+            sm.q_ready[k] = 0;
+            sm.q_done[k] = 0;
+        }
     }
     __syncthreads();
 
     const int warp = tid >> 5;
     if (warp < kCountWarps) {
-        count_group<kCompact>(p, sm);
+        count_group<kCompact>(p, sm, warp / kGroupWarps);
     } else if (warp < kProducerWarp) {
         look_group<kCompact>(p, sm);
     } else if ((tid & 31) == 0) {
