@@ -46,6 +46,10 @@ constexpr int kChainUnitElems = kChainUnitTiles * kTileElems;
 // ---------------------------------------------------------------------------
 constexpr unsigned long long kWsMagic = 0x3130305357534457ull;  // "DWSWS001"
 
+// Two 128-byte lines.  The ticket counter, hit by every producer's atomic,
+// has the second line to itself: waiting warps poll `abort`, and sharing a
+// line (let alone a sector) with the counter would queue those reads behind
+// the atomics at the L2, slowing the tickets in turn.
 struct WsHeader {
     unsigned long long magic;        // 0
     unsigned long long fingerprint;  // 8
@@ -53,10 +57,11 @@ struct WsHeader {
     int num_tensors;                 // 24
     unsigned int status;             // 28  first device error (dws_status_t), 0 = none
     long long detail;                // 32  detail of that error
-    unsigned long long ticket;       // 40  encode: next tile ticket
-    unsigned int abort;              // 48  encode: a bounded wait ran out, all waiters leave
-    unsigned int delta_bad;          // 52  apply/chain: offsets of some delta failed validation
-    unsigned char pad[256 - 56];
+    unsigned int abort;              // 40  encode: a bounded wait ran out, all waiters leave
+    unsigned int delta_bad;          // 44  apply/chain: offsets of some delta failed validation
+    unsigned char pad0[128 - 48];
+    unsigned long long ticket;       // 128 encode: next tile ticket
+    unsigned char pad1[256 - 136];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
 

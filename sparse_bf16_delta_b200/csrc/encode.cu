@@ -28,7 +28,7 @@
 //     while its CTA waits on a look-back makes every later tile wait on it
 //     in turn (convoys), and a stage held through a look-back caps the data
 //     in flight.
-//   * Look-back group (5 warps): each takes queued tiles in turn, resolves
+//   * Look-back group (3 warps): each takes queued tiles in turn, resolves
 //     the tile's exclusive prefix, publishes it, writes the tile's entries
 //     from the ring with consecutive lanes storing consecutive entries
 //     (coalesced), and releases its ring space.
@@ -52,7 +52,7 @@ constexpr int kGroupWarps = 4;  // warps per counting group
 constexpr int kGroupThreads = 32 * kGroupWarps;
 constexpr int kCountWarps = kGroups * kGroupWarps;
 constexpr int kElemsPerThread = kTileElems / kGroupThreads;  // 64
-constexpr int kLookWarps = 5;                     // the look-back group
+constexpr int kLookWarps = 3;                     // the look-back group
 constexpr int kProducerWarp = kCountWarps + kLookWarps;
 constexpr int kPublishThread = 64;  // of a group: publishes tile counts (its thread 0 keeps the queue)
 constexpr int kThreads = 32 * (kProducerWarp + 1);
