@@ -172,7 +172,7 @@ DWS_API dws_status_t dws_count(const dws_plan_t *plan,
  * afford a cudaMalloc and the device-wide synchronisation it implies.  The
  * source pages have no counterpart to this entry point; it computes exactly
  * what dws_encode computes.
- * The scan's scratch lives in a fixed 3 MiB array in device memory that every
+ * The scan's scratch lives in a fixed 5 MiB array in device memory that every
  * GPU loading libdws holds until the process exits; nothing is allocated.
  * numels: host array [num_tensors] of bf16 element counts (0 <= n < 2^31).
  * old_ptrs, new_ptrs, offsets, indices, values, capacity: as in dws_encode.

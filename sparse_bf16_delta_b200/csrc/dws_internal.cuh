@@ -26,6 +26,10 @@ namespace dws {
 // ---------------------------------------------------------------------------
 constexpr int kTileElems = 8192;
 constexpr int kTileShift = 13;
+// Tile status words sit one per 32-byte sector (every fourth word): all
+// look-backs read the newest tiles' words, and packing them densely puts
+// those reads on a few L2 lines (and slices).
+constexpr int kStatusStride = 4;
 static_assert((1 << kTileShift) == kTileElems, "tile size must be a power of two");
 constexpr int kChainUnitTiles = 1;
 constexpr int kChainUnitElems = kChainUnitTiles * kTileElems;
@@ -37,7 +41,7 @@ constexpr int kChainUnitElems = kChainUnitTiles * kTileElems;
 //   numel             int64[T]           tensor sizes          (static)
 //   first_tile        int64[T+1]         first tile of tensor  (static)
 //   tile_tensor       int32[ntiles]      tensor of each tile   (static)
-//   tile_status       uint64[ntiles]     encode scan state     (per call)
+//   tile_status       uint64[ntiles * kStatusStride]  encode scan state (per call)
 //   tile_desc         TileDesc[ntiles]   encode tile pointers  (per call)
 //
 // Every region starts on a 256-byte boundary.  The static regions are written
@@ -89,7 +93,8 @@ inline WsLayout ws_layout(int T, long long ntiles) {
     L.first_tile_off = round_up256(L.numel_off + sizeof(long long) * size_t(T));
     L.tile_tensor_off = round_up256(L.first_tile_off + sizeof(long long) * size_t(T + 1));
     L.tile_status_off = round_up256(L.tile_tensor_off + sizeof(int) * size_t(ntiles));
-    L.tile_desc_off = round_up256(L.tile_status_off + sizeof(unsigned long long) * size_t(ntiles));
+    L.tile_desc_off = round_up256(L.tile_status_off +
+                                  sizeof(unsigned long long) * size_t(ntiles) * kStatusStride);
     L.total = round_up256(L.tile_desc_off + sizeof(TileDesc) * size_t(ntiles));
     return L;
 }

@@ -35,10 +35,14 @@
 //   * detect: 16-byte shared-memory reads in a bank-conflict-free order, a
 //     64-bit change mask per thread, popc; block scan of the counts.
 //   * scan: decoupled look-back over the tile status words (flag + 62-bit
-//     count); warp 0 reads 256 predecessors per round trip (8 per lane) and,
-//     while waiting, re-reads only the words still unpublished (re-reading
-//     whole windows from every waiting warp floods the L2 with requests to
-//     the hottest lines).  Bounded by a wall-clock limit after which the
+//     count), one word per 32-byte sector so that the words every look-back
+//     reads (the newest tiles') spread over four times as many L2 lines.  A
+//     look-back reads the 32 nearest predecessors in one coalesced row, the
+//     next 224 only if those are all aggregates, and while waiting re-reads
+//     only the words still unpublished, with a backoff of 2 to 4 us
+//     (re-reading whole windows, or often, from every waiting warp floods
+//     the L2 slices holding the hottest lines, and every bulk copy through
+//     those slices waits).  Bounded by a wall-clock limit after which the
 //     kernel records DWS_ERR_TIMEOUT and every CTA leaves.
 #include <cuda_runtime.h>
 
@@ -149,52 +153,78 @@ __device__ void issue_stage(const EncodeParams &p, EncodeSmem &sm, int s, long l
     }
 }
 
-// Decoupled look-back, run by one warp.  Lane l reads predecessors
-// base - 8l - q (q = 0..7, newest first), 256 per round trip.  While some
-// needed predecessor is unpublished, only those words are read again (with
-// backoff): an aggregate stays valid even after it turns into a prefix, and
-// re-reading whole windows from every waiting warp floods the L2 with
-// requests to the hottest lines.  Returns -1 if the bounded wait ran out or
-// another tile gave up.
+// Decoupled look-back, run by one warp.  Row q of a window holds the 32
+// predecessors at distances 32q + lane (so a row is one coalesced read of
+// 256 bytes, 8 sectors), nearest row first.  The nearest row is read alone
+// first; the other seven only if it holds neither a prefix nor an
+// unpublished word.  The nearest word that is a prefix ends the look-back
+// (the aggregates before it are summed); the nearest unpublished word
+// blocks it, and while blocked only the unpublished words before the first
+// prefix are read again (with backoff): an aggregate stays valid even after
+// it turns into a prefix, and re-reading whole windows from every waiting
+// warp floods the L2 with requests to the hottest lines.  Returns -1 if the
+// bounded wait ran out or another tile gave up.
 constexpr int kProbePerLane = 8;
 constexpr int kWindow = 32 * kProbePerLane;
 
 __device__ long long look_back(const EncodeParams &p, const EncodeSmem &sm, long long ticket) {
     const int lane = threadIdx.x & 31;
     const unsigned long long *status = p.ws.tile_status;
-    long long base = ticket - 1;
+    long long base = ticket - 1;  // row q, lane l: word base - 32q - l
     unsigned long long acc = 0;
     unsigned long long t0 = 0;
-    unsigned int backoff = 32;
+    unsigned int backoff = 2000;
+    bool first_window = true;
     while (true) {
         unsigned long long w[kProbePerLane];
-#pragma unroll
-        for (int q = 0; q < kProbePerLane; ++q) {
-            const long long j = base - kProbePerLane * lane - q;
-            w[q] = (j >= 0) ? ld_relaxed_gpu(status + j) : kFlagPrefix;
+        {
+            const long long j = base - lane;
+            w[0] = (j >= 0) ? ld_relaxed_gpu(status + j * kStatusStride) : kFlagPrefix;
         }
-        int p_lane;
-        unsigned long long sum;
+        int rows = 1;  // rows read so far (1 or kProbePerLane)
+        if (!first_window) {
+#pragma unroll
+            for (int q = 1; q < kProbePerLane; ++q) {
+                const long long j = base - 32 * q - lane;
+                w[q] = (j >= 0) ? ld_relaxed_gpu(status + j * kStatusStride) : kFlagPrefix;
+            }
+            rows = kProbePerLane;
+        }
+        int stop_q, stop_l;  // the nearest prefix-or-unpublished word (stop_q == rows: none)
+        bool at_prefix;
         while (true) {
-            int first_p = kProbePerLane;
-            bool unready = false;
-            sum = 0;
+            stop_q = rows;
+            stop_l = 0;
+            at_prefix = false;
+            int pq = rows, pl = 0;  // the nearest prefix word
 #pragma unroll
             for (int q = 0; q < kProbePerLane; ++q) {
-                if (first_p == kProbePerLane) {
-                    const unsigned int flag = static_cast<unsigned int>(w[q] >> kFlagShift);
-                    if (flag == 0u) {
-                        unready = true;
-                    } else {
-                        sum += w[q] & kValueMask;
-                        if (flag == 2u) first_p = q;
+                if (q < rows && pq == rows) {  // rows past the nearest prefix do not matter
+                    const unsigned int f = static_cast<unsigned int>(w[q] >> kFlagShift);
+                    const unsigned int pm = __ballot_sync(0xffffffffu, f == 2u);
+                    const unsigned int xm = __ballot_sync(0xffffffffu, f == 0u);
+                    if (stop_q == rows && (pm | xm) != 0u) {
+                        stop_q = q;
+                        stop_l = __ffs(pm | xm) - 1;
+                        at_prefix = (pm >> stop_l) & 1u;
+                    }
+                    if (pq == rows && pm != 0u) {
+                        pq = q;
+                        pl = __ffs(pm) - 1;
                     }
                 }
             }
-            const unsigned int pmask = __ballot_sync(0xffffffffu, first_p < kProbePerLane);
-            p_lane = pmask ? (__ffs(pmask) - 1) : 32;
-            const bool blocks = (lane <= p_lane) && unready;
-            if (!__any_sync(0xffffffffu, blocks)) break;
+            if (stop_q == rows && rows < kProbePerLane) {
+                // the nearest 32 are all aggregates: read the rest of the window
+#pragma unroll
+                for (int q = 1; q < kProbePerLane; ++q) {
+                    const long long j = base - 32 * q - lane;
+                    w[q] = (j >= 0) ? ld_relaxed_gpu(status + j * kStatusStride) : kFlagPrefix;
+                }
+                rows = kProbePerLane;
+                continue;
+            }
+            if (stop_q == rows || at_prefix) break;
 
             int give_up = 0;
             if (lane == 0) {
@@ -211,23 +241,28 @@ __device__ long long look_back(const EncodeParams &p, const EncodeSmem &sm, long
             }
             if (__shfl_sync(0xffffffffu, give_up, 0)) return -1;
             __nanosleep(backoff);
-            if (backoff < 1024) backoff <<= 1;
-            if (blocks) {
+            if (backoff < 4000) backoff <<= 1;
 #pragma unroll
-                for (int q = 0; q < kProbePerLane; ++q) {
-                    if ((w[q] >> kFlagShift) == 0ull) {
-                        const long long j = base - kProbePerLane * lane - q;
-                        w[q] = ld_relaxed_gpu(status + j);
-                    }
+            for (int q = 0; q < kProbePerLane; ++q) {
+                const bool before_p = (q < pq) || (q == pq && lane < pl);
+                if (q < rows && before_p && (w[q] >> kFlagShift) == 0ull) {
+                    const long long j = base - 32 * q - lane;
+                    w[q] = ld_relaxed_gpu(status + j * kStatusStride);
                 }
             }
         }
-        unsigned long long v = (lane <= p_lane) ? sum : 0ull;
+        unsigned long long v = 0;
+#pragma unroll
+        for (int q = 0; q < kProbePerLane; ++q) {
+            const bool take = (q < rows) && (q < stop_q || (q == stop_q && lane <= stop_l));
+            if (take) v += w[q] & kValueMask;
+        }
 #pragma unroll
         for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
         acc += v;
-        if (p_lane < 32) return static_cast<long long>(acc);
+        if (stop_q < rows) return static_cast<long long>(acc);  // ended at a prefix
         base -= kWindow;
+        first_window = false;
     }
 }
 
@@ -438,7 +473,7 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
         // release afterwards (a release would wait for this global store).
         if (tid == kPublishThread && m.ticket != p.withhold) {
             const unsigned long long flag = (m.ticket == 0) ? kFlagPrefix : kFlagAggregate;
-            st_relaxed_gpu(p.ws.tile_status + m.ticket, flag | static_cast<unsigned long long>(total));
+            st_relaxed_gpu(p.ws.tile_status + m.ticket * kStatusStride, flag | static_cast<unsigned long long>(total));
         }
         if (kCompact) {
             int rr = pos + warp_off + incl - cnt;
@@ -522,7 +557,7 @@ __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
         if (prefix >= 0) {
             if (lane == 0) {
                 if (e.ticket != 0)
-                    st_relaxed_gpu(p.ws.tile_status + e.ticket,
+                    st_relaxed_gpu(p.ws.tile_status + e.ticket * kStatusStride,
                                    kFlagPrefix | static_cast<unsigned long long>(prefix + e.total));
                 if (e.local_start == 0) p.offsets[e.tensor] = prefix;
                 if (e.ticket == p.ws.num_tiles - 1) {
@@ -593,7 +628,7 @@ __global__ void prepare_kernel(WsView ws, const uint16_t *const *old_ptrs,
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
          i < ws.num_tiles; i += stride) {
-        ws.tile_status[i] = 0ull;
+        ws.tile_status[i * kStatusStride] = 0ull;
         TileDesc d;
         d.old_p = nullptr;
         d.new_p = nullptr;

@@ -35,7 +35,7 @@ namespace {
 
 constexpr int kNoAllocMaxTensors = 256;
 constexpr long long kNoAllocMaxTiles = 65536;
-constexpr size_t kNoAllocScratchBytes = 3u << 20;  // 3 MiB
+constexpr size_t kNoAllocScratchBytes = 5u << 20;  // 5 MiB
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 

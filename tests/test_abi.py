@@ -72,9 +72,9 @@ def test_plan_tiling_and_workspace_size():
         assert dws.dws_plan_num_tiles(p) == want_tiles
         ws = dws.dws_plan_workspace_bytes(p)
         assert ws % 256 == 0
-        # header + tensor table + 44 bytes per tile (map 4, scan state 8,
-        # descriptor 32), each region 256-aligned
-        lo = 256 + 16 * len(numels) + 8 + 44 * want_tiles
+        # header + tensor table + 68 bytes per tile (map 4, scan state 8 in
+        # a 32-byte slot, descriptor 32), each region 256-aligned
+        lo = 256 + 16 * len(numels) + 8 + 68 * want_tiles
         assert lo <= ws <= lo + 256 * 6
     finally:
         dws.dws_plan_destroy(p)
