@@ -481,11 +481,12 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
 // it in chunks of 32 entries, kScatDepth chunks in flight per warp, and the
 // stretch ends at the first entry past the window, which is where the next
 // window's stretch starts.
-constexpr int kScatThreads = 512;
+constexpr int kScatThreads = 1024;
 constexpr int kScatWarps = kScatThreads / 32;
 constexpr int kWinTiles = 32;
 constexpr int kWinElems = kWinTiles * kTileElems;
 constexpr int kScatDepth = 4;
+constexpr long long kMaxStretch = 1LL << 30;  // entries one phase streams at most
 
 struct ScatParams {
     WsView ws;
@@ -505,7 +506,7 @@ struct ScatSmem {
     unsigned long long next[2];            // first entry past the window (min over warps)
 };
 
-__global__ void __launch_bounds__(kScatThreads, 2) chain_scatter_kernel(ScatParams p) {
+__global__ void __launch_bounds__(kScatThreads, 1) chain_scatter_kernel(ScatParams p) {
     __shared__ __align__(16) ScatSmem sm;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -571,22 +572,34 @@ __global__ void __launch_bounds__(kScatThreads, 2) chain_scatter_kernel(ScatPara
             const long long *offs = sm.offs[ph];
             if (k == p.K - 1) __syncthreads();  // the window's set-up visible (later phases: below)
             const long long jmax = offs[nt];
-            long long j = sm.cur[k] + 32 * warp + lane;  // this lane's entry of the current chunk
-            const int *pi = d.indices + j;
-            const uint16_t *pv = d.values + j;
+            const long long j0 = sm.cur[k];
+            // Positions relative to the stretch start, in 32 bits: a stretch
+            // holds at most one window of valid entries (a delta's indices
+            // are unique); one that runs longer (bad entries) is cut at
+            // kMaxStretch and the next window goes on from there.
+            const long long span = jmax - j0;
+            const int n = static_cast<int>(span < kMaxStretch ? span : kMaxStretch);
+            const int *pi = d.indices + j0;
+            const uint16_t *pv = d.values + j0;
+            int r = 32 * warp + lane;  // this lane's entry of the current chunk
             if (!prefetched) {
 #pragma unroll
                 for (int q = 0; q < kScatDepth; ++q) {
-                    if (j + q * kStride < jmax) {
-                        ix[q] = __ldg(pi + q * kStride);
-                        vx[q] = __ldg(pv + q * kStride);
+                    if (r + q * kStride < n) {
+                        ix[q] = __ldg(pi + r + q * kStride);
+                        vx[q] = __ldg(pv + r + q * kStride);
                     }
                 }
             }
             // The warp's current tensor (its chunks only move forward) and
-            // that tensor's constants: segment, window offset, size, pointer.
+            // that tensor's constants: segment (relative to j0, clamped to
+            // [-1, n]), window offset, size, pointer.
+            auto clamp_rel = [&](long long x) -> int {
+                x -= j0;
+                return static_cast<int>(x < -1 ? -1 : (x > n ? n : x));
+            };
             int tw = 0;
-            long long seg_lo = offs[0], seg_hi = offs[1];
+            int seg_lo = clamp_rel(offs[0]), seg_hi = clamp_rel(offs[1]);
             int off_c = static_cast<int>(-sm.base[0]);  // window start - tensor start (elements)
             uint32_t numel_c = static_cast<uint32_t>(sm.numel[0]);
             uint16_t *ptr_c = sm.ptr[0];
@@ -594,32 +607,32 @@ __global__ void __launch_bounds__(kScatThreads, 2) chain_scatter_kernel(ScatPara
             for (;;) {
 #pragma unroll
                 for (int q = 0; q < kScatDepth; ++q) {
-                    const long long cstart = j - lane;
-                    if (cstart >= jmax) {  // whole chunk past the stretch (uniform)
+                    const int cs = r - lane;
+                    if (cs >= n) {  // whole chunk past the stretch (uniform)
                         stop = true;
                         break;
                     }
                     const int idx = ix[q];
                     const uint16_t val = vx[q];
-                    if (j + kScatDepth * kStride < jmax) {
-                        ix[q] = __ldg(pi + kScatDepth * kStride);
-                        vx[q] = __ldg(pv + kScatDepth * kStride);
+                    if (r + kScatDepth * kStride < n) {
+                        ix[q] = __ldg(pi + r + kScatDepth * kStride);
+                        vx[q] = __ldg(pv + r + kScatDepth * kStride);
                     }
-                    const bool valid = j < jmax;
-                    if (cstart >= seg_hi) {  // uniform: move to the chunk's first tensor
-                        while (tw + 1 < nt && offs[tw + 1] <= cstart) ++tw;
-                        seg_lo = offs[tw];
-                        seg_hi = offs[tw + 1];
+                    const bool valid = r < n;
+                    if (cs >= seg_hi) {  // uniform: move to the chunk's first tensor
+                        while (tw + 1 < nt && offs[tw + 1] <= j0 + cs) ++tw;
+                        seg_lo = clamp_rel(offs[tw]);
+                        seg_hi = clamp_rel(offs[tw + 1]);
                         off_c = static_cast<int>(-sm.base[tw]);
                         numel_c = static_cast<uint32_t>(sm.numel[tw]);
                         ptr_c = sm.ptr[tw];
                     }
-                    const long long clast = (cstart + 31 < jmax) ? cstart + 31 : jmax - 1;
+                    const int cl = (cs + 31 < n) ? cs + 31 : n - 1;
                     // 0: nothing, 1: store, 2: bad entry (consumed), 3: past the window
                     int cls = 0;
                     uint32_t rel = 0;  // element within the window (when cls == 1)
                     uint16_t *dst = ptr_c;
-                    if (cstart >= seg_lo && clast < seg_hi) {
+                    if (cs >= seg_lo && cl < seg_hi) {
                         // Common case, all 32-bit: the chunk lies in one tensor.
                         // (off_c < numel <= 2^31 - 1; rel wraps for indices
                         // below the window, which `before` catches.)
@@ -629,21 +642,22 @@ __global__ void __launch_bounds__(kScatThreads, 2) chain_scatter_kernel(ScatPara
                         if (valid) cls = (!ok || before) ? 2 : (rel >= static_cast<uint32_t>(win_len) ? 3 : 1);
                     } else if (valid) {
                         // The chunk crosses a tensor boundary: per-lane tensor.
+                        const long long j = j0 + r;
                         int tl = tw;
                         while (tl + 1 < nt && offs[tl + 1] <= j) ++tl;
                         if (j < offs[tl] || idx < 0 || static_cast<long long>(idx) >= sm.numel[tl]) {
                             cls = 2;
                         } else {
-                            const long long r = sm.base[tl] + idx;
-                            cls = (r >= win_len) ? 3 : (r < 0 ? 2 : 1);
-                            rel = static_cast<uint32_t>(r);
+                            const long long e = sm.base[tl] + idx;
+                            cls = (e >= win_len) ? 3 : (e < 0 ? 2 : 1);
+                            rel = static_cast<uint32_t>(e);
                             dst = sm.ptr[tl];
                         }
                     }
                     const unsigned int past = __ballot_sync(0xffffffffu, cls == 3);
                     if (past != 0u) {
                         const int first = __ffs(past) - 1;
-                        if (lane == first) atomicMin(&sm.next[ph], static_cast<unsigned long long>(j));
+                        if (lane == first) atomicMin(&sm.next[ph], static_cast<unsigned long long>(j0 + r));
                         if (lane > first) cls = 0;
                         stop = true;
                     }
@@ -656,27 +670,29 @@ __global__ void __launch_bounds__(kScatThreads, 2) chain_scatter_kernel(ScatPara
                         // Mark this delta's elements: one OR per lane, or two
                         // for a run of 32 consecutive elements (a clustered
                         // change), where per-lane ORs would all hit one word.
-                        const uint32_t prev = __shfl_up_sync(0xffffffffu, rel, 1);
-                        const unsigned int run = __ballot_sync(0xffffffffu, ins && (lane == 0 || rel > prev));
                         const uint32_t r0 = __shfl_sync(0xffffffffu, rel, 0);
                         const uint32_t r31 = __shfl_sync(0xffffffffu, rel, 31);
-                        if (run == 0xffffffffu && r31 - r0 == 31u) {
-                            if (lane == 0) atomicOr(&sm.written[r0 >> 5], ~0u << (r0 & 31u));
-                            if (lane == 31 && (r31 & 31u) != 31u)
-                                atomicOr(&sm.written[r31 >> 5], (2u << (r31 & 31u)) - 1u);
-                        } else if (ins) {
-                            atomicOr(&sm.written[word], bit);
+                        bool marked = false;
+                        if (r31 - r0 == 31u) {  // uniform; a run if all 32 ascend
+                            const uint32_t prev = __shfl_up_sync(0xffffffffu, rel, 1);
+                            const unsigned int run =
+                                __ballot_sync(0xffffffffu, ins && (lane == 0 || rel > prev));
+                            if (run == 0xffffffffu) {
+                                if (lane == 0) atomicOr(&sm.written[r0 >> 5], ~0u << (r0 & 31u));
+                                if (lane == 31 && (r31 & 31u) != 31u)
+                                    atomicOr(&sm.written[r31 >> 5], (2u << (r31 & 31u)) - 1u);
+                                marked = true;
+                            }
                         }
+                        if (!marked && ins) atomicOr(&sm.written[word], bit);
                     }
                     if (store) {
                         if (dst != nullptr) dst[idx] = val;
                     } else if (cls == 2) {
-                        record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, j);
+                        record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, j0 + r);
                     }
                     if (stop) break;
-                    j += kStride;
-                    pi += kStride;
-                    pv += kStride;
+                    r += kStride;
                 }
                 if (stop) break;
             }
@@ -702,7 +718,8 @@ __global__ void __launch_bounds__(kScatThreads, 2) chain_scatter_kernel(ScatPara
             __syncthreads();  // every entry of this delta stored before the next (earlier) one
             if (tid == 0) {
                 const unsigned long long nx = sm.next[ph];
-                sm.cur[k] = (nx < static_cast<unsigned long long>(jmax)) ? static_cast<long long>(nx) : jmax;
+                const long long end = j0 + n;
+                sm.cur[k] = (nx < static_cast<unsigned long long>(end)) ? static_cast<long long>(nx) : end;
             }
         }
     }
