@@ -92,6 +92,7 @@ struct EncodeParams {
     long long capacity;
     long long wait_limit_ns;
     long long withhold;
+    int vec_out;  // indices 16-byte and values 8-byte aligned: entries leave four at a time
 };
 
 struct EncodeSmem {
@@ -440,6 +441,15 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
             warp_off += (w < warp) ? v : 0;
             total += v;
         }
+        // The count is published at once, before any wait for ring space:
+        // every later tile's look-back, on every SM, may be waiting for it,
+        // and the rings those look-backs would drain are what this tile may
+        // be waiting for.  Published by a thread that does no shared-memory
+        // release afterwards (a release would wait for this global store).
+        if (tid == kPublishThread && m.ticket != p.withhold) {
+            const unsigned long long flag = (m.ticket == 0) ? kFlagPrefix : kFlagAggregate;
+            st_relaxed_gpu(p.ws.tile_status + m.ticket * kStatusStride, flag | static_cast<unsigned long long>(total));
+        }
         // Room in the ring for this tile's entries: known free space first,
         // else thread 0 polls the flags until the look-back group has
         // written out enough older tiles.
@@ -468,12 +478,6 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
                 failed = true;
                 break;
             }
-        }
-        // The count is published by a thread that does no shared-memory
-        // release afterwards (a release would wait for this global store).
-        if (tid == kPublishThread && m.ticket != p.withhold) {
-            const unsigned long long flag = (m.ticket == 0) ? kFlagPrefix : kFlagAggregate;
-            st_relaxed_gpu(p.ws.tile_status + m.ticket * kStatusStride, flag | static_cast<unsigned long long>(total));
         }
         if (kCompact) {
             int rr = pos + warp_off + incl - cnt;
@@ -531,6 +535,45 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
 // ---------------------------------------------------------------------------
 // Look-back group: warps kCountWarps .. kCountWarps + kLookWarps - 1
 // ---------------------------------------------------------------------------
+// The tile's entries, from the ring to indices[prefix ..] and values[prefix ..]
+// (those below capacity).  Consecutive lanes store consecutive entries; when
+// the outputs are aligned, each lane stores four entries at once (16 bytes of
+// indices, 8 of values) after a head that brings the position to a multiple
+// of four.
+__device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const Pending &e,
+                              long long prefix) {
+    const int lane = threadIdx.x & 31;
+    long long lim = p.capacity - prefix;
+    if (lim > e.total) lim = e.total;
+    const int n = lim > 0 ? static_cast<int>(lim) : 0;
+    const uint32_t ls = static_cast<uint32_t>(e.local_start);
+    auto one = [&](int k) {
+        const uint32_t v = ring[(e.pos + k) & (kRing - 1)];
+        st_stream_u32(p.indices + prefix + k, ls + (v & 0xffffu));
+        st_stream_u16(p.values + prefix + k, static_cast<uint16_t>(v >> 16));
+    };
+    if (!p.vec_out) {
+        for (int k = lane; k < n; k += 32) one(k);
+        return;
+    }
+    const int head = static_cast<int>((4 - (prefix & 3)) & 3) < n ? static_cast<int>((4 - (prefix & 3)) & 3) : n;
+    if (lane < head) one(lane);
+    const int groups = (n - head) >> 2;
+    for (int gi = lane; gi < groups; gi += 32) {
+        const int k = head + 4 * gi;
+        const uint32_t v0 = ring[(e.pos + k) & (kRing - 1)];
+        const uint32_t v1 = ring[(e.pos + k + 1) & (kRing - 1)];
+        const uint32_t v2 = ring[(e.pos + k + 2) & (kRing - 1)];
+        const uint32_t v3 = ring[(e.pos + k + 3) & (kRing - 1)];
+        st_stream_v4(p.indices + prefix + k,
+                     make_uint4(ls + (v0 & 0xffffu), ls + (v1 & 0xffffu), ls + (v2 & 0xffffu), ls + (v3 & 0xffffu)));
+        st_stream_v2(p.values + prefix + k,
+                     make_uint2((v0 >> 16) | (v1 & 0xffff0000u), (v2 >> 16) | (v3 & 0xffff0000u)));
+    }
+    const int tail = head + 4 * groups;
+    if (lane < n - tail) one(tail + lane);
+}
+
 template <bool kCompact>
 __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
     const int lane = threadIdx.x & 31;
@@ -566,16 +609,7 @@ __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
                     if (kCompact && nnz > p.capacity) record_error(p.ws.hdr, DWS_ERR_CAPACITY, nnz);
                 }
             }
-            if (kCompact) {
-                for (int k = lane; k < e.total; k += 32) {
-                    const long long out = prefix + k;
-                    if (out < p.capacity) {
-                        const uint32_t v = sm.ring[e.group][(e.pos + k) & (kRing - 1)];
-                        st_stream_u32(p.indices + out, static_cast<uint32_t>(e.local_start) + (v & 0xffffu));
-                        st_stream_u16(p.values + out, static_cast<uint16_t>(v >> 16));
-                    }
-                }
-            }
+            if (kCompact) write_entries(p, sm.ring[e.group], e, prefix);
         } else if (e.ticket != p.withhold) {
             if (lane == 0) *reinterpret_cast<volatile int *>(&sm.stop) = 1;
         }
@@ -739,6 +773,8 @@ cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
     p.capacity = compact ? capacity : 0;
     p.wait_limit_ns = wait_limit_ns > 0 ? wait_limit_ns : 2000000000LL;
     p.withhold = withhold_tile;
+    p.vec_out = ((reinterpret_cast<uintptr_t>(indices) & 15u) == 0 &&
+                 (reinterpret_cast<uintptr_t>(values) & 7u) == 0) ? 1 : 0;
 
     long long grid = static_cast<long long>(di.sm_count) * di.encode_ctas_per_sm;
     if (grid > ws.num_tiles) grid = ws.num_tiles;

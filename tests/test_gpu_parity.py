@@ -135,6 +135,40 @@ def test_encode_capacity_overflow_reports_required_nnz(dws):
     assert (idx[cap:].cpu().numpy() == -7).all() and (val[cap:].cpu().numpy() == -7).all()
 
 
+@pytest.mark.parametrize("shift", [1, 2, 3])
+def test_encode_into_unaligned_outputs(dws, shift):
+    # indices / values views that start 1-3 entries into their buffers (not
+    # 16- / 8-byte aligned): entries leave one at a time.  Clustered runs of
+    # changes make some tiles dense.
+    rng = np.random.default_rng(37 + shift)
+    sizes = (50_000, 8192 * 3 + 5, 1, 4096)
+    hs, hn = [], []
+    for n in sizes:
+        a = rng.integers(0, 1 << 16, n, dtype=np.uint16)
+        b = a.copy()
+        m = rng.random(n) < 0.05
+        if n > 5000:
+            m[1000:5000] = True
+        b[m] ^= np.uint16(0x0100)
+        hs.append(a)
+        hn.append(b)
+    want = oracle.encode(hs, hn)
+    nnz = int(want[0][-1])
+    olds, news = [dev_bits(a) for a in hs], [dev_bits(b) for b in hn]
+    plan = dws.DeltaPlan.for_tensors(olds)
+    offsets = torch.empty(len(olds) + 1, dtype=torch.int64, device="cuda")
+    ib = torch.full((nnz + 8,), -7, dtype=torch.int32, device="cuda")
+    vb = torch.full((nnz + 8,), -7, dtype=torch.int16, device="cuda")
+    idx, val = ib[shift:shift + nnz], vb[shift:shift + nnz]
+    ot, nt = dws.ptr_table(olds), dws.ptr_table(news)
+    plan.encode_into(ot, nt, offsets, idx, val)
+    plan.raise_on_error()
+    np.testing.assert_array_equal(offsets.cpu().numpy(), want[0])
+    np.testing.assert_array_equal(idx.cpu().numpy(), want[1])
+    np.testing.assert_array_equal(val.cpu().numpy().view(np.uint16), want[2])
+    assert (ib[:shift].cpu().numpy() == -7).all() and (ib[shift + nnz:].cpu().numpy() == -7).all()
+
+
 def test_encode_identical_and_all_changed(dws):
     rng = np.random.default_rng(29)
     a = rng.integers(0, 1 << 16, 1_000_003, dtype=np.uint16)
