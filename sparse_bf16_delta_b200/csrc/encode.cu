@@ -314,6 +314,26 @@ __device__ void produce(const EncodeParams &p, EncodeSmem &sm) {
 // ---------------------------------------------------------------------------
 // Counting groups: group g is threads g * kGroupThreads .. + kGroupThreads - 1
 // ---------------------------------------------------------------------------
+// A warp whose 2048 elements all changed (a clustered run): each thread's
+// 64 entries are its slice itself, read as 16-byte chunks in a rotated,
+// bank-conflict-free order, with no bit scan.  Kept out of line so that the
+// common path's code is left as it is.
+__device__ __noinline__ void dense_slice_to_ring(uint32_t *ring, int rr0, int o0, const uint16_t *new_s,
+                                                 int tid) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const int cr = (c + tid) & 7;
+        const uint4 w = *reinterpret_cast<const uint4 *>(new_s + o0 + 8 * cr);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const int k = 8 * cr + 2 * h;
+            ring[(rr0 + k) & (kRing - 1)] = static_cast<uint32_t>(o0 + k) | (ww[h] << 16);
+            ring[(rr0 + k + 1) & (kRing - 1)] = static_cast<uint32_t>(o0 + k + 1) | (ww[h] & 0xffff0000u);
+        }
+    }
+}
+
 template <bool kCompact>
 __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) {
     const int tid = threadIdx.x - g * kGroupThreads;  // thread within the group
@@ -479,7 +499,9 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
                 break;
             }
         }
-        if (kCompact) {
+        if (kCompact && __all_sync(0xffffffffu, (mask_lo & mask_hi) == 0xffffffffu)) {
+            dense_slice_to_ring(ring, pos + warp_off + incl - cnt, kElemsPerThread * tid, new_s, tid);
+        } else if (kCompact) {
             int rr = pos + warp_off + incl - cnt;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
