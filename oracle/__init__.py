@@ -81,6 +81,14 @@ def _load():
     lib.ref_absorption_changed.argtypes = [ctypes.c_uint16, f32]
     lib.ref_absorption_predict.restype = i64
     lib.ref_absorption_predict.argtypes = [vp, vp, f32, vp, i64]
+    lib.ref_pack_positions.restype = i64
+    lib.ref_pack_positions.argtypes = [i32, vp, vp, vp, vp, vp]
+    lib.ref_hash_bytes.restype = ctypes.c_uint64
+    lib.ref_hash_bytes.argtypes = [vp, i64]
+    lib.ref_hash_bf16.restype = ctypes.c_uint64
+    lib.ref_hash_bf16.argtypes = [vp, i64]
+    lib.ref_bf16_to_f64_bits.restype = ctypes.c_uint64
+    lib.ref_bf16_to_f64_bits.argtypes = [ctypes.c_uint16]
     _lib = lib
     return lib
 
@@ -234,3 +242,44 @@ def absorption_predict(w, u, lr: float):
     if n < 0:
         raise ValueError("non-finite weight")
     return changed, int(n)
+
+
+def pos_width(numel: int) -> int:
+    """Bytes per position of a parameter of `numel` elements (2 or 4)."""
+    return 2 if numel <= 65536 else 4
+
+
+def pack_positions(numels, offsets, indices):
+    """Wire positions: (byte block uint8[total], pos_offsets int64[T+1])."""
+    lib = _load()
+    n = _c(numels, np.int64)
+    o = _c(offsets, np.int64)
+    i = _c(indices, np.int32)
+    T = n.size
+    if o.size != T + 1:
+        raise ValueError("offsets must have T+1 entries")
+    total = int(sum(pos_width(int(n[t])) * int(o[t + 1] - o[t]) for t in range(T)))
+    out = np.zeros(max(1, total), dtype=np.uint8)
+    po = np.zeros(T + 1, dtype=np.int64)
+    got = lib.ref_pack_positions(T, _ptr(n), _ptr(o), _ptr(i), _ptr(out), _ptr(po))
+    if got < 0:
+        raise ValueError("invalid sizes or offsets")
+    return out[:got], po
+
+
+def checksum_parts(positions, values):
+    """(hash of the position bytes, hash of the bf16 values), both uint64."""
+    lib = _load()
+    p = _c(positions, np.uint8)
+    v = _c(np.asarray(values).view(np.uint16), np.uint16)
+    return int(lib.ref_hash_bytes(_ptr(p), p.size)), int(lib.ref_hash_bf16(_ptr(v), v.size))
+
+
+def checksum(positions, values) -> int:
+    """The wire checksum: hash(positions) ^ (hash(values) << 1) (65 bits)."""
+    hp, hv = checksum_parts(positions, values)
+    return hp ^ (hv << 1)
+
+
+def bf16_to_f64_bits(b: int) -> int:
+    return int(_load().ref_bf16_to_f64_bits(b))

@@ -186,3 +186,52 @@ int64_t ref_absorption_predict(const uint16_t *w, const float *u, float lr,
     }
     return count;
 }
+
+/* ------------------------------------------------------------------------
+ * Wire positions and checksum ([verl] review, key source snippets,
+ * encode.py: DeltaParam pos_start / pos_end / pos_width, checksum()).
+ * ------------------------------------------------------------------------ */
+
+int64_t ref_pack_positions(int32_t T, const int64_t *numels, const int64_t *offsets,
+                           const int32_t *indices, uint8_t *positions,
+                           int64_t *pos_offsets)
+{
+    int64_t at = 0;
+    for (int32_t t = 0; t < T; ++t) {
+        if (numels[t] < 0 || offsets[t + 1] < offsets[t]) return -1;
+        const int width = (numels[t] <= 65536) ? 2 : 4;
+        pos_offsets[t] = at;
+        for (int64_t j = offsets[t]; j < offsets[t + 1]; ++j) {
+            const uint32_t x = (uint32_t)indices[j];
+            for (int b = 0; b < width; ++b) positions[at + b] = (uint8_t)(x >> (8 * b));
+            at += width;
+        }
+    }
+    pos_offsets[T] = at;
+    return at;
+}
+
+uint64_t ref_bf16_to_f64_bits(uint16_t b)
+{
+    const uint32_t bits = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    const double d = (double)f;
+    uint64_t u;
+    memcpy(&u, &d, sizeof u);
+    return u;
+}
+
+uint64_t ref_hash_bytes(const uint8_t *b, int64_t n)
+{
+    uint64_t h = 0;
+    for (int64_t i = 0; i < n; ++i) h ^= (uint64_t)b[i];
+    return h;
+}
+
+uint64_t ref_hash_bf16(const uint16_t *v, int64_t n)
+{
+    uint64_t h = 0;
+    for (int64_t i = 0; i < n; ++i) h ^= ref_bf16_to_f64_bits(v[i]);
+    return h;
+}

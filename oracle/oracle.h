@@ -100,6 +100,32 @@ int32_t ref_absorption_changed(uint16_t w, float x);
 int64_t ref_absorption_predict(const uint16_t *w, const float *u, float lr,
                                uint8_t *changed, int64_t n);
 
+/* Wire positions, [verl] review, key source snippets, encode.py: a flush
+ * carries its positions as one uint8 byte block; each parameter's positions
+ * occupy bytes [pos_start, pos_end) of it, pos_width (2 or 4) bytes each.
+ * The page does not say when 2 is used; the reading taken here: 2 bytes when
+ * every position of the parameter fits in 16 bits (numels[t] <= 65536), else
+ * 4.  Positions are written little-endian, parameters in table order.
+ * pos_offsets (T+1 entries) receives the byte starts; pos_offsets[T] = total.
+ * Returns the total number of bytes, or -1 on a negative numel or
+ * non-monotone offsets.  `positions` must hold the total. */
+int64_t ref_pack_positions(int32_t T, const int64_t *numels, const int64_t *offsets,
+                           const int32_t *indices, uint8_t *positions,
+                           int64_t *pos_offsets);
+
+/* The wire checksum, [verl] encode.py checksum(): hash(positions) XOR
+ * (hash(values) << 1), where hash() XOR-reduces the elements after widening
+ * each one to its 64-bit equivalent (an unsigned byte zero-extended; a bf16
+ * value converted to an IEEE double) and reading that as a uint64.  The two
+ * hashes are returned separately: the shift makes the checksum a 65-bit
+ * number. */
+uint64_t ref_hash_bytes(const uint8_t *b, int64_t n);
+uint64_t ref_hash_bf16(const uint16_t *v, int64_t n);
+
+/* The 64-bit pattern of the double equal to a bf16 value (for NaN, the C
+ * conversion on this host). */
+uint64_t ref_bf16_to_f64_bits(uint16_t b);
+
 #ifdef __cplusplus
 }
 #endif

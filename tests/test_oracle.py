@@ -11,6 +11,7 @@ from __future__ import annotations
 import ctypes
 import itertools
 import math
+import struct
 
 import numpy as np
 import pytest
@@ -397,3 +398,76 @@ def test_sparsity_formula_reproduces_the_log_line():
     sparsity = 1 - changed / total
     assert round(100 * sparsity, 2) == float(d["sparsity_percent"][0])
     assert round(sparsity, 4) == float(d["sparsity_metadata"][0])
+
+
+# ---------------------------------------------------------------- wire positions and checksum
+
+
+def test_wire_checksum_golden_worked_example():
+    d = G.keyed("wire_checksum.txt")
+    numels = [int(x) for x in d["numels"]]
+    offsets = np.array([int(x) for x in d["offsets"]], dtype=np.int64)
+    indices = np.array([int(x) for x in d["indices"]], dtype=np.int32)
+    blob, po = oracle.pack_positions(numels, offsets, indices)
+    np.testing.assert_array_equal(blob, G.hex8(d["positions"]))
+    np.testing.assert_array_equal(po, [int(x) for x in d["pos_offsets"]])
+    values = G.hex16(d["values"])
+    hp, hv = oracle.checksum_parts(blob, values)
+    assert hp == int(d["hash_positions"][0], 16)
+    assert hv == int(d["hash_values"][0], 16)
+    assert oracle.checksum(blob, values) == int(d["checksum"][0], 16)
+
+
+def test_pack_positions_brute_force_and_width_rule():
+    rng = np.random.default_rng(91)
+    for _ in range(20):
+        numels = [int(x) for x in rng.choice([0, 1, 100, 65535, 65536, 65537, 10 ** 6], 6)]
+        counts = [0 if n == 0 else int(rng.integers(0, min(n, 50) + 1)) for n in numels]
+        idx, offs = [], [0]
+        for n, c in zip(numels, counts):
+            idx.extend(sorted(rng.choice(n, c, replace=False).tolist()) if c else [])
+            offs.append(offs[-1] + c)
+        blob, po = oracle.pack_positions(numels, np.array(offs), np.array(idx, dtype=np.int32))
+        want, wpo = b"", [0]
+        for t, n in enumerate(numels):
+            fmt = "<H" if n <= 65536 else "<I"
+            for j in range(offs[t], offs[t + 1]):
+                want += struct.pack(fmt, idx[j])
+            wpo.append(len(want))
+        assert blob.tobytes() == want
+        assert po.tolist() == wpo
+
+
+def test_bf16_to_double_bits_all_finite_patterns():
+    # Exact widening: every finite bf16 value is a double; numpy's float32 ->
+    # float64 conversion of the same bits gives the pattern independently.
+    b = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    f64 = (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64).view(np.uint64)
+    got = np.array([oracle.bf16_to_f64_bits(int(x)) for x in b], dtype=np.uint64)
+    finite = ((b >> 7) & 0xFF) != 0xFF
+    np.testing.assert_array_equal(got[finite], f64[finite])
+    # infinities keep their sign, NaNs stay NaN (quiet) with their sign
+    assert oracle.bf16_to_f64_bits(0x7F80) == 0x7FF0000000000000
+    assert oracle.bf16_to_f64_bits(0xFF80) == 0xFFF0000000000000
+    for x in (0x7FC0, 0x7F81, 0xFFC1):
+        u = oracle.bf16_to_f64_bits(x)
+        assert (u >> 52) & 0x7FF == 0x7FF and u & ((1 << 52) - 1) != 0 and (u >> 51) & 1 == 1
+        assert (u >> 63) == (x >> 15)
+
+
+def test_checksum_matches_torch_hash_tensor():
+    # The library routine the pages' checksum() calls, on CPU, over bytes and
+    # over bf16 values of every class (zeros, subnormals, normals, infinities,
+    # NaNs with payloads).
+    import torch
+    rng = np.random.default_rng(92)
+    blob = rng.integers(0, 256, 100_003, dtype=np.uint8)
+    vals = rng.integers(0, 1 << 16, 50_001, dtype=np.uint16)
+    vals[:8] = [0x0000, 0x8000, 0x0001, 0x807F, 0x7F80, 0xFF80, 0x7FC1, 0xFF81]
+    hp, hv = oracle.checksum_parts(blob, vals)
+    assert hp == int(torch.hash_tensor(torch.from_numpy(blob)).item())
+    tv = torch.from_numpy(vals.view(np.int16).copy()).view(torch.bfloat16)
+    assert hv == int(torch.hash_tensor(tv).item())
+    for sub in (vals[:8], vals[8:1000]):
+        t = torch.from_numpy(sub.view(np.int16).copy()).view(torch.bfloat16)
+        assert oracle.checksum_parts(blob[:0], sub)[1] == int(torch.hash_tensor(t).item())
