@@ -761,6 +761,34 @@ def run_ours(args):
                          {"min_ms": round(mn_e, 4), "nnz": nnz2, "sparsity": round(1 - nnz2 / N, 6)})])
         rows.update([row("apply_llama3_8b_lr1e-5", ms_a, 8 * nnz2, weight_bytes, peak,
                          {"min_ms": round(mn_a, 4), "exact": ok})])
+        # wire form of the same delta: positions block (2 or 4 bytes each) and checksum
+        pcap = 4 * nnz2
+        positions = torch.empty(max(2, pcap), dtype=torch.uint8, device=dev)
+        pos_offsets = torch.empty(T + 1, dtype=torch.int64, device=dev)
+        hashes = torch.empty(2, dtype=torch.int64, device=dev)
+        cs = torch.cuda.current_stream().cuda_stream
+
+        def pack():
+            dws.dws_pack_positions(plan.handle, offs2.data_ptr(), idx2.data_ptr(), nnz2,
+                                   positions.data_ptr(), pcap, pos_offsets.data_ptr(),
+                                   plan.workspace.data_ptr(), plan.workspace_bytes, cs)
+
+        ms_p, mn_p = time_reps(pack, args.rows_reps)
+        pbytes = int(pos_offsets[-1].item())
+        offs_h = offs2.cpu().numpy()
+        ok_p = plan.status()[0] == dws.DWS_OK and pbytes == 4 * nnz2 - 2 * sum(
+            int(offs_h[t + 1] - offs_h[t]) for t in range(T) if sizes[t] <= 65536)
+        rows.update([row("pack_positions_llama3_8b_lr1e-5", ms_p, 4 * nnz2 + pbytes + 8 * (T + 1),
+                         weight_bytes, peak, {"min_ms": round(mn_p, 4), "block_bytes": pbytes,
+                                              "sizes_ok": ok_p})])
+
+        def csum():
+            dws.dws_checksum(positions.data_ptr(), pbytes, val2.data_ptr(), nnz2, hashes.data_ptr(), cs)
+
+        ms_k, mn_k = time_reps(csum, args.rows_reps)
+        rows.update([row("checksum_llama3_8b_lr1e-5", ms_k, pbytes + 2 * nnz2, weight_bytes, peak,
+                         {"min_ms": round(mn_k, 4)})])
+        del positions, pos_offsets, hashes
         del old_flat, new_flat, snap_flat, old, new, snap, idx2, val2, d2, offs2
         import gc
         gc.collect()

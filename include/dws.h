@@ -255,6 +255,46 @@ DWS_API dws_status_t dws_apply_chain_ex(const dws_plan_t *plan, void *const *sna
                                 void *workspace, size_t workspace_bytes, dws_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Wire form of a delta, [verl] review of PR #6974, key source snippets,
+ * encode.py: a flush carries its positions as one uint8 byte block, each
+ * parameter's positions at bytes [pos_start, pos_end) with pos_width (2 or
+ * 4) bytes per position, plus the bf16 values and
+ *   checksum = hash(positions) ^ (hash(values) << 1),
+ * hash() being torch.hash_tensor's XOR of the elements widened to 64 bits.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes per position of tensor t: 2 if the tensor has at most 65536
+ * elements (every position fits in 16 bits), else 4.  The pages do not give
+ * the rule; this is the reading taken.  0 for an invalid plan or t. */
+DWS_API int32_t dws_pos_width(const dws_plan_t *plan, int32_t t);
+
+/* The byte block of a delta's positions: tensor t's entries
+ * [offsets[t], offsets[t+1]) as pos_width(t)-byte little-endian integers at
+ * bytes [pos_offsets[t], pos_offsets[t+1]), tensors in plan order.
+ * offsets, indices: one delta in the dws_encode layout (device); count as in
+ * dws_apply.  positions: device, 2-byte aligned, pos_capacity bytes.
+ * pos_offsets: device int64[T+1], written; pos_offsets[T] = block size.
+ * Errors: host -- DWS_ERR_INVALID (null or odd `positions`, negative sizes),
+ * workspace errors as dws_apply; device (dws_status) -- DWS_ERR_BAD_DELTA
+ * for offsets that fail validation (nothing written) or an index outside its
+ * tensor (that position skipped), DWS_ERR_CAPACITY (detail = size needed)
+ * when the block exceeds pos_capacity (positions past it are not written). */
+DWS_API dws_status_t dws_pack_positions(const dws_plan_t *plan, const int64_t *offsets,
+                                const int32_t *indices, int64_t count, uint8_t *positions,
+                                int64_t pos_capacity, int64_t *pos_offsets,
+                                void *workspace, size_t workspace_bytes, dws_stream_t stream);
+
+/* hashes[0] = XOR of the pos_bytes bytes at `positions`, each zero-extended
+ * to 64 bits; hashes[1] = XOR of the 64-bit patterns of the doubles equal to
+ * the nnz bf16 `values` (NaNs quieted, sign and payload kept).  The checksum
+ * is hashes[0] ^ (hashes[1] << 1), 65 bits wide, which is why the two are
+ * returned apart.  hashes: device uint64[2], overwritten.  values 2-byte
+ * aligned.  DWS_ERR_INVALID on null pointers or negative sizes. */
+DWS_API dws_status_t dws_checksum(const uint8_t *positions, int64_t pos_bytes,
+                          const uint16_t *values, int64_t nnz, uint64_t *hashes,
+                          dws_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * XOR-mask variant, [XOR] paragraph 1: mask = old ^ new bit by bit, the same
  * size as the model; the receiver gets new = old ^ mask with no
  * floating-point arithmetic.  Works on any bytes (e.g. packed NVFP4).

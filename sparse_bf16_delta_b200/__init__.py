@@ -70,6 +70,9 @@ _sig("dws_encode_noalloc", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _vp,
 _sig("dws_apply", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_apply_chain", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _vp, _sz, _vp])
 _sig("dws_apply_chain_ex", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _i32, _vp, _sz, _vp])
+_sig("dws_pos_width", _i32, [_vp, _i32])
+_sig("dws_pack_positions", _i32, [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp])
+_sig("dws_checksum", _i32, [_vp, _i64, _vp, _i64, _vp, _vp])
 _sig("dws_xor_encode", _i32, [_vp, _vp, _vp, _i64, _vp])
 _sig("dws_xor_apply", _i32, [_vp, _vp, _i64, _vp])
 _sig("dws_xor_apply_layers", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i64, _vp, _vp])
@@ -176,6 +179,20 @@ def dws_apply_chain_ex(plan, snap_ptrs, deltas, K, mode, workspace, workspace_by
     """dws_apply_chain with an explicit replay mode (DWS_CHAIN_*)."""
     return _lib.dws_apply_chain_ex(plan, snap_ptrs, deltas, K, mode, workspace, workspace_bytes,
                                    stream)
+
+
+def dws_pos_width(plan, t) -> int:
+    return _lib.dws_pos_width(plan, t)
+
+
+def dws_pack_positions(plan, offsets, indices, count, positions, pos_capacity, pos_offsets,
+                       workspace, workspace_bytes, stream) -> int:
+    return _lib.dws_pack_positions(plan, offsets, indices, count, positions, pos_capacity,
+                                   pos_offsets, workspace, workspace_bytes, stream)
+
+
+def dws_checksum(positions, pos_bytes, values, nnz, hashes, stream) -> int:
+    return _lib.dws_checksum(positions, pos_bytes, values, nnz, hashes, stream)
 
 
 def dws_xor_encode(old_bytes, new_bytes, mask, nbytes, stream) -> int:
@@ -368,6 +385,23 @@ class DeltaPlan:
                          self.workspace.data_ptr(), self.workspace_bytes,
                          _stream_handle(stream)), "dws_apply")
 
+    # -- wire form --
+    def pos_width(self, t: int) -> int:
+        return dws_pos_width(self.handle, t)
+
+    def pack_positions(self, delta: Delta, stream=None):
+        """(positions uint8[block size], pos_offsets int64[T+1]) of a delta."""
+        torch = _torch()
+        cap = 4 * delta.count
+        positions = torch.empty(max(2, cap), dtype=torch.uint8, device=self.device)
+        pos_offsets = torch.empty(self.num_tensors + 1, dtype=torch.int64, device=self.device)
+        o, i, _, c = delta.as_ref()
+        _check(dws_pack_positions(self.handle, o, i, c, positions.data_ptr(), cap,
+                                  pos_offsets.data_ptr(), self.workspace.data_ptr(),
+                                  self.workspace_bytes, _stream_handle(stream)), "dws_pack_positions")
+        self.raise_on_error("dws_pack_positions", stream)
+        return positions[:int(pos_offsets[-1].item())], pos_offsets
+
     def apply_chain(self, snap_table, deltas, stream=None, mode=DWS_CHAIN_AUTO):
         arr = make_delta_array([d.as_ref() for d in deltas])
         if mode == DWS_CHAIN_AUTO:
@@ -378,6 +412,20 @@ class DeltaPlan:
             _check(dws_apply_chain_ex(self.handle, snap_table.data_ptr(), arr, len(deltas), mode,
                                       self.workspace.data_ptr(), self.workspace_bytes,
                                       _stream_handle(stream)), "dws_apply_chain_ex")
+
+
+def checksum(positions, pos_bytes: int, values, stream=None) -> int:
+    """The wire checksum hash(positions) ^ (hash(values) << 1) of a byte block
+    and bf16 values (device tensors); synchronises to read the two hashes."""
+    torch = _torch()
+    dev = values.device if values.numel() else positions.device
+    hashes = torch.empty(2, dtype=torch.int64, device=dev)
+    nnz = int(values.numel())
+    _check(dws_checksum(positions.data_ptr() if pos_bytes else 0, int(pos_bytes),
+                        values.data_ptr() if nnz else 0, nnz, hashes.data_ptr(),
+                        _stream_handle(stream)), "dws_checksum")
+    hp, hv = (int(x) & 0xFFFFFFFFFFFFFFFF for x in hashes.cpu().tolist())
+    return hp ^ (hv << 1)
 
 
 def xor_encode(old, new, mask=None, stream=None):

@@ -63,17 +63,6 @@ __global__ void delta_check_kernel(CheckParams p) {
 
 __global__ void delta_flag_clear_kernel(WsView ws) { ws.hdr->delta_bad = 0u; }
 
-// Largest t in [lo, hi] with offsets[t] <= j (offsets validated non-decreasing).
-__device__ __forceinline__ int tensor_of_entry(const long long *offsets, int lo, int hi,
-                                               long long j) {
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (offsets[mid] <= j) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
-
 // ---------------------------------------------------------------------------
 // Single delta: direct scatter
 // ---------------------------------------------------------------------------
@@ -86,27 +75,6 @@ struct ApplyParams {
     uint16_t *const *snap_ptrs;
     DeltaRef d;
 };
-
-// Warp-cooperative: the largest t in [0, T-1] with offsets[t] <= j (offsets
-// non-decreasing, offsets[0] = 0 <= j).  Each round probes 32 evenly spaced
-// tensors, so T = 291 takes two dependent loads and T = 12000 three.
-__device__ int warp_tensor_of_entry(const long long *offsets, int T, long long j) {
-    const int lane = threadIdx.x & 31;
-    int lo = 0, hi = T - 1;  // the answer lies in [lo, hi]
-    while (true) {
-        const int span = hi - lo + 1;
-        const int step = (span + 31) / 32;
-        const int t = lo + lane * step;
-        const bool le = (t <= hi) && (__ldg(offsets + t) <= j);
-        const unsigned int b = __ballot_sync(0xffffffffu, le);  // a prefix of lanes; lane 0 set
-        const int c = __popc(b);
-        if (step == 1) return lo + c - 1;
-        const int nlo = lo + (c - 1) * step;
-        const int nhi = lo + c * step - 1;
-        lo = nlo;
-        hi = nhi < hi ? nhi : hi;
-    }
-}
 
 __global__ void __launch_bounds__(kApplyThreads) apply_kernel(ApplyParams p) {
     __shared__ int s_t[2];

@@ -287,6 +287,42 @@ dws_status_t dws_apply_chain_ex(const dws_plan_t *plan, void *const *snap_ptrs,
                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int32_t dws_pos_width(const dws_plan_t *plan, int32_t t) {
+    if (plan == nullptr || t < 0 || t >= plan->T) return 0;
+    const long long *numel =
+        reinterpret_cast<const long long *>(plan->image.data() + plan->layout.numel_off);
+    return numel[t] <= 65536 ? 2 : 4;
+}
+
+dws_status_t dws_pack_positions(const dws_plan_t *plan, const int64_t *offsets,
+                                const int32_t *indices, int64_t count, uint8_t *positions,
+                                int64_t pos_capacity, int64_t *pos_offsets, void *workspace,
+                                size_t workspace_bytes, dws_stream_t stream) {
+    dws_status_t st = check_ws(plan, workspace, workspace_bytes);
+    if (st != DWS_OK) return st;
+    if (offsets == nullptr || pos_offsets == nullptr || count < 0 || pos_capacity < 0)
+        return DWS_ERR_INVALID;
+    if (count > 0 && indices == nullptr) return DWS_ERR_INVALID;
+    if (pos_capacity > 0 && (positions == nullptr || (reinterpret_cast<uintptr_t>(positions) & 1u)))
+        return DWS_ERR_INVALID;
+    dws::DeltaRef d{reinterpret_cast<const long long *>(offsets),
+                    reinterpret_cast<const int *>(indices), nullptr, count};
+    return from_cuda(dws::launch_pack_positions(view_of(plan, workspace), d, positions, pos_capacity,
+                                                reinterpret_cast<long long *>(pos_offsets),
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dws_status_t dws_checksum(const uint8_t *positions, int64_t pos_bytes, const uint16_t *values,
+                          int64_t nnz, uint64_t *hashes, dws_stream_t stream) {
+    if (hashes == nullptr || pos_bytes < 0 || nnz < 0) return DWS_ERR_INVALID;
+    if ((pos_bytes > 0 && positions == nullptr) || (nnz > 0 && values == nullptr))
+        return DWS_ERR_INVALID;
+    if (reinterpret_cast<uintptr_t>(values) & 1u) return DWS_ERR_INVALID;
+    return from_cuda(dws::launch_checksum(positions, pos_bytes, values, nnz,
+                                          reinterpret_cast<unsigned long long *>(hashes),
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
 dws_status_t dws_xor_encode(const void *old_bytes, const void *new_bytes, void *mask,
                             int64_t nbytes, dws_stream_t stream) {
     if (nbytes < 0) return DWS_ERR_INVALID;

@@ -318,6 +318,39 @@ __device__ __forceinline__ void st_stream_u16(void *p, uint16_t v) {
     asm volatile("st.global.cs.u16 [%0], %1;" ::"l"(p), "h"(v) : "memory");
 }
 
+// Tensor of delta entry j (a delta's offsets are non-decreasing).
+// Largest t in [lo, hi] with offsets[t] <= j (offsets validated non-decreasing).
+__device__ __forceinline__ int tensor_of_entry(const long long *offsets, int lo, int hi,
+                                               long long j) {
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offsets[mid] <= j) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Warp-cooperative: the largest t in [0, T-1] with offsets[t] <= j (offsets
+// non-decreasing, offsets[0] = 0 <= j).  Each round probes 32 evenly spaced
+// tensors, so T = 291 takes two dependent loads and T = 12000 three.
+__device__ __forceinline__ int warp_tensor_of_entry(const long long *offsets, int T, long long j) {
+    const int lane = threadIdx.x & 31;
+    int lo = 0, hi = T - 1;  // the answer lies in [lo, hi]
+    while (true) {
+        const int span = hi - lo + 1;
+        const int step = (span + 31) / 32;
+        const int t = lo + lane * step;
+        const bool le = (t <= hi) && (__ldg(offsets + t) <= j);
+        const unsigned int b = __ballot_sync(0xffffffffu, le);  // a prefix of lanes; lane 0 set
+        const int c = __popc(b);
+        if (step == 1) return lo + c - 1;
+        const int nlo = lo + (c - 1) * step;
+        const int nhi = lo + c * step - 1;
+        lo = nlo;
+        hi = nhi < hi ? nhi : hi;
+    }
+}
+
 #endif  // __CUDACC__
 
 // ---------------------------------------------------------------------------
@@ -357,6 +390,11 @@ cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs,
                                long long total_elems, cudaStream_t s);
 cudaError_t launch_apply_chain_scatter(const WsView &ws, uint16_t *const *snap_ptrs,
                                        const DeltaRef *deltas, int K, cudaStream_t s);
+
+cudaError_t launch_pack_positions(const WsView &ws, const DeltaRef &d, uint8_t *positions,
+                                  long long pos_capacity, long long *pos_offsets, cudaStream_t s);
+cudaError_t launch_checksum(const uint8_t *positions, long long nbytes, const uint16_t *values,
+                            long long nval, unsigned long long *out, cudaStream_t s);
 
 cudaError_t launch_xor(const uint8_t *a, const uint8_t *b, uint8_t *out, long long nbytes,
                        cudaStream_t s);

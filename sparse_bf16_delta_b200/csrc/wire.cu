@@ -1,0 +1,264 @@
+// wire.cu -- the wire form of a delta: per-parameter position widths and the
+// integrity checksum ([verl] review of PR #6974, key source snippets,
+// encode.py: DeltaParam pos_start / pos_end / pos_width, DeltaFlush
+// positions and values, checksum()).
+//
+// dws_pack_positions: the positions of a delta as one byte block, parameter
+//   by parameter in plan order, each position in pos_width bytes
+//   little-endian.  pos_width is 2 for a parameter of at most 65536 elements
+//   (every position fits in 16 bits) and 4 otherwise.  A one-CTA pass scans
+//   the per-parameter byte counts into pos_offsets; then every block of 2048
+//   entries finds its parameters (warp-cooperative search over the delta's
+//   offsets) and stores 2-byte halves.
+//
+// dws_checksum: hash(positions) and hash(values), where hash() XOR-reduces
+//   the elements widened to 64 bits: a byte zero-extended, a bf16 value
+//   converted to the IEEE double equal to it and read as a uint64 (NaNs
+//   quieted with their sign and payload kept).  The checksum of the pages is
+//   hash(positions) ^ (hash(values) << 1), a 65-bit number, so the two
+//   hashes are returned separately.  One grid-stride pass with 16-byte
+//   loads; each CTA XORs its result into the outputs once.
+#include <cuda_runtime.h>
+
+#include "dws_internal.cuh"
+
+namespace dws {
+namespace {
+
+constexpr long long kSmallTensor = 65536;  // at most this many elements: 2-byte positions
+constexpr int kPackThreads = 256;
+constexpr int kPackPerThread = 8;
+constexpr int kPackEntries = kPackThreads * kPackPerThread;
+constexpr int kScanThreads = 1024;
+
+__device__ __forceinline__ int pos_width_of(long long numel) { return numel <= kSmallTensor ? 2 : 4; }
+
+// pos_offsets[t] = sum over t' < t of width(t') * (offsets[t'+1] - offsets[t']);
+// pos_offsets[T] = the block's size.  One CTA, chunks of kScanThreads tensors.
+__global__ void __launch_bounds__(kScanThreads) pos_offsets_kernel(WsView ws, const long long *offsets,
+                                                                   long long *pos_offsets,
+                                                                   long long pos_capacity) {
+    __shared__ long long warp_sums[kScanThreads / 32];
+    __shared__ long long carry;
+    if (!ws_matches(ws)) return;
+    if (ld_relaxed_gpu_u32(&ws.hdr->delta_bad) != 0u) return;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int T = ws.num_tensors;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < T; base += kScanThreads) {
+        const int t = base + tid;
+        long long v = 0;
+        if (t < T) v = pos_width_of(ws.numel[t]) * (offsets[t + 1] - offsets[t]);
+        long long incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const long long u = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += u;
+        }
+        if (lane == 31) warp_sums[warp] = incl;
+        __syncthreads();
+        long long before = carry;
+        for (int w = 0; w < warp; ++w) before += warp_sums[w];
+        if (t < T) pos_offsets[t] = before + incl - v;
+        __syncthreads();
+        if (tid == kScanThreads - 1) carry = before + incl;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        pos_offsets[T] = carry;
+        if (carry > pos_capacity) record_error(ws.hdr, DWS_ERR_CAPACITY, carry);
+    }
+}
+
+struct PackParams {
+    WsView ws;
+    DeltaRef d;
+    const long long *pos_offsets;
+    uint8_t *positions;
+    long long pos_capacity;
+};
+
+__global__ void __launch_bounds__(kPackThreads) pack_positions_kernel(PackParams p) {
+    __shared__ int s_t[2];
+    __shared__ int s_go;
+    __shared__ long long s_end;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int T = p.ws.num_tensors;
+    const long long base = static_cast<long long>(blockIdx.x) * kPackEntries;
+    const long long cap = p.d.count;
+    if (base >= cap) return;  // uniform
+    int idx[kPackPerThread];
+#pragma unroll
+    for (int r = 0; r < kPackPerThread; ++r) {
+        const long long j = base + tid + r * kPackThreads;
+        if (j < cap) idx[r] = __ldg(p.d.indices + j);
+    }
+    if (warp < 2) {
+        const long long last = (base + kPackEntries < cap ? base + kPackEntries : cap) - 1;
+        const int t = warp_tensor_of_entry(p.d.offsets, T, warp == 0 ? base : last);
+        if (lane == 0) s_t[warp] = t;
+    }
+    if (tid == 64) {
+        const WsHeader *h = p.ws.hdr;
+        const bool ok = (h->magic == kWsMagic && h->fingerprint == p.ws.fingerprint &&
+                         h->num_tiles == p.ws.num_tiles && h->num_tensors == T);
+        if (!ok) record_error(p.ws.hdr, DWS_ERR_WORKSPACE, 0);
+        const long long nnz = p.d.offsets[T];
+        const long long total = nnz < cap ? nnz : cap;
+        s_end = (base + kPackEntries < total) ? base + kPackEntries : total;
+        s_go = ok && (ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) == 0u) && base < s_end;
+    }
+    __syncthreads();
+    if (!s_go) return;
+    const long long end = s_end;
+    const int t0 = s_t[0], t1 = s_t[1];
+#pragma unroll
+    for (int r = 0; r < kPackPerThread; ++r) {
+        const long long j = base + tid + r * kPackThreads;
+        if (j >= end) continue;
+        const int t = (t0 == t1) ? t0 : tensor_of_entry(p.d.offsets, t0, t1, j);
+        const long long n = p.ws.numel[t];
+        const int i = idx[r];
+        if (i < 0 || static_cast<long long>(i) >= n) {
+            record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, j);
+            continue;
+        }
+        const int w = pos_width_of(n);
+        const long long at = p.pos_offsets[t] + (j - p.d.offsets[t]) * w;
+        if (at + w > p.pos_capacity) continue;  // recorded by the offsets pass
+        uint16_t *dst = reinterpret_cast<uint16_t *>(p.positions + at);  // at is even
+        dst[0] = static_cast<uint16_t>(i & 0xffff);
+        if (w == 4) dst[1] = static_cast<uint16_t>(static_cast<uint32_t>(i) >> 16);
+    }
+}
+
+// The double equal to a bf16 value, as bits: sign, exponent rebased from
+// 127 to 1023, mantissa moved up; subnormals normalised; infinities kept;
+// NaNs quieted (bit 51 set) with sign and payload kept.
+__device__ __forceinline__ unsigned long long bf16_to_f64_bits(uint32_t b) {
+    const unsigned long long sign = static_cast<unsigned long long>(b >> 15) << 63;
+    const uint32_t e = (b >> 7) & 0xffu;
+    const uint32_t m = b & 0x7fu;
+    if (e == 0xffu) {
+        const unsigned long long q = m ? ((1ull << 51) | (static_cast<unsigned long long>(m) << 45)) : 0ull;
+        return sign | (0x7ffull << 52) | q;
+    }
+    if (e == 0u) {
+        if (m == 0u) return sign;
+        const int top = 31 - __clz(m);  // m = 2^top + rest, value = m * 2^-133
+        const unsigned long long frac = static_cast<unsigned long long>(m - (1u << top)) << (52 - top);
+        return sign | (static_cast<unsigned long long>(top + 1023 - 133) << 52) | frac;
+    }
+    return sign | (static_cast<unsigned long long>(e - 127 + 1023) << 52) |
+           (static_cast<unsigned long long>(m) << 45);
+}
+
+constexpr int kSumThreads = 512;
+
+__device__ __forceinline__ unsigned long long fold_bytes(unsigned long long x) {
+    x ^= x >> 32;
+    x ^= x >> 16;
+    x ^= x >> 8;
+    return x & 0xffull;
+}
+
+__global__ void __launch_bounds__(kSumThreads) checksum_kernel(const uint8_t *pos, long long nbytes,
+                                                               const uint16_t *val, long long nval,
+                                                               unsigned long long *out) {
+    const long long stride = static_cast<long long>(gridDim.x) * kSumThreads;
+    const long long gid = static_cast<long long>(blockIdx.x) * kSumThreads + threadIdx.x;
+    unsigned long long hp = 0, hv = 0;
+    // bytes: unaligned head and tail one by one, the middle as 16-byte words
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(pos);
+    long long head = static_cast<long long>((16 - (pa & 15u)) & 15u);
+    if (head > nbytes) head = nbytes;
+    const long long nvec = (nbytes - head) >> 4;
+    if (gid < head) hp ^= pos[gid];
+    const uint4 *pv = reinterpret_cast<const uint4 *>(pos + head);
+    unsigned long long words = 0;
+    for (long long k = gid; k < nvec; k += stride) {
+        const uint4 w = ld_stream_v4(pv + k);
+        words ^= (static_cast<unsigned long long>(w.y) << 32 | w.x) ^ (static_cast<unsigned long long>(w.w) << 32 | w.z);
+    }
+    hp ^= fold_bytes(words);
+    for (long long k = head + (nvec << 4) + gid; k < nbytes; k += stride) hp ^= pos[k];
+    // values: unaligned head, 8 per 16-byte word, tail
+    const uintptr_t va = reinterpret_cast<uintptr_t>(val);
+    long long vhead = ((va & 15u) == 0) ? 0 : static_cast<long long>((16 - (va & 15u)) >> 1);
+    if ((va & 1u) != 0u || vhead > nval) vhead = nval;  // odd address: all one by one
+    const long long vvec = (nval - vhead) >> 3;
+    if (gid < vhead) hv ^= bf16_to_f64_bits(val[gid]);
+    const uint4 *vv = reinterpret_cast<const uint4 *>(val + vhead);
+    for (long long k = gid; k < vvec; k += stride) {
+        const uint4 w = ld_stream_v4(vv + k);
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            hv ^= bf16_to_f64_bits(ws[q] & 0xffffu) ^ bf16_to_f64_bits(ws[q] >> 16);
+    }
+    for (long long k = vhead + (vvec << 3) + gid; k < nval; k += stride) hv ^= bf16_to_f64_bits(val[k]);
+    // CTA reduction, one atomic per output per CTA
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) {
+        hp ^= __shfl_xor_sync(0xffffffffu, hp, d);
+        hv ^= __shfl_xor_sync(0xffffffffu, hv, d);
+    }
+    __shared__ unsigned long long sp[kSumThreads / 32], sv[kSumThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) {
+        sp[warp] = hp;
+        sv[warp] = hv;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned long long a = 0, b = 0;
+        for (int w = 0; w < kSumThreads / 32; ++w) {
+            a ^= sp[w];
+            b ^= sv[w];
+        }
+        if (a) atomicXor(out, a);
+        if (b) atomicXor(out + 1, b);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_pack_positions(const WsView &ws, const DeltaRef &d, uint8_t *positions,
+                                  long long pos_capacity, long long *pos_offsets, cudaStream_t s) {
+    cudaError_t e = launch_delta_check(ws, &d, 1, s);
+    if (e != cudaSuccess) return e;
+    pos_offsets_kernel<<<1, kScanThreads, 0, s>>>(ws, d.offsets, pos_offsets, pos_capacity);
+    e = launched();
+    if (e != cudaSuccess) return e;
+    if (d.count <= 0) return cudaSuccess;
+    PackParams p;
+    p.ws = ws;
+    p.d = d;
+    p.pos_offsets = pos_offsets;
+    p.positions = positions;
+    p.pos_capacity = pos_capacity;
+    const long long blocks = (d.count + kPackEntries - 1) / kPackEntries;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    pack_positions_kernel<<<static_cast<unsigned int>(blocks), kPackThreads, 0, s>>>(p);
+    return launched();
+}
+
+cudaError_t launch_checksum(const uint8_t *positions, long long nbytes, const uint16_t *values,
+                            long long nval, unsigned long long *out, cudaStream_t s) {
+    DeviceInfo di;
+    cudaError_t e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(out, 0, 2 * sizeof(unsigned long long), s);
+    if (e != cudaSuccess) return e;
+    const long long work = (nbytes >> 4) + (nval >> 3) + 1;
+    long long grid = (work + kSumThreads - 1) / kSumThreads;
+    const long long cap = 4LL * di.sm_count;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    checksum_kernel<<<static_cast<unsigned int>(grid), kSumThreads, 0, s>>>(positions, nbytes, values,
+                                                                            nval, out);
+    return launched();
+}
+
+}  // namespace dws
