@@ -198,7 +198,7 @@ def encode_traffic_per_elem():
     vals = {}
     for ln in open(summ):
         if ln.startswith("- ") and ":" in ln:
-            k, _, v = ln[2:].partition(":")
+            k, _, v = ln[2:].rpartition(": ")
             vals[k.strip()] = v.strip().strip("`")
     if vals.get("encode.cu sha256[:16]") != h:
         return None, None
