@@ -442,7 +442,8 @@ def test_bf16_to_double_bits_all_finite_patterns():
     # Exact widening: every finite bf16 value is a double; numpy's float32 ->
     # float64 conversion of the same bits gives the pattern independently.
     b = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
-    f64 = (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64).view(np.uint64)
+    with np.errstate(invalid="ignore"):  # NaN patterns are compared apart below
+        f64 = (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64).view(np.uint64)
     got = np.array([oracle.bf16_to_f64_bits(int(x)) for x in b], dtype=np.uint64)
     finite = ((b >> 7) & 0xFF) != 0xFF
     np.testing.assert_array_equal(got[finite], f64[finite])
