@@ -144,6 +144,20 @@ DWS_API dws_status_t dws_encode(const dws_plan_t *plan,
                         int64_t capacity,
                         void *workspace, size_t workspace_bytes, dws_stream_t stream);
 
+/* dws_encode with global int64 positions: [verl] sparse_gather.py
+ * shard_delta_indices diffs a rank's local shard of a parameter and returns
+ * global_idx = local_idx (as int64) + offset, the shard's first element in the
+ * full parameter.  Here entry j of tensor t holds index_base[t] + its local
+ * index.  index_base: device int64[num_tensors] (caller-owned; e.g. for an
+ * FSDP Shard(0) slice, its first row times the elements per row).
+ * indices: device int64[capacity].  Everything else, including errors, as
+ * dws_encode; DWS_ERR_INVALID also for a null index_base. */
+DWS_API dws_status_t dws_encode_global(const dws_plan_t *plan,
+                               const void *const *old_ptrs, const void *const *new_ptrs,
+                               const int64_t *index_base, int64_t *offsets, int64_t *indices,
+                               uint16_t *values, int64_t capacity,
+                               void *workspace, size_t workspace_bytes, dws_stream_t stream);
+
 /* dws_encode with explicit controls of the scan's bounded wait.
  * wait_limit_ns: how long a tile waits for its predecessor's count before it
  *   records DWS_ERR_TIMEOUT and every waiting tile gives up (<= 0: 2 s).

@@ -283,3 +283,14 @@ def checksum(positions, values) -> int:
 
 def bf16_to_f64_bits(b: int) -> int:
     return int(_load().ref_bf16_to_f64_bits(b))
+
+
+def encode_global(olds, news, index_base):
+    """Encode with global int64 positions ([verl] review, key source snippets,
+    sparse_gather.py shard_delta_indices: global_idx = local_idx + offset):
+    (offsets, int64 positions, values), entry j of tensor t at
+    index_base[t] + its local index."""
+    offsets, indices, values = encode(olds, news)
+    counts = np.diff(offsets)
+    base = np.repeat(np.asarray(index_base, dtype=np.int64), counts)
+    return offsets, indices.astype(np.int64) + base, values

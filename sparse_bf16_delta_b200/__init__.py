@@ -71,6 +71,7 @@ _sig("dws_apply", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_apply_chain", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _vp, _sz, _vp])
 _sig("dws_apply_chain_ex", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _i32, _vp, _sz, _vp])
 _sig("dws_pos_width", _i32, [_vp, _i32])
+_sig("dws_encode_global", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_pack_positions", _i32, [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp])
 _sig("dws_checksum", _i32, [_vp, _i64, _vp, _i64, _vp, _vp])
 _sig("dws_xor_encode", _i32, [_vp, _vp, _vp, _i64, _vp])
@@ -179,6 +180,12 @@ def dws_apply_chain_ex(plan, snap_ptrs, deltas, K, mode, workspace, workspace_by
     """dws_apply_chain with an explicit replay mode (DWS_CHAIN_*)."""
     return _lib.dws_apply_chain_ex(plan, snap_ptrs, deltas, K, mode, workspace, workspace_bytes,
                                    stream)
+
+
+def dws_encode_global(plan, old_ptrs, new_ptrs, index_base, offsets, indices, values, capacity,
+                      workspace, workspace_bytes, stream) -> int:
+    return _lib.dws_encode_global(plan, old_ptrs, new_ptrs, index_base, offsets, indices, values,
+                                  capacity, workspace, workspace_bytes, stream)
 
 
 def dws_pos_width(plan, t) -> int:
@@ -384,6 +391,22 @@ class DeltaPlan:
         _check(dws_apply(self.handle, snap_table.data_ptr(), o, i, v, c,
                          self.workspace.data_ptr(), self.workspace_bytes,
                          _stream_handle(stream)), "dws_apply")
+
+    def encode_global(self, old_table, new_table, index_base, stream=None) -> Delta:
+        """Encode with int64 global positions (index_base[t] + local index);
+        index_base: device int64 tensor [T].  Sized exactly (count first)."""
+        torch = _torch()
+        offsets = self.count(old_table, new_table, stream=stream)
+        nnz = int(offsets[-1].item())
+        indices = torch.empty(nnz, dtype=torch.int64, device=self.device)
+        values = torch.empty(nnz, dtype=torch.int16, device=self.device)
+        _check(dws_encode_global(self.handle, old_table.data_ptr(), new_table.data_ptr(),
+                                 index_base.data_ptr(), offsets.data_ptr(),
+                                 indices.data_ptr() if nnz else 0, values.data_ptr() if nnz else 0,
+                                 nnz, self.workspace.data_ptr(), self.workspace_bytes,
+                                 _stream_handle(stream)), "dws_encode_global")
+        self.raise_on_error("dws_encode_global", stream)
+        return Delta(offsets, indices, values)
 
     # -- wire form --
     def pos_width(self, t: int) -> int:

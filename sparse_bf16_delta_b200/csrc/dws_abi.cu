@@ -118,20 +118,23 @@ dws_status_t encode_common(const dws_plan_t *plan, const void *const *old_ptrs,
                            const void *const *new_ptrs, int64_t *offsets, int32_t *indices,
                            uint16_t *values, int64_t capacity, void *workspace,
                            size_t workspace_bytes, dws_stream_t stream, bool compact,
-                           int64_t wait_limit_ns, int64_t withhold) {
+                           int64_t wait_limit_ns, int64_t withhold, int64_t *indices64 = nullptr,
+                           const int64_t *index_base = nullptr) {
     dws_status_t st = check_ws(plan, workspace, workspace_bytes);
     if (st != DWS_OK) return st;
     if (old_ptrs == nullptr || new_ptrs == nullptr || offsets == nullptr) return DWS_ERR_INVALID;
     if (compact) {
         if (capacity < 0) return DWS_ERR_INVALID;
-        if (capacity > 0 && (indices == nullptr || values == nullptr)) return DWS_ERR_INVALID;
+        if (capacity > 0 && ((indices == nullptr && indices64 == nullptr) || values == nullptr))
+            return DWS_ERR_INVALID;
     }
     const WsView v = view_of(plan, workspace);
     return from_cuda(dws::launch_encode(
         v, reinterpret_cast<const uint16_t *const *>(old_ptrs),
         reinterpret_cast<const uint16_t *const *>(new_ptrs), reinterpret_cast<long long *>(offsets),
         reinterpret_cast<int *>(indices), values, compact ? capacity : 0, compact,
-        wait_limit_ns, withhold, reinterpret_cast<cudaStream_t>(stream)));
+        wait_limit_ns, withhold, reinterpret_cast<cudaStream_t>(stream),
+        reinterpret_cast<long long *>(indices64), reinterpret_cast<const long long *>(index_base)));
 }
 
 }  // namespace
@@ -226,6 +229,19 @@ dws_status_t dws_encode_ex(const dws_plan_t *plan, const void *const *old_ptrs,
                            int64_t debug_withhold_tile) {
     return encode_common(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, workspace,
                          workspace_bytes, stream, true, wait_limit_ns, debug_withhold_tile);
+}
+
+dws_status_t dws_encode_global(const dws_plan_t *plan, const void *const *old_ptrs,
+                               const void *const *new_ptrs, const int64_t *index_base,
+                               int64_t *offsets, int64_t *indices, uint16_t *values,
+                               int64_t capacity, void *workspace, size_t workspace_bytes,
+                               dws_stream_t stream) {
+    if (index_base == nullptr) return DWS_ERR_INVALID;
+    if (capacity > 0 && indices == nullptr) return DWS_ERR_INVALID;
+    // With no capacity nothing is written: the plain kernel computes the offsets.
+    return encode_common(plan, old_ptrs, new_ptrs, offsets, nullptr, values, capacity, workspace,
+                         workspace_bytes, stream, true, 0, -1, capacity > 0 ? indices : nullptr,
+                         index_base);
 }
 
 dws_status_t dws_count(const dws_plan_t *plan, const void *const *old_ptrs,

@@ -310,6 +310,14 @@ __device__ __forceinline__ void st_stream_v2(void *p, uint2 v) {
     asm volatile("st.global.cs.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
 
+__device__ __forceinline__ void st_stream_v2u64(void *p, unsigned long long a, unsigned long long b) {
+    asm volatile("st.global.cs.v2.u64 [%0], {%1,%2};" ::"l"(p), "l"(a), "l"(b) : "memory");
+}
+
+__device__ __forceinline__ void st_stream_u64(void *p, unsigned long long v) {
+    asm volatile("st.global.cs.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
 __device__ __forceinline__ void st_stream_u32(void *p, uint32_t v) {
     asm volatile("st.global.cs.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -373,7 +381,8 @@ cudaError_t launch_fill_tile_map(const WsView &ws, cudaStream_t s);
 cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
                           const uint16_t *const *new_ptrs, long long *offsets, int *indices,
                           uint16_t *values, long long capacity, bool compact,
-                          long long wait_limit_ns, long long withhold_tile, cudaStream_t s);
+                          long long wait_limit_ns, long long withhold_tile, cudaStream_t s,
+                          long long *indices64 = nullptr, const long long *index_base = nullptr);
 
 struct DeltaRef {
     const long long *offsets;

@@ -93,6 +93,8 @@ struct EncodeParams {
     long long wait_limit_ns;
     long long withhold;
     int vec_out;  // indices 16-byte and values 8-byte aligned: entries leave four at a time
+    long long *indices64;          // global positions (dws_encode_global), else null
+    const long long *index_base;   // per tensor: added to the local index (global positions)
 };
 
 struct EncodeSmem {
@@ -562,6 +564,8 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
 // the outputs are aligned, each lane stores four entries at once (16 bytes of
 // indices, 8 of values) after a head that brings the position to a multiple
 // of four.
+// kWide: int64 global positions, index_base[tensor] + local index.
+template <bool kWide>
 __device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const Pending &e,
                               long long prefix) {
     const int lane = threadIdx.x & 31;
@@ -569,9 +573,15 @@ __device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const
     if (lim > e.total) lim = e.total;
     const int n = lim > 0 ? static_cast<int>(lim) : 0;
     const uint32_t ls = static_cast<uint32_t>(e.local_start);
+    long long gs = 0;  // global position of the tile's first element
+    if (kWide) gs = p.index_base[e.tensor] + e.local_start;
     auto one = [&](int k) {
         const uint32_t v = ring[(e.pos + k) & (kRing - 1)];
-        st_stream_u32(p.indices + prefix + k, ls + (v & 0xffffu));
+        if (kWide) {
+            st_stream_u64(p.indices64 + prefix + k, static_cast<unsigned long long>(gs + (v & 0xffffu)));
+        } else {
+            st_stream_u32(p.indices + prefix + k, ls + (v & 0xffffu));
+        }
         st_stream_u16(p.values + prefix + k, static_cast<uint16_t>(v >> 16));
     };
     if (!p.vec_out) {
@@ -587,8 +597,16 @@ __device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const
         const uint32_t v1 = ring[(e.pos + k + 1) & (kRing - 1)];
         const uint32_t v2 = ring[(e.pos + k + 2) & (kRing - 1)];
         const uint32_t v3 = ring[(e.pos + k + 3) & (kRing - 1)];
-        st_stream_v4(p.indices + prefix + k,
-                     make_uint4(ls + (v0 & 0xffffu), ls + (v1 & 0xffffu), ls + (v2 & 0xffffu), ls + (v3 & 0xffffu)));
+        if (kWide) {
+            st_stream_v2u64(p.indices64 + prefix + k, static_cast<unsigned long long>(gs + (v0 & 0xffffu)),
+                            static_cast<unsigned long long>(gs + (v1 & 0xffffu)));
+            st_stream_v2u64(p.indices64 + prefix + k + 2, static_cast<unsigned long long>(gs + (v2 & 0xffffu)),
+                            static_cast<unsigned long long>(gs + (v3 & 0xffffu)));
+        } else {
+            st_stream_v4(p.indices + prefix + k,
+                         make_uint4(ls + (v0 & 0xffffu), ls + (v1 & 0xffffu), ls + (v2 & 0xffffu),
+                                    ls + (v3 & 0xffffu)));
+        }
         st_stream_v2(p.values + prefix + k,
                      make_uint2((v0 >> 16) | (v1 & 0xffff0000u), (v2 >> 16) | (v3 & 0xffff0000u)));
     }
@@ -596,7 +614,7 @@ __device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const
     if (lane < n - tail) one(tail + lane);
 }
 
-template <bool kCompact>
+template <bool kCompact, bool kWide>
 __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
     const int lane = threadIdx.x & 31;
     const int j = (threadIdx.x >> 5) - kCountWarps;
@@ -631,7 +649,7 @@ __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
                     if (kCompact && nnz > p.capacity) record_error(p.ws.hdr, DWS_ERR_CAPACITY, nnz);
                 }
             }
-            if (kCompact) write_entries(p, sm.ring[e.group], e, prefix);
+            if (kCompact) write_entries<kWide>(p, sm.ring[e.group], e, prefix);
         } else if (e.ticket != p.withhold) {
             if (lane == 0) *reinterpret_cast<volatile int *>(&sm.stop) = 1;
         }
@@ -642,7 +660,7 @@ __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
     }
 }
 
-template <bool kCompact>
+template <bool kCompact, bool kWide>
 __global__ void __launch_bounds__(kThreads, 1) encode_kernel(EncodeParams p) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     EncodeSmem &sm = *reinterpret_cast<EncodeSmem *>(smem_raw);
@@ -671,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(EncodeParams p) {
     if (warp < kCountWarps) {
         count_group<kCompact>(p, sm, warp / kGroupWarps);
     } else if (warp < kProducerWarp) {
-        look_group<kCompact>(p, sm);
+        look_group<kCompact, kWide>(p, sm);
     } else if ((tid & 31) == 0) {
         produce(p, sm);
     }
@@ -749,16 +767,19 @@ __global__ void fill_tile_map_kernel(WsView ws) {
 size_t encode_smem_bytes() { return sizeof(EncodeSmem); }
 
 cudaError_t encode_set_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(encode_kernel<true>,
+    cudaError_t e = cudaFuncSetAttribute(encode_kernel<true, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sizeof(EncodeSmem)));
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(encode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(encode_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sizeof(EncodeSmem)));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(encode_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(sizeof(EncodeSmem)));
 }
 
 cudaError_t encode_occupancy(int *ctas_per_sm) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, encode_kernel<true>,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, encode_kernel<true, false>,
                                                          kThreads, sizeof(EncodeSmem));
 }
 
@@ -776,7 +797,8 @@ cudaError_t launch_fill_tile_map(const WsView &ws, cudaStream_t s) {
 cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
                           const uint16_t *const *new_ptrs, long long *offsets, int *indices,
                           uint16_t *values, long long capacity, bool compact,
-                          long long wait_limit_ns, long long withhold_tile, cudaStream_t s) {
+                          long long wait_limit_ns, long long withhold_tile, cudaStream_t s,
+                          long long *indices64, const long long *index_base) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
@@ -795,17 +817,24 @@ cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
     p.capacity = compact ? capacity : 0;
     p.wait_limit_ns = wait_limit_ns > 0 ? wait_limit_ns : 2000000000LL;
     p.withhold = withhold_tile;
-    p.vec_out = ((reinterpret_cast<uintptr_t>(indices) & 15u) == 0 &&
-                 (reinterpret_cast<uintptr_t>(values) & 7u) == 0) ? 1 : 0;
+    p.indices64 = indices64;
+    p.index_base = index_base;
+    const uintptr_t ia = indices64 != nullptr ? reinterpret_cast<uintptr_t>(indices64)
+                                              : reinterpret_cast<uintptr_t>(indices);
+    p.vec_out = ((ia & 15u) == 0 && (reinterpret_cast<uintptr_t>(values) & 7u) == 0) ? 1 : 0;
 
     long long grid = static_cast<long long>(di.sm_count) * di.encode_ctas_per_sm;
     if (grid > ws.num_tiles) grid = ws.num_tiles;
     if (grid < 1) grid = 1;
     const size_t smem = sizeof(EncodeSmem);
     if (compact) {
-        encode_kernel<true><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
+        if (indices64 != nullptr) {
+            encode_kernel<true, true><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
+        } else {
+            encode_kernel<true, false><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
+        }
     } else {
-        encode_kernel<false><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
+        encode_kernel<false, false><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
     }
     return launched();
 }

@@ -472,3 +472,32 @@ def test_checksum_matches_torch_hash_tensor():
     for sub in (vals[:8], vals[8:1000]):
         t = torch.from_numpy(sub.view(np.int16).copy()).view(torch.bfloat16)
         assert oracle.checksum_parts(blob[:0], sub)[1] == int(torch.hash_tensor(t).item())
+
+
+def test_encode_global_matches_the_pages_shard_routine():
+    # shard_delta_indices, written with torch's own ops on CPU: integer-view
+    # compare, nonzero, then + offset in int64.  Offsets past 2^32 pin the
+    # width.
+    rng = np.random.default_rng(95)
+    sizes = [1000, 0, 70_001, 5]
+    bases = [0, 123, 5_000_000_000, 2 ** 31 - 3]
+    olds = [rng.integers(0, 1 << 16, n, dtype=np.uint16) for n in sizes]
+    news = []
+    for a in olds:
+        b = a.copy()
+        if a.size:
+            m = rng.random(a.size) < 0.1
+            b[m] ^= np.uint16(0x0040)
+        news.append(b)
+    o, gi, v = oracle.encode_global(olds, news, bases)
+    want_i, want_v = [], []
+    for a, b, off in zip(olds, news, bases):
+        ta = torch.from_numpy(a.view(np.int16).copy())
+        tb = torch.from_numpy(b.view(np.int16).copy())
+        local = (tb != ta).nonzero(as_tuple=False).view(-1)
+        want_i.append((local.to(torch.int64) + off).numpy())
+        want_v.append(tb[local].numpy().view(np.uint16))
+    assert gi.dtype == np.int64
+    np.testing.assert_array_equal(gi, np.concatenate(want_i))
+    np.testing.assert_array_equal(v, np.concatenate(want_v))
+    assert gi.max() > 2 ** 32
