@@ -744,6 +744,23 @@ def run_ours(args):
         ms_c, _ = time_reps(lambda: plan.count(ot, nt, offsets), args.rows_reps)
         rows = {}
         rows.update([row("count_llama3_8b_lr%g" % args.lr, ms_c, 4 * N, weight_bytes, peak)])
+        # the same step with int64 global positions (shard offset per tensor)
+        bases = torch.tensor([(t + 1) * (1 << 33) for t in range(T)], dtype=torch.int64, device=dev)
+        gidx = torch.empty(nnz, dtype=torch.int64, device=dev)
+        gval = torch.empty(nnz, dtype=torch.int16, device=dev)
+        goffs = torch.empty(T + 1, dtype=torch.int64, device=dev)
+        cs0 = torch.cuda.current_stream().cuda_stream
+
+        def enc_global():
+            dws.dws_encode_global(plan.handle, ot.data_ptr(), nt.data_ptr(), bases.data_ptr(),
+                                  goffs.data_ptr(), gidx.data_ptr(), gval.data_ptr(), nnz,
+                                  plan.workspace.data_ptr(), plan.workspace_bytes, cs0)
+
+        ms_g, mn_g = time_reps(enc_global, args.rows_reps)
+        ok_g = plan.status()[0] == dws.DWS_OK and bool(torch.equal(goffs, offsets))
+        rows.update([row("encode_global_int64_llama3_8b_lr%g" % args.lr, ms_g, 4 * N + 10 * nnz,
+                         weight_bytes, peak, {"min_ms": round(mn_g, 4), "offsets_equal": ok_g})])
+        del gidx, gval, goffs, bases
         lr2 = 1e-5
         for t in range(T):
             new[t].copy_(make_new(lr2)(t, sizes[t]))
