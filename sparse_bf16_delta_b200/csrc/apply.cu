@@ -7,21 +7,27 @@
 // after the latest anchor) the deltas in order, the later one winning.
 //
 // dws_apply -- one delta, direct scatter.  Each CTA takes 2048 consecutive
-//   entries (coalesced index/value reads), finds their tensors by binary
-//   search over offsets, range-checks every index and stores the 2-byte
-//   values.  DRAM traffic is the touched 32-byte sectors (read-modify-write)
-//   plus 6 bytes per entry, which is less than streaming the snapshot through
-//   at the densities the workloads have.
+//   entries (coalesced index/value reads) and, before its one barrier, has
+//   them, the workspace header and two warp-cooperative searches for its
+//   first and last tensor in flight together; then it range- and
+//   order-checks every index and stores the 2-byte values.  DRAM traffic is
+//   the touched 32-byte sectors (read-modify-write in L2) plus 6 bytes per
+//   entry, which is less than streaming the snapshot through at the
+//   densities the workloads have.
 //
-// dws_apply_chain -- K deltas, one launch, merge mode.  Each CTA owns a
-//   contiguous range of snapshot tiles (8192 elements).  Per tile: a 1-D bulk
-//   async copy brings the snapshot tile into shared memory while the CTA reads
-//   every delta's entries for the tile (one cursor per delta, advanced tile
-//   by tile, so each delta is binary-searched only once per CTA) and tags them
-//   into a shared array with atomicMax on ((k+1) << 16 | value): the highest k,
-//   i.e. the latest delta, wins regardless of thread order.  The merged tile
-//   goes back with a bulk store.  Traffic: the snapshot read and written once
-//   plus 6 bytes per entry, instead of K read-modify-write scatters.
+// dws_apply_chain -- K deltas, one launch, two modes:
+//   scatter (the default; chain_scatter_kernel): one CTA per SM owns whole
+//   windows of 32 tiles; per window the deltas are replayed from the last to
+//   the first, an element being stored only if its written-bit is clear, so
+//   every element is written once, by the latest delta that touches it, and
+//   untouched sectors are not moved at all.  Per delta, a window's entries
+//   are one contiguous stretch, streamed by all warps in 32-entry chunks.
+//   tile merge (chain_kernel): each CTA owns a contiguous range of snapshot
+//   tiles; per tile a 1-D bulk async copy brings the tile into shared memory
+//   while the CTA tags every delta's entries for it into a shared array with
+//   atomicMax on ((k+1) << 16 | value) (the latest delta wins regardless of
+//   thread order); the merged tile goes back with a bulk store.  It moves
+//   the whole snapshot even where the deltas touch nothing.
 #include <cuda_runtime.h>
 
 #include "dws_internal.cuh"
@@ -475,7 +481,8 @@ struct ScatSmem {
 };
 
 __global__ void __launch_bounds__(kScatThreads, 1) chain_scatter_kernel(ScatParams p) {
-    __shared__ __align__(16) ScatSmem sm;
+    extern __shared__ __align__(128) unsigned char scat_smem_raw[];
+    ScatSmem &sm = *reinterpret_cast<ScatSmem *>(scat_smem_raw);
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
@@ -698,13 +705,16 @@ __global__ void __launch_bounds__(kScatThreads, 1) chain_scatter_kernel(ScatPara
 size_t chain_smem_bytes() { return sizeof(ChainSmem); }
 
 cudaError_t chain_set_attributes() {
-    return cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sizeof(ChainSmem)));
+    cudaError_t e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(ChainSmem)));
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(chain_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sizeof(ScatSmem)));
 }
 
 cudaError_t scatter_occupancy(int *ctas_per_sm) {
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, chain_scatter_kernel,
-                                                         kScatThreads, 0);
+                                                         kScatThreads, sizeof(ScatSmem));
 }
 
 cudaError_t chain_occupancy(int *ctas_per_sm) {
@@ -794,7 +804,7 @@ cudaError_t launch_apply_chain_scatter(const WsView &ws, uint16_t *const *snap_p
     const long long win_per_cta = (windows + grid - 1) / grid;
     p.tiles_per_cta = win_per_cta * kWinTiles;
     grid = (ws.num_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
-    chain_scatter_kernel<<<static_cast<unsigned int>(grid), kScatThreads, 0, s>>>(p);
+    chain_scatter_kernel<<<static_cast<unsigned int>(grid), kScatThreads, sizeof(ScatSmem), s>>>(p);
     return launched();
 }
 
