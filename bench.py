@@ -761,6 +761,22 @@ def run_ours(args):
         rows.update([row("encode_global_int64_llama3_8b_lr%g" % args.lr, ms_g, 4 * N + 10 * nnz,
                          weight_bytes, peak, {"min_ms": round(mn_g, 4), "offsets_equal": ok_g})])
         del gidx, gval, goffs, bases
+        # the same step with the wire checksum computed on the fly
+        hashes = torch.empty(2, dtype=torch.int64, device=dev)
+        coffs = torch.empty(T + 1, dtype=torch.int64, device=dev)
+        cidx = torch.empty(nnz, dtype=torch.int32, device=dev)
+        cval = torch.empty(nnz, dtype=torch.int16, device=dev)
+
+        def enc_checksum():
+            dws.dws_encode_checksum(plan.handle, ot.data_ptr(), nt.data_ptr(), coffs.data_ptr(),
+                                    cidx.data_ptr(), cval.data_ptr(), nnz, hashes.data_ptr(),
+                                    plan.workspace.data_ptr(), plan.workspace_bytes, cs0)
+
+        ms_s, mn_s = time_reps(enc_checksum, args.rows_reps)
+        ok_s = plan.status()[0] == dws.DWS_OK and bool(torch.equal(cidx, indices))
+        rows.update([row("encode_checksum_llama3_8b_lr%g" % args.lr, ms_s, 4 * N + 6 * nnz,
+                         weight_bytes, peak, {"min_ms": round(mn_s, 4), "indices_equal": ok_s})])
+        del hashes, coffs, cidx, cval
         lr2 = 1e-5
         for t in range(T):
             new[t].copy_(make_new(lr2)(t, sizes[t]))

@@ -158,6 +158,19 @@ DWS_API dws_status_t dws_encode_global(const dws_plan_t *plan,
                                uint16_t *values, int64_t capacity,
                                void *workspace, size_t workspace_bytes, dws_stream_t stream);
 
+/* dws_encode that also returns the wire checksum of the delta it writes
+ * (see dws_checksum): hashes[0] = XOR of the bytes of every position at its
+ * tensor's pos_width, hashes[1] = XOR of the double bits of every value,
+ * i.e. what dws_pack_positions + dws_checksum would give, without the extra
+ * pass over the delta.  Only entries below `capacity` are hashed.
+ * hashes: device uint64[2], overwritten.  Otherwise as dws_encode;
+ * DWS_ERR_INVALID also for a null `hashes`. */
+DWS_API dws_status_t dws_encode_checksum(const dws_plan_t *plan,
+                                 const void *const *old_ptrs, const void *const *new_ptrs,
+                                 int64_t *offsets, int32_t *indices, uint16_t *values,
+                                 int64_t capacity, uint64_t *hashes,
+                                 void *workspace, size_t workspace_bytes, dws_stream_t stream);
+
 /* dws_encode with explicit controls of the scan's bounded wait.
  * wait_limit_ns: how long a tile waits for its predecessor's count before it
  *   records DWS_ERR_TIMEOUT and every waiting tile gives up (<= 0: 2 s).

@@ -72,6 +72,7 @@ _sig("dws_apply_chain", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _vp,
 _sig("dws_apply_chain_ex", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _i32, _vp, _sz, _vp])
 _sig("dws_pos_width", _i32, [_vp, _i32])
 _sig("dws_encode_global", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
+_sig("dws_encode_checksum", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _vp])
 _sig("dws_pack_positions", _i32, [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp])
 _sig("dws_checksum", _i32, [_vp, _i64, _vp, _i64, _vp, _vp])
 _sig("dws_xor_encode", _i32, [_vp, _vp, _vp, _i64, _vp])
@@ -186,6 +187,12 @@ def dws_encode_global(plan, old_ptrs, new_ptrs, index_base, offsets, indices, va
                       workspace, workspace_bytes, stream) -> int:
     return _lib.dws_encode_global(plan, old_ptrs, new_ptrs, index_base, offsets, indices, values,
                                   capacity, workspace, workspace_bytes, stream)
+
+
+def dws_encode_checksum(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, hashes,
+                        workspace, workspace_bytes, stream) -> int:
+    return _lib.dws_encode_checksum(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
+                                    hashes, workspace, workspace_bytes, stream)
 
 
 def dws_pos_width(plan, t) -> int:
@@ -407,6 +414,24 @@ class DeltaPlan:
                                  _stream_handle(stream)), "dws_encode_global")
         self.raise_on_error("dws_encode_global", stream)
         return Delta(offsets, indices, values)
+
+    def encode_checksum(self, old_table, new_table, stream=None):
+        """(Delta, checksum): the exact encode and the wire checksum of the
+        delta it wrote, hash(positions) ^ (hash(values) << 1)."""
+        torch = _torch()
+        offsets = self.count(old_table, new_table, stream=stream)
+        nnz = int(offsets[-1].item())
+        indices = torch.empty(nnz, dtype=torch.int32, device=self.device)
+        values = torch.empty(nnz, dtype=torch.int16, device=self.device)
+        hashes = torch.empty(2, dtype=torch.int64, device=self.device)
+        _check(dws_encode_checksum(self.handle, old_table.data_ptr(), new_table.data_ptr(),
+                                   offsets.data_ptr(), indices.data_ptr() if nnz else 0,
+                                   values.data_ptr() if nnz else 0, nnz, hashes.data_ptr(),
+                                   self.workspace.data_ptr(), self.workspace_bytes,
+                                   _stream_handle(stream)), "dws_encode_checksum")
+        self.raise_on_error("dws_encode_checksum", stream)
+        hp, hv = (int(x) & 0xFFFFFFFFFFFFFFFF for x in hashes.cpu().tolist())
+        return Delta(offsets, indices, values), hp ^ (hv << 1)
 
     # -- wire form --
     def pos_width(self, t: int) -> int:

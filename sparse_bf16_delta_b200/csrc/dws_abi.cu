@@ -119,7 +119,7 @@ dws_status_t encode_common(const dws_plan_t *plan, const void *const *old_ptrs,
                            uint16_t *values, int64_t capacity, void *workspace,
                            size_t workspace_bytes, dws_stream_t stream, bool compact,
                            int64_t wait_limit_ns, int64_t withhold, int64_t *indices64 = nullptr,
-                           const int64_t *index_base = nullptr) {
+                           const int64_t *index_base = nullptr, uint64_t *hashes = nullptr) {
     dws_status_t st = check_ws(plan, workspace, workspace_bytes);
     if (st != DWS_OK) return st;
     if (old_ptrs == nullptr || new_ptrs == nullptr || offsets == nullptr) return DWS_ERR_INVALID;
@@ -134,7 +134,8 @@ dws_status_t encode_common(const dws_plan_t *plan, const void *const *old_ptrs,
         reinterpret_cast<const uint16_t *const *>(new_ptrs), reinterpret_cast<long long *>(offsets),
         reinterpret_cast<int *>(indices), values, compact ? capacity : 0, compact,
         wait_limit_ns, withhold, reinterpret_cast<cudaStream_t>(stream),
-        reinterpret_cast<long long *>(indices64), reinterpret_cast<const long long *>(index_base)));
+        reinterpret_cast<long long *>(indices64), reinterpret_cast<const long long *>(index_base),
+        reinterpret_cast<unsigned long long *>(hashes)));
 }
 
 }  // namespace
@@ -242,6 +243,15 @@ dws_status_t dws_encode_global(const dws_plan_t *plan, const void *const *old_pt
     return encode_common(plan, old_ptrs, new_ptrs, offsets, nullptr, values, capacity, workspace,
                          workspace_bytes, stream, true, 0, -1, capacity > 0 ? indices : nullptr,
                          index_base);
+}
+
+dws_status_t dws_encode_checksum(const dws_plan_t *plan, const void *const *old_ptrs,
+                                 const void *const *new_ptrs, int64_t *offsets, int32_t *indices,
+                                 uint16_t *values, int64_t capacity, uint64_t *hashes,
+                                 void *workspace, size_t workspace_bytes, dws_stream_t stream) {
+    if (hashes == nullptr) return DWS_ERR_INVALID;
+    return encode_common(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, workspace,
+                         workspace_bytes, stream, true, 0, -1, nullptr, nullptr, hashes);
 }
 
 dws_status_t dws_count(const dws_plan_t *plan, const void *const *old_ptrs,

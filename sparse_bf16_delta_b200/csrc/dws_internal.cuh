@@ -359,6 +359,35 @@ __device__ __forceinline__ int warp_tensor_of_entry(const long long *offsets, in
     }
 }
 
+// The double equal to a bf16 value, as bits: sign, exponent rebased from
+// 127 to 1023, mantissa moved up; subnormals normalised; infinities kept;
+// NaNs quieted (bit 51 set) with sign and payload kept.
+__device__ __forceinline__ unsigned long long bf16_to_f64_bits(uint32_t b) {
+    const unsigned long long sign = static_cast<unsigned long long>(b >> 15) << 63;
+    const uint32_t e = (b >> 7) & 0xffu;
+    const uint32_t m = b & 0x7fu;
+    if (e == 0xffu) {
+        const unsigned long long q = m ? ((1ull << 51) | (static_cast<unsigned long long>(m) << 45)) : 0ull;
+        return sign | (0x7ffull << 52) | q;
+    }
+    if (e == 0u) {
+        if (m == 0u) return sign;
+        const int top = 31 - __clz(m);  // m = 2^top + rest, value = m * 2^-133
+        const unsigned long long frac = static_cast<unsigned long long>(m - (1u << top)) << (52 - top);
+        return sign | (static_cast<unsigned long long>(top + 1023 - 133) << 52) | frac;
+    }
+    return sign | (static_cast<unsigned long long>(e - 127 + 1023) << 52) |
+           (static_cast<unsigned long long>(m) << 45);
+}
+
+// XOR of the bytes of a position stored in `width` (2 or 4) little-endian
+// bytes: its contribution to the hash of a positions block.
+__device__ __forceinline__ unsigned long long pos_bytes_xor(uint32_t pos, int width) {
+    uint32_t x = pos ^ (pos >> 8);
+    if (width == 4) x ^= (pos >> 16) ^ (pos >> 24);
+    return x & 0xffu;
+}
+
 #endif  // __CUDACC__
 
 // ---------------------------------------------------------------------------
@@ -382,7 +411,8 @@ cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
                           const uint16_t *const *new_ptrs, long long *offsets, int *indices,
                           uint16_t *values, long long capacity, bool compact,
                           long long wait_limit_ns, long long withhold_tile, cudaStream_t s,
-                          long long *indices64 = nullptr, const long long *index_base = nullptr);
+                          long long *indices64 = nullptr, const long long *index_base = nullptr,
+                          unsigned long long *hashes = nullptr);
 
 struct DeltaRef {
     const long long *offsets;

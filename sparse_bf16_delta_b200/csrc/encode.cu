@@ -95,6 +95,7 @@ struct EncodeParams {
     int vec_out;  // indices 16-byte and values 8-byte aligned: entries leave four at a time
     long long *indices64;          // global positions (dws_encode_global), else null
     const long long *index_base;   // per tensor: added to the local index (global positions)
+    unsigned long long *hashes;    // wire checksum halves (dws_encode_checksum), else null
 };
 
 struct EncodeSmem {
@@ -565,9 +566,12 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
 // indices, 8 of values) after a head that brings the position to a multiple
 // of four.
 // kWide: int64 global positions, index_base[tensor] + local index.
-template <bool kWide>
+// kSum: also XOR the written entries into the wire checksum halves (the
+// bytes of each position at its tensor's pos_width, the double bits of each
+// value) kept in *hp / *hv.
+template <bool kWide, bool kSum>
 __device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const Pending &e,
-                              long long prefix) {
+                              long long prefix, unsigned long long *hp, unsigned long long *hv) {
     const int lane = threadIdx.x & 31;
     long long lim = p.capacity - prefix;
     if (lim > e.total) lim = e.total;
@@ -575,8 +579,17 @@ __device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const
     const uint32_t ls = static_cast<uint32_t>(e.local_start);
     long long gs = 0;  // global position of the tile's first element
     if (kWide) gs = p.index_base[e.tensor] + e.local_start;
+    int width = 4;
+    if (kSum) width = p.ws.numel[e.tensor] <= 65536 ? 2 : 4;
+    auto sum = [&](uint32_t v) {
+        if (kSum) {
+            *hp ^= pos_bytes_xor(ls + (v & 0xffffu), width);
+            *hv ^= bf16_to_f64_bits(v >> 16);
+        }
+    };
     auto one = [&](int k) {
         const uint32_t v = ring[(e.pos + k) & (kRing - 1)];
+        sum(v);
         if (kWide) {
             st_stream_u64(p.indices64 + prefix + k, static_cast<unsigned long long>(gs + (v & 0xffffu)));
         } else {
@@ -597,6 +610,10 @@ __device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const
         const uint32_t v1 = ring[(e.pos + k + 1) & (kRing - 1)];
         const uint32_t v2 = ring[(e.pos + k + 2) & (kRing - 1)];
         const uint32_t v3 = ring[(e.pos + k + 3) & (kRing - 1)];
+        sum(v0);
+        sum(v1);
+        sum(v2);
+        sum(v3);
         if (kWide) {
             st_stream_v2u64(p.indices64 + prefix + k, static_cast<unsigned long long>(gs + (v0 & 0xffffu)),
                             static_cast<unsigned long long>(gs + (v1 & 0xffffu)));
@@ -614,17 +631,36 @@ __device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const
     if (lane < n - tail) one(tail + lane);
 }
 
-template <bool kCompact, bool kWide>
+template <bool kCompact, bool kWide, bool kSum>
 __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
     const int lane = threadIdx.x & 31;
     const int j = (threadIdx.x >> 5) - kCountWarps;
+    unsigned long long hp = 0, hv = 0;  // this lane's share of the checksum halves (kSum)
+    // Leaves through here: the warp's checksum share goes out with one
+    // atomic per half (per-tile atomics on two words would be a hot spot).
+    auto leave = [&]() {
+        if (kSum) {
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) {
+                hp ^= __shfl_xor_sync(0xffffffffu, hp, d);
+                hv ^= __shfl_xor_sync(0xffffffffu, hv, d);
+            }
+            if (lane == 0) {
+                if (hp) atomicXor(p.hashes, hp);
+                if (hv) atomicXor(p.hashes + 1, hv);
+            }
+        }
+    };
     for (int i = j;; i += kLookWarps) {
         // Wait for queue entry i, or for the end.
         unsigned int backoff = 32;
         for (;;) {
             if (ld_acquire_cta(&sm.q_ready[i % kQueue]) == i + 1) break;
             const int fin = ld_acquire_cta(&sm.q_final);
-            if (i >= fin || *reinterpret_cast<volatile int *>(&sm.stop) != 0) return;
+            if (i >= fin || *reinterpret_cast<volatile int *>(&sm.stop) != 0) {
+                leave();
+                return;
+            }
             __nanosleep(backoff);
             if (backoff < 512) backoff <<= 1;
         }
@@ -649,7 +685,7 @@ __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
                     if (kCompact && nnz > p.capacity) record_error(p.ws.hdr, DWS_ERR_CAPACITY, nnz);
                 }
             }
-            if (kCompact) write_entries<kWide>(p, sm.ring[e.group], e, prefix);
+            if (kCompact) write_entries<kWide, kSum>(p, sm.ring[e.group], e, prefix, &hp, &hv);
         } else if (e.ticket != p.withhold) {
             if (lane == 0) *reinterpret_cast<volatile int *>(&sm.stop) = 1;
         }
@@ -660,7 +696,7 @@ __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
     }
 }
 
-template <bool kCompact, bool kWide>
+template <bool kCompact, bool kWide, bool kSum>
 __global__ void __launch_bounds__(kThreads, 1) encode_kernel(EncodeParams p) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     EncodeSmem &sm = *reinterpret_cast<EncodeSmem *>(smem_raw);
@@ -689,7 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(EncodeParams p) {
     if (warp < kCountWarps) {
         count_group<kCompact>(p, sm, warp / kGroupWarps);
     } else if (warp < kProducerWarp) {
-        look_group<kCompact, kWide>(p, sm);
+        look_group<kCompact, kWide, kSum>(p, sm);
     } else if ((tid & 31) == 0) {
         produce(p, sm);
     }
@@ -767,19 +803,22 @@ __global__ void fill_tile_map_kernel(WsView ws) {
 size_t encode_smem_bytes() { return sizeof(EncodeSmem); }
 
 cudaError_t encode_set_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(encode_kernel<true, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sizeof(EncodeSmem)));
+    const int bytes = static_cast<int>(sizeof(EncodeSmem));
+    cudaError_t e = cudaFuncSetAttribute(encode_kernel<true, false, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(encode_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sizeof(EncodeSmem)));
+    e = cudaFuncSetAttribute(encode_kernel<true, true, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(encode_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sizeof(EncodeSmem)));
+    e = cudaFuncSetAttribute(encode_kernel<true, false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(encode_kernel<false, false, false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
 cudaError_t encode_occupancy(int *ctas_per_sm) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, encode_kernel<true, false>,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, encode_kernel<true, false, false>,
                                                          kThreads, sizeof(EncodeSmem));
 }
 
@@ -798,7 +837,8 @@ cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
                           const uint16_t *const *new_ptrs, long long *offsets, int *indices,
                           uint16_t *values, long long capacity, bool compact,
                           long long wait_limit_ns, long long withhold_tile, cudaStream_t s,
-                          long long *indices64, const long long *index_base) {
+                          long long *indices64, const long long *index_base,
+                          unsigned long long *hashes) {
     DeviceInfo di;
     cudaError_t e = device_info(&di);
     if (e != cudaSuccess) return e;
@@ -819,6 +859,11 @@ cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
     p.withhold = withhold_tile;
     p.indices64 = indices64;
     p.index_base = index_base;
+    p.hashes = hashes;
+    if (hashes != nullptr) {
+        e = cudaMemsetAsync(hashes, 0, 2 * sizeof(unsigned long long), s);
+        if (e != cudaSuccess) return e;
+    }
     const uintptr_t ia = indices64 != nullptr ? reinterpret_cast<uintptr_t>(indices64)
                                               : reinterpret_cast<uintptr_t>(indices);
     p.vec_out = ((ia & 15u) == 0 && (reinterpret_cast<uintptr_t>(values) & 7u) == 0) ? 1 : 0;
@@ -829,12 +874,14 @@ cudaError_t launch_encode(const WsView &ws, const uint16_t *const *old_ptrs,
     const size_t smem = sizeof(EncodeSmem);
     if (compact) {
         if (indices64 != nullptr) {
-            encode_kernel<true, true><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
+            encode_kernel<true, true, false><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
+        } else if (hashes != nullptr) {
+            encode_kernel<true, false, true><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
         } else {
-            encode_kernel<true, false><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
+            encode_kernel<true, false, false><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
         }
     } else {
-        encode_kernel<false, false><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
+        encode_kernel<false, false, false><<<static_cast<unsigned int>(grid), kThreads, smem, s>>>(p);
     }
     return launched();
 }

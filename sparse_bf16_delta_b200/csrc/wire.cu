@@ -133,27 +133,6 @@ __global__ void __launch_bounds__(kPackThreads) pack_positions_kernel(PackParams
     }
 }
 
-// The double equal to a bf16 value, as bits: sign, exponent rebased from
-// 127 to 1023, mantissa moved up; subnormals normalised; infinities kept;
-// NaNs quieted (bit 51 set) with sign and payload kept.
-__device__ __forceinline__ unsigned long long bf16_to_f64_bits(uint32_t b) {
-    const unsigned long long sign = static_cast<unsigned long long>(b >> 15) << 63;
-    const uint32_t e = (b >> 7) & 0xffu;
-    const uint32_t m = b & 0x7fu;
-    if (e == 0xffu) {
-        const unsigned long long q = m ? ((1ull << 51) | (static_cast<unsigned long long>(m) << 45)) : 0ull;
-        return sign | (0x7ffull << 52) | q;
-    }
-    if (e == 0u) {
-        if (m == 0u) return sign;
-        const int top = 31 - __clz(m);  // m = 2^top + rest, value = m * 2^-133
-        const unsigned long long frac = static_cast<unsigned long long>(m - (1u << top)) << (52 - top);
-        return sign | (static_cast<unsigned long long>(top + 1023 - 133) << 52) | frac;
-    }
-    return sign | (static_cast<unsigned long long>(e - 127 + 1023) << 52) |
-           (static_cast<unsigned long long>(m) << 45);
-}
-
 constexpr int kSumThreads = 512;
 
 __device__ __forceinline__ unsigned long long fold_bytes(unsigned long long x) {

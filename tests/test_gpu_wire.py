@@ -132,3 +132,33 @@ def test_checksum_every_bf16_pattern(dws):
 def test_checksum_empty(dws):
     empty = torch.zeros(2, dtype=torch.uint8, device="cuda")
     assert dws.checksum(empty, 0, torch.zeros(0, dtype=torch.bfloat16, device="cuda")) == 0
+
+
+@pytest.mark.parametrize("rate", [0.02, 0.4])
+def test_encode_checksum_fused_equals_pack_then_checksum(dws, rate):
+    # The checksum the encode computes on the fly equals the one of the
+    # packed block (and the oracle's), over tensors of both widths, dense runs
+    # and a ragged tail.
+    rng = np.random.default_rng(330 + int(rate * 10))
+    sizes = [100, 65536, 65537, 8192 * 5 + 11, 0, 3]
+    olds, news = [], []
+    for n in sizes:
+        a = rng.integers(0, 1 << 16, n, dtype=np.uint16)
+        b = a.copy()
+        if n:
+            m = rng.random(n) < rate
+            b[m] ^= rng.integers(1, 1 << 16, int(m.sum()), dtype=np.uint16)
+            if n > 9000:
+                b[1024:9216] ^= np.uint16(0x0001)
+        olds.append(a)
+        news.append(b)
+    plan = dws.DeltaPlan(sizes)
+    ot = dws.ptr_table([dev_bits(a) for a in olds])
+    nt = dws.ptr_table([dev_bits(b) for b in news])
+    d, fused = plan.encode_checksum(ot, nt)
+    o, i, v = oracle.encode(olds, news)
+    np.testing.assert_array_equal(d.indices.cpu().numpy(), i)
+    blob, _ = oracle.pack_positions(sizes, o, i)
+    assert fused == oracle.checksum(blob, v)
+    gblob, _ = plan.pack_positions(d)
+    assert fused == dws.checksum(gblob, gblob.numel(), d.values)
