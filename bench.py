@@ -487,6 +487,25 @@ def rows_xor(args, dev, peak):
     out.update([row("xor_apply_layers_double_buffered_40x0.8GB", msp / 2, 5 * L * B, L * B, peak,
                     {"min_ms": round(mnp / 2, 4), "staging": "2 x 0.8 GB, D2D copy stream",
                      "exact": ok})])
+    # the same layers as a sparse delta of 16-bit words (indices + values):
+    # 680,000 changed bytes per layer travel as about 4 MB instead of 0.8 GB
+    ow = [o.view(torch.bfloat16) for o in olds]
+    nw = [n.view(torch.bfloat16) for n in news]
+    splan = dws.DeltaPlan.for_tensors(ow)
+    sot, snt = dws.ptr_table(ow), dws.ptr_table(nw)
+    sd = splan.encode_exact(sot, snt)
+    snnz = sd.nnz()
+    ms_e, mn_e = time_reps(lambda: splan.encode_into(sot, snt, sd.offsets, sd.indices, sd.values),
+                           args.rows_reps)
+    out.update([row("encode_sparse_nvfp4_40x0.8GB", ms_e, 2 * L * B + 6 * snnz, L * B, peak,
+                    {"min_ms": round(mn_e, 4), "nnz": snnz, "delta_bytes": 6 * snnz + 8 * (L + 1)})])
+    sst = dws.ptr_table(ow)
+    ms_a, mn_a = time_reps(lambda: splan.apply(sst, sd), args.rows_reps)
+    splan.raise_on_error("sparse xor apply")
+    ok = all(torch.equal(olds[l], news[l]) for l in (0, L - 1))
+    out.update([row("apply_sparse_nvfp4_40x0.8GB", ms_a, 8 * snnz, L * B, peak,
+                    {"min_ms": round(mn_a, 4), "exact": ok})])
+    del ow, nw, splan, sot, snt, sd, sst
     del olds, news, masks, bufs, staging
     gc.collect()
     torch.cuda.empty_cache()

@@ -477,6 +477,38 @@ def test_chain_rejects_negative_index(dws, mode):
     assert h[11] == 7 and h.sum() == 7
 
 
+# ---------------------------------------------------------------- sparse delta of XOR layers
+
+
+def test_sparse_delta_of_packed_byte_layers(dws):
+    # Packed low-precision layers (bytes) encoded as a sparse delta of 16-bit
+    # words: the changed words are exactly the words holding the generator's
+    # flipped bytes, the values are the new words, and applying the delta to
+    # the old layers gives the new ones.
+    nb = 1_000_002
+    olds, news, poss = [], [], []
+    for l in range(3):
+        o, n, pos = W.xor_layer(l, "cuda", nbytes=nb, flips=850)
+        olds.append(o)
+        news.append(n)
+        poss.append(pos)
+    ow = [o.view(torch.bfloat16) for o in olds]
+    nw = [n.view(torch.bfloat16) for n in news]
+    plan = dws.DeltaPlan.for_tensors(ow)
+    d = plan.encode_exact(dws.ptr_table(ow), dws.ptr_table(nw))
+    offs = d.offsets.cpu().numpy()
+    for l in range(3):
+        words = torch.unique(poss[l] // 2).cpu().numpy()
+        np.testing.assert_array_equal(d.indices[offs[l]:offs[l + 1]].cpu().numpy(), words)
+    want = oracle.encode([host_bits(t) for t in ow], [host_bits(t) for t in nw])
+    assert_delta_equal(delta_to_host(d), want)
+    snaps = [o.clone() for o in olds]
+    plan.apply(dws.ptr_table([t.view(torch.bfloat16) for t in snaps]), d)
+    plan.raise_on_error()
+    for t, n in zip(snaps, news):
+        assert torch.equal(t, n)
+
+
 # ---------------------------------------------------------------- XOR
 
 
