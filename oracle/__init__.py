@@ -16,6 +16,9 @@ tests can hand it numpy arrays.  Sources, by page title and section:
 * verl PR #6974 review, key source snippets, ``sparse_gather.py``
   (``shard_delta_indices``: integer-view compare, ``nonzero``, gather).
 * humans& weight-sync summary, first paragraph (XOR mask delta).
+
+``st_file.py`` (plain Python, json + struct) writes and reads a delta in the
+safetensors format of the TRL page's §4.1.
 """
 from __future__ import annotations
 

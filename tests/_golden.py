@@ -9,7 +9,7 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 
 def _lines(name):
-    with open(os.path.join(GOLDEN, name)) as f:
+    with open(os.path.join(GOLDEN, name), encoding="utf-8") as f:
         for raw in f:
             line = raw.split("#", 1)[0].strip()
             if line:
