@@ -31,11 +31,15 @@ library, which shares no code with this file):
   the data is the encode's two arrays as they stand.
 A reader takes any key order and any data layout; the parameters applied are
 exactly those that ``changed_params`` lists (§4.3), and a file whose tensor
-entries disagree with that list is refused.
+entries disagree with that list is refused.  It takes the JSON grammar
+strictly: a repeated key in an object, NaN/Infinity, a count or offset that
+is not a plain non-negative integer (``true``, ``1.0``), or a model_version
+that is not a decimal integer of 64 bits is refused.
 """
 from __future__ import annotations
 
 import json
+import re
 import struct
 
 import numpy as np
@@ -49,6 +53,25 @@ class DeltaFileError(ValueError):
 
 def _dumps(obj) -> str:
     return json.dumps(obj, ensure_ascii=False, separators=(",", ":"))
+
+
+def _no_repeats(pairs):
+    keys = [k for k, _ in pairs]
+    if len(set(keys)) != len(keys):
+        raise DeltaFileError("a JSON object repeats a key")
+    return dict(pairs)
+
+
+def _no_constants(name):
+    raise DeltaFileError(f"non-standard JSON constant {name}")
+
+
+def _loads(text: str):
+    return json.loads(text, object_pairs_hook=_no_repeats, parse_constant=_no_constants)
+
+
+def _count(x) -> bool:
+    return type(x) is int and x >= 0
 
 
 def sparsity(nnz: int, total: int) -> str:
@@ -95,7 +118,7 @@ def read_delta(blob: bytes, names):
     if hlen > len(blob) - 8:
         raise DeltaFileError("header runs past the end")
     try:
-        header = json.loads(blob[8:8 + hlen].decode("utf-8"))
+        header = _loads(blob[8:8 + hlen].decode("utf-8"))
     except (UnicodeDecodeError, json.JSONDecodeError) as e:
         raise DeltaFileError(f"header is not UTF-8 JSON: {e}") from None
     if not isinstance(header, dict):
@@ -104,16 +127,25 @@ def read_delta(blob: bytes, names):
     meta = header.pop("__metadata__", None)
     if not isinstance(meta, dict) or meta.get("sparse") != "True":
         raise DeltaFileError("not a delta (metadata sparse != True)")
+    version, changed = meta.get("model_version"), meta.get("changed_params")
+    if not isinstance(version, str) or not re.fullmatch(r"-?[0-9]+", version):
+        raise DeltaFileError("model_version is not a decimal integer")
+    version = int(version)
+    if not -(1 << 63) <= version < (1 << 63):
+        raise DeltaFileError("model_version does not fit 64 bits")
+    if not isinstance(changed, str):
+        raise DeltaFileError("changed_params missing")
     try:
-        version = int(meta["model_version"])
-        changed = json.loads(meta["changed_params"])
-    except (KeyError, ValueError) as e:
-        raise DeltaFileError(f"bad metadata: {e}") from None
+        changed = _loads(changed)
+    except json.JSONDecodeError as e:
+        raise DeltaFileError(f"changed_params is not JSON: {e}") from None
     if not isinstance(changed, list) or not all(isinstance(n, str) for n in changed):
         raise DeltaFileError("changed_params is not a list of names")
     if len(set(changed)) != len(changed):
         raise DeltaFileError("changed_params repeats a name")
     slot = {n: t for t, n in enumerate(names)}
+    if len(slot) != len(names):
+        raise ValueError("the table repeats a name")
     listed = set(changed)
     for key in header:
         base = key.rsplit(".", 1)[0] if key.endswith((".indices", ".values")) else None
@@ -124,8 +156,12 @@ def read_delta(blob: bytes, names):
         e = header.get(key)
         if not isinstance(e, dict) or e.get("dtype") != dtype:
             raise DeltaFileError(f"{key!r}: missing or not {dtype}")
-        shape, (a, b) = e["shape"], e["data_offsets"]
-        if len(shape) != 1 or not 0 <= a <= b <= len(data) or b - a != shape[0] * DTYPE_BYTES[dtype]:
+        shape, span = e.get("shape"), e.get("data_offsets")
+        if not (isinstance(shape, list) and len(shape) == 1 and _count(shape[0])
+                and isinstance(span, list) and len(span) == 2 and all(map(_count, span))):
+            raise DeltaFileError(f"{key!r}: shape or data_offsets malformed")
+        a, b = span
+        if not a <= b <= len(data) or b - a != shape[0] * DTYPE_BYTES[dtype]:
             raise DeltaFileError(f"{key!r}: shape and data offsets disagree")
         return shape[0], bytes(data[a:b])
 

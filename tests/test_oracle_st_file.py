@@ -167,3 +167,40 @@ def test_empty_delta_and_sparsity_edges():
     # no elements at all: sparsity 1; every element changed: 0
     assert st_file.sparsity(0, 0) == "1.000000"
     assert st_file.sparsity(5, 5) == "0.000000"
+
+
+def _raw(header_text: str, data: bytes = b"") -> bytes:
+    t = header_text.encode("utf-8")
+    return struct.pack("<Q", len(t)) + t + data
+
+
+def test_reader_takes_the_json_grammar_strictly():
+    # What Python's json module would let through but a safetensors header
+    # may not hold: repeated keys, NaN, true or 1.0 as a count, a padded or
+    # signed-plus model_version.  Each is refused; the well-formed variant
+    # of the same file (first line) is read.
+    md = '"__metadata__":{"sparse":"True","model_version":"%s","changed_params":"[\\"a\\"]"}'
+    good_entries = ('"a.indices":{"dtype":"I32","shape":[%s],"data_offsets":[0,4]},'
+                    '"a.values":{"dtype":"BF16","shape":[1],"data_offsets":[4,6]}')
+    data = struct.pack("<iH", 3, 0x3F80)
+    ok = _raw("{" + md % "5" + "," + good_entries % "1" + "}", data)
+    o, i, v, ver = st_file.read_delta(ok, ["a"])
+    assert o.tolist() == [0, 1] and i.tolist() == [3] and v.tolist() == [0x3F80] and ver == 5
+    assert st_file.read_delta(_raw(" {" + md % "-0" + "," + good_entries % "1" + "}  ", data),
+                              ["a"])[3] == 0
+    bad = [
+        "{" + md % "5" + "," + good_entries % "true" + "}",
+        "{" + md % "5" + "," + good_entries % "1.0" + "}",
+        "{" + md % "5" + "," + good_entries % "NaN" + "}",
+        "{" + md % " 5" + "," + good_entries % "1" + "}",
+        "{" + md % "+5" + "," + good_entries % "1" + "}",
+        "{" + md % "9223372036854775808" + "," + good_entries % "1" + "}",
+        "{" + md % "5" + "," + good_entries % "1" + "," + good_entries % "1" + "}",
+        "{" + md % "5" + "," + good_entries % "1" + "} x",
+        "[" + md % "5" + "]",
+    ]
+    for text in bad:
+        with pytest.raises(st_file.DeltaFileError):
+            st_file.read_delta(_raw(text, data), ["a"])
+    with pytest.raises(ValueError):
+        st_file.read_delta(ok, ["a", "a"])
