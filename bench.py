@@ -487,6 +487,29 @@ def rows_xor(args, dev, peak):
     out.update([row("xor_apply_layers_double_buffered_40x0.8GB", msp / 2, 5 * L * B, L * B, peak,
                     {"min_ms": round(mnp / 2, 4), "staging": "2 x 0.8 GB, D2D copy stream",
                      "exact": ok})])
+    # the same pipeline with the masks in pinned host memory (the host link
+    # bounds it): 4 layers, against a plain pinned H2D copy of one layer
+    LH = 4
+    hmasks = [torch.empty(B, dtype=torch.uint8, pin_memory=True) for _ in range(LH)]
+    for l in range(LH):
+        hmasks[l].copy_(masks[l])
+    ms_h2d, _ = time_reps(lambda: staging[0].copy_(hmasks[0], non_blocking=True), args.rows_reps)
+
+    def pipe_host2():
+        dws.xor_apply_layers(bufs[:LH], hmasks, staging[0], staging[1], copy_stream=cs)
+        dws.xor_apply_layers(bufs[:LH], hmasks, staging[0], staging[1], copy_stream=cs)
+
+    msh, mnh = time_reps(pipe_host2, max(2, args.rows_reps // 2))
+    dws.xor_apply(bufs[0], masks[0])
+    torch.cuda.synchronize()
+    ok_h = torch.equal(bufs[0], news[0])
+    dws.xor_apply(bufs[0], masks[0])
+    link = LH * B / (msh / 2) / 1e6
+    out["xor_apply_layers_pinned_host_4x0.8GB"] = {
+        "ms": round(msh / 2, 3), "min_ms": round(mnh / 2, 3), "link_GBps": round(link, 1),
+        "h2d_copy_GBps": round(B / ms_h2d / 1e6, 1), "link_frac": round(link / (B / ms_h2d / 1e6), 4),
+        "bound": "host link (plain pinned H2D copy of 0.8 GB timed in the same run)", "exact": ok_h}
+    del hmasks
     # the same layers as a sparse delta of 16-bit words (indices + values):
     # 680,000 changed bytes per layer travel as about 4 MB instead of 0.8 GB
     ow = [o.view(torch.bfloat16) for o in olds]
@@ -505,6 +528,28 @@ def rows_xor(args, dev, peak):
     ok = all(torch.equal(olds[l], news[l]) for l in (0, L - 1))
     out.update([row("apply_sparse_nvfp4_40x0.8GB", ms_a, 8 * snnz, L * B, peak,
                     {"min_ms": round(mn_a, 4), "exact": ok})])
+    # that delta arriving from pinned host memory: H2D of its 6 bytes per
+    # entry, then the apply (the dense masks would move all 32 GB)
+    hd = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in
+          (sd.offsets, sd.indices, sd.values)]
+    for h, x in zip(hd, (sd.offsets, sd.indices, sd.values)):
+        h.copy_(x)
+    rd = dws.Delta(torch.empty_like(sd.offsets), torch.empty_like(sd.indices),
+                   torch.empty_like(sd.values))
+
+    def host_apply():
+        for x, h in zip((rd.offsets, rd.indices, rd.values), hd):
+            x.copy_(h, non_blocking=True)
+        splan.apply(sst, rd)
+
+    ms_ha, mn_ha = time_reps(host_apply, args.rows_reps)
+    splan.raise_on_error("sparse xor apply from host")
+    hbytes = sum(h.numel() * h.element_size() for h in hd)
+    out["apply_sparse_from_pinned_host_nvfp4_40x0.8GB"] = {
+        "ms": round(ms_ha, 3), "min_ms": round(mn_ha, 3), "h2d_bytes": hbytes,
+        "link_GBps": round(hbytes / ms_ha / 1e6, 1),
+        "exact": all(torch.equal(olds[l], news[l]) for l in (0, L - 1))}
+    del hd, rd
     del ow, nw, splan, sot, snt, sd, sst
     del olds, news, masks, bufs, staging
     gc.collect()
@@ -564,6 +609,67 @@ def rows_stress_chain(args, dev, peak):
     gc.collect()
     torch.cuda.empty_cache()
     log(f"rows: stress chain done in {time.time() - t0:.1f}s")
+    return out
+
+
+def delta_file_rows(dws, plan, names, delta, args):
+    """The delta as a safetensors file: device arrays -> pinned host file
+    (header on the host + two D2H copies) and back (parse + H2D copies),
+    against plain pinned copies of the same bytes timed in the same run."""
+    import numpy as np
+    import torch
+    out = {}
+    T = len(names)
+    nnz = delta.count
+    arr = dws.make_name_array(names)
+    oh = delta.offsets.cpu().numpy()
+    cs = torch.cuda.current_stream().cuda_stream
+    st, fbytes = dws.dws_st_delta_write(plan.handle, arr, oh.ctypes.data, 1, delta.indices.data_ptr(),
+                                        delta.values.data_ptr(), None, 0, cs)
+    fbuf = torch.empty(fbytes, dtype=torch.uint8, pin_memory=True)
+
+    def write():
+        dws.dws_st_delta_write(plan.handle, arr, oh.ctypes.data, 1, delta.indices.data_ptr(),
+                               delta.values.data_ptr(), fbuf.data_ptr(), fbytes, cs)
+
+    ms_w, mn_w = time_reps(write, args.rows_reps)
+    hb = fbytes - 6 * nnz
+    body = fbuf[hb:]
+
+    def plain_d2h():
+        body[:4 * nnz].copy_(delta.indices.view(torch.uint8), non_blocking=True)
+        body[4 * nnz:].copy_(delta.values.view(torch.uint8), non_blocking=True)
+
+    ms_pd, _ = time_reps(plain_d2h, args.rows_reps)
+    out["delta_file_write_llama3_8b"] = {
+        "ms": round(ms_w, 3), "min_ms": round(mn_w, 3), "file_bytes": fbytes, "header_bytes": hb,
+        "GBps": round(fbytes / ms_w / 1e6, 1), "plain_d2h_ms": round(ms_pd, 3),
+        "link_frac": round(ms_pd / ms_w, 4),
+        "bound": "host link (plain pinned D2H copies of the same bytes timed in the same run)"}
+    oh2 = np.zeros(T + 1, dtype=np.int64)
+    r_off = torch.empty_like(delta.offsets)
+    r_idx = torch.empty_like(delta.indices)
+    r_val = torch.empty_like(delta.values)
+
+    def read():
+        dws.dws_st_delta_read(plan.handle, arr, fbuf.data_ptr(), fbytes, oh2.ctypes.data,
+                              r_off.data_ptr(), r_idx.data_ptr(), r_val.data_ptr(), nnz, cs)
+
+    ms_r, mn_r = time_reps(read, args.rows_reps)
+    torch.cuda.synchronize()
+    ok = (torch.equal(r_off, delta.offsets) and torch.equal(r_idx, delta.indices)
+          and torch.equal(r_val, delta.values))
+
+    def plain_h2d():
+        r_idx.view(torch.uint8).copy_(body[:4 * nnz], non_blocking=True)
+        r_val.view(torch.uint8).copy_(body[4 * nnz:], non_blocking=True)
+
+    ms_ph, _ = time_reps(plain_h2d, args.rows_reps)
+    out["delta_file_read_llama3_8b"] = {
+        "ms": round(ms_r, 3), "min_ms": round(mn_r, 3), "GBps": round(fbytes / ms_r / 1e6, 1),
+        "plain_h2d_ms": round(ms_ph, 3), "link_frac": round(ms_ph / ms_r, 4), "exact": ok,
+        "bound": "host link (plain pinned H2D copies of the same bytes timed in the same run)"}
+    del fbuf, body, r_off, r_idx, r_val
     return out
 
 
@@ -796,6 +902,7 @@ def run_ours(args):
         rows.update([row("encode_checksum_llama3_8b_lr%g" % args.lr, ms_s, 4 * N + 6 * nnz,
                          weight_bytes, peak, {"min_ms": round(mn_s, 4), "indices_equal": ok_s})])
         del hashes, coffs, cidx, cval
+        rows.update(delta_file_rows(dws, plan, [nm for nm, _ in shapes], delta, args))
         lr2 = 1e-5
         for t in range(T):
             new[t].copy_(make_new(lr2)(t, sizes[t]))

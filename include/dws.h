@@ -322,6 +322,76 @@ DWS_API dws_status_t dws_checksum(const uint8_t *positions, int64_t pos_bytes,
                           dws_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The delta file, [TRL] §4.1 and §4.3: a delta as a safetensors file (u64
+ * little-endian header length, UTF-8 JSON header, data) holding, for every
+ * parameter with at least one change, "{name}.indices" (I32, [n]) and
+ * "{name}.values" (BF16, [n]), with string metadata sparse = "True",
+ * model_version (decimal), sparsity (1 - nnz / elements, "%.6f") and
+ * changed_params (a JSON list of those names, table order).  Host code; the
+ * data moves with cudaMemcpyAsync on `stream`.
+ * ------------------------------------------------------------------------ */
+
+/* The header of the delta file of a delta with these offsets: the 8-byte
+ * length and the padded JSON, *header_bytes bytes in all; the file's data
+ * follows it: the offsets[T] int32 indices, then the offsets[T] bf16 values.
+ * Host only (no CUDA call), for callers that move the data themselves.
+ * Arguments, layout and errors as dws_st_delta_write; out (host, capacity
+ * bytes) NULL asks for the size only. */
+DWS_API dws_status_t dws_st_delta_header(const dws_plan_t *plan, const char *const *names,
+                                 const int64_t *offsets, int64_t model_version,
+                                 uint8_t *out, int64_t capacity, int64_t *header_bytes);
+
+/* Write the delta file of one delta in the dws_encode layout.  Layout of the
+ * file: [8-byte length][JSON: __metadata__, then name.indices and
+ * name.values per changed tensor in table order; compact, padded with spaces
+ * to 8 bytes][indices of all entries][values of all entries] -- the data is
+ * the two device arrays as they stand.
+ * names: host array of T distinct NUL-terminated UTF-8 strings.
+ * offsets: HOST int64[T+1] (a copy of the delta's offsets).
+ * indices, values: the delta's arrays (device, or any memory the CUDA runtime
+ * can copy from), offsets[T] entries each.
+ * file: host buffer of `capacity` bytes (pinned for an asynchronous copy);
+ * NULL asks for the size only (indices and values may then be NULL too).
+ * *file_bytes receives the file's size.  The
+ * header is written before the call returns; the data when `stream` reaches
+ * the two copies -- synchronise before using or freeing `file`.
+ * Errors: DWS_ERR_INVALID (null arguments, a name missing, not UTF-8 or
+ * repeated), DWS_ERR_BAD_DELTA (offsets not starting at 0, decreasing, or a
+ * count above its tensor's size), DWS_ERR_CAPACITY (capacity < *file_bytes;
+ * nothing written), DWS_ERR_CUDA. */
+DWS_API dws_status_t dws_st_delta_write(const dws_plan_t *plan, const char *const *names,
+                                const int64_t *offsets, int64_t model_version,
+                                const int32_t *indices, const uint16_t *values,
+                                uint8_t *file, int64_t capacity, int64_t *file_bytes,
+                                dws_stream_t stream);
+
+/* Read a delta file (any safetensors key order and data layout) into the
+ * dws_encode layout of the plan's table, ready for dws_apply.  The tensors
+ * applied are exactly those changed_params lists ([TRL] §4.3); the file is
+ * refused (DWS_ERR_BAD_DELTA, nothing enqueued) if it is not a delta
+ * (sparse != "True"), its header is not strict JSON in UTF-8 (a repeated key,
+ * NaN, a count that is not a plain integer), model_version is not a 64-bit
+ * decimal integer, changed_params names a parameter outside the table or
+ * twice, a listed parameter lacks an entry, an entry has another dtype, a
+ * shape that disagrees with its data_offsets, a range outside the data, or
+ * indices and values of different lengths, or the file holds an entry of a
+ * parameter it does not list.  Index values are not checked here: dws_apply
+ * validates them on the device.
+ * file: host memory, file_size bytes; it must stay valid until `stream`
+ * reaches the copies.  offsets_host: host int64[T+1], written (also the
+ * source of the copy into `offsets`: keep it until the stream gets there).
+ * offsets: device int64[T+1]; indices, values: device, `capacity` entries.
+ * *nnz receives the entry count and *model_version (nullable) the version.
+ * Errors: DWS_ERR_INVALID (null arguments, table names missing, not UTF-8 or
+ * repeated), DWS_ERR_BAD_DELTA as above, DWS_ERR_CAPACITY (nnz > capacity;
+ * *nnz and offsets_host set, nothing enqueued), DWS_ERR_CUDA. */
+DWS_API dws_status_t dws_st_delta_read(const dws_plan_t *plan, const char *const *names,
+                               const uint8_t *file, int64_t file_size, int64_t *offsets_host,
+                               int64_t *offsets, int32_t *indices, uint16_t *values,
+                               int64_t capacity, int64_t *nnz, int64_t *model_version,
+                               dws_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * XOR-mask variant, [XOR] paragraph 1: mask = old ^ new bit by bit, the same
  * size as the model; the receiver gets new = old ^ mask with no
  * floating-point arithmetic.  Works on any bytes (e.g. packed NVFP4).

@@ -75,6 +75,11 @@ _sig("dws_encode_global", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _
 _sig("dws_encode_checksum", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _vp])
 _sig("dws_pack_positions", _i32, [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp])
 _sig("dws_checksum", _i32, [_vp, _i64, _vp, _i64, _vp, _vp])
+_sig("dws_st_delta_header", _i32, [_vp, _vp, _vp, _i64, _vp, _i64, ctypes.POINTER(_i64)])
+_sig("dws_st_delta_write", _i32,
+     [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, ctypes.POINTER(_i64), _vp])
+_sig("dws_st_delta_read", _i32, [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _i64,
+                                 ctypes.POINTER(_i64), ctypes.POINTER(_i64), _vp])
 _sig("dws_xor_encode", _i32, [_vp, _vp, _vp, _i64, _vp])
 _sig("dws_xor_apply", _i32, [_vp, _vp, _i64, _vp])
 _sig("dws_xor_apply_layers", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i64, _vp, _vp])
@@ -209,6 +214,33 @@ def dws_checksum(positions, pos_bytes, values, nnz, hashes, stream) -> int:
     return _lib.dws_checksum(positions, pos_bytes, values, nnz, hashes, stream)
 
 
+def dws_st_delta_header(plan, names, offsets, model_version, out, capacity):
+    """Returns (status, header_bytes).  ``names``: see ``make_name_array``;
+    ``offsets``, ``out``: host pointers."""
+    n = ctypes.c_int64(0)
+    st = _lib.dws_st_delta_header(plan, names, offsets, model_version, out, capacity,
+                                  ctypes.byref(n))
+    return int(st), int(n.value)
+
+
+def dws_st_delta_write(plan, names, offsets, model_version, indices, values, file, capacity,
+                       stream):
+    """Returns (status, file_bytes)."""
+    n = ctypes.c_int64(0)
+    st = _lib.dws_st_delta_write(plan, names, offsets, model_version, indices, values, file,
+                                 capacity, ctypes.byref(n), stream)
+    return int(st), int(n.value)
+
+
+def dws_st_delta_read(plan, names, file, file_size, offsets_host, offsets, indices, values,
+                      capacity, stream):
+    """Returns (status, nnz, model_version)."""
+    nnz, ver = ctypes.c_int64(0), ctypes.c_int64(0)
+    st = _lib.dws_st_delta_read(plan, names, file, file_size, offsets_host, offsets, indices,
+                                values, capacity, ctypes.byref(nnz), ctypes.byref(ver), stream)
+    return int(st), int(nnz.value), int(ver.value)
+
+
 def dws_xor_encode(old_bytes, new_bytes, mask, nbytes, stream) -> int:
     return _lib.dws_xor_encode(old_bytes, new_bytes, mask, nbytes, stream)
 
@@ -248,6 +280,14 @@ def make_delta_array(deltas):
     arr = (dws_delta_t * max(1, len(deltas)))()
     for k, (o, i, v, c) in enumerate(deltas):
         arr[k] = dws_delta_t(o, i, v, c)
+    return arr
+
+
+def make_name_array(names):
+    """Tensor names (str) -> ctypes array of NUL-terminated UTF-8 strings."""
+    arr = (ctypes.c_char_p * max(1, len(names)))()
+    for k, n in enumerate(names):
+        arr[k] = n.encode("utf-8")
     return arr
 
 
@@ -449,6 +489,78 @@ class DeltaPlan:
                                   self.workspace_bytes, _stream_handle(stream)), "dws_pack_positions")
         self.raise_on_error("dws_pack_positions", stream)
         return positions[:int(pos_offsets[-1].item())], pos_offsets
+
+    # -- delta file (safetensors) --
+    def _host_offsets(self, offsets):
+        import numpy as np
+        if hasattr(offsets, "detach"):
+            offsets = offsets.detach().cpu().numpy()
+        o = np.ascontiguousarray(offsets, dtype=np.int64)
+        if o.size != self.num_tensors + 1:
+            raise ValueError("offsets must have T+1 entries")
+        return o
+
+    def delta_file_header(self, names, offsets, model_version: int) -> bytes:
+        """The delta file's header (length prefix + JSON) for these offsets."""
+        o = self._host_offsets(offsets)
+        arr = make_name_array(names)
+        st, n = dws_st_delta_header(self.handle, arr, o.ctypes.data, int(model_version), None, 0)
+        _check(st, "dws_st_delta_header")
+        buf = ctypes.create_string_buffer(max(1, n))
+        st, n = dws_st_delta_header(self.handle, arr, o.ctypes.data, int(model_version),
+                                    ctypes.addressof(buf), n)
+        _check(st, "dws_st_delta_header")
+        return buf.raw[:n]
+
+    def write_delta_file(self, delta: Delta, names, model_version: int, out=None, stream=None):
+        """The delta file of `delta` in a host uint8 tensor (pinned when this
+        call allocates it; `out` may pass a big enough one).  Reads the
+        offsets to the host and waits for the stream: the bytes are there on
+        return."""
+        torch = _torch()
+        o = self._host_offsets(delta.offsets)
+        arr = make_name_array(names)
+        _, i, v, _ = delta.as_ref()
+        st, need = dws_st_delta_write(self.handle, arr, o.ctypes.data, int(model_version), i, v,
+                                      None, 0, 0)
+        _check(st, "dws_st_delta_write")
+        if out is None or out.numel() < need:
+            out = torch.empty(max(1, need), dtype=torch.uint8, pin_memory=True)
+        sh = _stream_handle(stream)
+        st, need = dws_st_delta_write(self.handle, arr, o.ctypes.data, int(model_version), i, v,
+                                      out.data_ptr(), int(out.numel()), sh)
+        _check(st, "dws_st_delta_write")
+        (stream or torch.cuda.current_stream()).synchronize()
+        return out[:need]
+
+    def read_delta_file(self, file, names, capacity=None, stream=None):
+        """(Delta on the device, model_version) from a delta file held in a
+        host uint8 tensor or a bytes-like object.  Without `capacity` the
+        header is parsed twice (size, then copies).  Waits for the stream."""
+        import numpy as np
+        torch = _torch()
+        if not hasattr(file, "data_ptr"):
+            file = torch.frombuffer(bytearray(file), dtype=torch.uint8) if len(file) else \
+                torch.empty(0, dtype=torch.uint8)
+        arr = make_name_array(names)
+        oh = np.zeros(self.num_tensors + 1, dtype=np.int64)
+        offsets = torch.empty(self.num_tensors + 1, dtype=torch.int64, device=self.device)
+        fp, fs = (file.data_ptr() if file.numel() else 0), int(file.numel())
+        sh = _stream_handle(stream)
+        if capacity is None:
+            st, capacity, _ = dws_st_delta_read(self.handle, arr, fp, fs, oh.ctypes.data,
+                                                offsets.data_ptr(), 0, 0, 0, sh)
+            if st not in (DWS_OK, DWS_ERR_CAPACITY):
+                raise DwsError(st, "dws_st_delta_read")
+        indices = torch.empty(capacity, dtype=torch.int32, device=self.device)
+        values = torch.empty(capacity, dtype=torch.int16, device=self.device)
+        st, nnz, ver = dws_st_delta_read(self.handle, arr, fp, fs, oh.ctypes.data,
+                                         offsets.data_ptr(), indices.data_ptr() if capacity else 0,
+                                         values.data_ptr() if capacity else 0, capacity, sh)
+        if st != DWS_OK:
+            raise DwsError(st, "dws_st_delta_read", nnz if st == DWS_ERR_CAPACITY else None)
+        (stream or torch.cuda.current_stream()).synchronize()
+        return Delta(offsets, indices[:nnz], values[:nnz]), ver
 
     def apply_chain(self, snap_table, deltas, stream=None, mode=DWS_CHAIN_AUTO):
         arr = make_delta_array([d.as_ref() for d in deltas])

@@ -80,6 +80,13 @@ struct dws_plan {
     std::vector<unsigned char> image;  // header + numel + first_tile, as uploaded
 };
 
+bool dws::plan_numels(const dws_plan_t *plan, int32_t *num_tensors, const long long **numels) {
+    if (plan == nullptr) return false;
+    *num_tensors = plan->T;
+    *numels = reinterpret_cast<const long long *>(plan->image.data() + plan->layout.numel_off);
+    return true;
+}
+
 namespace {
 
 uint64_t fnv1a(uint64_t h, uint64_t v) {

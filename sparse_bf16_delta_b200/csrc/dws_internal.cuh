@@ -438,4 +438,8 @@ cudaError_t launch_checksum(const uint8_t *positions, long long nbytes, const ui
 cudaError_t launch_xor(const uint8_t *a, const uint8_t *b, uint8_t *out, long long nbytes,
                        cudaStream_t s);
 
+// The plan's tensor count and per-tensor element counts (host memory owned by
+// the plan).  False for a null plan.
+bool plan_numels(const dws_plan_t *plan, int32_t *num_tensors, const long long **numels);
+
 }  // namespace dws
