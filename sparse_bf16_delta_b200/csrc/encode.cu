@@ -18,9 +18,12 @@
 //     released: two 1-D bulk async copies (cp.async.bulk, global -> own
 //     shared memory, mbarrier transaction count, L2 evict-first) bring both
 //     snapshots' 16 KiB of the tile.
-//   * Two counting groups of 4 warps take the stage fills in turn (group g
+//   * Two counting groups of 8 warps take the stage fills in turn (group g
 //     the fills g, g + 2, ...), so two tiles are counted at once and one
-//     group's barriers and latencies overlap the other's work.  Per tile:
+//     group's barriers and latencies overlap the other's work.  Eight warps
+//     a group (32 elements a thread) keep a stage busy for half the time
+//     four did, which matters most when many elements change: each thread
+//     moves its own changed entries into the ring.  Per tile:
 //     detect, block scan, publish the tile's count, move the changed
 //     (offset, value) pairs into the group's shared ring, queue the tile,
 //     release the stage.  A stage is busy only from its refill to its
@@ -33,7 +36,7 @@
 //     from the ring with consecutive lanes storing consecutive entries
 //     (coalesced), and releases its ring space.
 //   * detect: 16-byte shared-memory reads in a bank-conflict-free order, a
-//     64-bit change mask per thread, popc; block scan of the counts.
+//     32-bit change mask per thread, popc; block scan of the counts.
 //   * scan: decoupled look-back over the tile status words (flag + 62-bit
 //     count), one word per 32-byte sector so that the words every look-back
 //     reads (the newest tiles') spread over four times as many L2 lines.  A
@@ -52,10 +55,10 @@ namespace dws {
 namespace {
 
 constexpr int kGroups = 2;      // counting groups; group g counts stage fills g, g + 2, ...
-constexpr int kGroupWarps = 4;  // warps per counting group
+constexpr int kGroupWarps = 8;  // warps per counting group
 constexpr int kGroupThreads = 32 * kGroupWarps;
 constexpr int kCountWarps = kGroups * kGroupWarps;
-constexpr int kElemsPerThread = kTileElems / kGroupThreads;  // 64
+constexpr int kElemsPerThread = kTileElems / kGroupThreads;  // 32
 constexpr int kLookWarps = 3;                     // the look-back group
 constexpr int kProducerWarp = kCountWarps + kLookWarps;
 constexpr int kPublishThread = 64;  // of a group: publishes tile counts (its thread 0 keeps the queue)
@@ -64,7 +67,7 @@ constexpr int kStages = 4;
 constexpr int kRing = 8192;  // per group: pending (offset | value << 16) entries
 constexpr int kQueue = 64;   // pending tiles
 constexpr int kCountBar = 1;  // named barrier of group g: kCountBar + g
-static_assert(kElemsPerThread == 64, "each counting thread owns 8 chunks of 8 elements");
+static_assert(kElemsPerThread == 32, "each counting thread owns 4 chunks of 8 elements");
 static_assert(kStages % kGroups == 0, "a stage always serves the same group");
 static_assert((kRing & (kRing - 1)) == 0 && kRing >= kTileElems, "ring holds any tile");
 
@@ -317,15 +320,15 @@ __device__ void produce(const EncodeParams &p, EncodeSmem &sm) {
 // ---------------------------------------------------------------------------
 // Counting groups: group g is threads g * kGroupThreads .. + kGroupThreads - 1
 // ---------------------------------------------------------------------------
-// A warp whose 2048 elements all changed (a clustered run): each thread's
-// 64 entries are its slice itself, read as 16-byte chunks in a rotated,
+// A warp whose 1024 elements all changed (a clustered run): each thread's
+// 32 entries are its slice itself, read as 16-byte chunks in a rotated,
 // bank-conflict-free order, with no bit scan.  Kept out of line so that the
 // common path's code is left as it is.
 __device__ __noinline__ void dense_slice_to_ring(uint32_t *ring, int rr0, int o0, const uint16_t *new_s,
                                                  int tid) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const int cr = (c + tid) & 7;
+    for (int c = 0; c < 4; ++c) {
+        const int cr = (c + (tid >> 1)) & 3;
         const uint4 w = *reinterpret_cast<const uint4 *>(new_s + o0 + 8 * cr);
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -392,12 +395,12 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
 
         uint16_t *old_s = sm.buf[s][0];
         uint16_t *new_s = sm.buf[s][1];
-        uint32_t mask_lo = 0, mask_hi = 0;  // elements 64 tid + [0, 32) and + [32, 64)
+        uint32_t mask = 0;  // elements 32 tid + [0, 32)
         if (work) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int slot = (tid + j) & 7;  // conflict-free 16-byte reads
-                const int e0 = (8 * tid + slot) * 8;
+            for (int j = 0; j < 4; ++j) {
+                const int slot = ((tid >> 1) + j) & 3;  // conflict-free 16-byte reads
+                const int e0 = (4 * tid + slot) * 8;
                 uint4 a, b;
                 if (e0 + 8 <= d.bulk) {
                     a = *reinterpret_cast<const uint4 *>(old_s + e0);
@@ -425,11 +428,10 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
                                        (((x1 & 0xffffu) != 0) << 2) | (((x1 >> 16) != 0) << 3) |
                                        (((x2 & 0xffffu) != 0) << 4) | (((x2 >> 16) != 0) << 5) |
                                        (((x3 & 0xffffu) != 0) << 6) | (((x3 >> 16) != 0) << 7);
-                if (slot < 4) mask_lo |= bits8 << (8 * slot);
-                else mask_hi |= bits8 << (8 * (slot - 4));
+                mask |= bits8 << (8 * slot);
             }
         }
-        const int cnt = __popc(mask_lo) + __popc(mask_hi);
+        const int cnt = __popc(mask);
         int incl = cnt;
 #pragma unroll
         for (int dd = 1; dd < 32; dd <<= 1) {
@@ -502,20 +504,17 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
                 break;
             }
         }
-        if (kCompact && __all_sync(0xffffffffu, (mask_lo & mask_hi) == 0xffffffffu)) {
+        if (kCompact && __all_sync(0xffffffffu, mask == 0xffffffffu)) {
             dense_slice_to_ring(ring, pos + warp_off + incl - cnt, kElemsPerThread * tid, new_s, tid);
         } else if (kCompact) {
             int rr = pos + warp_off + incl - cnt;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t mm = h ? mask_hi : mask_lo;
-                while (mm) {
-                    const int bit = __ffs(mm) - 1;
-                    mm &= mm - 1;
-                    const int o = kElemsPerThread * tid + 32 * h + bit;
-                    ring[rr & (kRing - 1)] = static_cast<uint32_t>(o) | (static_cast<uint32_t>(new_s[o]) << 16);
-                    ++rr;
-                }
+            uint32_t mm = mask;
+            while (mm) {
+                const int bit = __ffs(mm) - 1;
+                mm &= mm - 1;
+                const int o = kElemsPerThread * tid + bit;
+                ring[rr & (kRing - 1)] = static_cast<uint32_t>(o) | (static_cast<uint32_t>(new_s[o]) << 16);
+                ++rr;
             }
         }
         named_bar(bar, kGroupThreads);  // (C) entries in the ring, stage s consumed
