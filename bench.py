@@ -824,24 +824,37 @@ def run_ours(args):
     }
 
     # ---- e2e: new snapshot from pinned host memory, delta through the host --
+    # as the delta file of the pages' wire format: the trainer side writes it
+    # into pinned host memory, the receiver side reads it back and applies it.
     if not args.no_e2e:
+        import numpy as np
         host_new = torch.empty_like(new_flat, device="cpu").pin_memory()
         host_new.copy_(new_flat)
+        names_arr = dws.make_name_array([nm for nm, _ in shapes])
         h_off = torch.empty_like(offsets, device="cpu").pin_memory()
-        h_idx = torch.empty_like(indices, device="cpu").pin_memory()
-        h_val = torch.empty_like(values, device="cpu").pin_memory()
+        h_off_np = h_off.numpy()
+        h_off.copy_(offsets)
+        st_, fcap = dws.dws_st_delta_write(plan.handle, names_arr, h_off_np.ctypes.data, 1, 0, 0,
+                                           None, 0, 0)
+        fbuf = torch.empty(fcap, dtype=torch.uint8, pin_memory=True)
+        oh2 = np.zeros(T + 1, dtype=np.int64)
         r_off, r_idx, r_val = torch.empty_like(offsets), torch.empty_like(indices), torch.empty_like(values)
         rdelta = dws.Delta(r_off, r_idx, r_val)
+        cs_e = torch.cuda.current_stream()
+        codes = []
 
         def e2e_step():
             new_flat.copy_(host_new, non_blocking=True)
             plan.encode_into(ot, nt, offsets, indices, values)
             h_off.copy_(offsets, non_blocking=True)
-            h_idx.copy_(indices, non_blocking=True)
-            h_val.copy_(values, non_blocking=True)
-            r_off.copy_(h_off, non_blocking=True)
-            r_idx.copy_(h_idx, non_blocking=True)
-            r_val.copy_(h_val, non_blocking=True)
+            cs_e.synchronize()  # the file's header needs the counts
+            cw, fb = dws.dws_st_delta_write(plan.handle, names_arr, h_off_np.ctypes.data, 1,
+                                            indices.data_ptr(), values.data_ptr(), fbuf.data_ptr(),
+                                            fcap, cs_e.cuda_stream)
+            cr, _, _ = dws.dws_st_delta_read(plan.handle, names_arr, fbuf.data_ptr(), fb,
+                                             oh2.ctypes.data, r_off.data_ptr(), r_idx.data_ptr(),
+                                             r_val.data_ptr(), r_idx.numel(), cs_e.cuda_stream)
+            codes.append((cw, cr))
             plan.apply(st, rdelta)
 
         e2e_step()
@@ -855,14 +868,16 @@ def run_ours(args):
         b.record()
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b), world, dev) / args.e2e_steps
-        dbytes = 8 * (T + 1) + 6 * nnz
-        ok = bool(torch.equal(snap_flat, new_flat)) and plan.status()[0] == dws.DWS_OK
+        ok = (bool(torch.equal(snap_flat, new_flat)) and plan.status()[0] == dws.DWS_OK
+              and all(c == (dws.DWS_OK, dws.DWS_OK) for c in codes))
         line["e2e"] = {"value": round(replicas_value(world, weight_bytes, e_ms), 2), "unit": "GB/s",
-                       "h2d_bytes_per_step": 2 * new_flat.numel() + dbytes,
-                       "d2h_bytes_per_step": dbytes, "ms_per_step": round(e_ms, 3),
-                       "steps": args.e2e_steps, "exact": ok,
-                       "path": "pinned host new snapshot -> H2D -> dws_encode -> delta D2H -> H2D -> dws_apply"}
-        del host_new, h_off, h_idx, h_val, r_off, r_idx, r_val
+                       "h2d_bytes_per_step": 2 * new_flat.numel() + 6 * nnz + 8 * (T + 1),
+                       "d2h_bytes_per_step": 8 * (T + 1) + 6 * nnz, "ms_per_step": round(e_ms, 3),
+                       "steps": args.e2e_steps, "exact": ok, "delta_file_bytes": fcap,
+                       "path": ("pinned host new snapshot -> H2D -> dws_encode -> offsets D2H -> "
+                                "dws_st_delta_write (delta file into pinned host memory) -> "
+                                "dws_st_delta_read (back into device arrays) -> dws_apply")}
+        del host_new, h_off, fbuf, r_off, r_idx, r_val, rdelta
 
     # ---- encode / apply at lr 1e-5 and count-only ----------------------------
     if not args.no_rows:
