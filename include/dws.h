@@ -144,6 +144,21 @@ DWS_API dws_status_t dws_encode(const dws_plan_t *plan,
                         int64_t capacity,
                         void *workspace, size_t workspace_bytes, dws_stream_t stream);
 
+/* dws_encode that also delivers the entry count where the caller wants it,
+ * so that no host code has to read it element by element ([verl] review:
+ * per-parameter .item() calls serialised the host; one transfer replaces
+ * them).  After the encode, on `stream`: offsets[T] is copied to nnz_dev
+ * (nullable; device int64) and to nnz_host (nullable; host int64, pinned
+ * for the copy to stay asynchronous -- cudaMallocHost, cudaHostAlloc or a
+ * pinned torch tensor).  The values are there once the stream has reached
+ * the copies (synchronise the stream, or an event recorded after the call).
+ * Everything else, including errors, as dws_encode. */
+DWS_API dws_status_t dws_encode_nnz(const dws_plan_t *plan,
+                            const void *const *old_ptrs, const void *const *new_ptrs,
+                            int64_t *offsets, int32_t *indices, uint16_t *values,
+                            int64_t capacity, int64_t *nnz_dev, int64_t *nnz_host,
+                            void *workspace, size_t workspace_bytes, dws_stream_t stream);
+
 /* dws_encode with global int64 positions: [verl] sparse_gather.py
  * shard_delta_indices diffs a rank's local shard of a parameter and returns
  * global_idx = local_idx (as int64) + offset, the shard's first element in the

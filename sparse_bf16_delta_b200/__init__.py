@@ -10,7 +10,7 @@ in libdws's CUDA kernels:
 
 Importing this package loads ``libdws.so`` from the package directory and
 raises ``ImportError`` if it is missing: there is no CPU fallback.  Build it
-with ``python -m sparse_bf16_delta_b200._build`` (or ``__graft_entry__.build()``).
+with ``python sparse_bf16_delta_b200/_build.py`` (or ``__graft_entry__.build()``).
 """
 from __future__ import annotations
 
@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libdws.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"libdws.so not found at {LIB_PATH}; build it with "
-        "`python -m sparse_bf16_delta_b200._build` (needs nvcc for sm_100a)")
+        "`python sparse_bf16_delta_b200/_build.py` (needs nvcc for sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -64,6 +64,7 @@ _sig("dws_tile_elems", _i64, [])
 _sig("dws_plan_workspace_bytes", _sz, [_vp])
 _sig("dws_plan_upload", _i32, [_vp, _vp, _sz, _vp])
 _sig("dws_encode", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
+_sig("dws_encode_nnz", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _vp])
 _sig("dws_encode_ex", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp, _i64, _i64])
 _sig("dws_count", _i32, [_vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _sig("dws_encode_noalloc", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp])
@@ -148,6 +149,12 @@ def dws_encode(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, wor
                workspace_bytes, stream) -> int:
     return _lib.dws_encode(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
                            workspace, workspace_bytes, stream)
+
+
+def dws_encode_nnz(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, nnz_dev,
+                   nnz_host, workspace, workspace_bytes, stream) -> int:
+    return _lib.dws_encode_nnz(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
+                               nnz_dev, nnz_host, workspace, workspace_bytes, stream)
 
 
 def dws_encode_ex(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, workspace,
@@ -425,6 +432,19 @@ class DeltaPlan:
         self.raise_on_error("dws_encode", stream)
         nnz = int(offsets[-1].item())
         return Delta(offsets, indices[:nnz], values[:nnz])
+
+    def encode_into_nnz(self, old_table, new_table, offsets, indices, values, nnz_dev=None,
+                        nnz_host=None, stream=None):
+        """encode_into that also copies the entry count to a device int64
+        tensor and/or a pinned host int64 tensor after the encode (valid once
+        the stream has reached the copies)."""
+        _check(dws_encode_nnz(self.handle, old_table.data_ptr(), new_table.data_ptr(),
+                              offsets.data_ptr(), indices.data_ptr() if indices.numel() else 0,
+                              values.data_ptr() if values.numel() else 0, int(indices.numel()),
+                              nnz_dev.data_ptr() if nnz_dev is not None else 0,
+                              nnz_host.data_ptr() if nnz_host is not None else 0,
+                              self.workspace.data_ptr(), self.workspace_bytes,
+                              _stream_handle(stream)), "dws_encode_nnz")
 
     def encode_exact(self, old_table, new_table, stream=None) -> Delta:
         """Count first, then encode into exactly-sized buffers (two passes)."""

@@ -230,6 +230,22 @@ dws_status_t dws_encode(const dws_plan_t *plan, const void *const *old_ptrs,
                          workspace_bytes, stream, true, 0, -1);
 }
 
+dws_status_t dws_encode_nnz(const dws_plan_t *plan, const void *const *old_ptrs,
+                            const void *const *new_ptrs, int64_t *offsets, int32_t *indices,
+                            uint16_t *values, int64_t capacity, int64_t *nnz_dev, int64_t *nnz_host,
+                            void *workspace, size_t workspace_bytes, dws_stream_t stream) {
+    dws_status_t st = encode_common(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
+                                    workspace, workspace_bytes, stream, true, 0, -1);
+    if (st != DWS_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t *total = offsets + plan->T;
+    cudaError_t e = cudaSuccess;
+    if (nnz_dev != nullptr) e = cudaMemcpyAsync(nnz_dev, total, sizeof(int64_t), cudaMemcpyDefault, s);
+    if (e == cudaSuccess && nnz_host != nullptr)
+        e = cudaMemcpyAsync(nnz_host, total, sizeof(int64_t), cudaMemcpyDefault, s);
+    return from_cuda(e);
+}
+
 dws_status_t dws_encode_ex(const dws_plan_t *plan, const void *const *old_ptrs,
                            const void *const *new_ptrs, int64_t *offsets, int32_t *indices,
                            uint16_t *values, int64_t capacity, void *workspace,

@@ -2,8 +2,23 @@
 comparing libdws outputs with the CPU oracle."""
 from __future__ import annotations
 
+import importlib.util
+import os
+
 import numpy as np
 import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def build_module():
+    """sparse_bf16_delta_b200/_build.py, loaded by path (importing the package
+    would need the library it builds)."""
+    path = os.path.join(ROOT, "sparse_bf16_delta_b200", "_build.py")
+    spec = importlib.util.spec_from_file_location("dws_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
 
 
 def host_bits(t: torch.Tensor) -> np.ndarray:

@@ -20,8 +20,8 @@ def _declared_symbols():
 
 @pytest.fixture(scope="module")
 def lib():
-    from sparse_bf16_delta_b200 import _build
-    path = _build.build()
+    from tests._dev import build_module
+    path = build_module().build()
     return ctypes.CDLL(path)
 
 
@@ -34,8 +34,8 @@ def test_header_declares_the_boundary():
 
 
 def test_library_exports_every_declared_symbol(lib):
-    from sparse_bf16_delta_b200 import _build
-    out = subprocess.run(["nm", "-D", "--defined-only", _build.LIB_PATH], capture_output=True,
+    from tests._dev import build_module
+    out = subprocess.run(["nm", "-D", "--defined-only", build_module().LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
     missing = [s for s in _declared_symbols() if s not in exported]
@@ -95,6 +95,8 @@ def test_host_side_argument_errors_need_no_device():
         assert dws.dws_apply_chain(p, 1, arr, 65, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_encode_global(p, 1, 1, None, 1, 1, 1, 10, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_encode_checksum(p, 1, 1, 1, 1, 1, 10, None, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_encode_nnz(p, 1, 1, 1, 1, 1, 10, 1, 1, None, 0, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_encode_nnz(p, 1, 1, 1, 1, 1, -1, 1, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_pack_positions(p, 1, 1, 4, 0x1001, 8, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_checksum(1, -1, 1, 1, 0x1000, None) == dws.DWS_ERR_INVALID
         assert dws.dws_pos_width(p, 0) == 2 and dws.dws_pos_width(p, 1) == 0

@@ -169,6 +169,37 @@ def test_encode_into_unaligned_outputs(dws, shift):
     assert (ib[:shift].cpu().numpy() == -7).all() and (ib[shift + nnz:].cpu().numpy() == -7).all()
 
 
+def test_encode_reports_nnz_to_device_and_pinned_host(dws):
+    # The entry count arrives in a device scalar and a pinned host scalar
+    # after the encode, on the encode's stream, equal to the oracle's.
+    rng = np.random.default_rng(91)
+    pairs = [_random_pair(rng, n, 0.05) for n in (0, 7, 8192 * 3 + 11, 70000)]
+    olds = [dev_bits(a) for a, _ in pairs]
+    news = [dev_bits(b) for _, b in pairs]
+    want = oracle.encode([a for a, _ in pairs], [b for _, b in pairs])
+    plan = dws.DeltaPlan.for_tensors(olds)
+    cap = int(want[0][-1]) + 5
+    offsets = torch.empty(len(pairs) + 1, dtype=torch.int64, device="cuda")
+    indices = torch.full((cap,), -1, dtype=torch.int32, device="cuda")
+    values = torch.full((cap,), -1, dtype=torch.int16, device="cuda")
+    nnz_dev = torch.full((1,), -1, dtype=torch.int64, device="cuda")
+    nnz_host = torch.full((1,), -1, dtype=torch.int64).pin_memory()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        plan.encode_into_nnz(dws.ptr_table(olds), dws.ptr_table(news), offsets, indices, values,
+                             nnz_dev=nnz_dev, nnz_host=nnz_host, stream=s)
+    s.synchronize()
+    plan.raise_on_error("dws_encode_nnz")
+    assert int(nnz_host[0]) == int(nnz_dev.item()) == int(want[0][-1])
+    nnz = int(want[0][-1])
+    assert_delta_equal((offsets.cpu().numpy(), indices[:nnz].cpu().numpy(),
+                        values[:nnz].cpu().numpy().view(np.uint16)), want)
+    # either output may be left out
+    plan.encode_into_nnz(dws.ptr_table(olds), dws.ptr_table(news), offsets, indices, values)
+    torch.cuda.synchronize()
+    plan.raise_on_error("dws_encode_nnz")
+
+
 def test_encode_identical_and_all_changed(dws):
     rng = np.random.default_rng(29)
     a = rng.integers(0, 1 << 16, 1_000_003, dtype=np.uint16)

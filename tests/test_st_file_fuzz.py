@@ -19,8 +19,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def fuzzer(tmp_path_factory):
-    from sparse_bf16_delta_b200 import _build
-    nvcc = _build.nvcc()
+    from tests._dev import build_module
+    nvcc = build_module().nvcc()
     if (shutil.which(nvcc) is None and not os.path.exists(nvcc)) or shutil.which("g++") is None:
         pytest.skip("nvcc and g++ are needed to build the fuzzer")
     d = tmp_path_factory.mktemp("fuzz")

@@ -27,8 +27,8 @@ from tests.test_oracle_st_file import _random_delta  # noqa: E402
 
 @pytest.fixture(scope="module")
 def dws():
-    from sparse_bf16_delta_b200 import _build
-    _build.build()
+    from tests._dev import build_module
+    build_module().build()
     import sparse_bf16_delta_b200 as m
     return m
 
