@@ -7,7 +7,10 @@
  * (per tensor: ascending int32 element indices and the bf16 values there),
  * the receiver-side scatter of one delta or of a chain of deltas onto an
  * anchor snapshot, and the dense XOR-mask variant for packed low-precision
- * weights.  Everything is integer work on raw bits and bit-exact.
+ * weights; around them, the wire form of a delta (narrow positions and a
+ * checksum), the encode with int64 global positions of a rank's shard, and
+ * the delta as a safetensors file moved straight between device arrays and
+ * host memory.  Everything is integer work on raw bits and bit-exact.
  *
  * Sources, by page title and section:
  *   [TRL]  "Shipping a Trillion Parameters With a Hub Bucket: Delta Weight
@@ -34,7 +37,9 @@
  *     a delta, a bounded wait that ran out) are recorded in the workspace's
  *     status word and read with dws_status().
  *   - "device array" means an array in device memory; "host array" an array
- *     in host memory that may be freed as soon as the call returns.
+ *     in host memory that may be freed as soon as the call returns (the
+ *     delta-file functions and dws_xor_apply_layers say which of their host
+ *     buffers must outlive the copies they enqueue).
  *   - Calls that share one workspace must be ordered on one stream (or by
  *     events): the workspace holds per-call scratch.
  *   - Element indices are local to their tensor, 0-based, row-major flat,
