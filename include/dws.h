@@ -435,7 +435,9 @@ DWS_API dws_status_t dws_xor_apply(void *buf, const void *mask, int64_t nbytes, 
  * staging_bytes is split into staging-sized units.  Events order the two
  * streams; copy_stream first waits for work already queued on apply_stream,
  * and when the call's work on apply_stream is done, all of it is done.
- * bufs, masks, nbytes: host arrays of L entries (device/host pointers).
+ * bufs, masks, nbytes: host arrays of L entries (device/host pointers); the
+ * arrays may be freed on return, the masks they point to only once the call's
+ * work on apply_stream is done.
  * staging0/1: device buffers of staging_bytes each (caller-owned). */
 DWS_API dws_status_t dws_xor_apply_layers(void *const *bufs, const void *const *masks,
                                   const int64_t *nbytes, int32_t L,
