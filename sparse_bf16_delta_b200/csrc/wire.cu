@@ -9,7 +9,8 @@
 //   (every position fits in 16 bits) and 4 otherwise.  A one-CTA pass scans
 //   the per-parameter byte counts into pos_offsets; then every block of 2048
 //   entries finds its parameters (warp-cooperative search over the delta's
-//   offsets) and stores 2-byte halves.
+//   offsets) and stores each position whole (4 bytes) where its address is
+//   4-byte aligned, else as 2-byte halves.
 //
 // dws_checksum: hash(positions) and hash(values), where hash() XOR-reduces
 //   the elements widened to 64 bits: a byte zero-extended, a bf16 value
@@ -127,9 +128,14 @@ __global__ void __launch_bounds__(kPackThreads) pack_positions_kernel(PackParams
         const int w = pos_width_of(n);
         const long long at = p.pos_offsets[t] + (j - p.d.offsets[t]) * w;
         if (at + w > p.pos_capacity) continue;  // recorded by the offsets pass
-        uint16_t *dst = reinterpret_cast<uint16_t *>(p.positions + at);  // at is even
-        dst[0] = static_cast<uint16_t>(i & 0xffff);
-        if (w == 4) dst[1] = static_cast<uint16_t>(static_cast<uint32_t>(i) >> 16);
+        uint8_t *dst = p.positions + at;  // even
+        if (w == 4 && (reinterpret_cast<uintptr_t>(dst) & 3u) == 0) {
+            *reinterpret_cast<uint32_t *>(dst) = static_cast<uint32_t>(i);
+        } else {
+            uint16_t *d16 = reinterpret_cast<uint16_t *>(dst);
+            d16[0] = static_cast<uint16_t>(i & 0xffff);
+            if (w == 4) d16[1] = static_cast<uint16_t>(static_cast<uint32_t>(i) >> 16);
+        }
     }
 }
 
