@@ -55,6 +55,25 @@ def _check_segments(delta, olds, news, tensors):
         np.testing.assert_array_equal(delta.values[lo:hi].cpu().numpy().view(np.uint16), v)
 
 
+def _check_absorption(delta, olds, s, k, lr, tensors):
+    """The absorption rule, evaluated independently from the old weights and
+    the step's noise (exact midpoints in double precision), predicts exactly
+    the positions the encode listed, tensor by tensor."""
+    offs = delta.offsets.cpu().numpy()
+    for t in tensors:
+        u = W.update_noise(olds[t].numel(), W.step_seed(s, k, t), "cuda").cpu().numpy()
+        changed, cnt = oracle.absorption_predict(host_bits(olds[t]), u, lr)
+        assert cnt == offs[t + 1] - offs[t], t
+        np.testing.assert_array_equal(np.flatnonzero(changed),
+                                      delta.indices[offs[t]:offs[t + 1]].cpu().numpy())
+        del u, changed
+
+
+_LAYER0 = ["self_attn.q_proj", "self_attn.k_proj", "self_attn.v_proj", "self_attn.o_proj",
+           "mlp.gate_proj", "mlp.up_proj", "mlp.down_proj", "input_layernorm",
+           "post_attention_layernorm"]
+
+
 @pytest.mark.parametrize("lr", [3e-6, 1e-5])
 def test_llama3_8b_encode_apply_full(dws, lr):
     s = W.SEEDS["llama3_8b"]
@@ -76,14 +95,11 @@ def test_llama3_8b_encode_apply_full(dws, lr):
              [names.index("model.layers.31.input_layernorm.weight"), names.index("model.norm.weight"),
               names.index("lm_head.weight")]
     _check_segments(d, old, new, sample)
-    # the absorption rule predicts exactly the encoded positions (layer 0 q_proj, a norm)
-    offs = d.offsets.cpu().numpy()
-    for t in (names.index("model.layers.0.self_attn.q_proj.weight"),
-              names.index("model.layers.0.input_layernorm.weight")):
-        u = W.update_noise(sizes[t], W.step_seed(s, 1, t), dev).cpu().numpy()
-        changed, cnt = oracle.absorption_predict(host_bits(old[t]), u, lr)
-        assert cnt == offs[t + 1] - offs[t]
-        np.testing.assert_array_equal(np.flatnonzero(changed), d.indices[offs[t]:offs[t + 1]].cpu().numpy())
+    # the absorption rule predicts exactly the encoded positions: the embedding,
+    # every weight and norm of layer 0, the final norm (12 tensors)
+    _check_absorption(d, old, s, 1, lr,
+                      [names.index("model.embed_tokens.weight"), names.index("model.norm.weight")] +
+                      [names.index(f"model.layers.0.{m}.weight") for m in _LAYER0])
     # apply onto a copy of old gives new, bit for bit, everywhere
     snap_flat = old_flat.clone()
     snap = [snap_flat[v.storage_offset():][:v.numel()] for v in old]
@@ -112,6 +128,11 @@ def test_qwen3_0p6b_chain_full(dws):
         assert list(np.diff(d.offsets.cpu().numpy())) == _counts_by_torch(prev, cur)
         if k == 1:
             _check_segments(d, prev, cur, range(len(sizes)))  # the whole step, every tensor
+            names = [nm for nm, _ in shapes]
+            _check_absorption(d, prev, s, 1, 3e-6,
+                              [names.index("model.embed_tokens.weight")] +
+                              [names.index(f"model.layers.0.{m}.weight")
+                               for m in _LAYER0 + ["self_attn.q_norm", "self_attn.k_norm"]])
         elif k == 10:
             _check_segments(d, prev, cur, [0, 1, 5, 6, 7, 10, 309])
         deltas.append(d)
