@@ -119,3 +119,10 @@ def test_product_path_does_not_reach_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "oracle.h" not in text and "liboracle" not in text, f
+    # and the other way: the oracle reaches neither the package nor libdws
+    for dirpath, _, files in os.walk(os.path.join(ROOT, "oracle")):
+        for f in files:
+            if f.endswith((".py", ".c", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "sparse_bf16_delta_b200" not in text and "libdws" not in text, f
+                assert "dws.h" not in text and "dws_internal" not in text, f
