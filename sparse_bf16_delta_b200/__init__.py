@@ -511,6 +511,14 @@ class DeltaPlan:
         return positions[:int(pos_offsets[-1].item())], pos_offsets
 
     # -- delta file (safetensors) --
+    @staticmethod
+    def _host_bytes(buf, what):
+        """The file buffer is read and written by host code: a contiguous
+        uint8 tensor in CPU memory."""
+        if buf.device.type != "cpu" or buf.dtype != _torch().uint8 or not buf.is_contiguous():
+            raise ValueError(f"{what} must be a contiguous uint8 tensor in host memory")
+        return buf
+
     def _host_offsets(self, offsets):
         import numpy as np
         if hasattr(offsets, "detach"):
@@ -544,6 +552,8 @@ class DeltaPlan:
         st, need = dws_st_delta_write(self.handle, arr, o.ctypes.data, int(model_version), i, v,
                                       None, 0, 0)
         _check(st, "dws_st_delta_write")
+        if out is not None:
+            self._host_bytes(out, "out")
         if out is None or out.numel() < need:
             out = torch.empty(max(1, need), dtype=torch.uint8, pin_memory=True)
         sh = _stream_handle(stream)
@@ -562,6 +572,7 @@ class DeltaPlan:
         if not hasattr(file, "data_ptr"):
             file = torch.frombuffer(bytearray(file), dtype=torch.uint8) if len(file) else \
                 torch.empty(0, dtype=torch.uint8)
+        self._host_bytes(file, "file")
         arr = make_name_array(names)
         oh = np.zeros(self.num_tensors + 1, dtype=np.int64)
         offsets = torch.empty(self.num_tensors + 1, dtype=torch.int64, device=self.device)

@@ -231,3 +231,19 @@ def test_reader_matches_oracle_on_mutated_files(dws, seed):
                 assert got[2] == want[2]
             decisions[want[0]] += 1
     assert decisions["accepted"] > 40 and decisions["refused"] > 200, decisions
+
+
+def test_binding_refuses_file_buffers_outside_host_memory(dws):
+    # The header is written and parsed by host code, so a device (here a
+    # meta-device) or non-byte buffer is refused before libdws sees it.
+    import types
+
+    import torch
+    fake = types.SimpleNamespace(num_tensors=1, handle=0, _host_bytes=dws.DeltaPlan._host_bytes)
+    with pytest.raises(ValueError):
+        dws.DeltaPlan.read_delta_file(fake, torch.empty(16, dtype=torch.uint8, device="meta"), ["a"])
+    with pytest.raises(ValueError):
+        dws.DeltaPlan.read_delta_file(fake, torch.empty(4, dtype=torch.int32), ["a"])
+    with pytest.raises(ValueError):
+        dws.DeltaPlan.read_delta_file(fake, torch.empty(32, dtype=torch.uint8)[::2], ["a"])
+    dws.DeltaPlan._host_bytes(torch.empty(8, dtype=torch.uint8), "file")  # accepted
