@@ -28,6 +28,7 @@ timing reduction.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import datetime
 import hashlib
 import json
@@ -236,16 +237,39 @@ def layer_order(shapes):
     return order or list(range(len(shapes)))
 
 
+PINNED_CORE = {"core": None}
+
+
+@contextlib.contextmanager
+def one_core():
+    """Run the calling thread on one of its allowed cores (the lowest) and put
+    its affinity back afterwards; without affinity support it runs unpinned."""
+    try:
+        allowed = os.sched_getaffinity(0)
+        core = min(allowed)
+        os.sched_setaffinity(0, {core})
+    except (AttributeError, OSError, ValueError):
+        yield None
+        return
+    try:
+        PINNED_CORE["core"] = core
+        yield core
+    finally:
+        os.sched_setaffinity(0, allowed)
+
+
 def time_oracle(pairs):
-    """Seconds the oracle spends on encode + apply over the (old, new) pairs."""
+    """Seconds the oracle spends on encode + apply over the (old, new) pairs,
+    on one pinned core (the oracle is single-threaded)."""
     import oracle
     tot = 0.0
-    for a, b in pairs:
-        snap = a.copy()
-        t0 = time.perf_counter()
-        o, i, v = oracle.encode([a], [b])
-        oracle.apply([snap], o, i, v)
-        tot += time.perf_counter() - t0
+    with one_core():
+        for a, b in pairs:
+            snap = a.copy()
+            t0 = time.perf_counter()
+            o, i, v = oracle.encode([a], [b])
+            oracle.apply([snap], o, i, v)
+            tot += time.perf_counter() - t0
     return tot
 
 
@@ -315,7 +339,7 @@ def run_reference(args):
         "config": {"workload": "llama3_8b-shaped bf16 parameter set (bounded sample per step)",
                    "lr": args.lr, "parallelism": "replicas"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample, "cpu": cpu_model()},
+                         "sample": sample, "cpu": cpu_model(), "pinned_core": PINNED_CORE["core"]},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -979,7 +1003,7 @@ def run_ours(args):
             "sample": (f"the first {c} decoder-layer tensors of the same Llama-3-8B-shaped set "
                        f"({n} elements, {2 * n / 1e9:.2f} GB of weights), oracle encode + apply "
                        f"in {sec:.1f} s on one thread"),
-            "cpu": cpu_model(), "host_threads": os.cpu_count()}
+            "cpu": cpu_model(), "host_threads": os.cpu_count(), "pinned_core": PINNED_CORE["core"]}
 
     if rank == 0:
         print(json.dumps(line), flush=True)
