@@ -101,6 +101,19 @@ def replicas_value(world, bytes_per_rank, ms_per_step):
     return world * bytes_per_rank / (ms_per_step / 1e3) / 1e9
 
 
+def theoretical_hbm_gbs(props):
+    """HBM peak from the device attributes: memory clock (kHz) x 2 (double
+    data rate) x bus width (bits) / 8, in GB/s; None if unknown."""
+    try:
+        khz = float(props.memory_clock_rate)
+        bits = float(props.memory_bus_width)
+    except (AttributeError, TypeError, ValueError):
+        return None
+    if khz <= 0 or bits <= 0:
+        return None
+    return khz * 1e3 * 2 * bits / 8 / 1e9
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -775,6 +788,7 @@ def run_ours(args):
     e_enc0, e_enc1, e_app1 = events(K), events(K), events(K)
     start, end = events(2)
     props = torch.cuda.get_device_properties(dev)
+    theo = theoretical_hbm_gbs(props)
     clocks = Clocks(local, str(getattr(props, "uuid", "")) or None)
     clocks.start()
     launches0 = dws.dws_launch_count()
@@ -841,7 +855,9 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "kernel": "encode (dws_encode: workspace reset + fused detect/scan/compact)",
-                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "theoretical_peak": round(theo, 1) if theo else None,
+                     "frac_of_theoretical": round(achieved / theo, 4) if theo else None},
         "gpu_launches": int(launches),
         "clocks": clk,
         "exact": exact,

@@ -84,3 +84,17 @@ def test_reference_arm_runs_on_rank_zero_only():
     line = json.loads(lines[0][-1])
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_theoretical_hbm_peak_from_device_attributes():
+    # B200: 3,996 MHz HBM3e, 8 stacks x 1024 bits: 8.18 TB/s; an H100 SXM's
+    # 2,619 MHz x 5120 bits gives its 3.35 TB/s; missing attributes give None.
+    import types
+
+    import bench
+    b200 = types.SimpleNamespace(memory_clock_rate=3_996_000, memory_bus_width=8192)
+    assert abs(bench.theoretical_hbm_gbs(b200) - 8183.8) < 0.1
+    h100 = types.SimpleNamespace(memory_clock_rate=2_619_000, memory_bus_width=5120)
+    assert abs(bench.theoretical_hbm_gbs(h100) - 3352.3) < 0.1
+    assert bench.theoretical_hbm_gbs(types.SimpleNamespace()) is None
+    assert bench.theoretical_hbm_gbs(types.SimpleNamespace(memory_clock_rate=0, memory_bus_width=8)) is None
