@@ -15,6 +15,7 @@
 // writer made).
 #include <cuda_runtime.h>
 
+#include <charconv>
 #include <clocale>
 #include <cstdio>
 #include <cstring>
@@ -94,7 +95,15 @@ void put_utf8(std::string &out, unsigned cp) {
 // byte as it is (UTF-8 stays raw).
 void put_json_string(std::string &out, std::string_view s) {
     out += '"';
-    for (unsigned char c : s) {
+    size_t i = 0;
+    while (i < s.size()) {
+        // the run of bytes that need no escape goes in at once
+        size_t j = i;
+        while (j < s.size() && s[j] != '"' && s[j] != '\\' && static_cast<unsigned char>(s[j]) >= 0x20) ++j;
+        out.append(s.data() + i, j - i);
+        if (j == s.size()) break;
+        const unsigned char c = static_cast<unsigned char>(s[j]);
+        i = j + 1;
         switch (c) {
         case '"': out += "\\\""; break;
         case '\\': out += "\\\\"; break;
@@ -103,24 +112,21 @@ void put_json_string(std::string &out, std::string_view s) {
         case '\n': out += "\\n"; break;
         case '\r': out += "\\r"; break;
         case '\t': out += "\\t"; break;
-        default:
-            if (c < 0x20) {
-                static const char hex[] = "0123456789abcdef";
-                out += "\\u00";
-                out += hex[c >> 4];
-                out += hex[c & 15];
-            } else {
-                out += static_cast<char>(c);
-            }
+        default: {  // the other C0 controls
+            static const char hex[] = "0123456789abcdef";
+            out += "\\u00";
+            out += hex[c >> 4];
+            out += hex[c & 15];
+        }
         }
     }
     out += '"';
 }
 
 void put_int(std::string &out, long long v) {
-    char buf[32];
-    std::snprintf(buf, sizeof buf, "%lld", v);
-    out += buf;
+    char buf[24];
+    const std::to_chars_result r = std::to_chars(buf, buf + sizeof buf, v);
+    out.append(buf, static_cast<size_t>(r.ptr - buf));
 }
 
 // x with 6 decimals, '.' as the separator whatever the process locale.
@@ -135,32 +141,56 @@ std::string fixed6(double x) {
 
 // ---- JSON reading ---------------------------------------------------------
 
-struct JVal {
+// A parsed JSON document, held flat so that a header of tens of thousands of
+// entries costs a few allocations, not one per value: the nodes in one array,
+// the children of each array or object as one contiguous run of node indices
+// (with the keys of an object's children beside them), every decoded string
+// in one arena.
+struct JNode {
     enum Kind : unsigned char { kNull, kBool, kNum, kStr, kArr, kObj };
     Kind kind = kNull;
-    bool is_count = false;  // kNum: a plain integer >= 0 (or -0) within 64 bits
-    unsigned long long count = 0;
-    std::string str;
-    std::vector<JVal> arr;
-    std::vector<std::pair<std::string, JVal>> obj;
-
-    const JVal *get(std::string_view k) const {
-        for (const auto &kv : obj)
-            if (kv.first == k) return &kv.second;
-        return nullptr;
-    }
+    bool is_count = false;         // kNum: a plain integer >= 0 (or -0) within 64 bits
+    unsigned long long count = 0;  // kNum: its value when is_count
+    size_t a = 0, n = 0;           // kStr: arena offset and length; kArr/kObj: first child slot, children
 };
 
-// Recursive-descent parser of RFC 8259 JSON over [p, e); no extensions (no
-// NaN/Infinity, no comments, no trailing commas), objects with a repeated
-// key are refused, nesting deeper than kMaxDepth is refused.
+struct JDoc {
+    static constexpr size_t npos = ~size_t(0);
+    std::vector<JNode> nodes;
+    std::vector<size_t> kids;                          // child node index per slot
+    std::vector<std::pair<size_t, size_t>> keys;       // key (arena offset, length) per slot
+    std::string arena;
+
+    std::string_view str(size_t node) const {
+        return std::string_view(arena.data() + nodes[node].a, nodes[node].n);
+    }
+    std::string_view key(size_t slot) const {
+        return std::string_view(arena.data() + keys[slot].first, keys[slot].second);
+    }
+    // The value under key k of object `obj` (linear: for the small objects).
+    size_t get(size_t obj, std::string_view k) const {
+        const JNode &o = nodes[obj];
+        for (size_t s = o.a; s < o.a + o.n; ++s)
+            if (key(s) == k) return kids[s];
+        return npos;
+    }
+    JNode::Kind kind(size_t node) const { return node == npos ? JNode::kNull : nodes[node].kind; }
+};
+
+// Recursive-descent parser of RFC 8259 JSON over [p, e) into a JDoc; no
+// extensions (no NaN/Infinity, no comments, no trailing commas), objects with
+// a repeated key are refused, nesting deeper than kMaxDepth is refused.
 class JsonParser {
   public:
-    JsonParser(const char *p, const char *e) : p_(p), e_(e) {}
+    JsonParser(const char *p, const char *e, JDoc &doc) : p_(p), e_(e), d_(doc) {
+        const size_t bytes = static_cast<size_t>(e - p);
+        d_.nodes.reserve(bytes / 16 + 4);
+        d_.arena.reserve(bytes / 2 + 16);
+    }
 
-    bool document(JVal &v) {
+    bool document(size_t *root) {
         ws();
-        if (!value(v, 0)) return false;
+        if (!value(root, 0)) return false;
         ws();
         return p_ == e_;
     }
@@ -169,6 +199,9 @@ class JsonParser {
     static constexpr int kMaxDepth = 512;
     const char *p_;
     const char *e_;
+    JDoc &d_;
+    std::vector<size_t> stack_kids_;                     // children of the open containers
+    std::vector<std::pair<size_t, size_t>> stack_keys_;  // and their keys
 
     void ws() {
         while (p_ < e_ && (*p_ == ' ' || *p_ == '\t' || *p_ == '\n' || *p_ == '\r')) ++p_;
@@ -181,77 +214,92 @@ class JsonParser {
         return true;
     }
 
-    bool value(JVal &v, int depth) {
+    size_t add(JNode::Kind k) {
+        JNode nd;
+        nd.kind = k;
+        d_.nodes.push_back(nd);
+        return d_.nodes.size() - 1;
+    }
+
+    bool value(size_t *out, int depth) {
         if (depth > kMaxDepth || p_ >= e_) return false;
         switch (*p_) {
-        case '{': return object(v, depth);
-        case '[': return array(v, depth);
-        case '"': v.kind = JVal::kStr; return string(v.str);
-        case 't': v.kind = JVal::kBool; return word("true");
-        case 'f': v.kind = JVal::kBool; return word("false");
-        case 'n': v.kind = JVal::kNull; return word("null");
-        default: return number(v);
+        case '{': return container(out, depth, true);
+        case '[': return container(out, depth, false);
+        case '"': {
+            size_t off = 0, len = 0;
+            if (!string(&off, &len)) return false;
+            *out = add(JNode::kStr);
+            d_.nodes[*out].a = off;
+            d_.nodes[*out].n = len;
+            return true;
+        }
+        case 't': *out = add(JNode::kBool); return word("true");
+        case 'f': *out = add(JNode::kBool); return word("false");
+        case 'n': *out = add(JNode::kNull); return word("null");
+        default: *out = add(JNode::kNum); return number(&d_.nodes[*out]);
         }
     }
 
-    bool object(JVal &v, int depth) {
-        v.kind = JVal::kObj;
+    // An object (with keys) or an array: children collected on the stack,
+    // then moved to one run of slots when the container closes.
+    bool container(size_t *out, int depth, bool is_obj) {
+        const size_t node = add(is_obj ? JNode::kObj : JNode::kArr);
+        *out = node;
+        const size_t base = stack_kids_.size();
+        const char close = is_obj ? '}' : ']';
         ++p_;
         ws();
-        if (p_ < e_ && *p_ == '}') {
+        if (p_ < e_ && *p_ == close) {
             ++p_;
-            return true;
-        }
-        for (;;) {
-            ws();
-            if (p_ >= e_ || *p_ != '"') return false;
-            std::string key;
-            if (!string(key)) return false;
-            ws();
-            if (p_ >= e_ || *p_ != ':') return false;
-            ++p_;
-            ws();
-            v.obj.emplace_back(std::move(key), JVal());
-            if (!value(v.obj.back().second, depth + 1)) return false;
-            ws();
-            if (p_ >= e_) return false;
-            if (*p_ == ',') {
+        } else {
+            for (;;) {
+                ws();
+                std::pair<size_t, size_t> k(0, 0);
+                if (is_obj) {
+                    if (p_ >= e_ || *p_ != '"') return false;
+                    if (!string(&k.first, &k.second)) return false;
+                    ws();
+                    if (p_ >= e_ || *p_ != ':') return false;
+                    ++p_;
+                    ws();
+                }
+                size_t child = 0;
+                if (!value(&child, depth + 1)) return false;
+                stack_kids_.push_back(child);
+                stack_keys_.push_back(k);
+                ws();
+                if (p_ >= e_) return false;
+                if (*p_ == ',') {
+                    ++p_;
+                    continue;
+                }
+                if (*p_ != close) return false;
                 ++p_;
-                continue;
+                break;
             }
-            if (*p_ != '}') return false;
-            ++p_;
-            break;
+        }
+        const size_t n = stack_kids_.size() - base;
+        d_.nodes[node].a = d_.kids.size();
+        d_.nodes[node].n = n;
+        d_.kids.insert(d_.kids.end(), stack_kids_.begin() + base, stack_kids_.end());
+        d_.keys.insert(d_.keys.end(), stack_keys_.begin() + base, stack_keys_.end());
+        stack_kids_.resize(base);
+        stack_keys_.resize(base);
+        if (!is_obj || n < 2) return true;
+        // no key twice (the arena is not growing while this runs)
+        const size_t first = d_.nodes[node].a;
+        if (n <= 16) {
+            for (size_t i = first; i < first + n; ++i)
+                for (size_t j = i + 1; j < first + n; ++j)
+                    if (d_.key(i) == d_.key(j)) return false;
+            return true;
         }
         std::unordered_set<std::string_view> seen;
-        seen.reserve(v.obj.size());
-        for (const auto &kv : v.obj)
-            if (!seen.insert(kv.first).second) return false;
+        seen.reserve(n);
+        for (size_t i = first; i < first + n; ++i)
+            if (!seen.insert(d_.key(i)).second) return false;
         return true;
-    }
-
-    bool array(JVal &v, int depth) {
-        v.kind = JVal::kArr;
-        ++p_;
-        ws();
-        if (p_ < e_ && *p_ == ']') {
-            ++p_;
-            return true;
-        }
-        for (;;) {
-            ws();
-            v.arr.emplace_back();
-            if (!value(v.arr.back(), depth + 1)) return false;
-            ws();
-            if (p_ >= e_) return false;
-            if (*p_ == ',') {
-                ++p_;
-                continue;
-            }
-            if (*p_ != ']') return false;
-            ++p_;
-            return true;
-        }
     }
 
     bool hex4(unsigned &cp) {
@@ -269,17 +317,25 @@ class JsonParser {
         return true;
     }
 
-    bool string(std::string &out) {
+    // A string literal, decoded into the arena at [*off, *off + *len).
+    bool string(size_t *off, size_t *len) {
+        std::string &out = d_.arena;
+        *off = out.size();
         ++p_;  // the opening quote
         for (;;) {
+            // the run of plain bytes up to the next quote, escape or control
+            const char *q = p_;
+            while (q < e_ && *q != '"' && *q != '\\' && static_cast<unsigned char>(*q) >= 0x20) ++q;
+            out.append(p_, static_cast<size_t>(q - p_));
+            p_ = q;
             if (p_ >= e_) return false;
             unsigned char c = static_cast<unsigned char>(*p_++);
-            if (c == '"') return true;
-            if (c < 0x20) return false;
-            if (c != '\\') {
-                out += static_cast<char>(c);
-                continue;
+            if (c == '"') {
+                *len = out.size() - *off;
+                return true;
             }
+            if (c < 0x20) return false;
+            // c == '\\'
             if (p_ >= e_) return false;
             switch (*p_++) {
             case '"': out += '"'; break;
@@ -315,8 +371,7 @@ class JsonParser {
 
     static bool digit(char c) { return c >= '0' && c <= '9'; }
 
-    bool number(JVal &v) {
-        v.kind = JVal::kNum;
+    bool number(JNode *v) {
         bool neg = false, plain = true, fits = true;
         unsigned long long u = 0;
         if (p_ < e_ && *p_ == '-') {
@@ -346,14 +401,14 @@ class JsonParser {
             if (p_ >= e_ || !digit(*p_)) return false;
             while (p_ < e_ && digit(*p_)) ++p_;
         }
-        v.is_count = plain && fits && (!neg || u == 0);
-        v.count = v.is_count ? u : 0;
+        v->is_count = plain && fits && (!neg || u == 0);
+        v->count = v->is_count ? u : 0;
         return true;
     }
 };
 
 // A decimal integer string ("-"? digits) that fits in 64 bits.
-bool parse_version(const std::string &s, long long *out) {
+bool parse_version(std::string_view s, long long *out) {
     size_t i = 0;
     bool neg = false;
     if (i < s.size() && s[i] == '-') neg = true, ++i;
@@ -393,21 +448,23 @@ dws_status_t check_names(const char *const *names, int32_t T,
 
 // One tensor entry {"dtype": dtype, "shape": [n], "data_offsets": [a, b]}
 // whose range lies in the data and holds n elements of elem bytes.
-bool tensor_entry(const JVal *e, const char *dtype, unsigned long long elem,
+bool tensor_entry(const JDoc &doc, size_t e, const char *dtype, unsigned long long elem,
                   unsigned long long data_bytes, unsigned long long *n,
                   unsigned long long *begin) {
-    if (e == nullptr || e->kind != JVal::kObj) return false;
-    const JVal *dt = e->get("dtype");
-    const JVal *shape = e->get("shape");
-    const JVal *span = e->get("data_offsets");
-    if (dt == nullptr || dt->kind != JVal::kStr || dt->str != dtype) return false;
-    if (shape == nullptr || shape->kind != JVal::kArr || shape->arr.size() != 1 ||
-        !shape->arr[0].is_count)
+    if (doc.kind(e) != JNode::kObj) return false;
+    const size_t dt = doc.get(e, "dtype");
+    const size_t shape = doc.get(e, "shape");
+    const size_t span = doc.get(e, "data_offsets");
+    if (doc.kind(dt) != JNode::kStr || doc.str(dt) != dtype) return false;
+    if (doc.kind(shape) != JNode::kArr || doc.nodes[shape].n != 1) return false;
+    if (doc.kind(span) != JNode::kArr || doc.nodes[span].n != 2) return false;
+    const JNode &c0 = doc.nodes[doc.kids[doc.nodes[shape].a]];
+    const JNode &a0 = doc.nodes[doc.kids[doc.nodes[span].a]];
+    const JNode &b0 = doc.nodes[doc.kids[doc.nodes[span].a + 1]];
+    if (c0.kind != JNode::kNum || !c0.is_count || a0.kind != JNode::kNum || !a0.is_count ||
+        b0.kind != JNode::kNum || !b0.is_count)
         return false;
-    if (span == nullptr || span->kind != JVal::kArr || span->arr.size() != 2 ||
-        !span->arr[0].is_count || !span->arr[1].is_count)
-        return false;
-    unsigned long long a = span->arr[0].count, b = span->arr[1].count, c = shape->arr[0].count;
+    const unsigned long long a = a0.count, b = b0.count, c = c0.count;
     if (a > b || b > data_bytes) return false;
     if (c > (b - a) / elem || c * elem != b - a) return false;
     *n = c;
@@ -435,7 +492,10 @@ dws_status_t build_header(const dws_plan_t *plan, const char *const *names,
     }
     const long long nnz = offsets[T];
 
+    size_t name_bytes = 0;
+    for (int32_t t = 0; t < T; ++t) name_bytes += name[t].size();
     std::string changed = "[";
+    changed.reserve(name_bytes + 3 * static_cast<size_t>(T) + 2);
     for (int32_t t = 0; t < T; ++t) {
         if (offsets[t + 1] == offsets[t]) continue;
         if (changed.size() > 1) changed += ',';
@@ -444,6 +504,7 @@ dws_status_t build_header(const dws_plan_t *plan, const char *const *names,
     changed += ']';
 
     std::string h(8, '\0');
+    h.reserve(256 + 2 * changed.size() + 2 * name_bytes + 160 * static_cast<size_t>(T));
     h += "{\"__metadata__\":{\"sparse\":\"True\",\"model_version\":\"";
     put_int(h, model_version);
     h += "\",\"sparsity\":\"";
@@ -550,69 +611,79 @@ dws_status_t dws_st_delta_read(const dws_plan_t *plan, const char *const *names,
     if (hl > static_cast<unsigned long long>(file_size - 8)) return DWS_ERR_BAD_DELTA;
     const char *hdr = reinterpret_cast<const char *>(file + 8);
     if (!valid_utf8(file + 8, hl)) return DWS_ERR_BAD_DELTA;
-    JVal root;
-    if (!JsonParser(hdr, hdr + hl).document(root) || root.kind != JVal::kObj)
+    JDoc doc;
+    size_t root = 0;
+    if (!JsonParser(hdr, hdr + hl, doc).document(&root) || doc.kind(root) != JNode::kObj)
         return DWS_ERR_BAD_DELTA;
     const uint8_t *data = file + 8 + hl;
     const unsigned long long data_bytes = static_cast<unsigned long long>(file_size - 8) - hl;
 
     // Metadata: a delta (sparse "True"), its version, the list it applies.
-    const JVal *meta = root.get("__metadata__");
-    if (meta == nullptr || meta->kind != JVal::kObj) return DWS_ERR_BAD_DELTA;
-    const JVal *sparse = meta->get("sparse");
-    const JVal *ver = meta->get("model_version");
-    const JVal *listed = meta->get("changed_params");
-    if (sparse == nullptr || sparse->kind != JVal::kStr || sparse->str != "True")
-        return DWS_ERR_BAD_DELTA;
+    const size_t meta = doc.get(root, "__metadata__");
+    if (doc.kind(meta) != JNode::kObj) return DWS_ERR_BAD_DELTA;
+    const size_t sparse = doc.get(meta, "sparse");
+    const size_t ver = doc.get(meta, "model_version");
+    const size_t listed = doc.get(meta, "changed_params");
+    if (doc.kind(sparse) != JNode::kStr || doc.str(sparse) != "True") return DWS_ERR_BAD_DELTA;
     long long version = 0;
-    if (ver == nullptr || ver->kind != JVal::kStr || !parse_version(ver->str, &version))
+    if (doc.kind(ver) != JNode::kStr || !parse_version(doc.str(ver), &version))
         return DWS_ERR_BAD_DELTA;
-    if (listed == nullptr || listed->kind != JVal::kStr) return DWS_ERR_BAD_DELTA;
-    JVal list;
-    if (!JsonParser(listed->str.data(), listed->str.data() + listed->str.size()).document(list) ||
-        list.kind != JVal::kArr)
+    if (doc.kind(listed) != JNode::kStr) return DWS_ERR_BAD_DELTA;
+    const std::string_view listed_text = doc.str(listed);
+    JDoc ldoc;
+    size_t lroot = 0;
+    if (!JsonParser(listed_text.data(), listed_text.data() + listed_text.size(), ldoc).document(&lroot) ||
+        ldoc.kind(lroot) != JNode::kArr)
         return DWS_ERR_BAD_DELTA;
     std::unordered_map<std::string_view, int32_t> slot;
     slot.reserve(T);
     for (int32_t t = 0; t < T; ++t) slot.emplace(name[t], t);
+    const JNode &lnode = ldoc.nodes[lroot];
+    std::vector<std::string_view> list;  // the listed names, in their order
+    list.reserve(lnode.n);
     std::unordered_set<std::string_view> changed;
-    changed.reserve(list.arr.size());
-    for (const JVal &n : list.arr) {
-        if (n.kind != JVal::kStr || !changed.insert(n.str).second) return DWS_ERR_BAD_DELTA;
-        if (slot.find(n.str) == slot.end()) return DWS_ERR_BAD_DELTA;
+    changed.reserve(lnode.n);
+    for (size_t s = lnode.a; s < lnode.a + lnode.n; ++s) {
+        const size_t c = ldoc.kids[s];
+        if (ldoc.kind(c) != JNode::kStr) return DWS_ERR_BAD_DELTA;
+        const std::string_view n = ldoc.str(c);
+        if (!changed.insert(n).second) return DWS_ERR_BAD_DELTA;
+        if (slot.find(n) == slot.end()) return DWS_ERR_BAD_DELTA;
+        list.push_back(n);
     }
 
     // Every tensor entry belongs to a listed parameter.
-    std::unordered_map<std::string_view, const JVal *> entry;
-    entry.reserve(root.obj.size());
-    for (const auto &kv : root.obj) {
-        if (kv.first == "__metadata__") continue;
-        std::string_view k(kv.first);
+    const JNode &rnode = doc.nodes[root];
+    std::unordered_map<std::string_view, size_t> entry;
+    entry.reserve(rnode.n);
+    for (size_t s = rnode.a; s < rnode.a + rnode.n; ++s) {
+        const std::string_view k = doc.key(s);
+        if (k == "__metadata__") continue;
         std::string_view base;
         if (ends_with(k, ".indices")) base = k.substr(0, k.size() - 8);
         else if (ends_with(k, ".values")) base = k.substr(0, k.size() - 7);
         else return DWS_ERR_BAD_DELTA;
         if (changed.find(base) == changed.end()) return DWS_ERR_BAD_DELTA;
-        entry.emplace(k, &kv.second);
+        entry.emplace(k, doc.kids[s]);
     }
 
     // Each listed parameter: its two entries, equal lengths.
     struct Part { unsigned long long n = 0, ib = 0, vb = 0; bool present = false; };
     std::vector<Part> part(T);
     std::string key;
-    for (const JVal &n : list.arr) {
-        const int32_t t = slot[n.str];
+    for (const std::string_view n : list) {
+        const int32_t t = slot.find(n)->second;
         Part &p = part[t];
         unsigned long long nv = 0;
-        key.assign(n.str);
+        key.assign(n);
         key += ".indices";
         auto it = entry.find(key);
-        if (it == entry.end() || !tensor_entry(it->second, "I32", 4, data_bytes, &p.n, &p.ib))
+        if (it == entry.end() || !tensor_entry(doc, it->second, "I32", 4, data_bytes, &p.n, &p.ib))
             return DWS_ERR_BAD_DELTA;
-        key.assign(n.str);
+        key.assign(n);
         key += ".values";
         it = entry.find(key);
-        if (it == entry.end() || !tensor_entry(it->second, "BF16", 2, data_bytes, &nv, &p.vb))
+        if (it == entry.end() || !tensor_entry(doc, it->second, "BF16", 2, data_bytes, &nv, &p.vb))
             return DWS_ERR_BAD_DELTA;
         if (nv != p.n) return DWS_ERR_BAD_DELTA;
         p.present = true;
