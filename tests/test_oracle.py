@@ -194,6 +194,44 @@ def test_chain_replays_qwen_shaped_steps():
         np.testing.assert_array_equal(a, b)
 
 
+@pytest.mark.parametrize("seed", [5, 6, 7])
+def test_apply_and_chain_match_numpy_assignment(seed):
+    # Arbitrary deltas (not from an encode): K of them over T tensors, each an
+    # ascending random subset with random values, overlapping across deltas
+    # with different values.  The oracle's apply and chain must equal numpy's
+    # own indexed assignment `snap[t][idx] = val`, delta after delta (a
+    # transposed offset, a wrong tensor, or an order reversal fails this).
+    rng = np.random.default_rng(seed)
+    numels = [int(x) for x in rng.choice([0, 1, 17, 1000, 8193], 6)]
+    anchor = [rng.integers(0, 1 << 16, n, dtype=np.uint16) for n in numels]
+    deltas = []
+    for _ in range(int(rng.integers(1, 9))):
+        offs, idx, val = [0], [], []
+        for n in numels:
+            c = int(rng.integers(0, n + 1)) if n else 0
+            pick = np.sort(rng.choice(n, c, replace=False)) if c else np.zeros(0, np.int64)
+            idx.append(pick.astype(np.int32))
+            val.append(rng.integers(0, 1 << 16, c, dtype=np.uint16))
+            offs.append(offs[-1] + c)
+        deltas.append((np.array(offs, np.int64), np.concatenate(idx), np.concatenate(val)))
+    want = [a.copy() for a in anchor]
+    for o, i, v in deltas:
+        for t in range(len(numels)):
+            want[t][i[o[t]:o[t + 1]]] = v[o[t]:o[t + 1]]
+    got = [a.copy() for a in anchor]
+    oracle.apply_chain(got, deltas)
+    for g, w in zip(got, want):
+        np.testing.assert_array_equal(g, w)
+    one = [a.copy() for a in anchor]
+    oracle.apply(one, *deltas[0])
+    first = [a.copy() for a in anchor]
+    for t in range(len(numels)):
+        o, i, v = deltas[0]
+        first[t][i[o[t]:o[t + 1]]] = v[o[t]:o[t + 1]]
+    for g, w in zip(one, first):
+        np.testing.assert_array_equal(g, w)
+
+
 # ---------------------------------------------------------------- XOR
 
 
