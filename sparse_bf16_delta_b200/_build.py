@@ -1,7 +1,7 @@
 """Build libdws.so in-tree with nvcc for sm_100a (B200).
 
 Standard library only, and run as a script (``python sparse_bf16_delta_b200/_build.py``)
-or loaded by path: importing the package would load the library this builds."""
+or loaded by path: importing the package would load the library it compiles."""
 from __future__ import annotations
 
 import glob
