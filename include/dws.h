@@ -376,9 +376,10 @@ DWS_API dws_status_t dws_st_delta_header(const dws_plan_t *plan, const char *con
  * header is written before the call returns; the data when `stream` reaches
  * the two copies -- synchronise before using or freeing `file`.
  * Errors: DWS_ERR_INVALID (null arguments, a name missing, not UTF-8 or
- * repeated), DWS_ERR_BAD_DELTA (offsets not starting at 0, decreasing, or a
- * count above its tensor's size), DWS_ERR_CAPACITY (capacity < *file_bytes;
- * nothing written), DWS_ERR_CUDA. */
+ * repeated, or host memory for the header not available), DWS_ERR_BAD_DELTA
+ * (offsets not starting at 0, decreasing, or a count above its tensor's
+ * size), DWS_ERR_CAPACITY (capacity < *file_bytes; nothing written),
+ * DWS_ERR_CUDA. */
 DWS_API dws_status_t dws_st_delta_write(const dws_plan_t *plan, const char *const *names,
                                 const int64_t *offsets, int64_t model_version,
                                 const int32_t *indices, const uint16_t *values,
@@ -403,8 +404,9 @@ DWS_API dws_status_t dws_st_delta_write(const dws_plan_t *plan, const char *cons
  * offsets: device int64[T+1]; indices, values: device, `capacity` entries.
  * *nnz receives the entry count and *model_version (nullable) the version.
  * Errors: DWS_ERR_INVALID (null arguments, table names missing, not UTF-8 or
- * repeated), DWS_ERR_BAD_DELTA as above, DWS_ERR_CAPACITY (nnz > capacity;
- * *nnz and offsets_host set, nothing enqueued), DWS_ERR_CUDA. */
+ * repeated, or host memory for parsing the header not available),
+ * DWS_ERR_BAD_DELTA as above, DWS_ERR_CAPACITY (nnz > capacity; *nnz and
+ * offsets_host set, nothing enqueued), DWS_ERR_CUDA. */
 DWS_API dws_status_t dws_st_delta_read(const dws_plan_t *plan, const char *const *names,
                                const uint8_t *file, int64_t file_size, int64_t *offsets_host,
                                int64_t *offsets, int32_t *indices, uint16_t *values,

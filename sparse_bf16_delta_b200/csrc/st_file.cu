@@ -15,11 +15,13 @@
 // writer made).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <charconv>
 #include <clocale>
 #include <cstdio>
 #include <cstring>
 #include <locale.h>
+#include <new>
 #include <string>
 #include <string_view>
 #include <unordered_map>
@@ -183,9 +185,10 @@ struct JDoc {
 class JsonParser {
   public:
     JsonParser(const char *p, const char *e, JDoc &doc) : p_(p), e_(e), d_(doc) {
+        // a first guess from the text's size, capped: a larger document grows
         const size_t bytes = static_cast<size_t>(e - p);
-        d_.nodes.reserve(bytes / 16 + 4);
-        d_.arena.reserve(bytes / 2 + 16);
+        d_.nodes.reserve(std::min<size_t>(bytes / 16 + 4, size_t(1) << 20));
+        d_.arena.reserve(std::min<size_t>(bytes / 2 + 16, size_t(64) << 20));
     }
 
     bool document(size_t *root) {
@@ -548,13 +551,9 @@ dws_status_t build_header(const dws_plan_t *plan, const char *const *names,
     return DWS_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-dws_status_t dws_st_delta_header(const dws_plan_t *plan, const char *const *names,
-                                 const int64_t *offsets, int64_t model_version, uint8_t *out,
-                                 int64_t capacity, int64_t *header_bytes) {
+dws_status_t st_delta_header(const dws_plan_t *plan, const char *const *names,
+                             const int64_t *offsets, int64_t model_version, uint8_t *out,
+                             int64_t capacity, int64_t *header_bytes) {
     if (header_bytes == nullptr || capacity < 0) return DWS_ERR_INVALID;
     std::string h;
     long long nnz = 0;
@@ -567,10 +566,10 @@ dws_status_t dws_st_delta_header(const dws_plan_t *plan, const char *const *name
     return DWS_OK;
 }
 
-dws_status_t dws_st_delta_write(const dws_plan_t *plan, const char *const *names,
-                                const int64_t *offsets, int64_t model_version,
-                                const int32_t *indices, const uint16_t *values, uint8_t *file,
-                                int64_t capacity, int64_t *file_bytes, dws_stream_t stream) {
+dws_status_t st_delta_write(const dws_plan_t *plan, const char *const *names,
+                            const int64_t *offsets, int64_t model_version,
+                            const int32_t *indices, const uint16_t *values, uint8_t *file,
+                            int64_t capacity, int64_t *file_bytes, dws_stream_t stream) {
     if (file_bytes == nullptr || capacity < 0) return DWS_ERR_INVALID;
     std::string h;
     long long nnz = 0;
@@ -590,11 +589,11 @@ dws_status_t dws_st_delta_write(const dws_plan_t *plan, const char *const *names
     return from_cuda(e);
 }
 
-dws_status_t dws_st_delta_read(const dws_plan_t *plan, const char *const *names,
-                               const uint8_t *file, int64_t file_size, int64_t *offsets_host,
-                               int64_t *offsets, int32_t *indices, uint16_t *values,
-                               int64_t capacity, int64_t *nnz_out, int64_t *model_version,
-                               dws_stream_t stream) {
+dws_status_t st_delta_read(const dws_plan_t *plan, const char *const *names,
+                           const uint8_t *file, int64_t file_size, int64_t *offsets_host,
+                           int64_t *offsets, int32_t *indices, uint16_t *values,
+                           int64_t capacity, int64_t *nnz_out, int64_t *model_version,
+                           dws_stream_t stream) {
     int32_t T = 0;
     const long long *numel = nullptr;
     if (!dws::plan_numels(plan, &T, &numel) || offsets_host == nullptr || offsets == nullptr ||
@@ -732,6 +731,48 @@ dws_status_t dws_st_delta_read(const dws_plan_t *plan, const char *const *names,
         }
     }
     return from_cuda(e);
+}
+
+}  // namespace
+
+// The exported entry points: a host allocation that fails (a header larger
+// than the memory at hand) is reported as DWS_ERR_INVALID instead of an
+// exception crossing the C boundary.
+extern "C" {
+
+dws_status_t dws_st_delta_header(const dws_plan_t *plan, const char *const *names,
+                                 const int64_t *offsets, int64_t model_version, uint8_t *out,
+                                 int64_t capacity, int64_t *header_bytes) {
+    try {
+        return st_delta_header(plan, names, offsets, model_version, out, capacity, header_bytes);
+    } catch (const std::bad_alloc &) {
+        return DWS_ERR_INVALID;
+    }
+}
+
+dws_status_t dws_st_delta_write(const dws_plan_t *plan, const char *const *names,
+                                const int64_t *offsets, int64_t model_version,
+                                const int32_t *indices, const uint16_t *values, uint8_t *file,
+                                int64_t capacity, int64_t *file_bytes, dws_stream_t stream) {
+    try {
+        return st_delta_write(plan, names, offsets, model_version, indices, values, file, capacity,
+                              file_bytes, stream);
+    } catch (const std::bad_alloc &) {
+        return DWS_ERR_INVALID;
+    }
+}
+
+dws_status_t dws_st_delta_read(const dws_plan_t *plan, const char *const *names,
+                               const uint8_t *file, int64_t file_size, int64_t *offsets_host,
+                               int64_t *offsets, int32_t *indices, uint16_t *values,
+                               int64_t capacity, int64_t *nnz_out, int64_t *model_version,
+                               dws_stream_t stream) {
+    try {
+        return st_delta_read(plan, names, file, file_size, offsets_host, offsets, indices, values,
+                             capacity, nnz_out, model_version, stream);
+    } catch (const std::bad_alloc &) {
+        return DWS_ERR_INVALID;
+    }
 }
 
 }  // extern "C"
