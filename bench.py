@@ -101,17 +101,17 @@ def replicas_value(world, bytes_per_rank, ms_per_step):
     return world * bytes_per_rank / (ms_per_step / 1e3) / 1e9
 
 
-def theoretical_hbm_gbs(props):
-    """HBM peak from the device attributes: memory clock (kHz) x 2 (double
-    data rate) x bus width (bits) / 8, in GB/s; None if unknown."""
+def theoretical_hbm_gbs(dws, device_index):
+    """HBM peak from the device attributes libdws reads from the CUDA runtime
+    (dws_device_memory): memory clock (kHz) x 2 (double data rate) x bus width
+    (bits) / 8, in GB/s, with its two inputs; (None, None, None) if unknown."""
     try:
-        khz = float(props.memory_clock_rate)
-        bits = float(props.memory_bus_width)
-    except (AttributeError, TypeError, ValueError):
-        return None
+        khz, bits = dws.dws_device_memory(device_index)
+    except Exception:
+        return None, None, None
     if khz <= 0 or bits <= 0:
-        return None
-    return khz * 1e3 * 2 * bits / 8 / 1e9
+        return None, khz, bits
+    return khz * 1e3 * 2 * bits / 8 / 1e9, khz, bits
 
 
 def measured_peaks():
@@ -788,7 +788,7 @@ def run_ours(args):
     e_enc0, e_enc1, e_app1 = events(K), events(K), events(K)
     start, end = events(2)
     props = torch.cuda.get_device_properties(dev)
-    theo = theoretical_hbm_gbs(props)
+    theo, mem_khz, bus_bits = theoretical_hbm_gbs(dws, dev.index if dev.index is not None else 0)
     clocks = Clocks(local, str(getattr(props, "uuid", "")) or None)
     clocks.start()
     launches0 = dws.dws_launch_count()
@@ -857,6 +857,8 @@ def run_ours(args):
                      "kernel": "encode (dws_encode: workspace reset + fused detect/scan/compact)",
                      "peak_kind": f"{peak_kind} HBM copy bandwidth",
                      "theoretical_peak": round(theo, 1) if theo else None,
+                     "theoretical_inputs": {"memory_clock_khz": mem_khz, "bus_width_bits": bus_bits,
+                                            "formula": "khz x 1e3 x 2 x bits / 8"},
                      "frac_of_theoretical": round(achieved / theo, 4) if theo else None},
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -943,6 +945,7 @@ def run_ours(args):
         del gidx, gval, goffs, bases
         # the same step with the wire checksum computed on the fly
         hashes = torch.empty(2, dtype=torch.int64, device=dev)
+        wire = torch.empty(2, dtype=torch.int64, device=dev)
         coffs = torch.empty(T + 1, dtype=torch.int64, device=dev)
         cidx = torch.empty(nnz, dtype=torch.int32, device=dev)
         cval = torch.empty(nnz, dtype=torch.int16, device=dev)
@@ -950,13 +953,14 @@ def run_ours(args):
         def enc_checksum():
             dws.dws_encode_checksum(plan.handle, ot.data_ptr(), nt.data_ptr(), coffs.data_ptr(),
                                     cidx.data_ptr(), cval.data_ptr(), nnz, hashes.data_ptr(),
-                                    plan.workspace.data_ptr(), plan.workspace_bytes, cs0)
+                                    wire.data_ptr(), plan.workspace.data_ptr(), plan.workspace_bytes,
+                                    cs0)
 
         ms_s, mn_s = time_reps(enc_checksum, args.rows_reps)
         ok_s = plan.status()[0] == dws.DWS_OK and bool(torch.equal(cidx, indices))
         rows.update([row("encode_checksum_llama3_8b_lr%g" % args.lr, ms_s, 4 * N + 6 * nnz,
                          weight_bytes, peak, {"min_ms": round(mn_s, 4), "indices_equal": ok_s})])
-        del hashes, coffs, cidx, cval
+        del hashes, wire, coffs, cidx, cval
         rows.update(delta_file_rows(dws, plan, [nm for nm, _ in shapes], delta, args))
         lr2 = 1e-5
         for t in range(T):
@@ -980,6 +984,7 @@ def run_ours(args):
         positions = torch.empty(max(2, pcap), dtype=torch.uint8, device=dev)
         pos_offsets = torch.empty(T + 1, dtype=torch.int64, device=dev)
         hashes = torch.empty(2, dtype=torch.int64, device=dev)
+        wire = torch.empty(2, dtype=torch.int64, device=dev)
         cs = torch.cuda.current_stream().cuda_stream
 
         def pack():
@@ -997,12 +1002,13 @@ def run_ours(args):
                                               "sizes_ok": ok_p})])
 
         def csum():
-            dws.dws_checksum(positions.data_ptr(), pbytes, val2.data_ptr(), nnz2, hashes.data_ptr(), cs)
+            dws.dws_checksum(positions.data_ptr(), pbytes, val2.data_ptr(), nnz2, hashes.data_ptr(),
+                             wire.data_ptr(), cs)
 
         ms_k, mn_k = time_reps(csum, args.rows_reps)
         rows.update([row("checksum_llama3_8b_lr1e-5", ms_k, pbytes + 2 * nnz2, weight_bytes, peak,
                          {"min_ms": round(mn_k, 4)})])
-        del positions, pos_offsets, hashes
+        del positions, pos_offsets, hashes, wire
         del old_flat, new_flat, snap_flat, old, new, snap, idx2, val2, d2, offs2
         import gc
         gc.collect()

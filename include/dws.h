@@ -180,15 +180,18 @@ DWS_API dws_status_t dws_encode_global(const dws_plan_t *plan,
 
 /* dws_encode that also returns the wire checksum of the delta it writes
  * (see dws_checksum): hashes[0] = XOR of the bytes of every position at its
- * tensor's pos_width, hashes[1] = XOR of the double bits of every value,
- * i.e. what dws_pack_positions + dws_checksum would give, without the extra
- * pass over the delta.  Only entries below `capacity` are hashed.
- * hashes: device uint64[2], overwritten.  Otherwise as dws_encode;
+ * tensor's pos_width, hashes[1] = XOR of the double bits of every value, and
+ * checksum = hashes[0] ^ (hashes[1] << 1), i.e. what dws_pack_positions +
+ * dws_checksum would give, without the extra pass over the delta.  Only
+ * entries below `capacity` are hashed.
+ * hashes: device uint64[2], overwritten.  checksum: device uint64[2]
+ * (nullable), overwritten with the 65-bit checksum as a 128-bit
+ * little-endian integer, as in dws_checksum.  Otherwise as dws_encode;
  * DWS_ERR_INVALID also for a null `hashes`. */
 DWS_API dws_status_t dws_encode_checksum(const dws_plan_t *plan,
                                  const void *const *old_ptrs, const void *const *new_ptrs,
                                  int64_t *offsets, int32_t *indices, uint16_t *values,
-                                 int64_t capacity, uint64_t *hashes,
+                                 int64_t capacity, uint64_t *hashes, uint64_t *checksum,
                                  void *workspace, size_t workspace_bytes, dws_stream_t stream);
 
 /* dws_encode with explicit controls of the scan's bounded wait.
@@ -225,6 +228,11 @@ DWS_API dws_status_t dws_count(const dws_plan_t *plan,
  * old_ptrs, new_ptrs, offsets, indices, values, capacity: as in dws_encode.
  * status_out: device array [2] (nullable) that receives the call's device
  *   status (a dws_status_t) and its detail, as dws_status() would report them.
+ *   The scratch array is private, so there is no dws_status() for this entry
+ *   point: with a null status_out a device-side error (a bounded wait that
+ *   ran out, a null tensor pointer in the tables) cannot be seen, and the
+ *   outputs may then be partial; only a capacity overflow still shows, as
+ *   offsets[T] > capacity.
  * Limits: at most 256 tensors and 65,536 tiles of 8192 elements
  *   (536,870,912 elements); larger requests return DWS_ERR_WORKSPACE and
  *   enqueue nothing.
@@ -232,7 +240,9 @@ DWS_API dws_status_t dws_count(const dws_plan_t *plan,
  *   behind; each call re-initialises what it reads.  Calls that overlap on the
  *   same GPU race: order them on one stream or with events.
  * The first call on a device looks up the array's address there; make it
- *   before capturing any stream on that device. */
+ *   before capturing any stream on that device.  Only a successful lookup is
+ *   kept: if it fails the call returns DWS_ERR_CUDA and the next call on that
+ *   device looks again. */
 DWS_API dws_status_t dws_encode_noalloc(const int64_t *numels, int32_t num_tensors,
                                         const void *const *old_ptrs, const void *const *new_ptrs,
                                         int64_t *offsets, int32_t *indices, uint16_t *values,
@@ -276,7 +286,15 @@ typedef struct dws_delta {
  * block owns a range of elements and replays all K deltas over it, so where
  * deltas touch the same element the later one wins, exactly as K sequential
  * dws_apply calls.  deltas: host array of K (1 <= K <= DWS_MAX_CHAIN).
- * Indices are range-checked (DWS_ERR_BAD_DELTA, entry skipped). */
+ * Every entry is checked as dws_apply checks it, in every mode: an index
+ * outside its tensor, or not above the entry before it in its tensor's
+ * segment (descending or repeated), is skipped and DWS_ERR_BAD_DELTA
+ * recorded (detail = its entry number in its delta); offsets that fail
+ * validation write nothing.  Elements named only by entries that pass are
+ * exactly as K sequential dws_apply calls leave them.  An entry above the one
+ * before it but not above every earlier entry of its segment (possible only
+ * after a flagged entry) may or may not be applied: after DWS_ERR_BAD_DELTA
+ * the elements such entries name are unspecified. */
 DWS_API dws_status_t dws_apply_chain(const dws_plan_t *plan, void *const *snap_ptrs,
                              const dws_delta_t *deltas, int32_t K,
                              void *workspace, size_t workspace_bytes, dws_stream_t stream);
@@ -333,13 +351,17 @@ DWS_API dws_status_t dws_pack_positions(const dws_plan_t *plan, const int64_t *o
 
 /* hashes[0] = XOR of the pos_bytes bytes at `positions`, each zero-extended
  * to 64 bits; hashes[1] = XOR of the 64-bit patterns of the doubles equal to
- * the nnz bf16 `values` (NaNs quieted, sign and payload kept).  The checksum
- * is hashes[0] ^ (hashes[1] << 1), 65 bits wide, which is why the two are
- * returned apart.  hashes: device uint64[2], overwritten.  values 2-byte
+ * the nnz bf16 `values` (NaNs quieted, sign and payload kept).
+ * checksum = hashes[0] ^ (hashes[1] << 1) taken on unbounded integers, as the
+ * page's Python does, so it is 65 bits wide: written as a 128-bit
+ * little-endian integer, checksum[0] = bits 0-63 and checksum[1] = bit 64
+ * (0 or 1; no higher bit is ever set).
+ * hashes: device uint64[2], overwritten.  checksum: device uint64[2]
+ * (nullable: only the hashes are wanted), overwritten.  values 2-byte
  * aligned.  DWS_ERR_INVALID on null pointers or negative sizes. */
 DWS_API dws_status_t dws_checksum(const uint8_t *positions, int64_t pos_bytes,
                           const uint16_t *values, int64_t nnz, uint64_t *hashes,
-                          dws_stream_t stream);
+                          uint64_t *checksum, dws_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * The delta file, [TRL] §4.1 and §4.3: a delta as a safetensors file (u64
@@ -457,6 +479,14 @@ DWS_API dws_status_t dws_xor_apply_layers(void *const *bufs, const void *const *
 DWS_API dws_status_t dws_status(void *workspace, int64_t *detail, dws_stream_t stream);
 
 DWS_API const char *dws_strerror(dws_status_t status);
+
+/* The device's memory clock (kHz) and global memory bus width (bits), as the
+ * CUDA runtime reports them (cudaDevAttrMemoryClockRate,
+ * cudaDevAttrGlobalMemoryBusWidth): the inputs of the theoretical DRAM peak,
+ * clock x 2 (double data rate) x width / 8 bytes per second.  A diagnostic
+ * for reporting bandwidth fractions.  Errors: DWS_ERR_INVALID (null outputs),
+ * DWS_ERR_CUDA (no such device). */
+DWS_API dws_status_t dws_device_memory(int32_t device, int32_t *clock_khz, int32_t *bus_bits);
 
 /* Number of kernels libdws has launched in this process so far (all devices,
  * all entry points).  A diagnostic: the difference across a region of calls is

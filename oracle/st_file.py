@@ -109,9 +109,13 @@ def write_delta(names, numels, offsets, indices, values, model_version: int) -> 
     return struct.pack("<Q", len(text)) + text + body
 
 
-def read_delta(blob: bytes, names):
+def read_delta(blob: bytes, names, numels=None):
     """Parse a delta file into the encode layout of the table `names`:
-    (offsets int64[T+1], indices int32[nnz], values uint16[nnz], model_version)."""
+    (offsets int64[T+1], indices int32[nnz], values uint16[nnz], model_version).
+    With `numels` (the table's element counts), a parameter listing more
+    entries than it has elements is refused: a delta names each changed
+    element of a parameter once ([TRL] §4.1), so it has at most numel of them,
+    the bound the writer keeps too."""
     if len(blob) < 8:
         raise DeltaFileError("shorter than the length prefix")
     (hlen,) = struct.unpack_from("<Q", blob, 0)
@@ -174,6 +178,8 @@ def read_delta(blob: bytes, names):
         nv, vb = entry(n + ".values", "BF16")
         if ni != nv:
             raise DeltaFileError(f"{n!r}: indices and values differ in length")
+        if numels is not None and ni > numels[slot[n]]:
+            raise DeltaFileError(f"{n!r}: more entries than the parameter has elements")
         parts[slot[n]] = (np.frombuffer(ib, dtype="<i4"), np.frombuffer(vb, dtype="<u2"))
     offsets = np.zeros(T + 1, dtype=np.int64)
     for t in range(T):

@@ -73,9 +73,9 @@ _sig("dws_apply_chain", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _vp,
 _sig("dws_apply_chain_ex", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _i32, _vp, _sz, _vp])
 _sig("dws_pos_width", _i32, [_vp, _i32])
 _sig("dws_encode_global", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
-_sig("dws_encode_checksum", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _vp])
+_sig("dws_encode_checksum", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _vp])
 _sig("dws_pack_positions", _i32, [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp])
-_sig("dws_checksum", _i32, [_vp, _i64, _vp, _i64, _vp, _vp])
+_sig("dws_checksum", _i32, [_vp, _i64, _vp, _i64, _vp, _vp, _vp])
 _sig("dws_st_delta_header", _i32, [_vp, _vp, _vp, _i64, _vp, _i64, ctypes.POINTER(_i64)])
 _sig("dws_st_delta_write", _i32,
      [_vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, ctypes.POINTER(_i64), _vp])
@@ -88,6 +88,7 @@ _sig("dws_status", _i32, [_vp, ctypes.POINTER(_i64), _vp])
 _sig("dws_strerror", ctypes.c_char_p, [_i32])
 _sig("dws_version", ctypes.c_char_p, [])
 _sig("dws_launch_count", ctypes.c_uint64, [])
+_sig("dws_device_memory", _i32, [_i32, ctypes.POINTER(_i32), ctypes.POINTER(_i32)])
 
 
 class DwsError(RuntimeError):
@@ -202,9 +203,9 @@ def dws_encode_global(plan, old_ptrs, new_ptrs, index_base, offsets, indices, va
 
 
 def dws_encode_checksum(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, hashes,
-                        workspace, workspace_bytes, stream) -> int:
+                        checksum, workspace, workspace_bytes, stream) -> int:
     return _lib.dws_encode_checksum(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
-                                    hashes, workspace, workspace_bytes, stream)
+                                    hashes, checksum, workspace, workspace_bytes, stream)
 
 
 def dws_pos_width(plan, t) -> int:
@@ -217,8 +218,8 @@ def dws_pack_positions(plan, offsets, indices, count, positions, pos_capacity, p
                                    pos_offsets, workspace, workspace_bytes, stream)
 
 
-def dws_checksum(positions, pos_bytes, values, nnz, hashes, stream) -> int:
-    return _lib.dws_checksum(positions, pos_bytes, values, nnz, hashes, stream)
+def dws_checksum(positions, pos_bytes, values, nnz, hashes, checksum, stream) -> int:
+    return _lib.dws_checksum(positions, pos_bytes, values, nnz, hashes, checksum, stream)
 
 
 def dws_st_delta_header(plan, names, offsets, model_version, out, capacity):
@@ -280,6 +281,14 @@ def dws_version() -> str:
 
 def dws_launch_count() -> int:
     return int(_lib.dws_launch_count())
+
+
+def dws_device_memory(device: int = 0):
+    """(memory clock kHz, bus width bits) of a device, from the CUDA runtime."""
+    khz, bits = _i32(0), _i32(0)
+    _check(_lib.dws_device_memory(int(device), ctypes.byref(khz), ctypes.byref(bits)),
+           "dws_device_memory")
+    return int(khz.value), int(bits.value)
 
 
 def make_delta_array(deltas):
@@ -476,22 +485,23 @@ class DeltaPlan:
         return Delta(offsets, indices, values)
 
     def encode_checksum(self, old_table, new_table, stream=None):
-        """(Delta, checksum): the exact encode and the wire checksum of the
-        delta it wrote, hash(positions) ^ (hash(values) << 1)."""
+        """(Delta, checksum): the exact encode and the 65-bit wire checksum
+        that libdws computed for the delta it wrote (dws_encode_checksum)."""
         torch = _torch()
         offsets = self.count(old_table, new_table, stream=stream)
         nnz = int(offsets[-1].item())
         indices = torch.empty(nnz, dtype=torch.int32, device=self.device)
         values = torch.empty(nnz, dtype=torch.int16, device=self.device)
         hashes = torch.empty(2, dtype=torch.int64, device=self.device)
+        wire = torch.empty(2, dtype=torch.int64, device=self.device)
         _check(dws_encode_checksum(self.handle, old_table.data_ptr(), new_table.data_ptr(),
                                    offsets.data_ptr(), indices.data_ptr() if nnz else 0,
                                    values.data_ptr() if nnz else 0, nnz, hashes.data_ptr(),
-                                   self.workspace.data_ptr(), self.workspace_bytes,
-                                   _stream_handle(stream)), "dws_encode_checksum")
+                                   wire.data_ptr(), self.workspace.data_ptr(),
+                                   self.workspace_bytes, _stream_handle(stream)),
+               "dws_encode_checksum")
         self.raise_on_error("dws_encode_checksum", stream)
-        hp, hv = (int(x) & 0xFFFFFFFFFFFFFFFF for x in hashes.cpu().tolist())
-        return Delta(offsets, indices, values), hp ^ (hv << 1)
+        return Delta(offsets, indices, values), _wire_int(wire)
 
     # -- wire form --
     def pos_width(self, t: int) -> int:
@@ -605,18 +615,24 @@ class DeltaPlan:
                                       _stream_handle(stream)), "dws_apply_chain_ex")
 
 
+def _wire_int(wire) -> int:
+    """The 128-bit little-endian integer libdws wrote into a 2-word device
+    tensor, as a Python int (reading only: libdws computed it)."""
+    return int.from_bytes(wire.cpu().numpy().tobytes(), "little")
+
+
 def checksum(positions, pos_bytes: int, values, stream=None) -> int:
-    """The wire checksum hash(positions) ^ (hash(values) << 1) of a byte block
-    and bf16 values (device tensors); synchronises to read the two hashes."""
+    """The wire checksum of a byte block and bf16 values (device tensors), as
+    libdws computes it (dws_checksum); synchronises to read it."""
     torch = _torch()
     dev = values.device if values.numel() else positions.device
     hashes = torch.empty(2, dtype=torch.int64, device=dev)
+    wire = torch.empty(2, dtype=torch.int64, device=dev)
     nnz = int(values.numel())
     _check(dws_checksum(positions.data_ptr() if pos_bytes else 0, int(pos_bytes),
-                        values.data_ptr() if nnz else 0, nnz, hashes.data_ptr(),
+                        values.data_ptr() if nnz else 0, nnz, hashes.data_ptr(), wire.data_ptr(),
                         _stream_handle(stream)), "dws_checksum")
-    hp, hv = (int(x) & 0xFFFFFFFFFFFFFFFF for x in hashes.cpu().tolist())
-    return hp ^ (hv << 1)
+    return _wire_int(wire)
 
 
 def xor_encode(old, new, mask=None, stream=None):

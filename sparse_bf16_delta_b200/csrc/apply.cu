@@ -184,7 +184,8 @@ struct ChainSmem {
     uint32_t tag[kChainUnitElems];
     long long cur[DWS_MAX_CHAIN];
     long long end[DWS_MAX_CHAIN];
-    int consumed[DWS_MAX_CHAIN];
+    long long seg[DWS_MAX_CHAIN];             // first entry of the current tensor's segment
+    unsigned long long stop[DWS_MAX_CHAIN];   // first entry of this round not taken
     int active[DWS_MAX_CHAIN];
     unsigned long long bar[2];
     UnitMeta meta[2];
@@ -299,7 +300,8 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
             if (lane == 0) {
                 sm.cur[k] = c;
                 sm.end[k] = hi;
-                sm.consumed[k] = 0;
+                sm.seg[k] = lo;
+                sm.stop[k] = ~0ull;
             }
         }
     }
@@ -325,6 +327,7 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
                 const DeltaRef d = p.d[tid];
                 if (sm.cur[tid] != sm.end[tid]) record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, sm.cur[tid]);
                 sm.cur[tid] = d.offsets[m.tensor];
+                sm.seg[tid] = sm.cur[tid];
                 sm.end[tid] = d.offsets[m.tensor + 1];
             }
         }
@@ -332,9 +335,15 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
         __syncthreads();
 
         // ---- entry phase: tag this unit's entries of every delta ----------
+        // Per round, L entries of every active delta from its cursor.  An
+        // entry inside the unit is tagged unless it is not above the entry
+        // before it in its tensor's segment; an entry below the unit is bad;
+        // both are taken (consumed).  The first entry past the unit ends the
+        // delta's stretch for this unit: the cursor moves to it.
         for (;;) {
             int idx[kChainSlotsPerThread];
             uint16_t val[kChainSlotsPerThread];
+            int pidx[kChainSlotsPerThread];
             bool valid[kChainSlotsPerThread];
 #pragma unroll
             for (int q = 0; q < kChainSlotsPerThread; ++q) {
@@ -347,6 +356,7 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
                         valid[q] = true;
                         idx[q] = __ldg(p.d[k].indices + j);
                         val[q] = __ldg(p.d[k].values + j);
+                        if (lane == 0 && j > sm.seg[k]) pidx[q] = __ldg(p.d[k].indices + j - 1);
                     }
                 }
             }
@@ -354,33 +364,47 @@ __global__ void __launch_bounds__(kChainThreads, 3) chain_kernel(ChainParams p) 
             for (int q = 0; q < kChainSlotsPerThread; ++q) {
                 const int sidx = tid + q * kChainThreads;
                 if (q * kChainThreads >= slots) break;  // uniform across the CTA
+                // 32 consecutive slots of a warp belong to one delta (L is a
+                // multiple of 32) and hold consecutive entries.
+                const int up = __shfl_up_sync(0xffffffffu, idx[q], 1);
                 bool take = false;
+                long long j = 0;
                 if (valid[q]) {
                     const int k = sidx / L;
+                    j = sm.cur[k] + (sidx - k * L);
+                    const int prev = (lane == 0) ? pidx[q] : up;
+                    const bool ordered = (j == sm.seg[k]) || (prev < idx[q]);
                     if (idx[q] < ls) {
-                        // Not ascending (or negative): skip, but consume it.
-                        record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, sm.cur[k] + (sidx - k * L));
+                        // Below the unit (not ascending, or negative): bad.
+                        record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, j);
                         take = true;
                     } else if (idx[q] - ls < m.count) {
-                        const uint32_t key = (static_cast<uint32_t>(k + 1) << 16) | val[q];
-                        atomicMax(&sm.tag[idx[q] - ls], key);
+                        if (ordered) {
+                            const uint32_t key = (static_cast<uint32_t>(k + 1) << 16) | val[q];
+                            atomicMax(&sm.tag[idx[q] - ls], key);
+                        } else {
+                            record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, j);
+                        }
                         take = true;
                     }
                 }
-                // 32 consecutive slots of a warp belong to one delta (L is a
-                // multiple of 32): count them with one shared atomic.
-                const unsigned int ballot = __ballot_sync(0xffffffffu, take);
-                if (lane == 0 && ballot != 0u && sidx < slots)
-                    atomicAdd(&sm.consumed[sidx / L], __popc(ballot));
+                const unsigned int left = __ballot_sync(0xffffffffu, valid[q] && !take);
+                if (left != 0u && lane == __ffs(left) - 1)
+                    atomicMin(&sm.stop[sidx / L], static_cast<unsigned long long>(j));
             }
             __syncthreads();
             int again = 0;
             if (tid < p.K) {
-                const int c = sm.consumed[tid];
-                sm.consumed[tid] = 0;
+                const unsigned long long st = sm.stop[tid];
+                sm.stop[tid] = ~0ull;
                 if (sm.active[tid]) {
-                    sm.cur[tid] += c;
-                    again = (c == L) && (sm.cur[tid] < sm.end[tid]);
+                    if (st != ~0ull) {
+                        sm.cur[tid] = static_cast<long long>(st);
+                    } else {
+                        const long long nc = sm.cur[tid] + L;
+                        sm.cur[tid] = nc < sm.end[tid] ? nc : sm.end[tid];
+                        again = sm.cur[tid] < sm.end[tid];
+                    }
                     sm.active[tid] = again;
                 }
             }
@@ -540,6 +564,7 @@ __global__ void __launch_bounds__(kScatThreads, 1) chain_scatter_kernel(ScatPara
 
         int ix[kScatDepth];
         uint16_t vx[kScatDepth];
+        int px[kScatDepth];  // lane 0: the index of the entry before its chunk
         bool prefetched = false;  // the phase's first chunks already requested (uniform)
         for (int k = p.K - 1; k >= 0; --k) {
             const DeltaRef d = p.d[k];
@@ -563,6 +588,7 @@ __global__ void __launch_bounds__(kScatThreads, 1) chain_scatter_kernel(ScatPara
                     if (r + q * kStride < n) {
                         ix[q] = __ldg(pi + r + q * kStride);
                         vx[q] = __ldg(pv + r + q * kStride);
+                        if (lane == 0 && j0 + r + q * kStride > 0) px[q] = __ldg(pi + r + q * kStride - 1);
                     }
                 }
             }
@@ -589,9 +615,13 @@ __global__ void __launch_bounds__(kScatThreads, 1) chain_scatter_kernel(ScatPara
                     }
                     const int idx = ix[q];
                     const uint16_t val = vx[q];
+                    // the previous entry's index (lane 0: loaded with the chunk)
+                    const int up = __shfl_up_sync(0xffffffffu, idx, 1);
+                    const int prev = (lane == 0) ? px[q] : up;
                     if (r + kScatDepth * kStride < n) {
                         ix[q] = __ldg(pi + r + kScatDepth * kStride);
                         vx[q] = __ldg(pv + r + kScatDepth * kStride);
+                        if (lane == 0) px[q] = __ldg(pi + r + kScatDepth * kStride - 1);
                     }
                     const bool valid = r < n;
                     if (cs >= seg_hi) {  // uniform: move to the chunk's first tensor
@@ -611,16 +641,23 @@ __global__ void __launch_bounds__(kScatThreads, 1) chain_scatter_kernel(ScatPara
                         // Common case, all 32-bit: the chunk lies in one tensor.
                         // (off_c < numel <= 2^31 - 1; rel wraps for indices
                         // below the window, which `before` catches.)
+                        // An entry not above the one before it in its
+                        // tensor's segment is bad (as in dws_apply).
                         const bool ok = static_cast<uint32_t>(idx) < numel_c;
                         const bool before = idx < off_c;
+                        const bool ordered = (r <= seg_lo) || (prev < idx);
                         rel = static_cast<uint32_t>(idx) - static_cast<uint32_t>(off_c);
-                        if (valid) cls = (!ok || before) ? 2 : (rel >= static_cast<uint32_t>(win_len) ? 3 : 1);
+                        if (valid)
+                            cls = (!ok || before || !ordered)
+                                      ? 2
+                                      : (rel >= static_cast<uint32_t>(win_len) ? 3 : 1);
                     } else if (valid) {
                         // The chunk crosses a tensor boundary: per-lane tensor.
                         const long long j = j0 + r;
                         int tl = tw;
                         while (tl + 1 < nt && offs[tl + 1] <= j) ++tl;
-                        if (j < offs[tl] || idx < 0 || static_cast<long long>(idx) >= sm.numel[tl]) {
+                        if (j < offs[tl] || idx < 0 || static_cast<long long>(idx) >= sm.numel[tl] ||
+                            (j > offs[tl] && prev >= idx)) {
                             cls = 2;
                         } else {
                             const long long e = sm.base[tl] + idx;
@@ -686,6 +723,7 @@ __global__ void __launch_bounds__(kScatThreads, 1) chain_scatter_kernel(ScatPara
                     if (jn + q * kStride < dn.count) {
                         ix[q] = __ldg(dn.indices + jn + q * kStride);
                         vx[q] = __ldg(dn.values + jn + q * kStride);
+                        if (lane == 0 && jn + q * kStride > 0) px[q] = __ldg(dn.indices + jn + q * kStride - 1);
                     }
                 }
                 prefetched = true;

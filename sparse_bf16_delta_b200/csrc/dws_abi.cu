@@ -271,10 +271,16 @@ dws_status_t dws_encode_global(const dws_plan_t *plan, const void *const *old_pt
 dws_status_t dws_encode_checksum(const dws_plan_t *plan, const void *const *old_ptrs,
                                  const void *const *new_ptrs, int64_t *offsets, int32_t *indices,
                                  uint16_t *values, int64_t capacity, uint64_t *hashes,
-                                 void *workspace, size_t workspace_bytes, dws_stream_t stream) {
+                                 uint64_t *checksum, void *workspace, size_t workspace_bytes,
+                                 dws_stream_t stream) {
     if (hashes == nullptr) return DWS_ERR_INVALID;
-    return encode_common(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity, workspace,
-                         workspace_bytes, stream, true, 0, -1, nullptr, nullptr, hashes);
+    dws_status_t st = encode_common(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
+                                    workspace, workspace_bytes, stream, true, 0, -1, nullptr,
+                                    nullptr, hashes);
+    if (st != DWS_OK || checksum == nullptr) return st;
+    return from_cuda(dws::launch_checksum_wire(reinterpret_cast<const unsigned long long *>(hashes),
+                                               reinterpret_cast<unsigned long long *>(checksum),
+                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
 dws_status_t dws_count(const dws_plan_t *plan, const void *const *old_ptrs,
@@ -362,14 +368,18 @@ dws_status_t dws_pack_positions(const dws_plan_t *plan, const int64_t *offsets,
 }
 
 dws_status_t dws_checksum(const uint8_t *positions, int64_t pos_bytes, const uint16_t *values,
-                          int64_t nnz, uint64_t *hashes, dws_stream_t stream) {
+                          int64_t nnz, uint64_t *hashes, uint64_t *checksum, dws_stream_t stream) {
     if (hashes == nullptr || pos_bytes < 0 || nnz < 0) return DWS_ERR_INVALID;
     if ((pos_bytes > 0 && positions == nullptr) || (nnz > 0 && values == nullptr))
         return DWS_ERR_INVALID;
     if (reinterpret_cast<uintptr_t>(values) & 1u) return DWS_ERR_INVALID;
-    return from_cuda(dws::launch_checksum(positions, pos_bytes, values, nnz,
-                                          reinterpret_cast<unsigned long long *>(hashes),
-                                          reinterpret_cast<cudaStream_t>(stream)));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = dws::launch_checksum(positions, pos_bytes, values, nnz,
+                                         reinterpret_cast<unsigned long long *>(hashes), s);
+    if (e == cudaSuccess && checksum != nullptr)
+        e = dws::launch_checksum_wire(reinterpret_cast<const unsigned long long *>(hashes),
+                                      reinterpret_cast<unsigned long long *>(checksum), s);
+    return from_cuda(e);
 }
 
 dws_status_t dws_xor_encode(const void *old_bytes, const void *new_bytes, void *mask,
@@ -492,6 +502,20 @@ const char *dws_strerror(dws_status_t status) {
         case DWS_ERR_WORKSPACE: return "workspace too small or not prepared for this plan";
     }
     return "unknown status";
+}
+
+dws_status_t dws_device_memory(int32_t device, int32_t *clock_khz, int32_t *bus_bits) {
+    if (clock_khz == nullptr || bus_bits == nullptr) return DWS_ERR_INVALID;
+    int khz = 0, bits = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&khz, cudaDevAttrMemoryClockRate, device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&bits, cudaDevAttrGlobalMemoryBusWidth, device);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DWS_ERR_CUDA;
+    }
+    *clock_khz = khz;
+    *bus_bits = bits;
+    return DWS_OK;
 }
 
 uint64_t dws_launch_count(void) { return dws::g_launches.load(std::memory_order_relaxed); }

@@ -434,6 +434,9 @@ cudaError_t launch_pack_positions(const WsView &ws, const DeltaRef &d, uint8_t *
                                   long long pos_capacity, long long *pos_offsets, cudaStream_t s);
 cudaError_t launch_checksum(const uint8_t *positions, long long nbytes, const uint16_t *values,
                             long long nval, unsigned long long *out, cudaStream_t s);
+// wire[0..1] = hashes[0] ^ (hashes[1] << 1) as a 128-bit little-endian integer.
+cudaError_t launch_checksum_wire(const unsigned long long *hashes, unsigned long long *wire,
+                                 cudaStream_t s);
 
 cudaError_t launch_xor(const uint8_t *a, const uint8_t *b, uint8_t *out, long long nbytes,
                        cudaStream_t s);

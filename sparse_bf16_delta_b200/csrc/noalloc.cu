@@ -23,9 +23,12 @@
 //
 // The first call on a device looks up the array's device address there
 // (cudaGetSymbolAddress with that device current); make that first call
-// before capturing any stream on that device.
+// before capturing any stream on that device.  Only a successful lookup is
+// kept: after a failed one (say, during a capture) the call returns
+// DWS_ERR_CUDA and the next call on that device tries again.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "dws_internal.cuh"
@@ -40,14 +43,23 @@ constexpr size_t kNoAllocScratchBytes = 5u << 20;  // 5 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_addr_once[kMaxDevices];
-void *g_addr[kMaxDevices];
-cudaError_t g_addr_err[kMaxDevices];
+std::mutex g_addr_mu[kMaxDevices];
+std::atomic<void *> g_addr[kMaxDevices];  // null until a lookup on that device succeeds
 
-void lookup_scratch(int dev) {
-    void *ptr = nullptr;
-    g_addr_err[dev] = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    g_addr[dev] = ptr;
+// The scratch array's address on device `dev` (the current device), or null
+// if the lookup failed; a failure is not remembered.
+void *scratch_address(int dev) {
+    void *ptr = g_addr[dev].load(std::memory_order_acquire);
+    if (ptr != nullptr) return ptr;
+    std::lock_guard<std::mutex> lock(g_addr_mu[dev]);
+    ptr = g_addr[dev].load(std::memory_order_relaxed);
+    if (ptr != nullptr) return ptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+        (void)cudaGetLastError();  // not left for the next launch check to find
+        return nullptr;
+    }
+    g_addr[dev].store(ptr, std::memory_order_release);
+    return ptr;
 }
 
 // Tables of a one-call plan, passed by value to the set-up kernel.
@@ -126,10 +138,10 @@ extern "C" DWS_API dws_status_t dws_encode_noalloc(const int64_t *numels, int32_
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DWS_ERR_CUDA;
-    std::call_once(g_addr_once[dev], lookup_scratch, dev);
-    if (g_addr_err[dev] != cudaSuccess || g_addr[dev] == nullptr) return DWS_ERR_CUDA;
+    void *scratch = scratch_address(dev);
+    if (scratch == nullptr) return DWS_ERR_CUDA;
 
-    unsigned char *base = static_cast<unsigned char *>(g_addr[dev]);
+    unsigned char *base = static_cast<unsigned char *>(scratch);
     WsView v;
     v.hdr = reinterpret_cast<WsHeader *>(base);
     v.numel = reinterpret_cast<const long long *>(base + L.numel_off);

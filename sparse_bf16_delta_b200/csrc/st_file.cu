@@ -685,6 +685,9 @@ dws_status_t st_delta_read(const dws_plan_t *plan, const char *const *names,
         if (it == entry.end() || !tensor_entry(doc, it->second, "BF16", 2, data_bytes, &nv, &p.vb))
             return DWS_ERR_BAD_DELTA;
         if (nv != p.n) return DWS_ERR_BAD_DELTA;
+        // each changed element at most once: no more entries than elements
+        // (the writer's bound as well)
+        if (p.n > static_cast<unsigned long long>(numel[t])) return DWS_ERR_BAD_DELTA;
         p.present = true;
     }
 

@@ -15,10 +15,12 @@
 // dws_checksum: hash(positions) and hash(values), where hash() XOR-reduces
 //   the elements widened to 64 bits: a byte zero-extended, a bf16 value
 //   converted to the IEEE double equal to it and read as a uint64 (NaNs
-//   quieted with their sign and payload kept).  The checksum of the pages is
-//   hash(positions) ^ (hash(values) << 1), a 65-bit number, so the two
-//   hashes are returned separately.  One grid-stride pass with 16-byte
-//   loads; each CTA XORs its result into the outputs once.
+//   quieted with their sign and payload kept).  One grid-stride pass with
+//   16-byte loads; each CTA XORs its result into the outputs once.  The
+//   checksum of the pages is hash(positions) ^ (hash(values) << 1) on
+//   unbounded integers, a 65-bit number: a one-thread kernel after the hashes
+//   writes it as a 128-bit little-endian integer (two uint64 words, bit 64 the
+//   only bit of the high word that can be set).
 #include <cuda_runtime.h>
 
 #include "dws_internal.cuh"
@@ -207,7 +209,22 @@ __global__ void __launch_bounds__(kSumThreads) checksum_kernel(const uint8_t *po
     }
 }
 
+// checksum = hash(positions) ^ (hash(values) << 1), the shift taken on a
+// 128-bit integer so that bit 63 of hash(values) lands in bit 64.
+__global__ void checksum_wire_kernel(const unsigned long long *hashes, unsigned long long *wire) {
+    if (threadIdx.x != 0) return;
+    const unsigned long long hp = hashes[0], hv = hashes[1];
+    wire[0] = hp ^ (hv << 1);
+    wire[1] = hv >> 63;
+}
+
 }  // namespace
+
+cudaError_t launch_checksum_wire(const unsigned long long *hashes, unsigned long long *wire,
+                                 cudaStream_t s) {
+    checksum_wire_kernel<<<1, 32, 0, s>>>(hashes, wire);
+    return launched();
+}
 
 cudaError_t launch_pack_positions(const WsView &ws, const DeltaRef &d, uint8_t *positions,
                                   long long pos_capacity, long long *pos_offsets, cudaStream_t s) {

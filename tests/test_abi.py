@@ -94,11 +94,12 @@ def test_host_side_argument_errors_need_no_device():
         assert dws.dws_apply_chain(p, 1, arr, 0, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_apply_chain(p, 1, arr, 65, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_encode_global(p, 1, 1, None, 1, 1, 1, 10, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
-        assert dws.dws_encode_checksum(p, 1, 1, 1, 1, 1, 10, None, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_encode_checksum(p, 1, 1, 1, 1, 1, 10, None, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_encode_nnz(p, 1, 1, 1, 1, 1, 10, 1, 1, None, 0, None) == dws.DWS_ERR_INVALID
         assert dws.dws_encode_nnz(p, 1, 1, 1, 1, 1, -1, 1, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_pack_positions(p, 1, 1, 4, 0x1001, 8, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
-        assert dws.dws_checksum(1, -1, 1, 1, 0x1000, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_checksum(1, -1, 1, 1, 0x1000, 0x2000, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_checksum(1, 4, 1, 1, None, 0x2000, None) == dws.DWS_ERR_INVALID
         assert dws.dws_pos_width(p, 0) == 2 and dws.dws_pos_width(p, 1) == 0
         assert dws.dws_apply_chain_ex(p, 1, arr, 1, 3, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_apply_chain_ex(p, 1, arr, 1, -1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID

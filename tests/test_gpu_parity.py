@@ -599,3 +599,89 @@ def test_xor_apply_layers_double_buffered(dws, pinned_masks):
     torch.cuda.current_stream().synchronize()
     for o, nw in zip(olds, news):
         assert torch.equal(o, nw)
+
+
+# ---------------------------------------------------------------- malformed deltas
+
+
+def _malformed_chain(rng, sizes):
+    """Three deltas over `sizes` (dws layout, host arrays) and, for each, the
+    mask of its entries that the pairwise rule flags: delta 0 holds descending
+    pairs (one inside a tile, one across tiles, one across 32-tile windows),
+    delta 1 repeated indices, delta 2 is well formed.  Each flagged entry is
+    followed by one above the entry before it, so no later entry of the
+    segment lies at or below an earlier one except the flagged ones."""
+    deltas, flags = [], []
+    for k in range(3):
+        offs, idx, val, bad = [0], [], [], []
+        for t, n in enumerate(sizes):
+            pos = np.sort(rng.choice(n, min(n, max(1, n // 40)), replace=False)).astype(np.int64)
+            pos = list(pos)
+            b = [False] * len(pos)
+            if k == 0 and t == 1:
+                # insert b < a right after a, then continue above a
+                # plan tiles: tensor 0 owns 0-6, so tensor 1's tile 25 opens
+                # the second 32-tile window
+                for a_at in (8195, 9000, 25 * 8192 + 10):
+                    a_i = next(i for i, x in enumerate(pos) if x >= a_at)
+                    below = pos[a_i] - (7 if a_at == 8195 else (5000 if a_at == 9000 else 8192 * 2))
+                    if a_i + 1 < len(pos) and pos[a_i + 1] > pos[a_i] + 1:
+                        pos.insert(a_i + 1, below)
+                        b.insert(a_i + 1, True)
+            if k == 1 and len(pos) > 4:
+                for dup_at in (1, len(pos) // 2, len(pos) - 2):
+                    pos.insert(dup_at + 1, pos[dup_at])
+                    b.insert(dup_at + 1, True)
+            idx += pos
+            bad += b
+            val += list(rng.integers(0, 1 << 16, len(pos), dtype=np.uint16))
+            offs.append(offs[-1] + len(pos))
+        deltas.append((np.array(offs, np.int64), np.array(idx, np.int32), np.array(val, np.uint16)))
+        flags.append(np.array(bad, bool))
+    return deltas, flags
+
+
+def test_chain_flags_unordered_and_repeated_entries_in_every_mode(dws):
+    # An entry at or below the one before it in its tensor's segment is
+    # flagged (DWS_ERR_BAD_DELTA) and skipped, by dws_apply and by both chain
+    # modes alike; every other position equals the sequential replay of the
+    # entries that are not flagged.
+    rng = np.random.default_rng(77)
+    sizes = [50_000, 8192 * 40 + 3, 7, 20_000]
+    deltas, flags = _malformed_chain(rng, sizes)
+    assert flags[0].sum() >= 3 and flags[1].sum() >= 3 and not flags[2].any()
+    anchor = [rng.integers(0, 1 << 16, n, dtype=np.uint16) for n in sizes]
+    valid = []
+    for (o, i, v), f in zip(deltas, flags):
+        keep = ~f
+        t_of = np.repeat(np.arange(len(sizes)), np.diff(o))
+        vo = np.concatenate([[0], np.cumsum(np.bincount(t_of[keep], minlength=len(sizes)))])
+        valid.append((vo.astype(np.int64), i[keep], v[keep]))
+    ref = [a.copy() for a in anchor]
+    oracle.apply_chain(ref, valid)
+
+    def dev(o, i, v):
+        return dws.Delta(torch.from_numpy(o).cuda(), torch.from_numpy(i).cuda(),
+                         torch.from_numpy(v.view(np.int16)).cuda())
+
+    plan = dws.DeltaPlan(sizes)
+    dd = [dev(*d) for d in deltas]
+    for mode in (1, 2):
+        snaps = [dev_bits(a) for a in anchor]
+        plan.apply_chain(dws.ptr_table(snaps), dd, mode=mode)
+        st, _ = plan.status()
+        assert st == dws.DWS_ERR_BAD_DELTA, mode
+        for s, r in zip(snaps, ref):
+            np.testing.assert_array_equal(host_bits(s), r)
+    # three sequential dws_apply calls do the same
+    snaps = [dev_bits(a) for a in anchor]
+    for d in dd:
+        plan.apply(dws.ptr_table(snaps), d)
+    st, _ = plan.status()
+    assert st == dws.DWS_ERR_BAD_DELTA
+    for s, r in zip(snaps, ref):
+        np.testing.assert_array_equal(host_bits(s), r)
+    # the well-formed delta alone is accepted
+    snaps = [dev_bits(a) for a in anchor]
+    plan.apply_chain(dws.ptr_table(snaps), [dd[2]], mode=2)
+    assert plan.status()[0] == dws.DWS_OK

@@ -2,6 +2,8 @@
 pos_width, and the XOR-hash checksum) against the CPU oracle, byte by byte."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -162,3 +164,50 @@ def test_encode_checksum_fused_equals_pack_then_checksum(dws, rate):
     assert fused == oracle.checksum(blob, v)
     gblob, _ = plan.pack_positions(d)
     assert fused == dws.checksum(gblob, gblob.numel(), d.values)
+
+
+def test_checksum_bit_64_comes_from_the_library(dws):
+    # A negative value widens to a double with bit 63 set, so hash(values)
+    # << 1 reaches bit 64: the 65-bit checksum is read back as written by
+    # libdws (a 128-bit little-endian integer), nothing combined in Python.
+    empty = torch.zeros(2, dtype=torch.uint8, device="cuda")
+    for pats in ([0xBF80], [0xBF80, 0x3F80], [0xFFC1, 0x0001, 0x8000]):
+        v = np.array(pats, dtype=np.uint16)
+        want = oracle.checksum(np.zeros(0, np.uint8), v)
+        got = dws.checksum(empty, 0, dev_bits(v))
+        assert got == want and (got >> 64) == (oracle.checksum_parts(np.zeros(0, np.uint8), v)[1] >> 63)
+    assert dws.checksum(empty, 0, dev_bits(np.array([0xBF80], np.uint16))) >> 64 == 1
+
+
+def test_checksum_through_the_c_abi_from_c(dws, tmp_path):
+    # tests/native/checksum_abi.c calls dws_checksum from C and prints the
+    # hashes and the checksum words; they must equal the oracle's.
+    import shutil
+    import subprocess
+    from tests._dev import ROOT
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("a C compiler is needed")
+    cuda = os.path.dirname(os.path.dirname(os.path.realpath(shutil.which("nvcc") or
+                                                            "/usr/local/cuda/bin/nvcc")))
+    libdir = os.path.dirname(dws.LIB_PATH)
+    exe = str(tmp_path / "checksum_abi")
+    subprocess.run([cc, "-O2", "-o", exe, os.path.join(ROOT, "tests", "native", "checksum_abi.c"),
+                    "-I", os.path.join(ROOT, "include"), "-I", os.path.join(cuda, "include"),
+                    "-L", libdir, "-l:libdws.so", f"-Wl,-rpath,{libdir}",
+                    "-L", os.path.join(cuda, "lib64"), "-lcudart", f"-Wl,-rpath,{cuda}/lib64"],
+                   check=True, capture_output=True)
+    rng = np.random.default_rng(340)
+    for nb, nv in ((0, 0), (13, 7), (100_003, 40_001)):
+        blob = rng.integers(0, 256, nb, dtype=np.uint8)
+        vals = rng.integers(0, 1 << 16, nv, dtype=np.uint16)
+        vals[:min(nv, 3)] |= np.uint16(0x8000)
+        inp = tmp_path / f"in_{nb}_{nv}.bin"
+        inp.write_bytes(np.array([nb, nv], np.int64).tobytes() + blob.tobytes() + vals.tobytes())
+        r = subprocess.run([exe, str(inp)], capture_output=True, text=True, timeout=120)
+        assert r.returncode == 0, r.stderr
+        h0, h1, c0, c1 = (int(x, 16) for x in r.stdout.split())
+        hp, hv = oracle.checksum_parts(blob, vals)
+        assert (h0, h1) == (hp, hv)
+        assert c0 | (c1 << 64) == oracle.checksum(blob, vals)
+        assert c1 in (0, 1)

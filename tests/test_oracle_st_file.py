@@ -204,3 +204,18 @@ def test_reader_takes_the_json_grammar_strictly():
             st_file.read_delta(_raw(text, data), ["a"])
     with pytest.raises(ValueError):
         st_file.read_delta(ok, ["a", "a"])
+
+
+def test_reader_refuses_more_entries_than_elements_when_given_the_sizes():
+    # [TRL] §4.1: a delta names each changed element of a parameter once, so
+    # a parameter with n elements has at most n entries.  A hand-written file
+    # listing 3 entries for "a": read without sizes, refused for a 2-element
+    # "a", read for a 3-element one.
+    md = '"__metadata__":{"sparse":"True","model_version":"1","changed_params":"[\\"a\\"]"}'
+    ent = ('"a.indices":{"dtype":"I32","shape":[3],"data_offsets":[0,12]},'
+           '"a.values":{"dtype":"BF16","shape":[3],"data_offsets":[12,18]}')
+    blob = _raw("{" + md + "," + ent + "}", struct.pack("<3i3H", 0, 1, 2, 1, 2, 3))
+    assert st_file.read_delta(blob, ["a"])[0].tolist() == [0, 3]
+    assert st_file.read_delta(blob, ["a"], [3])[1].tolist() == [0, 1, 2]
+    with pytest.raises(st_file.DeltaFileError):
+        st_file.read_delta(blob, ["a"], [2])

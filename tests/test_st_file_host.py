@@ -75,9 +75,9 @@ def c_read(dws, numels, names, blob):
     return "accepted", oh, ver
 
 
-def o_read(names, blob):
+def o_read(names, blob, numels=None):
     try:
-        o, _, _, ver = st_file.read_delta(blob, names)
+        o, _, _, ver = st_file.read_delta(blob, names, numels)
     except st_file.DeltaFileError:
         return "refused", None, None
     return "accepted", o, ver
@@ -171,6 +171,12 @@ def _crafted_files():
                 '{' + md % ',"v":"\\x"' + ',' + ent + '}', '{' + md % ',"v":"a\tb"' + ',' + ent + '}',
                 '{' + md % ',"v":"\\ud800\\uzzzz"' + ',' + ent + '}'):
         out.append((["a"], [4], raw(bad, data)))
+    # more entries than the parameter has elements (5 for a 4-element "a")
+    ent5 = ('"a.indices":{"dtype":"I32","shape":[5],"data_offsets":[0,20]},'
+            '"a.values":{"dtype":"BF16","shape":[5],"data_offsets":[20,30]}')
+    data5 = struct.pack("<5i5H", 0, 1, 2, 3, 4, *([0x4000] * 5))
+    out.append((["a"], [4], raw("{" + md % "" + "," + ent5 + "}", data5)))
+    out.append((["a"], [5], raw("{" + md % "" + "," + ent5 + "}", data5)))
     b = bytearray(raw("{" + md % ',"v":"é"' + "," + ent + "}", data))
     out.append((["a"], [4], bytes(b)))
     b[b.index(b"\xc3")] = 0xC0  # overlong / invalid UTF-8
@@ -184,7 +190,7 @@ def _crafted_files():
 def test_reader_matches_oracle_on_crafted_files(dws):
     seen = set()
     for names, numels, blob in _crafted_files():
-        want = o_read(names, blob)
+        want = o_read(names, blob, numels)
         got = c_read(dws, numels, names, blob)
         assert got[0] == want[0], (blob[:200], want[0])
         if want[0] == "accepted":
@@ -223,7 +229,7 @@ def test_reader_matches_oracle_on_mutated_files(dws, seed):
                 hl2 = len(b) - 8 - (len(blob) - 8 - hl)  # the data keeps its length
                 b[:8] = struct.pack("<Q", max(0, hl2))
             blob2 = bytes(b)
-            want = o_read(names, blob2)
+            want = o_read(names, blob2, numels)
             got = c_read(dws, numels, names, blob2)
             assert got[0] == want[0], (blob2[8:8 + hl + 2], want[0])
             if want[0] == "accepted":
