@@ -297,3 +297,30 @@ def encode_global(olds, news, index_base):
     counts = np.diff(offsets)
     base = np.repeat(np.asarray(index_base, dtype=np.int64), counts)
     return offsets, indices.astype(np.int64) + base, values
+
+
+def merge_shards(rank_offsets, rank_indices, rank_values):
+    """One delta from the ranks' deltas of their shards, as the page's
+    gather_v_batched_to_rank0 leaves it on rank 0 ([verl] review, key source
+    snippets, sparse_gather.py: after the gather, rank 0 splits each rank's
+    buffer by that rank's per-parameter counts and concatenates, per
+    parameter, the ranks' pieces in rank order).
+    rank_offsets: R arrays int64[T+1] (each rank's delta layout);
+    rank_indices, rank_values: R arrays holding at least rank_offsets[r][T]
+    entries (global int64 positions, bf16 bits).
+    Returns (offsets int64[T+1], indices int64[n], values uint16[n])."""
+    R = len(rank_offsets)
+    T = len(rank_offsets[0]) - 1
+    offsets = [0]
+    idx, val = [], []
+    for t in range(T):
+        n = 0
+        for r in range(R):
+            a, b = int(rank_offsets[r][t]), int(rank_offsets[r][t + 1])
+            idx.append(np.asarray(rank_indices[r][a:b], dtype=np.int64))
+            val.append(np.asarray(rank_values[r][a:b]).view(np.uint16))
+            n += b - a
+        offsets.append(offsets[-1] + n)
+    idx.append(np.zeros(0, np.int64))
+    val.append(np.zeros(0, np.uint16))
+    return np.array(offsets, dtype=np.int64), np.concatenate(idx), np.concatenate(val)

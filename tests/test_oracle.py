@@ -539,3 +539,61 @@ def test_encode_global_matches_the_pages_shard_routine():
     np.testing.assert_array_equal(gi, np.concatenate(want_i))
     np.testing.assert_array_equal(v, np.concatenate(want_v))
     assert gi.max() > 2 ** 32
+
+
+# ---------------------------------------------------------------- gather of shards to rank 0
+
+
+def test_merge_shards_hand_worked():
+    # Two ranks, two parameters: rank 0 has 2 entries of p0 and 1 of p1, rank
+    # 1 one of p0 and none of p1.  Rank 0's merged delta lists p0's entries
+    # rank by rank, then p1's (a dropped rank, a rank-major instead of
+    # parameter-major order or wrong offsets fail it).
+    o, i, v = oracle.merge_shards(
+        [np.array([0, 2, 3]), np.array([0, 1, 1])],
+        [np.array([1, 5, 0]), np.array([9])],
+        [np.array([0xA, 0xB, 0xC], np.uint16), np.array([0xD], np.uint16)])
+    assert o.tolist() == [0, 3, 4]
+    assert i.tolist() == [1, 5, 9, 0]
+    assert v.tolist() == [0xA, 0xB, 0xD, 0xC]
+
+
+@pytest.mark.parametrize("world", [2, 3, 8])
+def test_merge_shards_of_row_shards_equals_the_unsharded_encode(world):
+    # FSDP Shard(0): rank r holds rows [r*c, (r+1)*c) of each parameter
+    # (torch.chunk sizes, so the last ranks may hold fewer rows or none).
+    # Each rank encodes its slice with global positions (offset = first row x
+    # row length, [verl] shard_delta_indices); merging the ranks' deltas must
+    # give the encode of the whole parameters with offset 0.
+    rng = np.random.default_rng(96 + world)
+    shapes = [(37, 64), (5, 3), (1, 1000), (16, 16), (0, 8)]
+    olds, news = [], []
+    for sh in shapes:
+        a = rng.integers(0, 1 << 16, sh, dtype=np.uint16)
+        b = a.copy()
+        m = rng.random(sh) < 0.2
+        b[m] ^= np.uint16(0x0101)
+        olds.append(a)
+        news.append(b)
+    rank_deltas = []
+    for r in range(world):
+        lo, hi, base = [], [], []
+        for a in olds:
+            rows = a.shape[0]
+            c = -(-rows // world) if rows else 0
+            r0, r1 = min(rows, r * c), min(rows, (r + 1) * c)
+            lo.append(a[r0:r1].reshape(-1))
+            base.append(r0 * (a.shape[1] if a.ndim > 1 else 1))
+        for k, b in enumerate(news):
+            rows = b.shape[0]
+            c = -(-rows // world) if rows else 0
+            r0, r1 = min(rows, r * c), min(rows, (r + 1) * c)
+            hi.append(b[r0:r1].reshape(-1))
+        rank_deltas.append(oracle.encode_global(lo, hi, base))
+    o, i, v = oracle.merge_shards(*zip(*rank_deltas))
+    wo, wi, wv = oracle.encode_global([a.reshape(-1) for a in olds], [b.reshape(-1) for b in news],
+                                      [0] * len(shapes))
+    np.testing.assert_array_equal(o, wo)
+    np.testing.assert_array_equal(i, wi)
+    np.testing.assert_array_equal(v, wv)
+    assert int(o[-1]) > 100
