@@ -178,6 +178,37 @@ DWS_API dws_status_t dws_encode_global(const dws_plan_t *plan,
                                uint16_t *values, int64_t capacity,
                                void *workspace, size_t workspace_bytes, dws_stream_t stream);
 
+/* Rank 0's side of gathering sharded deltas ([verl] review of PR #6974, key
+ * source snippets, sparse_gather.py gather_v_batched_to_rank0: one
+ * all_gather of the ranks' per-parameter counts, each rank's concatenated
+ * positions and values padded to the largest total and gathered to rank 0,
+ * which splits them by the counts).  Given the gathered buffers, writes ONE
+ * delta in the dws_encode_global layout: per tensor, the ranks' entries
+ * concatenated in rank order -- ascending whenever rank r's shard of every
+ * tensor precedes rank r+1's (FSDP Shard(0) slices with
+ * index_base = first row x row length).
+ * num_ranks: R >= 1.
+ * rank_offsets: device int64[R][T+1], rank r's offsets (the layout its
+ *   dws_encode_global wrote; the per-parameter counts are their differences).
+ * rank_indices: device int64[R * stride], rank r's entries at [r * stride,
+ *   r * stride + rank_offsets[r][T]) (8-byte aligned); rank_values: device
+ *   uint16[R * stride] likewise (2-byte aligned).  stride >= every rank's
+ *   total (the padded length).
+ * offsets: device int64[T+1], written: offsets[t] = sum over r of
+ *   rank_offsets[r][t].  indices (int64, 8-byte aligned), values: device
+ *   arrays of `capacity` entries.
+ * Errors: host -- DWS_ERR_INVALID (null or misaligned arrays, R out of
+ * [1, 65535], negative sizes), workspace errors as dws_apply; device
+ * (dws_status) -- DWS_ERR_BAD_DELTA (detail -1 - r) when rank r's offsets do
+ * not start at 0, decrease, or end past stride (then no entry is written);
+ * DWS_ERR_CAPACITY (detail = entries needed) when the total exceeds
+ * capacity (offsets complete, entries past capacity not written). */
+DWS_API dws_status_t dws_merge_shards(const dws_plan_t *plan, int32_t num_ranks,
+                              const int64_t *rank_offsets, const int64_t *rank_indices,
+                              const uint16_t *rank_values, int64_t stride, int64_t *offsets,
+                              int64_t *indices, uint16_t *values, int64_t capacity,
+                              void *workspace, size_t workspace_bytes, dws_stream_t stream);
+
 /* dws_encode that also returns the wire checksum of the delta it writes
  * (see dws_checksum): hashes[0] = XOR of the bytes of every position at its
  * tensor's pos_width, hashes[1] = XOR of the double bits of every value, and

@@ -72,6 +72,7 @@ _sig("dws_apply", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_apply_chain", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _vp, _sz, _vp])
 _sig("dws_apply_chain_ex", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _i32, _vp, _sz, _vp])
 _sig("dws_pos_width", _i32, [_vp, _i32])
+_sig("dws_merge_shards", _i32, [_vp, _i32, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_encode_global", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_encode_checksum", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _vp])
 _sig("dws_pack_positions", _i32, [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp])
@@ -206,6 +207,13 @@ def dws_encode_checksum(plan, old_ptrs, new_ptrs, offsets, indices, values, capa
                         checksum, workspace, workspace_bytes, stream) -> int:
     return _lib.dws_encode_checksum(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
                                     hashes, checksum, workspace, workspace_bytes, stream)
+
+
+def dws_merge_shards(plan, num_ranks, rank_offsets, rank_indices, rank_values, stride, offsets,
+                     indices, values, capacity, workspace, workspace_bytes, stream) -> int:
+    return _lib.dws_merge_shards(plan, num_ranks, rank_offsets, rank_indices, rank_values, stride,
+                                 offsets, indices, values, capacity, workspace, workspace_bytes,
+                                 stream)
 
 
 def dws_pos_width(plan, t) -> int:
@@ -502,6 +510,26 @@ class DeltaPlan:
                "dws_encode_checksum")
         self.raise_on_error("dws_encode_checksum", stream)
         return Delta(offsets, indices, values), _wire_int(wire)
+
+    def merge_shards(self, rank_offsets, rank_indices, rank_values, stream=None) -> Delta:
+        """One delta (int64 global positions) from R ranks' gathered deltas:
+        rank_offsets int64 [R, T+1], rank_indices int64 [R, stride],
+        rank_values int16 [R, stride] (device tensors, row r = rank r's
+        padded buffer).  Per tensor, the ranks' entries in rank order."""
+        torch = _torch()
+        R, stride = int(rank_indices.shape[0]), int(rank_indices.shape[1])
+        nnz = int(rank_offsets[:, -1].sum().item())
+        offsets = torch.empty(self.num_tensors + 1, dtype=torch.int64, device=self.device)
+        indices = torch.empty(nnz, dtype=torch.int64, device=self.device)
+        values = torch.empty(nnz, dtype=torch.int16, device=self.device)
+        ro, ri, rv = (x.contiguous() for x in (rank_offsets, rank_indices, rank_values))
+        _check(dws_merge_shards(self.handle, R, ro.data_ptr(), ri.data_ptr() if stride else 0,
+                                rv.data_ptr() if stride else 0, stride, offsets.data_ptr(),
+                                indices.data_ptr() if nnz else 0, values.data_ptr() if nnz else 0,
+                                nnz, self.workspace.data_ptr(), self.workspace_bytes,
+                                _stream_handle(stream)), "dws_merge_shards")
+        self.raise_on_error("dws_merge_shards", stream)
+        return Delta(offsets, indices, values)
 
     # -- wire form --
     def pos_width(self, t: int) -> int:

@@ -760,9 +760,13 @@ cudaError_t chain_occupancy(int *ctas_per_sm) {
                                                          sizeof(ChainSmem));
 }
 
-cudaError_t launch_delta_check(const WsView &ws, const DeltaRef *deltas, int K, cudaStream_t s) {
+cudaError_t launch_delta_flag_clear(const WsView &ws, cudaStream_t s) {
     delta_flag_clear_kernel<<<1, 1, 0, s>>>(ws);
-    cudaError_t e = launched();
+    return launched();
+}
+
+cudaError_t launch_delta_check(const WsView &ws, const DeltaRef *deltas, int K, cudaStream_t s) {
+    cudaError_t e = launch_delta_flag_clear(ws, s);
     if (e != cudaSuccess) return e;
     CheckParams p;
     p.ws = ws;

@@ -342,6 +342,28 @@ dws_status_t dws_apply_chain_ex(const dws_plan_t *plan, void *const *snap_ptrs,
                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
+dws_status_t dws_merge_shards(const dws_plan_t *plan, int32_t num_ranks,
+                              const int64_t *rank_offsets, const int64_t *rank_indices,
+                              const uint16_t *rank_values, int64_t stride, int64_t *offsets,
+                              int64_t *indices, uint16_t *values, int64_t capacity,
+                              void *workspace, size_t workspace_bytes, dws_stream_t stream) {
+    dws_status_t st = check_ws(plan, workspace, workspace_bytes);
+    if (st != DWS_OK) return st;
+    if (num_ranks < 1 || num_ranks > 65535 || rank_offsets == nullptr || offsets == nullptr ||
+        stride < 0 || capacity < 0)
+        return DWS_ERR_INVALID;
+    if (stride > 0 && (rank_indices == nullptr || rank_values == nullptr)) return DWS_ERR_INVALID;
+    if (capacity > 0 && (indices == nullptr || values == nullptr)) return DWS_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(rank_indices) & 7u) || (reinterpret_cast<uintptr_t>(indices) & 7u) ||
+        (reinterpret_cast<uintptr_t>(rank_values) & 1u) || (reinterpret_cast<uintptr_t>(values) & 1u))
+        return DWS_ERR_INVALID;
+    return from_cuda(dws::launch_merge_shards(
+        view_of(plan, workspace), num_ranks, reinterpret_cast<const long long *>(rank_offsets),
+        reinterpret_cast<const long long *>(rank_indices), rank_values, stride,
+        reinterpret_cast<long long *>(offsets), reinterpret_cast<long long *>(indices), values,
+        capacity, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int32_t dws_pos_width(const dws_plan_t *plan, int32_t t) {
     if (plan == nullptr || t < 0 || t >= plan->T) return 0;
     const long long *numel =

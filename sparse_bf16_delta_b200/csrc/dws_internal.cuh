@@ -421,7 +421,14 @@ struct DeltaRef {
     long long count;
 };
 
+// Clears the workspace's delta flag (set by a failed validation) on the stream.
+cudaError_t launch_delta_flag_clear(const WsView &ws, cudaStream_t s);
 cudaError_t launch_delta_check(const WsView &ws, const DeltaRef *deltas, int K, cudaStream_t s);
+// Rank 0's merge of gathered shard deltas (dws_merge_shards).
+cudaError_t launch_merge_shards(const WsView &ws, int R, const long long *rank_offsets,
+                                const long long *rank_indices, const uint16_t *rank_values,
+                                long long stride, long long *offsets, long long *indices,
+                                uint16_t *values, long long capacity, cudaStream_t s);
 cudaError_t launch_apply(const WsView &ws, uint16_t *const *snap_ptrs, const DeltaRef &d,
                          cudaStream_t s);
 cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs,

@@ -101,6 +101,13 @@ def test_host_side_argument_errors_need_no_device():
         assert dws.dws_checksum(1, -1, 1, 1, 0x1000, 0x2000, None) == dws.DWS_ERR_INVALID
         assert dws.dws_checksum(1, 4, 1, 1, None, 0x2000, None) == dws.DWS_ERR_INVALID
         assert dws.dws_pos_width(p, 0) == 2 and dws.dws_pos_width(p, 1) == 0
+        # dws_merge_shards: ranks out of range, null or misaligned arrays, negative sizes
+        assert dws.dws_merge_shards(p, 0, 8, 8, 8, 1, 8, 8, 8, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_merge_shards(p, 1, None, 8, 8, 1, 8, 8, 8, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_merge_shards(p, 1, 8, 12, 8, 1, 8, 8, 8, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_merge_shards(p, 1, 8, 8, 9, 1, 8, 8, 8, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_merge_shards(p, 1, 8, 8, 8, -1, 8, 8, 8, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
+        assert dws.dws_merge_shards(p, 1, 8, 8, 8, 1, 8, 8, 8, 1, 0x1000, 16, None) == dws.DWS_ERR_WORKSPACE
         assert dws.dws_apply_chain_ex(p, 1, arr, 1, 3, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_apply_chain_ex(p, 1, arr, 1, -1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_apply_chain_ex(p, 1, arr, 0, 2, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID

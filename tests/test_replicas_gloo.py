@@ -87,14 +87,23 @@ def test_reference_arm_runs_on_rank_zero_only():
 
 
 def test_theoretical_hbm_peak_from_device_attributes():
-    # B200: 3,996 MHz HBM3e, 8 stacks x 1024 bits: 8.18 TB/s; an H100 SXM's
-    # 2,619 MHz x 5120 bits gives its 3.35 TB/s; missing attributes give None.
+    # The two device attributes libdws reports (memory clock in kHz, bus
+    # width in bits) give clock x 2 (double data rate) x width / 8: an H100
+    # SXM's 2,619 MHz x 5120 bits is its 3.35 TB/s; 3,996 MHz x 7680 bits is
+    # 7.67 TB/s.  A failed query or a zero attribute gives no peak.
     import types
 
     import bench
-    b200 = types.SimpleNamespace(memory_clock_rate=3_996_000, memory_bus_width=8192)
-    assert abs(bench.theoretical_hbm_gbs(b200) - 8183.8) < 0.1
-    h100 = types.SimpleNamespace(memory_clock_rate=2_619_000, memory_bus_width=5120)
-    assert abs(bench.theoretical_hbm_gbs(h100) - 3352.3) < 0.1
-    assert bench.theoretical_hbm_gbs(types.SimpleNamespace()) is None
-    assert bench.theoretical_hbm_gbs(types.SimpleNamespace(memory_clock_rate=0, memory_bus_width=8)) is None
+
+    def fake(khz, bits):
+        return types.SimpleNamespace(dws_device_memory=lambda dev: (khz, bits))
+
+    peak, khz, bits = bench.theoretical_hbm_gbs(fake(2_619_000, 5120), 0)
+    assert abs(peak - 3352.3) < 0.1 and (khz, bits) == (2_619_000, 5120)
+    assert abs(bench.theoretical_hbm_gbs(fake(3_996_000, 7680), 0)[0] - 7672.3) < 0.1
+    assert bench.theoretical_hbm_gbs(fake(0, 8), 0)[0] is None
+
+    def broken(dev):
+        raise RuntimeError("no device")
+
+    assert bench.theoretical_hbm_gbs(types.SimpleNamespace(dws_device_memory=broken), 0) == (None, None, None)
