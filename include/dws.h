@@ -313,33 +313,38 @@ typedef struct dws_delta {
 
 /* Anchor + delta chain ([TRL] §4.1: an anchor every N syncs, sparse deltas in
  * between; a new replica takes the latest anchor and replays the deltas after
- * it).  Applies deltas[0..K-1] in order onto snap_ptrs in ONE launch: each
- * block owns a range of elements and replays all K deltas over it, so where
- * deltas touch the same element the later one wins, exactly as K sequential
- * dws_apply calls.  deltas: host array of K (1 <= K <= DWS_MAX_CHAIN).
- * Every entry is checked as dws_apply checks it, in every mode: an index
- * outside its tensor, or not above the entry before it in its tensor's
- * segment (descending or repeated), is skipped and DWS_ERR_BAD_DELTA
- * recorded (detail = its entry number in its delta); offsets that fail
- * validation write nothing.  Elements named only by entries that pass are
- * exactly as K sequential dws_apply calls leave them.  An entry above the one
- * before it but not above every earlier entry of its segment (possible only
- * after a flagged entry) may or may not be applied: after DWS_ERR_BAD_DELTA
- * the elements such entries name are unspecified. */
+ * it).  Applies deltas[0..K-1] in order onto snap_ptrs: where deltas touch
+ * the same element the later one wins, exactly as K sequential dws_apply
+ * calls on deltas that pass the checks below.  deltas: host array of K
+ * (1 <= K <= DWS_MAX_CHAIN).
+ * Every entry of every delta is checked before anything is written: its
+ * index must lie inside its tensor and be strictly above the entry before it
+ * in its tensor's segment (as dws_encode writes them), and the offsets must
+ * pass dws_apply's checks.  If any check fails, DWS_ERR_BAD_DELTA is recorded
+ * (detail = an offending entry's number in its delta, or -1 - k for delta
+ * k's offsets) and the snapshot is left exactly as it was: a receiver never
+ * holds a half-applied chain.  (dws_apply, one delta, instead skips each bad
+ * entry and applies the rest.)
+ * Runs one pass over the snapshot per 16 deltas; uses the workspace's
+ * per-call scratch (the encode's), so it must not overlap an encode on the
+ * same workspace. */
 DWS_API dws_status_t dws_apply_chain(const dws_plan_t *plan, void *const *snap_ptrs,
                              const dws_delta_t *deltas, int32_t K,
                              void *workspace, size_t workspace_bytes, dws_stream_t stream);
 
 /* How dws_apply_chain_ex replays the chain; both give the same snapshot.
- * DWS_CHAIN_AUTO: the library's choice (what dws_apply_chain does).
- * DWS_CHAIN_TILE_MERGE: every snapshot tile is read into shared memory, the
- *   entries of all K deltas are merged into it (the latest delta wins per
- *   element) and the whole tile is written back: 4 bytes per element of the
- *   snapshot plus 6 per entry, whatever the deltas touch.
+ * DWS_CHAIN_AUTO: the library's choice (what dws_apply_chain does): the tile
+ *   merge when the deltas' entry counts suggest that more than half of the
+ *   snapshot's 32-byte sectors are touched, else the scatter.
+ * DWS_CHAIN_TILE_MERGE: every tile some delta touches is read into shared
+ *   memory, the entries of all deltas for it are written in delta order and
+ *   the whole tile is written back (4 bytes per element of the touched tiles
+ *   plus 6 per entry); tiles no delta touches are not moved.
  * DWS_CHAIN_SCATTER: per window of tiles, the deltas are replayed from the last
  *   to the first and an element is stored only by the latest delta that
  *   touches it (a written-bit per element in shared memory); untouched parts of
- *   the snapshot are neither read nor written. */
+ *   the snapshot are neither read nor written (L2 reads and writes back the
+ *   touched 32-byte sectors). */
 #define DWS_CHAIN_AUTO 0
 #define DWS_CHAIN_TILE_MERGE 1
 #define DWS_CHAIN_SCATTER 2

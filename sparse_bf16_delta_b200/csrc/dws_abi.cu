@@ -15,10 +15,10 @@ namespace dws {
 size_t encode_smem_bytes();
 cudaError_t encode_set_attributes();
 cudaError_t encode_occupancy(int *ctas_per_sm);
-size_t chain_smem_bytes();
 cudaError_t chain_set_attributes();
 cudaError_t chain_occupancy(int *ctas_per_sm);
 cudaError_t scatter_occupancy(int *ctas_per_sm);
+cudaError_t index_occupancy(int *ctas_per_sm);
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -34,10 +34,12 @@ void init_device(int dev) {
     if (e == cudaSuccess) e = encode_occupancy(&di.encode_ctas_per_sm);
     if (e == cudaSuccess) e = chain_occupancy(&di.chain_ctas_per_sm);
     if (e == cudaSuccess) e = scatter_occupancy(&di.scatter_ctas_per_sm);
+    if (e == cudaSuccess) e = index_occupancy(&di.index_ctas_per_sm);
     if (e == cudaSuccess) {
         if (di.encode_ctas_per_sm < 1) di.encode_ctas_per_sm = 1;
         if (di.chain_ctas_per_sm < 1) di.chain_ctas_per_sm = 1;
         if (di.scatter_ctas_per_sm < 1) di.scatter_ctas_per_sm = 1;
+        if (di.index_ctas_per_sm < 1) di.index_ctas_per_sm = 1;
     }
     g_info[dev] = di;
     g_err[dev] = e;
@@ -120,6 +122,25 @@ dws_status_t check_ws(const dws_plan *p, const void *ws, size_t ws_bytes) {
 }
 
 dws_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? DWS_OK : DWS_ERR_CUDA; }
+
+// DWS_CHAIN_AUTO's choice, from what the host knows (the entry counts): the
+// merge moves every touched tile whole, the scatter only the touched 32-byte
+// sectors, each read and written back by L2.  With the deltas' union covering
+// a fraction u of the elements, about 1 - (1 - u)^16 of the sectors are
+// touched; above one half the merge moves fewer bytes, or about as many at a
+// better rate (whole-tile bulk copies against partial-sector writes).
+int32_t chain_auto_mode(const dws::DeltaRef *d, int32_t K, long long N) {
+    if (N <= 0) return DWS_CHAIN_SCATTER;
+    double keep = 1.0;  // fraction of elements no delta names (independent deltas)
+    for (int32_t k = 0; k < K; ++k) {
+        double f = double(d[k].count) / double(N);
+        if (f > 1.0) f = 1.0;
+        keep *= 1.0 - f;
+    }
+    double untouched_sector = 1.0;
+    for (int i = 0; i < 16; ++i) untouched_sector *= keep;
+    return (1.0 - untouched_sector) > 0.5 ? DWS_CHAIN_TILE_MERGE : DWS_CHAIN_SCATTER;
+}
 
 dws_status_t encode_common(const dws_plan_t *plan, const void *const *old_ptrs,
                            const void *const *new_ptrs, int64_t *offsets, int32_t *indices,
@@ -321,24 +342,22 @@ dws_status_t dws_apply_chain_ex(const dws_plan_t *plan, void *const *snap_ptrs,
     if (mode != DWS_CHAIN_AUTO && mode != DWS_CHAIN_TILE_MERGE && mode != DWS_CHAIN_SCATTER)
         return DWS_ERR_INVALID;
     dws::DeltaRef d[DWS_MAX_CHAIN];
-    long long total = 0;
     for (int32_t k = 0; k < K; ++k) {
         if (deltas[k].offsets == nullptr || deltas[k].count < 0) return DWS_ERR_INVALID;
         if (deltas[k].count > 0 && (deltas[k].indices == nullptr || deltas[k].values == nullptr))
             return DWS_ERR_INVALID;
+        if ((reinterpret_cast<uintptr_t>(deltas[k].indices) & 3u) ||
+            (reinterpret_cast<uintptr_t>(deltas[k].values) & 1u) ||
+            (reinterpret_cast<uintptr_t>(deltas[k].offsets) & 7u))
+            return DWS_ERR_INVALID;
         d[k] = dws::DeltaRef{reinterpret_cast<const long long *>(deltas[k].offsets),
                              reinterpret_cast<const int *>(deltas[k].indices), deltas[k].values,
                              deltas[k].count};
-        total += deltas[k].count;
     }
-    if (mode == DWS_CHAIN_AUTO) mode = DWS_CHAIN_SCATTER;
-    if (mode == DWS_CHAIN_SCATTER)
-        return from_cuda(dws::launch_apply_chain_scatter(
-            view_of(plan, workspace), reinterpret_cast<uint16_t *const *>(snap_ptrs), d, K,
-            reinterpret_cast<cudaStream_t>(stream)));
+    if (mode == DWS_CHAIN_AUTO) mode = chain_auto_mode(d, K, plan->N);
     return from_cuda(dws::launch_apply_chain(view_of(plan, workspace),
                                              reinterpret_cast<uint16_t *const *>(snap_ptrs), d, K,
-                                             total, plan->N,
+                                             mode == DWS_CHAIN_TILE_MERGE,
                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 

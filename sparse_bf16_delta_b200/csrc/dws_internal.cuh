@@ -20,9 +20,7 @@ namespace dws {
 // ---------------------------------------------------------------------------
 // Tiling shared by the encode scan and the chain replay: a tensor is cut into
 // tiles of kTileElems elements (16 KiB of bf16 per snapshot); a tile never
-// straddles two tensors and an empty tensor owns one empty tile.  The chain
-// replay works on units of up to kChainUnitTiles consecutive tiles of one
-// tensor.
+// straddles two tensors and an empty tensor owns one empty tile.
 // ---------------------------------------------------------------------------
 constexpr int kTileElems = 8192;
 constexpr int kTileShift = 13;
@@ -31,8 +29,10 @@ constexpr int kTileShift = 13;
 // those reads on a few L2 lines (and slices).
 constexpr int kStatusStride = 4;
 static_assert((1 << kTileShift) == kTileElems, "tile size must be a power of two");
-constexpr int kChainUnitTiles = 1;
-constexpr int kChainUnitElems = kChainUnitTiles * kTileElems;
+// The chain replay handles up to kChainGroup deltas per pass over the
+// snapshot; its tile index holds, per tile and delta of the pass, the first
+// entry at or past the tile (mod 2^32), kChainGroup words per tile.
+constexpr int kChainGroup = 16;
 
 // ---------------------------------------------------------------------------
 // Workspace layout (device memory owned by the caller)
@@ -43,6 +43,10 @@ constexpr int kChainUnitElems = kChainUnitTiles * kTileElems;
 //   tile_tensor       int32[ntiles]      tensor of each tile   (static)
 //   tile_status       uint64[ntiles * kStatusStride]  encode scan state (per call)
 //   tile_desc         TileDesc[ntiles]   encode tile pointers  (per call)
+//
+// The chain replay's tile index, uint32[(ntiles + 1) * kChainGroup] (per
+// call), overlays tile_status and tile_desc: 64 bytes per tile, the two
+// regions' size, plus one more row that the total leaves room for.
 //
 // Every region starts on a 256-byte boundary.  The static regions are written
 // by dws_plan_upload; the header's magic + fingerprint tie the workspace to
@@ -96,6 +100,9 @@ inline WsLayout ws_layout(int T, long long ntiles) {
     L.tile_desc_off = round_up256(L.tile_status_off +
                                   sizeof(unsigned long long) * size_t(ntiles) * kStatusStride);
     L.total = round_up256(L.tile_desc_off + sizeof(TileDesc) * size_t(ntiles));
+    const size_t index_end =
+        L.tile_status_off + sizeof(uint32_t) * size_t(kChainGroup) * size_t(ntiles + 1);
+    if (L.total < round_up256(index_end)) L.total = round_up256(index_end);
     return L;
 }
 
@@ -222,6 +229,34 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long *bar, uint32_t pari
     return true;
 }
 
+// try_wait that lets the hardware suspend the thread for up to `hint_ns`
+// while the phase is incomplete (instead of returning at once).
+__device__ __forceinline__ bool mbar_try_wait_hint(unsigned long long *bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+
+// mbar_wait for threads that may wait long: each test suspends the thread
+// in hardware for up to a microsecond, leaving the issue slots to the warps
+// that work.
+__device__ __forceinline__ bool mbar_wait_sleepy(unsigned long long *bar, uint32_t parity,
+                                                 unsigned long long limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_timer_ns();
+    while (!mbar_try_wait_hint(bar, parity, 1000u)) {
+        if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
 // --- 1-D bulk async copies (no tensor map, no multicast) --------------------
 // global -> this CTA's shared memory, completion counted on `bar`.
 // dst and src 16-byte aligned, bytes a multiple of 16.
@@ -248,6 +283,21 @@ __device__ __forceinline__ void bulk_commit() {
 // The issuing thread's committed bulk stores have finished READING shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// All but the n most recently committed bulk-store groups of the issuing
+// thread have finished READING shared memory (n > 7 waits for all).
+__device__ __forceinline__ void bulk_wait_read_n(int n) {
+    switch (n) {
+        case 1: asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); break;
+        case 2: asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory"); break;
+        case 3: asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory"); break;
+        case 4: asm volatile("cp.async.bulk.wait_group.read 4;" ::: "memory"); break;
+        case 5: asm volatile("cp.async.bulk.wait_group.read 5;" ::: "memory"); break;
+        case 6: asm volatile("cp.async.bulk.wait_group.read 6;" ::: "memory"); break;
+        case 7: asm volatile("cp.async.bulk.wait_group.read 7;" ::: "memory"); break;
+        default: asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); break;
+    }
 }
 
 // The issuing thread's committed bulk stores are complete.
@@ -398,6 +448,7 @@ struct DeviceInfo {
     int encode_ctas_per_sm;
     int chain_ctas_per_sm;
     int scatter_ctas_per_sm;
+    int index_ctas_per_sm;
 };
 
 // Per-device constants and one-time kernel attribute setup (thread-safe).
@@ -431,11 +482,12 @@ cudaError_t launch_merge_shards(const WsView &ws, int R, const long long *rank_o
                                 uint16_t *values, long long capacity, cudaStream_t s);
 cudaError_t launch_apply(const WsView &ws, uint16_t *const *snap_ptrs, const DeltaRef &d,
                          cudaStream_t s);
+// Chain replay (chain.cu): validation and tile index of every delta, then
+// one pass per group of up to kChainGroup deltas, by tile merge (merge =
+// true) or by reverse-order scatter.  Nothing is written unless every delta
+// passes validation.
 cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs,
-                               const DeltaRef *deltas, int K, long long total_entries,
-                               long long total_elems, cudaStream_t s);
-cudaError_t launch_apply_chain_scatter(const WsView &ws, uint16_t *const *snap_ptrs,
-                                       const DeltaRef *deltas, int K, cudaStream_t s);
+                               const DeltaRef *deltas, int K, bool merge, cudaStream_t s);
 
 cudaError_t launch_pack_positions(const WsView &ws, const DeltaRef &d, uint8_t *positions,
                                   long long pos_capacity, long long *pos_offsets, cudaStream_t s);

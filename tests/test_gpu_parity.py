@@ -338,7 +338,7 @@ def test_apply_with_bad_offsets_writes_nothing(dws):
 # ---------------------------------------------------------------- chain
 
 # Both replay modes of dws_apply_chain_ex must give the sequential replay.
-CHAIN_MODES = pytest.mark.parametrize("mode", [1, 2], ids=["tile_merge", "scatter"])
+CHAIN_MODES = pytest.mark.parametrize("mode", [0, 1, 2], ids=["auto", "tile_merge", "scatter"])
 
 
 @CHAIN_MODES
@@ -456,6 +456,93 @@ def test_chain_max_length_tiny_and_empty_tensors(dws, mode):
         np.testing.assert_array_equal(host_bits(s), c)
 
 
+def _host_chain(rng, sizes, rates, K):
+    """An anchor and K consecutive random steps (per-delta rates cycled),
+    with the oracle's deltas and the final snapshot."""
+    anchor = [rng.integers(0, 1 << 16, n, dtype=np.uint16) for n in sizes]
+    cur = [a.copy() for a in anchor]
+    host_deltas = []
+    for k in range(K):
+        rate = rates[k % len(rates)]
+        nxt = []
+        for c in cur:
+            x = c.copy()
+            if c.size:
+                m = rng.random(c.size) < rate
+                x[m] ^= rng.integers(1, 1 << 16, int(m.sum()), dtype=np.uint16)
+            nxt.append(x)
+        host_deltas.append(oracle.encode(cur, nxt))
+        cur = nxt
+    return anchor, host_deltas, cur
+
+
+@CHAIN_MODES
+@pytest.mark.parametrize("ishift,vshift", [(1, 3), (3, 1), (2, 0)])
+def test_chain_on_unaligned_delta_arrays(dws, mode, ishift, vshift):
+    # Index and value arrays that start 4/8/12 and 2/6 bytes past a 16-byte
+    # boundary: the staged middles, the heads and tails read from global
+    # memory, and the index pass's scalar loads.
+    rng = np.random.default_rng(90 + 7 * ishift + vshift)
+    sizes = [8192 * 5 + 11, 3000, 8192 * 2]
+    anchor, host_deltas, final = _host_chain(rng, sizes, [0.05, 0.4, 0.01], 5)
+    dd = []
+    for o, i, v in host_deltas:
+        ib = torch.zeros(i.size + 8, dtype=torch.int32, device="cuda")
+        vb = torch.zeros(v.size + 8, dtype=torch.int16, device="cuda")
+        ib[ishift:ishift + i.size] = torch.from_numpy(i).cuda()
+        vb[vshift:vshift + v.size] = torch.from_numpy(v.view(np.int16)).cuda()
+        dd.append(dws.Delta(torch.from_numpy(o).cuda(), ib[ishift:ishift + i.size],
+                            vb[vshift:vshift + v.size]))
+    plan = dws.DeltaPlan(sizes)
+    snaps = [dev_bits(a) for a in anchor]
+    plan.apply_chain(dws.ptr_table(snaps), dd, mode=mode)
+    plan.raise_on_error()
+    for s_, f in zip(snaps, final):
+        np.testing.assert_array_equal(host_bits(s_), f)
+
+
+@CHAIN_MODES
+def test_chain_denser_than_a_stage_holds(dws, mode):
+    # Every element changed by every delta: a tile's entries (8192 per delta)
+    # exceed what one merge stage holds, so part of them is read straight
+    # from global memory; then the same with one sparse delta in between.
+    rng = np.random.default_rng(91)
+    sizes = [8192 * 6 + 5, 100]
+    for rates in ([1.0], [1.0, 0.001, 0.9]):
+        anchor, host_deltas, final = _host_chain(rng, sizes, rates, 4)
+        dd = [dws.Delta(torch.from_numpy(o).cuda(), torch.from_numpy(i).cuda(),
+                        torch.from_numpy(v.view(np.int16)).cuda()) for o, i, v in host_deltas]
+        plan = dws.DeltaPlan(sizes)
+        snaps = [dev_bits(a) for a in anchor]
+        plan.apply_chain(dws.ptr_table(snaps), dd, mode=mode)
+        plan.raise_on_error()
+        for s_, f in zip(snaps, final):
+            np.testing.assert_array_equal(host_bits(s_), f)
+
+
+@CHAIN_MODES
+def test_chain_of_single_entries_over_many_tiles(dws, mode):
+    # Deltas of one entry each in a plan of thousands of tiles: the tile
+    # index's long runs of rows pointing at the same entry.
+    sizes = [8192 * 3000 + 1, 5, 8192 * 10]
+    rng = np.random.default_rng(92)
+    anchor = [rng.integers(0, 1 << 16, n, dtype=np.uint16) for n in sizes]
+    host_deltas, cur = [], [a.copy() for a in anchor]
+    for t, i in ((0, 8192 * 2999 + 7), (2, 3), (0, 0), (1, 4)):
+        nxt = [c.copy() for c in cur]
+        nxt[t][i] ^= np.uint16(0x0102)
+        host_deltas.append(oracle.encode(cur, nxt))
+        cur = nxt
+    dd = [dws.Delta(torch.from_numpy(o).cuda(), torch.from_numpy(i).cuda(),
+                    torch.from_numpy(v.view(np.int16)).cuda()) for o, i, v in host_deltas]
+    plan = dws.DeltaPlan(sizes)
+    snaps = [dev_bits(a) for a in anchor]
+    plan.apply_chain(dws.ptr_table(snaps), dd, mode=mode)
+    plan.raise_on_error()
+    for s_, f in zip(snaps, cur):
+        np.testing.assert_array_equal(host_bits(s_), f)
+
+
 @CHAIN_MODES
 def test_chain_single_delta_equals_apply(dws, mode):
     rng = np.random.default_rng(65)
@@ -487,10 +574,9 @@ def test_chain_rejects_index_beyond_numel(dws, mode):
                   torch.tensor([3, n + 5], dtype=torch.int32, device="cuda"),
                   torch.tensor([7, 7], dtype=torch.int16, device="cuda"))
     plan.apply_chain(dws.ptr_table([snap]), [d], mode=mode)
-    st, _ = plan.status()
-    assert st == dws.DWS_ERR_BAD_DELTA
-    h = host_bits(snap)
-    assert h[3] == 7 and h.sum() == 7
+    st, detail = plan.status()
+    assert st == dws.DWS_ERR_BAD_DELTA and detail == 1
+    assert host_bits(snap).sum() == 0  # a chain with a bad entry writes nothing
 
 
 @CHAIN_MODES
@@ -502,10 +588,9 @@ def test_chain_rejects_negative_index(dws, mode):
                   torch.tensor([-4, 11], dtype=torch.int32, device="cuda"),
                   torch.tensor([7, 7], dtype=torch.int16, device="cuda"))
     plan.apply_chain(dws.ptr_table([snap]), [d], mode=mode)
-    st, _ = plan.status()
-    assert st == dws.DWS_ERR_BAD_DELTA
-    h = host_bits(snap)
-    assert h[11] == 7 and h.sum() == 7
+    st, detail = plan.status()
+    assert st == dws.DWS_ERR_BAD_DELTA and detail == 0
+    assert host_bits(snap).sum() == 0  # a chain with a bad entry writes nothing
 
 
 # ---------------------------------------------------------------- sparse delta of XOR layers
@@ -641,11 +726,12 @@ def _malformed_chain(rng, sizes):
     return deltas, flags
 
 
-def test_chain_flags_unordered_and_repeated_entries_in_every_mode(dws):
-    # An entry at or below the one before it in its tensor's segment is
-    # flagged (DWS_ERR_BAD_DELTA) and skipped, by dws_apply and by both chain
-    # modes alike; every other position equals the sequential replay of the
-    # entries that are not flagged.
+def test_chain_with_unordered_or_repeated_entries_writes_nothing_in_every_mode(dws):
+    # Descending pairs (inside a tile, across tiles, across 32-tile windows)
+    # and repeated indices: every mode records DWS_ERR_BAD_DELTA and leaves
+    # the snapshot exactly as it was; dws_apply, one delta at a time, skips
+    # the flagged entries and applies the rest; without the malformed deltas
+    # the chain is applied.
     rng = np.random.default_rng(77)
     sizes = [50_000, 8192 * 40 + 3, 7, 20_000]
     deltas, flags = _malformed_chain(rng, sizes)
@@ -666,14 +752,15 @@ def test_chain_flags_unordered_and_repeated_entries_in_every_mode(dws):
 
     plan = dws.DeltaPlan(sizes)
     dd = [dev(*d) for d in deltas]
-    for mode in (1, 2):
-        snaps = [dev_bits(a) for a in anchor]
-        plan.apply_chain(dws.ptr_table(snaps), dd, mode=mode)
-        st, _ = plan.status()
-        assert st == dws.DWS_ERR_BAD_DELTA, mode
-        for s, r in zip(snaps, ref):
-            np.testing.assert_array_equal(host_bits(s), r)
-    # three sequential dws_apply calls do the same
+    for mode in (0, 1, 2):
+        for chain in (dd, [dd[2], dd[0]], [dd[1]], dd * 6):  # 18 deltas: two passes
+            snaps = [dev_bits(a) for a in anchor]
+            plan.apply_chain(dws.ptr_table(snaps), chain, mode=mode)
+            st, _ = plan.status()
+            assert st == dws.DWS_ERR_BAD_DELTA, (mode, len(chain))
+            for s, a in zip(snaps, anchor):
+                np.testing.assert_array_equal(host_bits(s), a)
+    # three sequential dws_apply calls skip the flagged entries
     snaps = [dev_bits(a) for a in anchor]
     for d in dd:
         plan.apply(dws.ptr_table(snaps), d)
@@ -681,7 +768,11 @@ def test_chain_flags_unordered_and_repeated_entries_in_every_mode(dws):
     assert st == dws.DWS_ERR_BAD_DELTA
     for s, r in zip(snaps, ref):
         np.testing.assert_array_equal(host_bits(s), r)
-    # the well-formed delta alone is accepted
-    snaps = [dev_bits(a) for a in anchor]
-    plan.apply_chain(dws.ptr_table(snaps), [dd[2]], mode=2)
-    assert plan.status()[0] == dws.DWS_OK
+    # the well-formed parts replay as the oracle says, in every mode
+    vd = [dev(*v) for v in valid]
+    for mode in (0, 1, 2):
+        snaps = [dev_bits(a) for a in anchor]
+        plan.apply_chain(dws.ptr_table(snaps), vd, mode=mode)
+        assert plan.status()[0] == dws.DWS_OK
+        for s, r in zip(snaps, ref):
+            np.testing.assert_array_equal(host_bits(s), r)
