@@ -13,14 +13,17 @@
 //     replay kernels then write nothing: a chain with a bad entry anywhere is
 //     not applied at all.
 //
-//   chain_merge_kernel  (DWS_CHAIN_TILE_MERGE) CTAs over contiguous ranges of
-//     tiles; per tile each thread owns 32 elements and each warp a share of
-//     the tile's entries (exactly the tile's, from the tile index), all
-//     loaded one tile ahead into registers with plain vector loads; every
-//     entry raises its element's tag in shared memory to (k + 1) << 16 |
-//     value with atomicMax (the latest delta wins whatever the thread order),
-//     then each thread merges its 32 elements and writes them back.  A tile
-//     no delta touches is neither read nor written.
+//   chain_merge_kernel  (DWS_CHAIN_TILE_MERGE) one persistent CTA per SM over
+//     a contiguous range of tiles.  A producer warp fills a 4-stage ring:
+//     per tile, one bulk copy of the snapshot tile and, per delta, bulk copies
+//     of exactly that tile's entries (the tile index gives their range), so
+//     the loads of the next tiles are in flight while 8 consumer warps merge
+//     the current one: every entry of every delta raises its element's tag
+//     to (k + 1) << 16 | value with atomicMax (the latest delta wins whatever
+//     the thread order), then one pass moves the tagged values into the
+//     tile.  The producer writes the merged tile back with one bulk store as
+//     soon as it is done.  A tile no delta touches is neither read nor
+//     written.
 //
 //   chain_scatter_kernel  (DWS_CHAIN_SCATTER) per window of 32 tiles the
 //     deltas are replayed from the last to the first, an element being
@@ -34,6 +37,8 @@
 
 namespace dws {
 namespace {
+
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
 
 // ---------------------------------------------------------------------------
 // Tile index and validation
@@ -143,15 +148,16 @@ __global__ void __launch_bounds__(kIdxThreads, 4) chain_index_kernel(IndexParams
         for (int q = 1; q < kIdxPerThread; ++q) viol |= !(x[q - 1] < x[q]);
         const bool ok = !viol && x[0] >= 0 && x[kIdxPerThread - 1] < nm;
         if (!ok) {
-            int pv = prev;  // rare: locate the first offending entry
+            // rare: the first offending entry (unrolled: x stays in registers)
+            unsigned int badm = 0;
+#pragma unroll
             for (int q = 0; q < kIdxPerThread; ++q) {
-                if (!(x[q] >= 0 && x[q] < nm && ((q == 0 && opens) || pv < x[q]))) {
-                    bad = true;
-                    bad_j = j0 + q;
-                    break;
-                }
-                pv = x[q];
+                const int pv = q == 0 ? prev : x[q - 1];
+                const bool e_ok = x[q] >= 0 && x[q] < nm && ((q == 0 && opens) || pv < x[q]);
+                badm |= e_ok ? 0u : (1u << q);
             }
+            bad = true;
+            bad_j = j0 + (badm ? __ffs(badm) - 1 : 0);
         }
         glast = ok ? ft + (x[kIdxPerThread - 1] >> kTileShift) : -2;
         if (p.write) {
@@ -331,25 +337,13 @@ __device__ __forceinline__ long long index_entry(const DeltaRef &d, const uint32
 }
 
 // ---------------------------------------------------------------------------
-// Tile merge (register streaming)
+// Tile merge
 // ---------------------------------------------------------------------------
-// Each CTA walks a contiguous range of tiles.  Per tile, thread t owns the
-// 32 elements [32 t, 32 t + 32) (four 16-byte vectors) and each warp a share
-// of the tile's entries, in work items of 32 entries of one delta (the tile
-// index gives every delta's range).  While tile i is merged, the loads of
-// tile i+1 -- its 32 elements per thread and its entries -- are in flight in
-// registers.  Merge: every entry raises its element's tag in shared memory to
-// (k + 1) << 16 | value (atomicMax: the latest delta wins whatever the thread
-// order); then each thread takes the tags of its elements, clears them, and
-// writes its 32 merged elements back with 16-byte stores.  A tile no delta
-// touches is neither read nor written; a tile whose elements cannot move as
-// whole 16-byte vectors (an unaligned tensor, a tensor's short last tile)
-// gets its tagged values stored one by one.
-constexpr int kMThreads = 256;
-constexpr int kMWarps = kMThreads / 32;
-constexpr int kMPer = kTileElems / kMThreads;  // 32 elements per thread
-constexpr int kMVec = kMPer / 8;               // 4 vectors of 8 elements
-constexpr int kMPre = 10;                      // entry items per warp held in registers
+constexpr int kMergeConsumerWarps = 8;
+constexpr int kMergeConsumers = 32 * kMergeConsumerWarps;
+constexpr int kMergeThreads = 32 + kMergeConsumers;
+constexpr int kStages = 4;
+constexpr int kStageEntries = 4096;  // entries staged per stage, all deltas together
 
 struct MergeParams {
     WsView ws;
@@ -360,113 +354,174 @@ struct MergeParams {
     DeltaRef d[kChainGroup];
 };
 
-struct MergeSmem {
-    uint32_t tag[kTileElems];
-    const int *idx[kChainGroup];
-    const uint16_t *val[kChainGroup];
-    long long cnt[kChainGroup];
-};
-
-// One tile as a warp sees it.  Lane k < K: delta k's first entry of the tile
-// (s), its entries (n) and the exclusive prefix of the items (c0, items of 32
-// entries of one delta, in delta order).
-struct TileView {
-    uint16_t *ptr;  // the tile's first element (null: untouched)
+// What the producer staged for one tile.
+struct StageMeta {
+    long long s[kChainGroup];  // first entry of the tile in delta k
+    int n[kChainGroup];        // entries of the tile in delta k
+    int ia[kChainGroup];       // staged indices: entries s + [ia, ib) at idx[io + ...] (ia may be < 0)
+    int ib[kChainGroup];
+    int io[kChainGroup];
+    int va[kChainGroup];       // staged values: entries s + [va, vb) at val[vo + ...]
+    int vb[kChainGroup];
+    int vo[kChainGroup];
+    int C[kChainGroup + 1];    // work items (32 entries of one delta): delta k's are [C[k], C[k+1])
+    uint16_t *ptr;  // tile start in the snapshot
     int local_start;
-    int count;      // elements
-    bool vec;       // whole 16-byte vectors: aligned pointer and a full tile
-    long long s;
-    int n;
-    int c0;
-    int items;      // the tile's items
+    int count;   // elements of the tile
+    int bulk;    // leading elements moved by bulk copies (multiple of 8)
+    int touched;
 };
 
-// This thread's loads of one tile, in flight: its 32 elements and its warp's
-// first kMPre items (item w + kMWarps * r is this warp's r-th): the entry's
-// index and its tag (k + 1) << 16 | value (0: no entry).
-struct TileLoads {
-    uint4 e[kMVec];
-    int ix[kMPre];
-    uint32_t tg[kMPre];
+struct MergeSmem {
+    uint32_t tag[kTileElems];  // (k + 1) << 16 | value of the latest delta k per element; 0: none
+    uint16_t tile[kStages][kTileElems];
+    int idx[kStages][kStageEntries];
+    uint16_t val[kStages][kStageEntries];
+    StageMeta meta[kStages];
+    unsigned long long full[kStages];  // producer -> consumers: tile staged
+    unsigned long long done[kStages];  // consumers -> producer: tile merged
+    int grp[kStages];                  // producer: store group of the stage's tile (-1: none)
+    long long cursor[kChainGroup];
+    int abort;
 };
 
-// The delta (lane) an item belongs to: items are in delta order.
-__device__ __forceinline__ int item_delta(int item, int c0, int n_items, int K) {
-    const int lane = threadIdx.x & 31;
-    const bool before = lane < K && c0 + n_items <= item;  // delta `lane` ends at or before item
-    return __popc(__ballot_sync(0xffffffffu, before));
+// Producer warp's view of the tensor that holds the current tile.
+struct TensorCursor {
+    int t;              // tensor
+    long long first;    // its first tile
+    long long next;     // first tile of the next tensor
+    long long numel;
+    uint16_t *ptr;
+};
+
+__device__ __forceinline__ void tensor_at(const MergeParams &p, int t, TensorCursor &c) {
+    c.t = t;
+    c.first = p.ws.first_tile[t];
+    c.next = p.ws.first_tile[t + 1];
+    c.numel = p.ws.numel[t];
+    c.ptr = p.snap_ptrs[t];
 }
 
-// Warp-wide: the view of tile i (tensor t, its first tile `first`, numel,
-// pointer), from the index rows of tiles i and i+1 (lane k: delta k).
-__device__ __forceinline__ void tile_view(const MergeParams &p, long long i, long long first, long long numel,
-                                          uint16_t *tptr, uint32_t row_i, uint32_t row_next, long long &cursor,
-                                          TileView &v) {
+// Producer warp: describe tile i and start its copies into stage st.  Lane k
+// (< K) owns delta k: its entries of the tile are [cursor, cursor + n) with
+// n the difference of two index rows (mod 2^32; a tile holds fewer).
+__device__ void merge_stage(const MergeParams &p, MergeSmem &sm, long long i, int st,
+                            const TensorCursor &tc, uint32_t row_next, long long &cursor,
+                            unsigned long long policy) {
     const int lane = threadIdx.x & 31;
-    const long long ls = (i - first) << kTileShift;
-    const long long rest = numel - ls;
-    v.local_start = static_cast<int>(ls);
-    v.count = static_cast<int>(rest < kTileElems ? (rest > 0 ? rest : 0) : kTileElems);
-    v.s = cursor;
-    v.n = lane < p.K ? static_cast<int>(row_next - row_i) : 0;
-    if (lane < p.K) cursor += v.n;
-    const int ni = (v.n + 31) >> 5;
-    int incl = ni;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int x = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += x;
+    StageMeta &m = sm.meta[st];
+    const long long ls = (i - tc.first) << kTileShift;
+    const long long rest = tc.numel - ls;
+    const int count = static_cast<int>(rest < kTileElems ? (rest > 0 ? rest : 0) : kTileElems);
+    const bool mine = lane < p.K;
+    int n = 0;
+    long long s = 0;
+    if (mine) {
+        s = cursor;
+        const uint32_t row_here = static_cast<uint32_t>(s);  // the row of tile i, as cursor's low bits
+        n = static_cast<int>(row_next - row_here);
+        cursor = s + n;
     }
-    v.c0 = incl - ni;
-    v.items = __shfl_sync(0xffffffffu, incl, 31);
-    const bool touched = v.items > 0 && v.count > 0 && tptr != nullptr &&
-                         (reinterpret_cast<uintptr_t>(tptr) & 1u) == 0;
-    v.ptr = touched ? tptr + ls : nullptr;
-    v.vec = touched && v.count == kTileElems && (reinterpret_cast<uintptr_t>(tptr) & 15u) == 0;
-}
-
-// Issues this thread's loads of tile v (elements when v.vec; the warp's first
-// kMPre items).
-__device__ __forceinline__ void tile_issue(const MergeParams &p, const MergeSmem &sm, const TileView &v,
-                                           TileLoads &L) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (v.vec) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(v.ptr + threadIdx.x * kMPer);
+    int total = n;
 #pragma unroll
-        for (int q = 0; q < kMVec; ++q) L.e[q] = ld_stream_v4(src + q);
+    for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+    const uintptr_t ua = reinterpret_cast<uintptr_t>(tc.ptr);
+    bool touched = total > 0 && count > 0;
+    if (touched && (tc.ptr == nullptr || (ua & 1u))) {
+        if (lane == 0) record_error(p.ws.hdr, DWS_ERR_INVALID, tc.t);
+        touched = false;
     }
-#pragma unroll
-    for (int r = 0; r < kMPre; ++r) {
-        const int item = warp + r * kMWarps;
-        L.ix[r] = 0;
-        L.tg[r] = 0u;
-        if (item < v.items) {  // uniform per warp
-            const int k = item_delta(item, v.c0, (v.n + 31) >> 5, p.K);
-            const int c0 = __shfl_sync(0xffffffffu, v.c0, k);
-            const int n = __shfl_sync(0xffffffffu, v.n, k);
-            const long long s = __shfl_sync(0xffffffffu, v.s, k);
-            const int el = ((item - c0) << 5) + lane;
-            const long long j = s + el;
-            if (el < n && j >= 0 && j < sm.cnt[k]) {  // (the index keeps it inside; the check is cheap)
-                L.ix[r] = __ldg(sm.idx[k] + j);
-                L.tg[r] = (static_cast<uint32_t>(k + 1) << 16) | __ldg(sm.val[k] + j);
-            }
+    const int bulk = (touched && (ua & 15u) == 0) ? (count & ~7) : 0;
+    // Entries: each delta's range widened to 16-byte boundaries (so that
+    // no entry of the tile has to come from global memory), kept inside the
+    // delta's arrays: only at the arrays' unaligned ends do a few entries
+    // stay outside it.  A prefix sum over the lanes places the ranges while
+    // there is room.
+    int ci = 0, cv = 0;
+    long long ia = 0, va = 0;  // absolute first staged entry
+    if (mine && touched && n > 0) {
+        const DeltaRef &dk = p.d[lane];
+        const uintptr_t lo_i = (reinterpret_cast<uintptr_t>(dk.indices) + 15) & ~uintptr_t(15);
+        const uintptr_t hi_i = reinterpret_cast<uintptr_t>(dk.indices + dk.count) & ~uintptr_t(15);
+        uintptr_t a = reinterpret_cast<uintptr_t>(dk.indices + s) & ~uintptr_t(15);
+        uintptr_t b = (reinterpret_cast<uintptr_t>(dk.indices + s + n) + 15) & ~uintptr_t(15);
+        if (a < lo_i) a = lo_i;
+        if (b > hi_i) b = hi_i;
+        if (b > a && ((a - reinterpret_cast<uintptr_t>(dk.indices)) & 3u) == 0) {
+            ci = static_cast<int>((b - a) >> 2);
+            ia = static_cast<long long>((a - reinterpret_cast<uintptr_t>(dk.indices)) >> 2);
+        }
+        const uintptr_t lo_v = (reinterpret_cast<uintptr_t>(dk.values) + 15) & ~uintptr_t(15);
+        const uintptr_t hi_v = reinterpret_cast<uintptr_t>(dk.values + dk.count) & ~uintptr_t(15);
+        uintptr_t c = reinterpret_cast<uintptr_t>(dk.values + s) & ~uintptr_t(15);
+        uintptr_t d = (reinterpret_cast<uintptr_t>(dk.values + s + n) + 15) & ~uintptr_t(15);
+        if (c < lo_v) c = lo_v;
+        if (d > hi_v) d = hi_v;
+        if (d > c && ((c - reinterpret_cast<uintptr_t>(dk.values)) & 1u) == 0) {
+            cv = static_cast<int>((d - c) >> 1);
+            va = static_cast<long long>((c - reinterpret_cast<uintptr_t>(dk.values)) >> 1);
         }
     }
+    int oi = ci, ov = cv;  // inclusive prefix over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, oi, o);
+        const int y = __shfl_up_sync(0xffffffffu, ov, o);
+        if (lane >= o) {
+            oi += x;
+            ov += y;
+        }
+    }
+    oi -= ci;  // exclusive
+    ov -= cv;
+    if (oi + ci > kStageEntries) ci = oi < kStageEntries ? ((kStageEntries - oi) & ~3) : 0;
+    if (ov + cv > kStageEntries) cv = ov < kStageEntries ? ((kStageEntries - ov) & ~7) : 0;
+    int fn = (n + 31) >> 5;  // inclusive prefix of the work items over the lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, fn, o);
+        if (lane >= o) fn += x;
+    }
+    if (lane < p.K) m.C[lane + 1] = fn;
+    if (lane == 0) m.C[0] = 0;
+    if (mine) {
+        m.s[lane] = s;
+        m.n[lane] = n;
+        // staged ranges relative to s (may start before it)
+        m.ia[lane] = static_cast<int>(ia - s);
+        m.ib[lane] = static_cast<int>(ia - s) + ci;
+        m.io[lane] = oi;
+        m.va[lane] = static_cast<int>(va - s);
+        m.vb[lane] = static_cast<int>(va - s) + cv;
+        m.vo[lane] = ov;
+    }
+    uint32_t bytes = static_cast<uint32_t>(ci) * 4u + static_cast<uint32_t>(cv) * 2u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+    if (lane == 0) {
+        m.ptr = touched ? tc.ptr + ls : nullptr;
+        m.local_start = static_cast<int>(ls);
+        m.count = count;
+        m.bulk = bulk;
+        m.touched = touched ? 1 : 0;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        bytes += static_cast<uint32_t>(bulk) * 2u;
+        mbar_arrive_expect_tx(&sm.full[st], bytes);  // releases the description above
+        if (bulk > 0)
+            bulk_load(sm.tile[st], tc.ptr + ls, static_cast<uint32_t>(bulk) * 2u, &sm.full[st], policy);
+    }
+    __syncwarp();
+    if (ci > 0)
+        bulk_load(&sm.idx[st][oi], p.d[lane].indices + ia, static_cast<uint32_t>(ci) * 4u,
+                  &sm.full[st], policy);
+    if (cv > 0)
+        bulk_load(&sm.val[st][ov], p.d[lane].values + va, static_cast<uint32_t>(cv) * 2u,
+                  &sm.full[st], policy);
 }
 
-// Tags one entry: the element at (index - local_start) of the tile gets the
-// entry's tag unless a later delta's is there.
-__device__ __forceinline__ void tag_entry(MergeSmem &sm, const MergeParams &p, const TileView &v, int index,
-                                          uint32_t tag) {
-    const int pos = index - v.local_start;  // in [0, count): the index pass's ranges
-    if (static_cast<unsigned>(pos) < static_cast<unsigned>(v.count))
-        atomicMax(&sm.tag[pos], tag);
-    else
-        record_error(p.ws.hdr, DWS_ERR_WORKSPACE, pos);  // never expected
-}
-
-__global__ void __launch_bounds__(kMThreads, 2) chain_merge_kernel(MergeParams p) {
+__global__ void __launch_bounds__(kMergeThreads, 1) chain_merge_kernel(MergeParams p) {
     extern __shared__ __align__(128) unsigned char merge_smem_raw[];
     MergeSmem &sm = *reinterpret_cast<MergeSmem *>(merge_smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -477,111 +532,182 @@ __global__ void __launch_bounds__(kMThreads, 2) chain_merge_kernel(MergeParams p
     long long te = tb + p.tiles_per_cta;
     if (te > p.ws.num_tiles) te = p.ws.num_tiles;
     if (tb >= te) return;
+    const long long ntl = te - tb;
 
-    for (int e = tid; e < kTileElems; e += kMThreads) sm.tag[e] = 0u;
-    if (tid < p.K) {
-        sm.idx[tid] = p.d[tid].indices;
-        sm.val[tid] = p.d[tid].values;
-        sm.cnt[tid] = p.d[tid].count;
-    }
-    // every warp keeps its own copy of the walk: tensor, cursors, index rows
-    int t = p.ws.tile_tensor[tb];
-    long long first = p.ws.first_tile[t], next = p.ws.first_tile[t + 1], numel = p.ws.numel[t];
-    uint16_t *tptr = p.snap_ptrs[t];
-    long long cursor = 0;  // lane k: delta k's first entry of the next tile to view
-    // lane k: index rows of tiles i+1 and i+2 (row i+3 is loaded one tile ahead)
-    uint32_t row0 = 0, row1 = 0, row2 = 0;
-    const long long nrows = p.ws.num_tiles;
-    if (lane < p.K) {
-        cursor = index_entry(p.d[lane], p.index, tb, lane, t);
-        row0 = p.index[tb * kChainGroup + lane];
-        row1 = p.index[(tb + 1) * kChainGroup + lane];
-        if (tb + 2 <= nrows) row2 = p.index[(tb + 2) * kChainGroup + lane];
+    if (tid == 0) {
+        sm.abort = 0;
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.done[s], 1);
+        }
+        mbar_fence_init();
     }
     __syncthreads();
 
-    TileView va, vb;
-    TileLoads la, lb;
-    tile_view(p, tb, first, numel, tptr, row0, row1, cursor, va);
-    tile_issue(p, sm, va, la);
+    if (warp == 0) {
+        // ---- producer warp ---------------------------------------------------
+        // Stages tile li once tile li - kStages is merged and its store has
+        // read the stage; stores are issued as soon as a tile is merged.
+        const unsigned long long policy = l2_evict_first_policy();
+        TensorCursor tc;
+        tensor_at(p, p.ws.tile_tensor[tb], tc);
+        long long cursor = 0;  // lane k: delta k's first entry of the next tile to stage
+        uint32_t rq0 = 0, rq1 = 0, rq2 = 0, rq3 = 0;  // index rows of tiles i+1 .. i+4
+        const long long nrows = p.ws.num_tiles;      // last row
+        if (lane < p.K) {
+            cursor = index_entry(p.d[lane], p.index, tb, lane, tc.t);
+            rq0 = p.index[(tb + 1) * kChainGroup + lane];
+            if (tb + 2 <= nrows) rq1 = p.index[(tb + 2) * kChainGroup + lane];
+            if (tb + 3 <= nrows) rq2 = p.index[(tb + 3) * kChainGroup + lane];
+            if (tb + 4 <= nrows) rq3 = p.index[(tb + 4) * kChainGroup + lane];
+        }
+        long long taken = 0;  // tiles whose completion the producer has taken
+        int committed = 0;    // store groups committed
+        // take tile c's completion: write it back
+        auto take = [&](long long c) {
+            const int cs = static_cast<int>(c % kStages);
+            const StageMeta &m = sm.meta[cs];
+            if (m.touched && m.bulk > 0) {
+                bulk_store(m.ptr, sm.tile[cs], static_cast<uint32_t>(m.bulk) * 2u);
+                bulk_commit();
+                sm.grp[cs] = committed++;
+            } else {
+                sm.grp[cs] = -1;
+            }
+        };
+        bool ok = true;
+        for (long long li = 0; li < ntl; ++li) {
+            const long long i = tb + li;
+            const int st = static_cast<int>(li % kStages);
+            while (i >= tc.next) tensor_at(p, tc.t + 1, tc);  // uniform
+            if (lane == 0) {
+                while (taken < li && mbar_try_wait(&sm.done[taken % kStages],
+                                                   static_cast<uint32_t>((taken / kStages) & 1)))
+                    take(taken++);
+                while (ok && taken <= li - kStages) {
+                    ok = mbar_wait_sleepy(&sm.done[taken % kStages], static_cast<uint32_t>((taken / kStages) & 1),
+                                          kWaitLimitNs);
+                    if (ok) take(taken++);
+                }
+                if (ok && li >= kStages && sm.grp[st] >= 0) bulk_wait_read_n(committed - 1 - sm.grp[st]);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            __syncwarp();
+            merge_stage(p, sm, i, st, tc, rq0, cursor, policy);
+            rq0 = rq1;
+            rq1 = rq2;
+            rq2 = rq3;
+            rq3 = (lane < p.K && i + 5 <= nrows) ? p.index[(i + 5) * kChainGroup + lane] : 0u;
+        }
+        if (lane == 0) {
+            // write back the last tiles
+            while (ok && taken < ntl) {
+                ok = mbar_wait_sleepy(&sm.done[taken % kStages], static_cast<uint32_t>((taken / kStages) & 1),
+                                      kWaitLimitNs);
+                if (ok) take(taken++);
+            }
+            if (!ok) {
+                atomicExch(&sm.abort, 1);
+                record_error(p.ws.hdr, DWS_ERR_TIMEOUT, tb);
+            }
+            bulk_wait_all();
+        }
+        return;
+    }
 
-    // One tile: view and start loading tile i + 1 into (nv, nl), then merge
-    // tile i from (cv, cl).  Called with the two buffers swapped on
-    // alternate tiles, so that no register holding a load in flight is
-    // copied (a copy would wait for the load).
-    auto step = [&](long long i, const TileView &cv, const TileLoads &cl, TileView &nv, TileLoads &nl) {
-        nv.items = 0;
-        nv.ptr = nullptr;
-        if (i + 1 < te) {
-            while (i + 1 >= next) {  // uniform: the next tensor
-                ++t;
-                first = p.ws.first_tile[t];
-                next = p.ws.first_tile[t + 1];
-                numel = p.ws.numel[t];
-                tptr = p.snap_ptrs[t];
+    // ---- consumers (8 warps) ------------------------------------------------
+    // Per tile: the entries of all deltas as one list; each entry raises its
+    // element's tag to (k + 1) << 16 | value with atomicMax, so the latest
+    // delta wins whatever the order the threads run in; then one pass moves
+    // the tagged values into the tile (or straight to global memory past the
+    // bulk-copied part) and clears the tags.
+    const int ct = tid - 32;  // 0 .. kMergeConsumers - 1
+    for (int e = ct; e < kTileElems; e += kMergeConsumers) sm.tag[e] = 0u;
+    named_bar(1, kMergeConsumers);
+    for (long long li = 0; li < ntl; ++li) {
+        const int st = static_cast<int>(li % kStages);
+        const bool got = mbar_wait_sleepy(&sm.full[st], static_cast<uint32_t>((li / kStages) & 1), kWaitLimitNs);
+        if (!named_bar_and(1, kMergeConsumers, got && ld_acquire_cta(&sm.abort) == 0)) {
+            if (ct == 0) record_error(p.ws.hdr, DWS_ERR_TIMEOUT, tb + li);
+            return;  // the producer's own waits are bounded too
+        }
+        const StageMeta &m = sm.meta[st];
+        if (m.touched) {
+            const int ls = m.local_start;
+            const int count = m.count;
+            const int items = m.C[p.K];
+            const int cw = ct >> 5;
+            int k = -1, c_lo = 0, c_hi = 0, n = 0, ia = 0, ib = 0, io = 0, va = 0, vb = 0, vo = 0;
+            bool staged = false;
+            const int *gi = nullptr;
+            const uint16_t *gv = nullptr;
+            for (int it = cw; it < items; it += kMergeConsumerWarps) {
+                while (it >= c_hi) {  // uniform per warp: items only move forward
+                    ++k;
+                    c_lo = m.C[k];
+                    c_hi = m.C[k + 1];
+                    n = m.n[k];
+                    ia = m.ia[k]; ib = m.ib[k]; io = m.io[k];
+                    va = m.va[k]; vb = m.vb[k]; vo = m.vo[k];
+                    staged = ia <= 0 && ib >= n && va <= 0 && vb >= n;
+                    gi = p.d[k].indices + m.s[k];
+                    gv = p.d[k].values + m.s[k];
+                }
+                const int el = ((it - c_lo) << 5) + lane;
+                if (el >= n) continue;
+                int ix;
+                uint32_t vx;
+                if (staged) {
+                    ix = sm.idx[st][io + el - ia];
+                    vx = sm.val[st][vo + el - va];
+                } else {
+                    // outside the staged range: from global memory, inside the
+                    // delta's arrays whatever the index says
+                    const bool in_arr = m.s[k] + el >= 0 && m.s[k] + el < p.d[k].count;
+                    ix = (el >= ia && el < ib) ? sm.idx[st][io + el - ia] : (in_arr ? __ldg(gi + el) : -1);
+                    vx = (el >= va && el < vb) ? sm.val[st][vo + el - va] : (in_arr ? __ldg(gv + el) : 0u);
+                }
+                const int pos = ix - ls;  // in [0, count): the index pass's ranges
+                if (static_cast<unsigned>(pos) < static_cast<unsigned>(count))
+                    atomicMax(&sm.tag[pos], (static_cast<uint32_t>(k + 1) << 16) | vx);
+                else
+                    record_error(p.ws.hdr, DWS_ERR_WORKSPACE, m.s[k] + el);  // never expected
             }
-            const uint32_t row3 = (lane < p.K && i + 3 <= nrows) ? p.index[(i + 3) * kChainGroup + lane] : 0u;
-            tile_view(p, i + 1, first, numel, tptr, row1, row2, cursor, nv);
-            tile_issue(p, sm, nv, nl);
-            row1 = row2;
-            row2 = row3;
-        }
-        if (cv.ptr == nullptr) return;  // uniform: untouched
-        // tag tile i's entries: the items held, then the rest
+            named_bar(1, kMergeConsumers);
+            const int bulk = m.bulk;
+            uint16_t *tile = sm.tile[st];
 #pragma unroll
-        for (int r = 0; r < kMPre; ++r)
-            if (cl.tg[r] != 0u) tag_entry(sm, p, cv, cl.ix[r], cl.tg[r]);
-        for (int item = warp + kMPre * kMWarps; item < cv.items; item += kMWarps) {
-            const int k = item_delta(item, cv.c0, (cv.n + 31) >> 5, p.K);
-            const int c0 = __shfl_sync(0xffffffffu, cv.c0, k);
-            const int n = __shfl_sync(0xffffffffu, cv.n, k);
-            const long long s = __shfl_sync(0xffffffffu, cv.s, k);
-            const int el = ((item - c0) << 5) + lane;
-            const long long j = s + el;
-            if (el < n && j >= 0 && j < sm.cnt[k])
-                tag_entry(sm, p, cv, __ldg(sm.idx[k] + j),
-                          (static_cast<uint32_t>(k + 1) << 16) | __ldg(sm.val[k] + j));
-        }
-        __syncthreads();
-        // merge this thread's 32 elements, clear their tags
-        const int e0 = tid * kMPer;
-        if (cv.vec) {
-            uint4 *dst = reinterpret_cast<uint4 *>(cv.ptr + e0);
+            for (int r = 0; r < kTileElems / (4 * kMergeConsumers); ++r) {
+                const int e0 = 4 * ct + r * 4 * kMergeConsumers;
+                if (e0 >= count) break;
+                const uint4 tg = *reinterpret_cast<const uint4 *>(&sm.tag[e0]);
+                if ((tg.x | tg.y | tg.z | tg.w) == 0u) continue;
+                *reinterpret_cast<uint4 *>(&sm.tag[e0]) = make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t t4[4] = {tg.x, tg.y, tg.z, tg.w};
+                if (e0 + 4 <= bulk) {
+                    uint2 w = *reinterpret_cast<const uint2 *>(&tile[e0]);
+                    uint32_t lo = w.x, hi = w.y;
+                    if (t4[0]) lo = (lo & 0xffff0000u) | (t4[0] & 0xffffu);
+                    if (t4[1]) lo = (lo & 0x0000ffffu) | (t4[1] << 16);
+                    if (t4[2]) hi = (hi & 0xffff0000u) | (t4[2] & 0xffffu);
+                    if (t4[3]) hi = (hi & 0x0000ffffu) | (t4[3] << 16);
+                    *reinterpret_cast<uint2 *>(&tile[e0]) = make_uint2(lo, hi);
+                } else {
 #pragma unroll
-            for (int q = 0; q < kMVec; ++q) {
-                uint32_t w[4] = {cl.e[q].x, cl.e[q].y, cl.e[q].z, cl.e[q].w};
-                const uint4 ta = *reinterpret_cast<const uint4 *>(&sm.tag[e0 + 8 * q]);
-                const uint4 tc = *reinterpret_cast<const uint4 *>(&sm.tag[e0 + 8 * q + 4]);
-                const uint32_t tg[8] = {ta.x, ta.y, ta.z, ta.w, tc.x, tc.y, tc.z, tc.w};
-                if ((ta.x | ta.y | ta.z | ta.w | tc.x | tc.y | tc.z | tc.w) != 0u) {
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) {
-                        if (tg[h]) {
-                            const uint32_t sh = (h & 1) * 16;
-                            w[h >> 1] = (w[h >> 1] & ~(0xffffu << sh)) | ((tg[h] & 0xffffu) << sh);
-                        }
+                    for (int q = 0; q < 4; ++q) {
+                        if (!t4[q] || e0 + q >= count) continue;
+                        if (e0 + q < bulk) tile[e0 + q] = static_cast<uint16_t>(t4[q] & 0xffffu);
+                        else m.ptr[e0 + q] = static_cast<uint16_t>(t4[q] & 0xffffu);
                     }
-                    *reinterpret_cast<uint4 *>(&sm.tag[e0 + 8 * q]) = make_uint4(0u, 0u, 0u, 0u);
-                    *reinterpret_cast<uint4 *>(&sm.tag[e0 + 8 * q + 4]) = make_uint4(0u, 0u, 0u, 0u);
-                }
-                st_stream_v4(dst + q, make_uint4(w[0], w[1], w[2], w[3]));
-            }
-        } else {
-#pragma unroll 4
-            for (int h = 0; h < kMPer; ++h) {
-                const int e = e0 + h;
-                const uint32_t tg = sm.tag[e];
-                if (tg) {
-                    sm.tag[e] = 0u;
-                    if (e < cv.count) cv.ptr[e] = static_cast<uint16_t>(tg & 0xffffu);
                 }
             }
+            if (bulk > 0) fence_proxy_async_smem();  // the bulk store reads the tile
+            named_bar(1, kMergeConsumers);
         }
-        __syncthreads();  // tags clear before the next tile's entries
-    };
-    for (long long i = tb; i < te; i += 2) {
-        step(i, va, la, vb, lb);
-        if (i + 1 < te) step(i + 1, vb, lb, va, la);
+        if (ct == 0) mbar_arrive(&sm.done[st]);
+    }
+    if (ct == 0) {
     }
 }
 
@@ -791,7 +917,7 @@ cudaError_t chain_set_attributes() {
 }
 
 cudaError_t chain_occupancy(int *ctas_per_sm) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, chain_merge_kernel, kMThreads,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, chain_merge_kernel, kMergeThreads,
                                                          sizeof(MergeSmem));
 }
 
@@ -854,7 +980,7 @@ cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs, con
             if (grid < 1) grid = 1;
             mp.tiles_per_cta = (ws.num_tiles + grid - 1) / grid;
             grid = (ws.num_tiles + mp.tiles_per_cta - 1) / mp.tiles_per_cta;
-            chain_merge_kernel<<<static_cast<unsigned int>(grid), kMThreads, sizeof(MergeSmem), s>>>(mp);
+            chain_merge_kernel<<<static_cast<unsigned int>(grid), kMergeThreads, sizeof(MergeSmem), s>>>(mp);
         } else {
             ScatParams sp;
             sp.ws = ws;
