@@ -32,6 +32,7 @@ import contextlib
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -63,8 +64,12 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--rows-reps", type=int, default=5)
+    ap.add_argument("--xor-layers", type=int, default=40,
+                    help="layers of 0.8 GB in the XOR rows (fewer: a small case for profiling)")
+    ap.add_argument("--stress-tensors", type=int, default=12000,
+                    help="tensors of the stress set (fewer: a small case for profiling)")
     ap.add_argument("--rows-only", default=None,
-                    help="comma list of qwen_chain, xor, stress_chain: time only these rows "
+                    help="comma list of single, qwen_chain, xor, stress_chain: time only these rows "
                          "(no Llama-3-8B step; a small case for profiling)")
     return ap.parse_args()
 
@@ -386,23 +391,94 @@ def time_reps(fn, reps, warm=1):
     return statistics.median(ts), min(ts)
 
 
-def row(name, ms, alg_bytes, weight_bytes, peak, extra=None):
+def touched_sectors(offsets, indices):
+    """Distinct 32-byte sectors (16 bf16 elements) a delta writes, counted
+    on the device; every tensor starts on a 256-byte boundary in the bench's
+    packed buffers, so sector k of a tensor is its elements [16k, 16k+16)."""
+    import torch
+    T = offsets.numel() - 1
+    counts = offsets[1:] - offsets[:-1]
+    if int(offsets[-1].item()) == 0:
+        return 0
+    tid = torch.repeat_interleave(torch.arange(T, device=offsets.device, dtype=torch.int64), counts)
+    key = (tid << 40) | (indices.to(torch.int64) >> 4)  # ascending: tensor order, then index
+    n = 1 + int((key[1:] != key[:-1]).sum().item())
+    del tid, key
+    return n
+
+
+def sector_model(nnz, sectors, ms, peak):
+    """The apply's DRAM traffic model: 6 bytes read per entry, and every
+    touched 32-byte sector read and written back whole by L2 (HBM has no
+    byte-masked writes): 6 nnz + 64 S bytes."""
+    b = 6 * nnz + 64 * sectors
+    return {"sectors": sectors, "sector_model_bytes": b,
+            "sector_model_GBps": round(b / ms / 1e6, 1), "sector_model_frac": round(b / ms / 1e6 / peak, 4)}
+
+
+def row(name, ms, alg_bytes, weight_bytes, peak, extra=None, elems=None):
+    """A bench row: time, algorithmic and weight GB/s, the fraction of the HBM
+    peak and elements per second (elems: the row's elements, default the bf16
+    elements of weight_bytes)."""
+    elems = weight_bytes // 2 if elems is None else elems
     d = {"ms": round(ms, 4), "alg_GBps": round(alg_bytes / ms / 1e6, 1),
          "weight_GBps": round(weight_bytes / ms / 1e6, 1),
+         "elems_per_s": round(elems / ms * 1e3, 1),
          "hbm_frac": round(alg_bytes / ms / 1e6 / peak, 4)}
     if extra:
         d.update(extra)
     return name, d
 
 
-ROW_GROUPS = ("qwen_chain", "xor", "stress_chain")
+ROW_GROUPS = ("single", "qwen_chain", "xor", "stress_chain")
 # (dws_apply_chain_ex mode, row-name suffix); 0 = the library's default
 CHAIN_MODES = ((0, ""), (1, "_tile_merge"), (2, "_scatter"))
+
+
+def rows_single(args, dev, peak):
+    """Workload 1 (one 1024x1024 bf16 tensor, one step at lr 3e-6): latency of
+    encode, apply, XOR encode and XOR apply, median of 50 launches.  4 MB in
+    all: it lives in L2, so these rows measure latency, not HBM bandwidth."""
+    import torch
+
+    import sparse_bf16_delta_b200 as dws
+    import workloads as W
+    old, new = W.single(dev)
+    a, b = old.tensors[0], new.tensors[0]
+    N = a.numel()
+    plan = dws.DeltaPlan.for_tensors([a])
+    ot, nt = dws.ptr_table([a]), dws.ptr_table([b])
+    d = plan.encode_exact(ot, nt)
+    nnz = d.nnz()
+    snap = a.clone()
+    st = dws.ptr_table([snap])
+    mask = torch.empty(2 * N, dtype=torch.uint8, device=dev)
+    buf = a.clone()
+    reps = max(50, args.rows_reps)
+    ms_e, mn_e = time_reps(lambda: plan.encode_into(ot, nt, d.offsets, d.indices, d.values), reps, warm=5)
+    ms_a, mn_a = time_reps(lambda: plan.apply(st, d), reps, warm=5)
+    ok = bool(torch.equal(snap, b)) and plan.status()[0] == dws.DWS_OK
+    ms_x, mn_x = time_reps(lambda: dws.xor_encode(a, b, mask), reps, warm=5)
+    ms_y, mn_y = time_reps(lambda: (dws.xor_apply(buf, mask), dws.xor_apply(buf, mask)), reps, warm=5)
+    ok_x = bool(torch.equal(buf, a))
+    lat = {"latency_row": True, "l2_resident": True, "reps": reps}
+    out = {}
+    out.update([row("encode_single_1024x1024", ms_e, 4 * N + 6 * nnz, 2 * N, peak,
+                    {**lat, "min_ms": round(mn_e, 4), "nnz": nnz})])
+    out.update([row("apply_single_1024x1024", ms_a, 8 * nnz, 2 * N, peak,
+                    {**lat, "min_ms": round(mn_a, 4), "exact": ok})])
+    out.update([row("xor_encode_single_1024x1024", ms_x, 6 * N, 2 * N, peak,
+                    {**lat, "min_ms": round(mn_x, 4)}, elems=2 * N)])
+    out.update([row("xor_apply_single_1024x1024", ms_y / 2, 6 * N, 2 * N, peak,
+                    {**lat, "min_ms": round(mn_y / 2, 4), "exact": ok_x}, elems=2 * N)])
+    return out
 
 
 def run_rows(args, dev, peak, groups=ROW_GROUPS):
     """The other hot-path rows, each on its own workload, timed with events."""
     out = {}
+    if "single" in groups:
+        out.update(rows_single(args, dev, peak))
     if "qwen_chain" in groups:
         out.update(rows_qwen_chain(args, dev, peak))
     if "xor" in groups:
@@ -457,6 +533,7 @@ def rows_qwen_chain(args, dev, peak):
         out.update([row("apply_chain_qwen3_0p6b_k10" + suffix, ms, 4 * N + 6 * tot, 2 * N, peak,
                         {"min_ms": round(mn, 4), "nnz_total": tot, "exact": ok})])
         del snap_flat, snap, st
+    out.update(merge_shards_row(args, dev, peak, plan, shapes, deltas[0]))
     mean_enc = statistics.mean(enc_ms)
     out.update([row("encode_qwen3_0p6b", mean_enc, 4 * N + 6 * tot / 10, 2 * N, peak,
                     {"nnz_mean": tot // 10, "sparsity_mean": round(1 - tot / 10 / N, 5)})])
@@ -464,6 +541,60 @@ def rows_qwen_chain(args, dev, peak):
     gc.collect()
     torch.cuda.empty_cache()
     log(f"rows: qwen chain done in {time.time() - t0:.1f}s")
+    return out
+
+
+def merge_shards_row(args, dev, peak, plan, shapes, d, R=8):
+    """Rank 0's merge of sharded deltas (dws_merge_shards): step 1 of the
+    Qwen3-0.6B chain split among R simulated ranks as FSDP Shard(0) would
+    (rank r holds rows [r c, (r+1) c) of every parameter, c = ceil(rows / R)),
+    each rank's delta in global int64 positions, padded and stacked as the
+    gather leaves them on rank 0; then merged back.  Reads and writes 10
+    bytes per entry."""
+    import torch
+
+    import sparse_bf16_delta_b200 as dws
+    T = len(shapes)
+    counts = d.offsets[1:] - d.offsets[:-1]
+    tid = torch.repeat_interleave(torch.arange(T, device=dev), counts)
+    rows = torch.tensor([sh[0] for _, sh in shapes], dtype=torch.int64, device=dev)
+    numel = torch.tensor([math.prod(sh) for _, sh in shapes], dtype=torch.int64, device=dev)
+    rowlen = numel // rows
+    chunk = (rows + R - 1) // R * rowlen
+    gidx = d.indices.to(torch.int64)
+    rank = torch.clamp(gidx // chunk[tid], max=R - 1)
+    per = []
+    for r in range(R):
+        m = rank == r
+        c = torch.bincount(tid[m], minlength=T)
+        o = torch.zeros(T + 1, dtype=torch.int64, device=dev)
+        o[1:] = torch.cumsum(c, 0)
+        per.append((o, gidx[m], d.values[m]))
+    stride = max(int(x[1].numel()) for x in per)
+    ro = torch.stack([x[0] for x in per])
+    ri = torch.zeros(R, stride, dtype=torch.int64, device=dev)
+    rv = torch.zeros(R, stride, dtype=torch.int16, device=dev)
+    for r, (_, i, v) in enumerate(per):
+        ri[r, :i.numel()] = i
+        rv[r, :v.numel()] = v
+    nnz = int(gidx.numel())
+    offs = torch.empty(T + 1, dtype=torch.int64, device=dev)
+    oidx = torch.empty(nnz, dtype=torch.int64, device=dev)
+    oval = torch.empty(nnz, dtype=torch.int16, device=dev)
+    cs = torch.cuda.current_stream().cuda_stream
+
+    def merge():
+        dws.dws_merge_shards(plan.handle, R, ro.data_ptr(), ri.data_ptr(), rv.data_ptr(), stride,
+                             offs.data_ptr(), oidx.data_ptr(), oval.data_ptr(), nnz,
+                             plan.workspace.data_ptr(), plan.workspace_bytes, cs)
+
+    ms, mn = time_reps(merge, args.rows_reps)
+    ok = (plan.status()[0] == dws.DWS_OK and torch.equal(offs, d.offsets) and torch.equal(oidx, gidx)
+          and torch.equal(oval, d.values))
+    out = [row(f"merge_shards_qwen3_0p6b_{R}ranks", ms, 20 * nnz + 8 * (T + 1) * (R + 1), 0, peak,
+               {"min_ms": round(mn, 4), "entries": nnz, "entries_per_s": round(nnz / ms * 1e3, 1),
+                "exact": ok}, elems=nnz)]
+    del ro, ri, rv, offs, oidx, oval, per
     return out
 
 
@@ -477,7 +608,8 @@ def rows_xor(args, dev, peak):
     import workloads as W
     out = {}
     t0 = time.time()
-    L, B = 40, 800_000_000
+    L, B = args.xor_layers, 800_000_000
+    tag = f"{L}x0.8GB"
     olds, news, masks = [], [], []
     for l in range(L):
         o, n, _ = W.xor_layer(l, dev, nbytes=B)
@@ -492,8 +624,8 @@ def rows_xor(args, dev, peak):
 
     ms, mn = time_reps(xor_enc, args.rows_reps)
     ok = all(int(torch.count_nonzero(masks[l])) == 680_000 for l in (0, L - 1))
-    out.update([row("xor_encode_nvfp4_40x0.8GB", ms, 3 * L * B, L * B, peak,
-                    {"min_ms": round(mn, 4), "launches": L, "exact_flip_count": ok})])
+    out.update([row("xor_encode_nvfp4_" + tag, ms, 3 * L * B, L * B, peak,
+                    {"min_ms": round(mn, 4), "launches": L, "exact_flip_count": ok}, elems=L * B)])
     # apply twice per rep so the buffers end where they started
     bufs = olds
 
@@ -504,8 +636,8 @@ def rows_xor(args, dev, peak):
             dws.xor_apply(bufs[l], masks[l])
 
     ms2, mn2 = time_reps(xor_app2, args.rows_reps)
-    out.update([row("xor_apply_nvfp4_40x0.8GB", ms2 / 2, 3 * L * B, L * B, peak,
-                    {"min_ms": round(mn2 / 2, 4)})])
+    out.update([row("xor_apply_nvfp4_" + tag, ms2 / 2, 3 * L * B, L * B, peak,
+                    {"min_ms": round(mn2 / 2, 4)}, elems=L * B)])
     # double-buffered layer pipeline, masks staged D2D (stand-in for the DE)
     staging = [torch.empty(B, dtype=torch.uint8, device=dev) for _ in range(2)]
     cs = torch.cuda.Stream()
@@ -521,12 +653,12 @@ def rows_xor(args, dev, peak):
     ok = torch.equal(bufs[0], news[0]) and torch.equal(bufs[L - 1], news[L - 1])
     dws.xor_apply(bufs[0], masks[0])
     dws.xor_apply(bufs[L - 1], masks[L - 1])
-    out.update([row("xor_apply_layers_double_buffered_40x0.8GB", msp / 2, 5 * L * B, L * B, peak,
+    out.update([row("xor_apply_layers_double_buffered_" + tag, msp / 2, 5 * L * B, L * B, peak,
                     {"min_ms": round(mnp / 2, 4), "staging": "2 x 0.8 GB, D2D copy stream",
-                     "exact": ok})])
+                     "exact": ok}, elems=L * B)])
     # the same pipeline with the masks in pinned host memory (the host link
     # bounds it): 4 layers, against a plain pinned H2D copy of one layer
-    LH = 4
+    LH = min(4, L)
     hmasks = [torch.empty(B, dtype=torch.uint8, pin_memory=True) for _ in range(LH)]
     for l in range(LH):
         hmasks[l].copy_(masks[l])
@@ -542,7 +674,7 @@ def rows_xor(args, dev, peak):
     ok_h = torch.equal(bufs[0], news[0])
     dws.xor_apply(bufs[0], masks[0])
     link = LH * B / (msh / 2) / 1e6
-    out["xor_apply_layers_pinned_host_4x0.8GB"] = {
+    out[f"xor_apply_layers_pinned_host_{LH}x0.8GB"] = {
         "ms": round(msh / 2, 3), "min_ms": round(mnh / 2, 3), "link_GBps": round(link, 1),
         "h2d_copy_GBps": round(B / ms_h2d / 1e6, 1), "link_frac": round(link / (B / ms_h2d / 1e6), 4),
         "bound": "host link (plain pinned H2D copy of 0.8 GB timed in the same run)", "exact": ok_h}
@@ -557,14 +689,16 @@ def rows_xor(args, dev, peak):
     snnz = sd.nnz()
     ms_e, mn_e = time_reps(lambda: splan.encode_into(sot, snt, sd.offsets, sd.indices, sd.values),
                            args.rows_reps)
-    out.update([row("encode_sparse_nvfp4_40x0.8GB", ms_e, 2 * L * B + 6 * snnz, L * B, peak,
-                    {"min_ms": round(mn_e, 4), "nnz": snnz, "delta_bytes": 6 * snnz + 8 * (L + 1)})])
+    out.update([row("encode_sparse_nvfp4_" + tag, ms_e, 2 * L * B + 6 * snnz, L * B, peak,
+                    {"min_ms": round(mn_e, 4), "nnz": snnz, "delta_bytes": 6 * snnz + 8 * (L + 1)},
+                    elems=L * B)])
     sst = dws.ptr_table(ow)
     ms_a, mn_a = time_reps(lambda: splan.apply(sst, sd), args.rows_reps)
     splan.raise_on_error("sparse xor apply")
     ok = all(torch.equal(olds[l], news[l]) for l in (0, L - 1))
-    out.update([row("apply_sparse_nvfp4_40x0.8GB", ms_a, 8 * snnz, L * B, peak,
-                    {"min_ms": round(mn_a, 4), "exact": ok})])
+    out.update([row("apply_sparse_nvfp4_" + tag, ms_a, 8 * snnz, L * B, peak,
+                    {"min_ms": round(mn_a, 4), "exact": ok,
+                     "entries_per_s": round(snnz / ms_a * 1e3, 1)}, elems=L * B)])
     # that delta arriving from pinned host memory: H2D of its 6 bytes per
     # entry, then the apply (the dense masks would move all 32 GB)
     hd = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in
@@ -582,7 +716,7 @@ def rows_xor(args, dev, peak):
     ms_ha, mn_ha = time_reps(host_apply, args.rows_reps)
     splan.raise_on_error("sparse xor apply from host")
     hbytes = sum(h.numel() * h.element_size() for h in hd)
-    out["apply_sparse_from_pinned_host_nvfp4_40x0.8GB"] = {
+    out["apply_sparse_from_pinned_host_nvfp4_" + tag] = {
         "ms": round(ms_ha, 3), "min_ms": round(mn_ha, 3), "h2d_bytes": hbytes,
         "link_GBps": round(hbytes / ms_ha / 1e6, 1),
         "exact": all(torch.equal(olds[l], news[l]) for l in (0, L - 1))}
@@ -606,8 +740,9 @@ def rows_stress_chain(args, dev, peak):
     out = {}
     t0 = time.time()
     s = W.SEEDS["stress"]
-    sizes = W.stress_sizes()
-    clustered = W.stress_clustered()
+    sizes = W.stress_sizes(count=args.stress_tensors)
+    clustered = W.stress_clustered(count=args.stress_tensors)
+    stag = f"{args.stress_tensors}t"
     anchor_flat, anchor = W.pack_flat(sizes, lambda t, n: W.init_tensor(n, W.weight_seed(s, t), dev, 0.02), dev)
     plan = dws.DeltaPlan.for_tensors(anchor)
     prev_flat, prev = W.pack_flat(sizes, lambda t, n: anchor[t], dev)
@@ -637,10 +772,10 @@ def rows_stress_chain(args, dev, peak):
         ms, mn = time_reps(lambda: plan.apply_chain(st, deltas, mode=mode), args.rows_reps)
         plan.raise_on_error("stress chain")
         ok = torch.equal(snap_flat, prev_flat) and nnzs == exp_nnz
-        out.update([row("apply_chain_stress_12000t_k10" + suffix, ms, 4 * N + 6 * tot, 2 * N, peak,
+        out.update([row("apply_chain_stress_" + stag + "_k10" + suffix, ms, 4 * N + 6 * tot, 2 * N, peak,
                         {"min_ms": round(mn, 4), "elements": N, "nnz_total": tot, "exact": ok})])
         del snap_flat, snap, st
-    out.update([row("encode_stress_12000t", statistics.mean(enc_ms), 4 * N + 6 * tot / 10, 2 * N, peak,
+    out.update([row("encode_stress_" + stag, statistics.mean(enc_ms), 4 * N + 6 * tot / 10, 2 * N, peak,
                     {"nnz_mean": tot // 10})])
     del deltas, anchor_flat, prev_flat, cur_flat, anchor, prev, cur, plan
     gc.collect()
@@ -828,6 +963,7 @@ def run_ours(args):
     if tpe is not None:
         traffic = int(tpe * N)
     app_alg = 8 * nnz
+    app_sectors = touched_sectors(offsets, indices)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -850,7 +986,10 @@ def run_ours(args):
                        "elems_per_s": round(N / enc_ms * 1e3, 1)},
             "apply": {"ms": round(app_ms, 4), "alg_bytes": app_alg,
                       "alg_GBps": round(app_alg / app_ms / 1e6, 1),
-                      "weight_GBps": round(weight_bytes / app_ms / 1e6, 1)},
+                      "weight_GBps": round(weight_bytes / app_ms / 1e6, 1),
+                      "elems_per_s": round(N / app_ms * 1e3, 1),
+                      "entries_per_s": round(nnz / app_ms * 1e3, 1),
+                      **sector_model(nnz, app_sectors, app_ms, peak)},
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -978,7 +1117,8 @@ def run_ours(args):
         rows.update([row("encode_llama3_8b_lr1e-5", ms_e, 4 * N + 6 * nnz2, weight_bytes, peak,
                          {"min_ms": round(mn_e, 4), "nnz": nnz2, "sparsity": round(1 - nnz2 / N, 6)})])
         rows.update([row("apply_llama3_8b_lr1e-5", ms_a, 8 * nnz2, weight_bytes, peak,
-                         {"min_ms": round(mn_a, 4), "exact": ok})])
+                         {"min_ms": round(mn_a, 4), "exact": ok, "entries_per_s": round(nnz2 / ms_a * 1e3, 1),
+                          **sector_model(nnz2, touched_sectors(offs2, idx2), ms_a, peak)})])
         # wire form of the same delta: positions block (2 or 4 bytes each) and checksum
         pcap = 4 * nnz2
         positions = torch.empty(max(2, pcap), dtype=torch.uint8, device=dev)
