@@ -333,18 +333,20 @@ DWS_API dws_status_t dws_apply_chain(const dws_plan_t *plan, void *const *snap_p
                              void *workspace, size_t workspace_bytes, dws_stream_t stream);
 
 /* How dws_apply_chain_ex replays the chain; both give the same snapshot.
- * DWS_CHAIN_AUTO: the library's choice (what dws_apply_chain does): the tile
- *   merge when the deltas' entry counts suggest that more than half of the
- *   snapshot's 32-byte sectors are touched, else the scatter.
+ * Both work tile by tile (8192 elements): every entry of every delta for the
+ * tile raises its element's tag in shared memory to (k + 1) << 16 | value,
+ * so the latest delta's value is kept whatever the order of the threads.
+ * DWS_CHAIN_AUTO: the library's choice (what dws_apply_chain does): the
+ *   scatter, the faster of the two on every chain measured (10 Qwen3-0.6B
+ *   steps, which touch nearly every sector, and the clustered stress set).
  * DWS_CHAIN_TILE_MERGE: every tile some delta touches is read into shared
- *   memory, the entries of all deltas for it are written in delta order and
- *   the whole tile is written back (4 bytes per element of the touched tiles
- *   plus 6 per entry); tiles no delta touches are not moved.
- * DWS_CHAIN_SCATTER: per window of tiles, the deltas are replayed from the last
- *   to the first and an element is stored only by the latest delta that
- *   touches it (a written-bit per element in shared memory); untouched parts of
- *   the snapshot are neither read nor written (L2 reads and writes back the
- *   touched 32-byte sectors). */
+ *   memory first and written back whole (4 bytes per element of the touched
+ *   tiles plus 6 per entry; whole-sector writes); tiles no delta touches are
+ *   not moved.
+ * DWS_CHAIN_SCATTER: only the elements some delta names are stored, each
+ *   once, with its latest value; untouched parts of the snapshot are neither
+ *   read nor written (L2 reads and writes back the touched 32-byte
+ *   sectors). */
 #define DWS_CHAIN_AUTO 0
 #define DWS_CHAIN_TILE_MERGE 1
 #define DWS_CHAIN_SCATTER 2

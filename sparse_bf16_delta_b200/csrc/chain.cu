@@ -3,42 +3,29 @@
 // between; a new replica takes the latest anchor and replays the deltas after
 // it, the later delta winning where two touch the same element).
 //
-// Three kernels per pass over the snapshot:
+// Two kernels per pass over the snapshot:
 //
 //   chain_index_kernel  reads every entry of every delta once (coalesced
 //     16-byte loads), checks it (index inside its tensor, strictly above the
 //     entry before it in its tensor's segment) and writes the chain's tile
 //     index: for tile g and delta k, the first entry of k at or past the start
 //     of g, mod 2^32.  A failed check sets the workspace's delta flag, and the
-//     replay kernels then write nothing: a chain with a bad entry anywhere is
+//     replay kernel then writes nothing: a chain with a bad entry anywhere is
 //     not applied at all.
 //
-//   chain_merge_kernel  (DWS_CHAIN_TILE_MERGE) one persistent CTA per SM over
-//     a contiguous range of tiles.  A producer warp fills a 4-stage ring:
-//     per tile, one bulk copy of the snapshot tile and, per delta, bulk copies
-//     of exactly that tile's entries (the tile index gives their range), so
-//     the loads of the next tiles are in flight while 8 consumer warps merge
-//     the current one: every entry of every delta raises its element's tag
-//     to (k + 1) << 16 | value with atomicMax (the latest delta wins whatever
-//     the thread order), then one pass moves the tagged values into the
-//     tile.  The producer writes the merged tile back with one bulk store as
-//     soon as it is done.  A tile no delta touches is neither read nor
-//     written.
-//
-//   chain_scatter_kernel  (DWS_CHAIN_SCATTER) per window of 32 tiles the
-//     deltas are replayed from the last to the first, an element being
-//     stored only if its written-bit in shared memory is clear, so every
-//     element is written once, by the latest delta that names it; untouched
-//     32-byte sectors are not moved at all.  The tile index gives each
-//     window's stretch of every delta.
+//   chain_tile_kernel  one CTA per tile: the tile index gives each delta's
+//     entries of the tile; every entry raises its element's tag in shared
+//     memory to (k + 1) << 16 | value with atomicMax, so the latest delta
+//     wins whatever the thread order; then the tagged elements are stored
+//     (DWS_CHAIN_SCATTER: untouched sectors are not moved), or the whole tile,
+//     read in first, is written back (DWS_CHAIN_TILE_MERGE: whole-sector
+//     writes).  A tile no delta touches is not moved in either mode.
 #include <cuda_runtime.h>
 
 #include "dws_internal.cuh"
 
 namespace dws {
 namespace {
-
-constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
 
 // ---------------------------------------------------------------------------
 // Tile index and validation
@@ -327,615 +314,276 @@ __global__ void __launch_bounds__(kIdxThreads, 4) chain_index_kernel(IndexParams
     }
 }
 
-// The first entry of delta `d` at or past the start of tile g (in tensor t),
-// from the tile index: the only value in [offsets[t], offsets[t+1]] with
-// these low 32 bits (a tensor has fewer than 2^31 entries).
-__device__ __forceinline__ long long index_entry(const DeltaRef &d, const uint32_t *index, long long g,
-                                                 int col, int t) {
-    const long long lo = d.offsets[t];
-    return lo + static_cast<long long>(index[g * kChainGroup + col] - static_cast<uint32_t>(lo));
-}
-
 // ---------------------------------------------------------------------------
-// Tile merge
+// Per-tile replay: one CTA per tile
 // ---------------------------------------------------------------------------
-constexpr int kMergeConsumerWarps = 8;
-constexpr int kMergeConsumers = 32 * kMergeConsumerWarps;
-constexpr int kMergeThreads = 32 + kMergeConsumers;
-constexpr int kStages = 4;
-constexpr int kStageEntries = 4096;  // entries staged per stage, all deltas together
+constexpr int kTileThreads = 256;
+constexpr int kTileWarps = kTileThreads / 32;
+constexpr int kItemEntries = 128;                         // 4 consecutive entries per lane
+constexpr int kTileItems = 3;                             // items per warp per round
+constexpr int kTileRoundItems = kTileWarps * kTileItems;  // items per round
+constexpr int kTileMinBlocks = 6;
 
-struct MergeParams {
+struct TileParams {
     WsView ws;
     uint16_t *const *snap_ptrs;
     const uint32_t *index;
-    long long tiles_per_cta;
     int K;
     DeltaRef d[kChainGroup];
 };
 
-// What the producer staged for one tile.
-struct StageMeta {
-    long long s[kChainGroup];  // first entry of the tile in delta k
-    int n[kChainGroup];        // entries of the tile in delta k
-    int ia[kChainGroup];       // staged indices: entries s + [ia, ib) at idx[io + ...] (ia may be < 0)
-    int ib[kChainGroup];
-    int io[kChainGroup];
-    int va[kChainGroup];       // staged values: entries s + [va, vb) at val[vo + ...]
-    int vb[kChainGroup];
-    int vo[kChainGroup];
-    int C[kChainGroup + 1];    // work items (32 entries of one delta): delta k's are [C[k], C[k+1])
-    uint16_t *ptr;  // tile start in the snapshot
-    int local_start;
-    int count;   // elements of the tile
-    int bulk;    // leading elements moved by bulk copies (multiple of 8)
-    int touched;
+struct TileShared {
+    // Delta k's entries of the tile are base + [lo, hi), base = the first
+    // entry rounded down to a multiple of 4, so that items start aligned;
+    // lim = entries from base to the end of the delta's arrays.
+    const int *ip[kChainGroup];
+    const uint16_t *vp[kChainGroup];
+    int lo[kChainGroup];
+    int hi[kChainGroup];
+    long long lim[kChainGroup];
+    int vec[kChainGroup];                       // 16-byte loads allowed (aligned arrays)
+    int C[kChainGroup + 1];                     // items of the deltas before k
+    uint16_t *dst;                              // tile start in the snapshot (null: skip)
+    int local;                                  // tile start within its tensor
+    int count;                                  // elements of the tile
 };
 
-struct MergeSmem {
-    uint32_t tag[kTileElems];  // (k + 1) << 16 | value of the latest delta k per element; 0: none
-    uint16_t tile[kStages][kTileElems];
-    int idx[kStages][kStageEntries];
-    uint16_t val[kStages][kStageEntries];
-    StageMeta meta[kStages];
-    unsigned long long full[kStages];  // producer -> consumers: tile staged
-    unsigned long long done[kStages];  // consumers -> producer: tile merged
-    int grp[kStages];                  // producer: store group of the stage's tile (-1: none)
-    long long cursor[kChainGroup];
-    int abort;
-};
-
-// Producer warp's view of the tensor that holds the current tile.
-struct TensorCursor {
-    int t;              // tensor
-    long long first;    // its first tile
-    long long next;     // first tile of the next tensor
-    long long numel;
-    uint16_t *ptr;
-};
-
-__device__ __forceinline__ void tensor_at(const MergeParams &p, int t, TensorCursor &c) {
-    c.t = t;
-    c.first = p.ws.first_tile[t];
-    c.next = p.ws.first_tile[t + 1];
-    c.numel = p.ws.numel[t];
-    c.ptr = p.snap_ptrs[t];
+__device__ __forceinline__ int int4_at(const int4 &v, int e) {
+    return e == 0 ? v.x : (e == 1 ? v.y : (e == 2 ? v.z : v.w));
+}
+__device__ __forceinline__ uint32_t u16x4_at(const uint2 &v, int e) {
+    const uint32_t w = e < 2 ? v.x : v.y;
+    return (e & 1) ? (w >> 16) : (w & 0xffffu);
 }
 
-// Producer warp: describe tile i and start its copies into stage st.  Lane k
-// (< K) owns delta k: its entries of the tile are [cursor, cursor + n) with
-// n the difference of two index rows (mod 2^32; a tile holds fewer).
-__device__ void merge_stage(const MergeParams &p, MergeSmem &sm, long long i, int st,
-                            const TensorCursor &tc, uint32_t row_next, long long &cursor,
-                            unsigned long long policy) {
-    const int lane = threadIdx.x & 31;
-    StageMeta &m = sm.meta[st];
-    const long long ls = (i - tc.first) << kTileShift;
-    const long long rest = tc.numel - ls;
-    const int count = static_cast<int>(rest < kTileElems ? (rest > 0 ? rest : 0) : kTileElems);
-    const bool mine = lane < p.K;
-    int n = 0;
-    long long s = 0;
-    if (mine) {
-        s = cursor;
-        const uint32_t row_here = static_cast<uint32_t>(s);  // the row of tile i, as cursor's low bits
-        n = static_cast<int>(row_next - row_here);
-        cursor = s + n;
-    }
-    int total = n;
+// Round r of this warp's items: item i = r * kTileRoundItems + warp + q *
+// kTileWarps covers entries base + 128 c + [0, 128) of delta k (c = i -
+// C[k]); lane l takes the 4 entries from base + 128 c + 4 l.  kq[q] = k
+// (warp-uniform; -1: no such item); vm[q] bit e: entry e is the tile's.
+// Every load of the round is in flight at once.
+__device__ __forceinline__ void tile_load_round(const TileShared &sm, int K, int r, int4 (&ix)[kTileItems],
+                                                uint2 (&vx)[kTileItems], int (&kq)[kTileItems],
+                                                unsigned int (&vm)[kTileItems]) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int i0 = r * kTileRoundItems + warp;
+    const int items = sm.C[K];
+    int k = 0;
+    while (k + 1 < K && sm.C[k + 1] <= i0) ++k;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
-    const uintptr_t ua = reinterpret_cast<uintptr_t>(tc.ptr);
-    bool touched = total > 0 && count > 0;
-    if (touched && (tc.ptr == nullptr || (ua & 1u))) {
-        if (lane == 0) record_error(p.ws.hdr, DWS_ERR_INVALID, tc.t);
-        touched = false;
-    }
-    const int bulk = (touched && (ua & 15u) == 0) ? (count & ~7) : 0;
-    // Entries: each delta's range widened to 16-byte boundaries (so that
-    // no entry of the tile has to come from global memory), kept inside the
-    // delta's arrays: only at the arrays' unaligned ends do a few entries
-    // stay outside it.  A prefix sum over the lanes places the ranges while
-    // there is room.
-    int ci = 0, cv = 0;
-    long long ia = 0, va = 0;  // absolute first staged entry
-    if (mine && touched && n > 0) {
-        const DeltaRef &dk = p.d[lane];
-        const uintptr_t lo_i = (reinterpret_cast<uintptr_t>(dk.indices) + 15) & ~uintptr_t(15);
-        const uintptr_t hi_i = reinterpret_cast<uintptr_t>(dk.indices + dk.count) & ~uintptr_t(15);
-        uintptr_t a = reinterpret_cast<uintptr_t>(dk.indices + s) & ~uintptr_t(15);
-        uintptr_t b = (reinterpret_cast<uintptr_t>(dk.indices + s + n) + 15) & ~uintptr_t(15);
-        if (a < lo_i) a = lo_i;
-        if (b > hi_i) b = hi_i;
-        if (b > a && ((a - reinterpret_cast<uintptr_t>(dk.indices)) & 3u) == 0) {
-            ci = static_cast<int>((b - a) >> 2);
-            ia = static_cast<long long>((a - reinterpret_cast<uintptr_t>(dk.indices)) >> 2);
-        }
-        const uintptr_t lo_v = (reinterpret_cast<uintptr_t>(dk.values) + 15) & ~uintptr_t(15);
-        const uintptr_t hi_v = reinterpret_cast<uintptr_t>(dk.values + dk.count) & ~uintptr_t(15);
-        uintptr_t c = reinterpret_cast<uintptr_t>(dk.values + s) & ~uintptr_t(15);
-        uintptr_t d = (reinterpret_cast<uintptr_t>(dk.values + s + n) + 15) & ~uintptr_t(15);
-        if (c < lo_v) c = lo_v;
-        if (d > hi_v) d = hi_v;
-        if (d > c && ((c - reinterpret_cast<uintptr_t>(dk.values)) & 1u) == 0) {
-            cv = static_cast<int>((d - c) >> 1);
-            va = static_cast<long long>((c - reinterpret_cast<uintptr_t>(dk.values)) >> 1);
+    for (int q = 0; q < kTileItems; ++q) {
+        const int i = i0 + q * kTileWarps;
+        kq[q] = -1;
+        vm[q] = 0u;
+        if (i < items) {  // warp-uniform
+            while (k + 1 < K && sm.C[k + 1] <= i) ++k;
+            kq[q] = k;
+            const int o = (i - sm.C[k]) * kItemEntries + 4 * lane;
+            const int lo = sm.lo[k], hi = sm.hi[k];
+            unsigned int m = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) m |= (o + e >= lo && o + e < hi) ? (1u << e) : 0u;
+            vm[q] = m;
+            if (m == 0xfu && sm.vec[k] && o + 3 < sm.lim[k]) {
+                ix[q] = __ldg(reinterpret_cast<const int4 *>(sm.ip[k] + o));
+                vx[q] = __ldg(reinterpret_cast<const uint2 *>(sm.vp[k] + o));
+            } else if (m != 0u) {
+                int xs[4] = {0, 0, 0, 0};
+                uint32_t vs[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if ((m >> e) & 1u) {
+                        xs[e] = __ldg(sm.ip[k] + o + e);
+                        vs[e] = __ldg(sm.vp[k] + o + e);
+                    }
+                }
+                ix[q] = make_int4(xs[0], xs[1], xs[2], xs[3]);
+                vx[q] = make_uint2(vs[0] | (vs[1] << 16), vs[2] | (vs[3] << 16));
+            }
         }
     }
-    int oi = ci, ov = cv;  // inclusive prefix over lanes
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int x = __shfl_up_sync(0xffffffffu, oi, o);
-        const int y = __shfl_up_sync(0xffffffffu, ov, o);
-        if (lane >= o) {
-            oi += x;
-            ov += y;
-        }
-    }
-    oi -= ci;  // exclusive
-    ov -= cv;
-    if (oi + ci > kStageEntries) ci = oi < kStageEntries ? ((kStageEntries - oi) & ~3) : 0;
-    if (ov + cv > kStageEntries) cv = ov < kStageEntries ? ((kStageEntries - ov) & ~7) : 0;
-    int fn = (n + 31) >> 5;  // inclusive prefix of the work items over the lanes
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int x = __shfl_up_sync(0xffffffffu, fn, o);
-        if (lane >= o) fn += x;
-    }
-    if (lane < p.K) m.C[lane + 1] = fn;
-    if (lane == 0) m.C[0] = 0;
-    if (mine) {
-        m.s[lane] = s;
-        m.n[lane] = n;
-        // staged ranges relative to s (may start before it)
-        m.ia[lane] = static_cast<int>(ia - s);
-        m.ib[lane] = static_cast<int>(ia - s) + ci;
-        m.io[lane] = oi;
-        m.va[lane] = static_cast<int>(va - s);
-        m.vb[lane] = static_cast<int>(va - s) + cv;
-        m.vo[lane] = ov;
-    }
-    uint32_t bytes = static_cast<uint32_t>(ci) * 4u + static_cast<uint32_t>(cv) * 2u;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-    if (lane == 0) {
-        m.ptr = touched ? tc.ptr + ls : nullptr;
-        m.local_start = static_cast<int>(ls);
-        m.count = count;
-        m.bulk = bulk;
-        m.touched = touched ? 1 : 0;
-    }
-    __syncwarp();
-    if (lane == 0) {
-        bytes += static_cast<uint32_t>(bulk) * 2u;
-        mbar_arrive_expect_tx(&sm.full[st], bytes);  // releases the description above
-        if (bulk > 0)
-            bulk_load(sm.tile[st], tc.ptr + ls, static_cast<uint32_t>(bulk) * 2u, &sm.full[st], policy);
-    }
-    __syncwarp();
-    if (ci > 0)
-        bulk_load(&sm.idx[st][oi], p.d[lane].indices + ia, static_cast<uint32_t>(ci) * 4u,
-                  &sm.full[st], policy);
-    if (cv > 0)
-        bulk_load(&sm.val[st][ov], p.d[lane].values + va, static_cast<uint32_t>(cv) * 2u,
-                  &sm.full[st], policy);
 }
 
-__global__ void __launch_bounds__(kMergeThreads, 1) chain_merge_kernel(MergeParams p) {
-    extern __shared__ __align__(128) unsigned char merge_smem_raw[];
-    MergeSmem &sm = *reinterpret_cast<MergeSmem *>(merge_smem_raw);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// One CTA replays every delta of the group onto one tile.  Each element has
+// a 32-bit tag in shared memory; every entry of delta k raises its element's
+// tag to (k + 1) << 16 | value with atomicMax, so that whatever the thread
+// order the tag ends with the latest delta's value, and no entry is read
+// twice.  Then one coalesced pass writes the tile:
+//   scatter (kMerge false): tags start at 0, and only tagged elements are
+//     stored to the snapshot (untouched sectors are not moved);
+//   merge (kMerge true): tags start as the tile's own values (version 0),
+//     and the whole tile is written back (whole-sector writes).
+// Warp 0 first turns the tile's two index rows into per-delta entry ranges;
+// the work is cut into items of 128 entries of one delta (4 per lane, 16-byte
+// loads when the arrays allow).  A tile no delta touches is not moved.
+template <bool kMerge>
+__global__ void __launch_bounds__(kTileThreads, kTileMinBlocks) chain_tile_kernel(TileParams p) {
+    __shared__ TileShared sm;
+    __shared__ __align__(16) uint32_t s_tag[kTileElems];
+    const int tid = threadIdx.x, lane = tid & 31;
+    const long long g = blockIdx.x;
+    const int K = p.K;
 
-    if (!ws_matches(p.ws)) return;
-    if (ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) != 0u) return;
-    const long long tb = static_cast<long long>(blockIdx.x) * p.tiles_per_cta;
-    long long te = tb + p.tiles_per_cta;
-    if (te > p.ws.num_tiles) te = p.ws.num_tiles;
-    if (tb >= te) return;
-    const long long ntl = te - tb;
-
-    if (tid == 0) {
-        sm.abort = 0;
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.done[s], 1);
+    if constexpr (!kMerge) {
+#pragma unroll
+        for (int q = 0; q < kTileElems / 4 / kTileThreads; ++q)
+            reinterpret_cast<uint4 *>(s_tag)[tid + q * kTileThreads] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (tid < 32) {
+        // The rows are requested before the header is checked: the workspace
+        // size was checked on the host, so every address here is inside it.
+        const int t = p.ws.tile_tensor[g];
+        uint32_t ra = 0, rb = 0;
+        if (lane < K) {
+            ra = p.index[g * kChainGroup + lane];
+            rb = p.index[(g + 1) * kChainGroup + lane];
         }
-        mbar_fence_init();
+        const WsHeader *h = p.ws.hdr;
+        bool ok = h->magic == kWsMagic && h->fingerprint == p.ws.fingerprint &&
+                  h->num_tiles == p.ws.num_tiles && h->num_tensors == p.ws.num_tensors;
+        if (!ok && lane == 0) record_error(p.ws.hdr, DWS_ERR_WORKSPACE, 0);
+        ok = ok && ld_relaxed_gpu_u32(&h->delta_bad) == 0u;
+        if (ok && (t < 0 || t >= p.ws.num_tensors)) {
+            if (lane == 0) record_error(p.ws.hdr, DWS_ERR_WORKSPACE, g);
+            ok = false;
+        }
+        long long s = 0;
+        int n = 0;
+        if (ok && lane < K) {
+            const DeltaRef d = p.d[lane];
+            const long long lo = d.offsets[t];
+            s = lo + static_cast<long long>(ra - static_cast<uint32_t>(lo));
+            long long e = lo + static_cast<long long>(rb - static_cast<uint32_t>(lo));
+            // kept inside the delta's arrays and one tile's worth
+            s = s < 0 ? 0 : (s > d.count ? d.count : s);
+            e = e > d.count ? d.count : e;
+            e = e - s > kTileElems ? s + kTileElems : e;
+            n = e > s ? static_cast<int>(e - s) : 0;
+            const long long base = s & ~3LL;
+            sm.ip[lane] = d.indices + base;
+            sm.vp[lane] = d.values + base;
+            sm.lo[lane] = static_cast<int>(s - base);
+            sm.hi[lane] = static_cast<int>(s - base) + n;
+            sm.lim[lane] = d.count - base;
+            sm.vec[lane] = ((reinterpret_cast<uintptr_t>(d.indices) & 15u) == 0 &&
+                            (reinterpret_cast<uintptr_t>(d.values) & 7u) == 0) ? 1 : 0;
+        }
+        // items of delta k: ceil(hi / 128), none if it has no entry here
+        int pre = n > 0 ? (static_cast<int>(s & 3LL) + n + kItemEntries - 1) / kItemEntries : 0;
+#pragma unroll
+        for (int o = 1; o < kChainGroup; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, pre, o);
+            if (lane >= o) pre += y;
+        }
+        if (lane < K) sm.C[lane + 1] = pre;
+        if (lane == 0) {
+            sm.C[0] = 0;
+            uint16_t *dst = nullptr;
+            int local = 0, count = 0;
+            if (ok) {
+                const long long ls = (g - p.ws.first_tile[t]) << kTileShift;
+                const long long rest = p.ws.numel[t] - ls;
+                count = static_cast<int>(rest < kTileElems ? (rest > 0 ? rest : 0) : kTileElems);
+                local = static_cast<int>(ls);
+                dst = p.snap_ptrs[t];
+                if (count > 0 && (dst == nullptr || (reinterpret_cast<uintptr_t>(dst) & 1u))) {
+                    record_error(p.ws.hdr, DWS_ERR_INVALID, t);
+                    dst = nullptr;
+                }
+                if (dst != nullptr) dst += ls;
+            }
+            sm.dst = dst;
+            sm.local = local;
+            sm.count = count;
+        }
     }
     __syncthreads();
+    uint16_t *const dst = sm.dst;
+    const int items = sm.C[K];
+    if (dst == nullptr || items == 0) return;  // uniform
+    const int local = sm.local, count = sm.count;
+    const bool vec = count == kTileElems && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0;
 
-    if (warp == 0) {
-        // ---- producer warp ---------------------------------------------------
-        // Stages tile li once tile li - kStages is merged and its store has
-        // read the stage; stores are issued as soon as a tile is merged.
-        const unsigned long long policy = l2_evict_first_policy();
-        TensorCursor tc;
-        tensor_at(p, p.ws.tile_tensor[tb], tc);
-        long long cursor = 0;  // lane k: delta k's first entry of the next tile to stage
-        uint32_t rq0 = 0, rq1 = 0, rq2 = 0, rq3 = 0;  // index rows of tiles i+1 .. i+4
-        const long long nrows = p.ws.num_tiles;      // last row
-        if (lane < p.K) {
-            cursor = index_entry(p.d[lane], p.index, tb, lane, tc.t);
-            rq0 = p.index[(tb + 1) * kChainGroup + lane];
-            if (tb + 2 <= nrows) rq1 = p.index[(tb + 2) * kChainGroup + lane];
-            if (tb + 3 <= nrows) rq2 = p.index[(tb + 3) * kChainGroup + lane];
-            if (tb + 4 <= nrows) rq3 = p.index[(tb + 4) * kChainGroup + lane];
+    const int rounds = (items + kTileRoundItems - 1) / kTileRoundItems;
+    int4 ix[kTileItems];
+    uint2 vx[kTileItems];
+    int kq[kTileItems];
+    unsigned int vm[kTileItems];
+    tile_load_round(sm, K, 0, ix, vx, kq, vm);
+    if constexpr (kMerge) {
+        // tags <- the tile's values (version 0), while the entries arrive
+        if (vec) {
+            uint4 t4[kTileElems / 8 / kTileThreads];
+#pragma unroll
+            for (int q = 0; q < kTileElems / 8 / kTileThreads; ++q)
+                t4[q] = ld_stream_v4(reinterpret_cast<const uint4 *>(dst) + tid + q * kTileThreads);
+#pragma unroll
+            for (int q = 0; q < kTileElems / 8 / kTileThreads; ++q) {
+                uint4 *o = reinterpret_cast<uint4 *>(s_tag + (tid + q * kTileThreads) * 8);
+                o[0] = make_uint4(t4[q].x & 0xffffu, t4[q].x >> 16, t4[q].y & 0xffffu, t4[q].y >> 16);
+                o[1] = make_uint4(t4[q].z & 0xffffu, t4[q].z >> 16, t4[q].w & 0xffffu, t4[q].w >> 16);
+            }
+        } else {
+            for (int i = tid; i < kTileElems; i += kTileThreads) s_tag[i] = i < count ? dst[i] : 0u;
         }
-        long long taken = 0;  // tiles whose completion the producer has taken
-        int committed = 0;    // store groups committed
-        // take tile c's completion: write it back
-        auto take = [&](long long c) {
-            const int cs = static_cast<int>(c % kStages);
-            const StageMeta &m = sm.meta[cs];
-            if (m.touched && m.bulk > 0) {
-                bulk_store(m.ptr, sm.tile[cs], static_cast<uint32_t>(m.bulk) * 2u);
-                bulk_commit();
-                sm.grp[cs] = committed++;
+    }
+    __syncthreads();  // tags initialised
+    for (int r = 0; r < rounds; ++r) {
+        if (r > 0) tile_load_round(sm, K, r, ix, vx, kq, vm);
+#pragma unroll
+        for (int q = 0; q < kTileItems; ++q) {
+            const uint32_t ver = static_cast<uint32_t>(kq[q] + 1) << 16;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if ((vm[q] >> e) & 1u) {
+                    // position within the tile; checked entries never fall outside
+                    const uint32_t pos = static_cast<uint32_t>(int4_at(ix[q], e) - local);
+                    if (pos < static_cast<uint32_t>(count)) atomicMax(&s_tag[pos], ver | u16x4_at(vx[q], e));
+                    else record_error(p.ws.hdr, DWS_ERR_WORKSPACE, g);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if constexpr (kMerge) {
+        if (vec) {
+#pragma unroll
+            for (int q = 0; q < kTileElems / 8 / kTileThreads; ++q) {
+                const uint4 *t = reinterpret_cast<const uint4 *>(s_tag + (tid + q * kTileThreads) * 8);
+                const uint4 a = t[0], b = t[1];
+                st_stream_v4(reinterpret_cast<uint4 *>(dst) + tid + q * kTileThreads,
+                             make_uint4((a.x & 0xffffu) | (a.y << 16), (a.z & 0xffffu) | (a.w << 16),
+                                        (b.x & 0xffffu) | (b.y << 16), (b.z & 0xffffu) | (b.w << 16)));
+            }
+        } else {
+            for (int i = tid; i < count; i += kTileThreads) dst[i] = static_cast<uint16_t>(s_tag[i]);
+        }
+    } else {
+        // 4 consecutive elements per thread, a warp 128: the tagged ones are
+        // stored, as one 8-byte store when all four are and it is aligned
+        const bool al8 = (reinterpret_cast<uintptr_t>(dst) & 7u) == 0;
+#pragma unroll 2
+        for (int q = 0; q < kTileElems / 4 / kTileThreads; ++q) {
+            const int e0 = (tid + q * kTileThreads) * 4;
+            const uint4 t = reinterpret_cast<const uint4 *>(s_tag)[tid + q * kTileThreads];
+            const bool h0 = t.x >> 16, h1 = t.y >> 16, h2 = t.z >> 16, h3 = t.w >> 16;
+            if (h0 && h1 && h2 && h3 && al8) {
+                *reinterpret_cast<uint2 *>(dst + e0) =
+                    make_uint2((t.x & 0xffffu) | (t.y << 16), (t.z & 0xffffu) | (t.w << 16));
             } else {
-                sm.grp[cs] = -1;
+                if (h0) dst[e0] = static_cast<uint16_t>(t.x);
+                if (h1) dst[e0 + 1] = static_cast<uint16_t>(t.y);
+                if (h2) dst[e0 + 2] = static_cast<uint16_t>(t.z);
+                if (h3) dst[e0 + 3] = static_cast<uint16_t>(t.w);
             }
-        };
-        bool ok = true;
-        for (long long li = 0; li < ntl; ++li) {
-            const long long i = tb + li;
-            const int st = static_cast<int>(li % kStages);
-            while (i >= tc.next) tensor_at(p, tc.t + 1, tc);  // uniform
-            if (lane == 0) {
-                while (taken < li && mbar_try_wait(&sm.done[taken % kStages],
-                                                   static_cast<uint32_t>((taken / kStages) & 1)))
-                    take(taken++);
-                while (ok && taken <= li - kStages) {
-                    ok = mbar_wait_sleepy(&sm.done[taken % kStages], static_cast<uint32_t>((taken / kStages) & 1),
-                                          kWaitLimitNs);
-                    if (ok) take(taken++);
-                }
-                if (ok && li >= kStages && sm.grp[st] >= 0) bulk_wait_read_n(committed - 1 - sm.grp[st]);
-            }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            __syncwarp();
-            merge_stage(p, sm, i, st, tc, rq0, cursor, policy);
-            rq0 = rq1;
-            rq1 = rq2;
-            rq2 = rq3;
-            rq3 = (lane < p.K && i + 5 <= nrows) ? p.index[(i + 5) * kChainGroup + lane] : 0u;
         }
-        if (lane == 0) {
-            // write back the last tiles
-            while (ok && taken < ntl) {
-                ok = mbar_wait_sleepy(&sm.done[taken % kStages], static_cast<uint32_t>((taken / kStages) & 1),
-                                      kWaitLimitNs);
-                if (ok) take(taken++);
-            }
-            if (!ok) {
-                atomicExch(&sm.abort, 1);
-                record_error(p.ws.hdr, DWS_ERR_TIMEOUT, tb);
-            }
-            bulk_wait_all();
-        }
-        return;
-    }
-
-    // ---- consumers (8 warps) ------------------------------------------------
-    // Per tile: the entries of all deltas as one list; each entry raises its
-    // element's tag to (k + 1) << 16 | value with atomicMax, so the latest
-    // delta wins whatever the order the threads run in; then one pass moves
-    // the tagged values into the tile (or straight to global memory past the
-    // bulk-copied part) and clears the tags.
-    const int ct = tid - 32;  // 0 .. kMergeConsumers - 1
-    for (int e = ct; e < kTileElems; e += kMergeConsumers) sm.tag[e] = 0u;
-    named_bar(1, kMergeConsumers);
-    for (long long li = 0; li < ntl; ++li) {
-        const int st = static_cast<int>(li % kStages);
-        const bool got = mbar_wait_sleepy(&sm.full[st], static_cast<uint32_t>((li / kStages) & 1), kWaitLimitNs);
-        if (!named_bar_and(1, kMergeConsumers, got && ld_acquire_cta(&sm.abort) == 0)) {
-            if (ct == 0) record_error(p.ws.hdr, DWS_ERR_TIMEOUT, tb + li);
-            return;  // the producer's own waits are bounded too
-        }
-        const StageMeta &m = sm.meta[st];
-        if (m.touched) {
-            const int ls = m.local_start;
-            const int count = m.count;
-            const int items = m.C[p.K];
-            const int cw = ct >> 5;
-            int k = -1, c_lo = 0, c_hi = 0, n = 0, ia = 0, ib = 0, io = 0, va = 0, vb = 0, vo = 0;
-            bool staged = false;
-            const int *gi = nullptr;
-            const uint16_t *gv = nullptr;
-            for (int it = cw; it < items; it += kMergeConsumerWarps) {
-                while (it >= c_hi) {  // uniform per warp: items only move forward
-                    ++k;
-                    c_lo = m.C[k];
-                    c_hi = m.C[k + 1];
-                    n = m.n[k];
-                    ia = m.ia[k]; ib = m.ib[k]; io = m.io[k];
-                    va = m.va[k]; vb = m.vb[k]; vo = m.vo[k];
-                    staged = ia <= 0 && ib >= n && va <= 0 && vb >= n;
-                    gi = p.d[k].indices + m.s[k];
-                    gv = p.d[k].values + m.s[k];
-                }
-                const int el = ((it - c_lo) << 5) + lane;
-                if (el >= n) continue;
-                int ix;
-                uint32_t vx;
-                if (staged) {
-                    ix = sm.idx[st][io + el - ia];
-                    vx = sm.val[st][vo + el - va];
-                } else {
-                    // outside the staged range: from global memory, inside the
-                    // delta's arrays whatever the index says
-                    const bool in_arr = m.s[k] + el >= 0 && m.s[k] + el < p.d[k].count;
-                    ix = (el >= ia && el < ib) ? sm.idx[st][io + el - ia] : (in_arr ? __ldg(gi + el) : -1);
-                    vx = (el >= va && el < vb) ? sm.val[st][vo + el - va] : (in_arr ? __ldg(gv + el) : 0u);
-                }
-                const int pos = ix - ls;  // in [0, count): the index pass's ranges
-                if (static_cast<unsigned>(pos) < static_cast<unsigned>(count))
-                    atomicMax(&sm.tag[pos], (static_cast<uint32_t>(k + 1) << 16) | vx);
-                else
-                    record_error(p.ws.hdr, DWS_ERR_WORKSPACE, m.s[k] + el);  // never expected
-            }
-            named_bar(1, kMergeConsumers);
-            const int bulk = m.bulk;
-            uint16_t *tile = sm.tile[st];
-#pragma unroll
-            for (int r = 0; r < kTileElems / (4 * kMergeConsumers); ++r) {
-                const int e0 = 4 * ct + r * 4 * kMergeConsumers;
-                if (e0 >= count) break;
-                const uint4 tg = *reinterpret_cast<const uint4 *>(&sm.tag[e0]);
-                if ((tg.x | tg.y | tg.z | tg.w) == 0u) continue;
-                *reinterpret_cast<uint4 *>(&sm.tag[e0]) = make_uint4(0u, 0u, 0u, 0u);
-                const uint32_t t4[4] = {tg.x, tg.y, tg.z, tg.w};
-                if (e0 + 4 <= bulk) {
-                    uint2 w = *reinterpret_cast<const uint2 *>(&tile[e0]);
-                    uint32_t lo = w.x, hi = w.y;
-                    if (t4[0]) lo = (lo & 0xffff0000u) | (t4[0] & 0xffffu);
-                    if (t4[1]) lo = (lo & 0x0000ffffu) | (t4[1] << 16);
-                    if (t4[2]) hi = (hi & 0xffff0000u) | (t4[2] & 0xffffu);
-                    if (t4[3]) hi = (hi & 0x0000ffffu) | (t4[3] << 16);
-                    *reinterpret_cast<uint2 *>(&tile[e0]) = make_uint2(lo, hi);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        if (!t4[q] || e0 + q >= count) continue;
-                        if (e0 + q < bulk) tile[e0 + q] = static_cast<uint16_t>(t4[q] & 0xffffu);
-                        else m.ptr[e0 + q] = static_cast<uint16_t>(t4[q] & 0xffffu);
-                    }
-                }
-            }
-            if (bulk > 0) fence_proxy_async_smem();  // the bulk store reads the tile
-            named_bar(1, kMergeConsumers);
-        }
-        if (ct == 0) mbar_arrive(&sm.done[st]);
-    }
-    if (ct == 0) {
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Reverse-order scatter over windows, with a written-bitmap
-// ---------------------------------------------------------------------------
-constexpr int kScatThreads = 1024;
-constexpr int kScatWarps = kScatThreads / 32;
-constexpr int kWinTiles = 32;
-constexpr int kWinElems = kWinTiles * kTileElems;
-constexpr int kScatDepth = 4;
-
-struct ScatParams {
-    WsView ws;
-    uint16_t *const *snap_ptrs;
-    const uint32_t *index;
-    long long tiles_per_cta;
-    int K;
-    DeltaRef d[kChainGroup];
-};
-
-struct ScatSmem {
-    uint32_t written[kWinElems / 32];
-    long long cur[kChainGroup];      // per delta: first entry of the current window
-    long long len[kChainGroup];      // per delta: entries of the current window
-    long long base[kWinTiles];       // per window tensor: (first_tile - window start) * tile
-    long long numel[kWinTiles];
-    uint16_t *ptr[kWinTiles];
-    long long offs[2][kWinTiles + 1];  // a delta's offsets of the window tensors (by parity)
-};
-
-__global__ void __launch_bounds__(kScatThreads, 1) chain_scatter_kernel(ScatParams p) {
-    extern __shared__ __align__(128) unsigned char scat_smem_raw[];
-    ScatSmem &sm = *reinterpret_cast<ScatSmem *>(scat_smem_raw);
-    const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const int warp = tid >> 5;
-
-    if (!ws_matches(p.ws)) return;
-    if (ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) != 0u) return;
-    const long long tb = static_cast<long long>(blockIdx.x) * p.tiles_per_cta;
-    long long te = tb + p.tiles_per_cta;
-    if (te > p.ws.num_tiles) te = p.ws.num_tiles;
-    if (tb >= te) return;
-
-    if (tid < p.K) sm.cur[tid] = index_entry(p.d[tid], p.index, tb, tid, p.ws.tile_tensor[tb]);
-
-    for (long long a = tb; a < te; a += kWinTiles) {
-        const long long b = (a + kWinTiles < te) ? a + kWinTiles : te;
-        const int win_words = static_cast<int>(b - a) * (kTileElems / 32);
-        const int t_lo = p.ws.tile_tensor[a];
-        const int nt = p.ws.tile_tensor[b - 1] - t_lo + 1;  // <= b - a: every tensor owns a tile
-        if (t_lo < 0 || nt < 1 || nt > kWinTiles || t_lo + nt > p.ws.num_tensors) {
-            if (tid == 0) record_error(p.ws.hdr, DWS_ERR_WORKSPACE, a);
-            return;  // uniform: every thread read the same table entries
-        }
-        __syncthreads();  // the previous window is complete
-        if (p.K > 1)
-            for (int w = tid; w < win_words; w += kScatThreads) sm.written[w] = 0u;
-        if (tid < nt) {
-            const int t = t_lo + tid;
-            const long long n = p.ws.numel[t];
-            uint16_t *ptr = p.snap_ptrs[t];
-            if (n > 0 && (ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 1u))) {
-                record_error(p.ws.hdr, DWS_ERR_INVALID, t);
-                ptr = nullptr;
-            }
-            sm.base[tid] = (p.ws.first_tile[t] - a) << kTileShift;
-            sm.numel[tid] = n;
-            sm.ptr[tid] = ptr;
-        }
-        if (tid < p.K) {
-            const int tn = b < p.ws.num_tiles ? p.ws.tile_tensor[b] : p.ws.num_tensors - 1;
-            sm.len[tid] = index_entry(p.d[tid], p.index, b, tid, tn) - sm.cur[tid];
-        }
-        constexpr long long kStride = 32LL * kScatWarps;
-        if (tid <= nt) sm.offs[(p.K - 1) & 1][tid] = p.d[p.K - 1].offsets[t_lo + tid];
-        __syncthreads();
-
-        int ix[kScatDepth];
-        uint16_t vx[kScatDepth];
-        bool prefetched = false;  // the phase's first chunks already requested (uniform)
-        for (int k = p.K - 1; k >= 0; --k) {
-            const DeltaRef d = p.d[k];
-            const int ph = k & 1;
-            const long long *offs = sm.offs[ph];
-            // the window's stretch of delta k, kept inside its arrays
-            const long long j0 = sm.cur[k] < 0 ? 0 : (sm.cur[k] > d.count ? d.count : sm.cur[k]);
-            const long long nl = sm.len[k] < 0 ? 0 : (j0 + sm.len[k] > d.count ? d.count - j0 : sm.len[k]);
-            const int n = static_cast<int>(nl < kWinElems ? nl : kWinElems);  // one window of one delta
-            const int *pi = d.indices + j0;
-            const uint16_t *pv = d.values + j0;
-            int r = 32 * warp + lane;  // this lane's entry of the current chunk
-            if (!prefetched) {
-#pragma unroll
-                for (int q = 0; q < kScatDepth; ++q) {
-                    if (r + q * kStride < n) {
-                        ix[q] = __ldg(pi + r + q * kStride);
-                        vx[q] = __ldg(pv + r + q * kStride);
-                    }
-                }
-            }
-            // The warp's current tensor (its chunks only move forward) and
-            // that tensor's constants: segment end relative to j0, window
-            // offset, size, pointer.
-            int tw = 0;
-            while (tw + 1 < nt && offs[tw + 1] <= j0 + r - lane) ++tw;
-            long long seg_hi = offs[tw + 1] - j0;
-            int off_c = static_cast<int>(-sm.base[tw]);
-            uint16_t *ptr_c = sm.ptr[tw];
-            for (bool more = r - lane < n; more;) {
-#pragma unroll
-                for (int q = 0; q < kScatDepth; ++q) {
-                    const int cs = r - lane;
-                    if (cs >= n) {  // the whole chunk is past the stretch (uniform)
-                        more = false;
-                        break;
-                    }
-                    const int idx = ix[q];
-                    const uint16_t val = vx[q];
-                    if (r + kScatDepth * kStride < n) {
-                        ix[q] = __ldg(pi + r + kScatDepth * kStride);
-                        vx[q] = __ldg(pv + r + kScatDepth * kStride);
-                    }
-                    const bool valid = r < n;
-                    if (cs >= seg_hi) {  // uniform: move to the chunk's first tensor
-                        while (tw + 1 < nt && offs[tw + 1] <= j0 + cs) ++tw;
-                        seg_hi = offs[tw + 1] - j0;
-                        off_c = static_cast<int>(-sm.base[tw]);
-                        ptr_c = sm.ptr[tw];
-                    }
-                    const int cl = (cs + 31 < n) ? cs + 31 : n - 1;
-                    uint32_t rel = 0;  // element within the window
-                    uint16_t *dst = ptr_c;
-                    if (cl < seg_hi) {
-                        // The chunk lies in one tensor (checked entries:
-                        // 0 <= idx - off_c < window length).
-                        rel = static_cast<uint32_t>(idx - off_c);
-                    } else if (valid) {
-                        const long long j = j0 + r;
-                        int tl = tw;
-                        while (tl + 1 < nt && offs[tl + 1] <= j) ++tl;
-                        rel = static_cast<uint32_t>(sm.base[tl] + idx);
-                        dst = sm.ptr[tl];
-                    }
-                    if (valid && rel >= static_cast<uint32_t>(kWinElems)) {  // never expected
-                        record_error(p.ws.hdr, DWS_ERR_WORKSPACE, j0 + r);
-                        rel = 0;
-                        dst = nullptr;
-                    }
-                    bool store = valid;
-                    if (p.K > 1) {  // uniform: a single delta needs no written-bits
-                        const uint32_t word = rel >> 5;
-                        const uint32_t bit = 1u << (rel & 31u);
-                        if (valid) store = (sm.written[word] & bit) == 0u;
-                        // Mark this delta's elements: one OR per lane, or two
-                        // for a run of 32 consecutive elements (a clustered
-                        // change), where per-lane ORs would all hit one word.
-                        const uint32_t r0 = __shfl_sync(0xffffffffu, rel, 0);
-                        const uint32_t r31 = __shfl_sync(0xffffffffu, rel, 31);
-                        bool marked = false;
-                        if (r31 - r0 == 31u && cs + 31 < n) {  // uniform; entries ascend
-                            if (lane == 0) atomicOr(&sm.written[r0 >> 5], ~0u << (r0 & 31u));
-                            if (lane == 31 && (r31 & 31u) != 31u)
-                                atomicOr(&sm.written[r31 >> 5], (2u << (r31 & 31u)) - 1u);
-                            marked = true;
-                        }
-                        if (!marked && valid) atomicOr(&sm.written[word], bit);
-                    }
-                    if (store && dst != nullptr) dst[idx] = val;
-                    r += kStride;
-                }
-            }
-            // This warp is done with delta k.  While the others finish,
-            // request the next (earlier) delta's offsets and first chunks.
-            prefetched = false;
-            if (k > 0) {
-                const DeltaRef dn = p.d[k - 1];
-                if (tid <= nt) sm.offs[ph ^ 1][tid] = dn.offsets[t_lo + tid];
-                const long long jn = sm.cur[k - 1] < 0 ? 0 : (sm.cur[k - 1] > dn.count ? dn.count : sm.cur[k - 1]);
-                const long long nn0 = sm.len[k - 1] < 0 ? 0 : (jn + sm.len[k - 1] > dn.count ? dn.count - jn : sm.len[k - 1]);
-                const long long nn = nn0 < kWinElems ? nn0 : kWinElems;
-                const int rn = 32 * warp + lane;
-#pragma unroll
-                for (int q = 0; q < kScatDepth; ++q) {
-                    if (rn + q * kStride < nn) {
-                        ix[q] = __ldg(dn.indices + jn + rn + q * kStride);
-                        vx[q] = __ldg(dn.values + jn + rn + q * kStride);
-                    }
-                }
-                prefetched = true;
-            }
-            __syncthreads();  // every entry of this delta stored before the next (earlier) one
-        }
-        if (tid < p.K) sm.cur[tid] += sm.len[tid];
     }
 }
 
 }  // namespace
 
-cudaError_t chain_set_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(chain_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sizeof(MergeSmem)));
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(chain_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sizeof(ScatSmem)));
-}
-
-cudaError_t chain_occupancy(int *ctas_per_sm) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, chain_merge_kernel, kMergeThreads,
-                                                         sizeof(MergeSmem));
-}
-
-cudaError_t index_occupancy(int *ctas_per_sm) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, chain_index_kernel, kIdxThreads, 0);
-}
-
-cudaError_t scatter_occupancy(int *ctas_per_sm) {
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, chain_scatter_kernel,
-                                                         kScatThreads, sizeof(ScatSmem));
-}
-
 cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs, const DeltaRef *deltas,
                                int K, bool merge, cudaStream_t s) {
-    DeviceInfo di;
-    cudaError_t e = device_info(&di);
-    if (e != cudaSuccess) return e;
-    e = launch_delta_check(ws, deltas, K, s);  // offsets of every delta
+    cudaError_t e = launch_delta_check(ws, deltas, K, s);  // offsets of every delta
     if (e != cudaSuccess) return e;
     uint32_t *index = reinterpret_cast<uint32_t *>(ws.tile_status);
 
@@ -968,35 +616,17 @@ cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs, con
         chain_index_kernel<<<dim3(static_cast<unsigned int>(gx), kg), kIdxThreads, 0, s>>>(ip);
         e = launched();
         if (e != cudaSuccess) return e;
-        if (merge) {
-            MergeParams mp;
-            mp.ws = ws;
-            mp.snap_ptrs = snap_ptrs;
-            mp.index = index;
-            mp.K = kg;
-            for (int k = 0; k < kg; ++k) mp.d[k] = deltas[k0 + k];
-            long long grid = static_cast<long long>(di.sm_count) * di.chain_ctas_per_sm;
-            if (grid > ws.num_tiles) grid = ws.num_tiles;
-            if (grid < 1) grid = 1;
-            mp.tiles_per_cta = (ws.num_tiles + grid - 1) / grid;
-            grid = (ws.num_tiles + mp.tiles_per_cta - 1) / mp.tiles_per_cta;
-            chain_merge_kernel<<<static_cast<unsigned int>(grid), kMergeThreads, sizeof(MergeSmem), s>>>(mp);
-        } else {
-            ScatParams sp;
-            sp.ws = ws;
-            sp.snap_ptrs = snap_ptrs;
-            sp.index = index;
-            sp.K = kg;
-            for (int k = 0; k < kg; ++k) sp.d[k] = deltas[k0 + k];
-            long long grid = static_cast<long long>(di.sm_count) * di.scatter_ctas_per_sm;
-            const long long windows = (ws.num_tiles + kWinTiles - 1) / kWinTiles;
-            if (grid > windows) grid = windows;
-            if (grid < 1) grid = 1;
-            // whole windows per CTA, so that only the last window of the plan is short
-            const long long win_per_cta = (windows + grid - 1) / grid;
-            sp.tiles_per_cta = win_per_cta * kWinTiles;
-            grid = (ws.num_tiles + sp.tiles_per_cta - 1) / sp.tiles_per_cta;
-            chain_scatter_kernel<<<static_cast<unsigned int>(grid), kScatThreads, sizeof(ScatSmem), s>>>(sp);
+        TileParams tp;
+        tp.ws = ws;
+        tp.snap_ptrs = snap_ptrs;
+        tp.index = index;
+        tp.K = kg;
+        for (int k = 0; k < kg; ++k) tp.d[k] = deltas[k0 + k];
+        if (ws.num_tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+        if (ws.num_tiles > 0) {
+            const unsigned int grid = static_cast<unsigned int>(ws.num_tiles);
+            if (merge) chain_tile_kernel<true><<<grid, kTileThreads, 0, s>>>(tp);
+            else chain_tile_kernel<false><<<grid, kTileThreads, 0, s>>>(tp);
         }
         e = launched();
         if (e != cudaSuccess) return e;

@@ -15,10 +15,6 @@ namespace dws {
 size_t encode_smem_bytes();
 cudaError_t encode_set_attributes();
 cudaError_t encode_occupancy(int *ctas_per_sm);
-cudaError_t chain_set_attributes();
-cudaError_t chain_occupancy(int *ctas_per_sm);
-cudaError_t scatter_occupancy(int *ctas_per_sm);
-cudaError_t index_occupancy(int *ctas_per_sm);
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -30,16 +26,9 @@ void init_device(int dev) {
     DeviceInfo di{};
     cudaError_t e = cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) e = encode_set_attributes();
-    if (e == cudaSuccess) e = chain_set_attributes();
     if (e == cudaSuccess) e = encode_occupancy(&di.encode_ctas_per_sm);
-    if (e == cudaSuccess) e = chain_occupancy(&di.chain_ctas_per_sm);
-    if (e == cudaSuccess) e = scatter_occupancy(&di.scatter_ctas_per_sm);
-    if (e == cudaSuccess) e = index_occupancy(&di.index_ctas_per_sm);
     if (e == cudaSuccess) {
         if (di.encode_ctas_per_sm < 1) di.encode_ctas_per_sm = 1;
-        if (di.chain_ctas_per_sm < 1) di.chain_ctas_per_sm = 1;
-        if (di.scatter_ctas_per_sm < 1) di.scatter_ctas_per_sm = 1;
-        if (di.index_ctas_per_sm < 1) di.index_ctas_per_sm = 1;
     }
     g_info[dev] = di;
     g_err[dev] = e;
@@ -129,19 +118,9 @@ dws_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? DWS_OK : DWS_E
 // a fraction u of the elements, about 1 - (1 - u)^16 of the sectors are
 // touched; above one half the merge moves fewer bytes, or about as many at a
 // better rate (whole-tile bulk copies against partial-sector writes).
-int32_t chain_auto_mode(const dws::DeltaRef *d, int32_t K, long long N) {
-    if (N <= 0) return DWS_CHAIN_SCATTER;
-    double keep = 1.0;  // fraction of elements no delta names (independent deltas)
-    for (int32_t k = 0; k < K; ++k) {
-        double f = double(d[k].count) / double(N);
-        if (f > 1.0) f = 1.0;
-        keep *= 1.0 - f;
-    }
-    double untouched_sector = 1.0;
-    for (int i = 0; i < 16; ++i) untouched_sector *= keep;
-    (void)untouched_sector;  // (the merge is not yet the faster mode at any density measured)
-    return DWS_CHAIN_SCATTER;
-}
+// The scatter moves only the touched sectors and was the faster mode on
+// every chain measured, dense or clustered.
+int32_t chain_auto_mode() { return DWS_CHAIN_SCATTER; }
 
 dws_status_t encode_common(const dws_plan_t *plan, const void *const *old_ptrs,
                            const void *const *new_ptrs, int64_t *offsets, int32_t *indices,
@@ -355,7 +334,7 @@ dws_status_t dws_apply_chain_ex(const dws_plan_t *plan, void *const *snap_ptrs,
                              reinterpret_cast<const int *>(deltas[k].indices), deltas[k].values,
                              deltas[k].count};
     }
-    if (mode == DWS_CHAIN_AUTO) mode = chain_auto_mode(d, K, plan->N);
+    if (mode == DWS_CHAIN_AUTO) mode = chain_auto_mode();
     return from_cuda(dws::launch_apply_chain(view_of(plan, workspace),
                                              reinterpret_cast<uint16_t *const *>(snap_ptrs), d, K,
                                              mode == DWS_CHAIN_TILE_MERGE,

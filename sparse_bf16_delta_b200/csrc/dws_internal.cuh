@@ -446,9 +446,6 @@ __device__ __forceinline__ unsigned long long pos_bytes_xor(uint32_t pos, int wi
 struct DeviceInfo {
     int sm_count;
     int encode_ctas_per_sm;
-    int chain_ctas_per_sm;
-    int scatter_ctas_per_sm;
-    int index_ctas_per_sm;
 };
 
 // Per-device constants and one-time kernel attribute setup (thread-safe).

@@ -424,7 +424,7 @@ def test_chain_on_unaligned_snapshots(dws, mode):
 def test_chain_max_length_tiny_and_empty_tensors(dws, mode):
     # 64 deltas (the maximum) of mixed densities, one of them empty, over a
     # plan of many tiny tensors, empty tensors and a few multi-tile ones, so
-    # that windows and CTA ranges cut through tensors and hold many of them.
+    # that index blocks cut through tensors and hold many of them.
     rng = np.random.default_rng(64)
     sizes = [0, 1, 5, 0, 8191, 8192, 8193, 3] + [int(x) for x in rng.integers(1, 600, 120)] + \
             [3 * 8192 + 17, 0, 300_001, 2, 70_000]
@@ -692,7 +692,7 @@ def test_xor_apply_layers_double_buffered(dws, pinned_masks):
 def _malformed_chain(rng, sizes):
     """Three deltas over `sizes` (dws layout, host arrays) and, for each, the
     mask of its entries that the pairwise rule flags: delta 0 holds descending
-    pairs (one inside a tile, one across tiles, one across 32-tile windows),
+    pairs (one inside a tile, one across adjacent tiles, one across distant tiles),
     delta 1 repeated indices, delta 2 is well formed.  Each flagged entry is
     followed by one above the entry before it, so no later entry of the
     segment lies at or below an earlier one except the flagged ones."""
@@ -705,8 +705,8 @@ def _malformed_chain(rng, sizes):
             b = [False] * len(pos)
             if k == 0 and t == 1:
                 # insert b < a right after a, then continue above a
-                # plan tiles: tensor 0 owns 0-6, so tensor 1's tile 25 opens
-                # the second 32-tile window
+                # the third pair reaches two tiles back (tensor 1's local
+                # tiles 25 and 23)
                 for a_at in (8195, 9000, 25 * 8192 + 10):
                     a_i = next(i for i, x in enumerate(pos) if x >= a_at)
                     below = pos[a_i] - (7 if a_at == 8195 else (5000 if a_at == 9000 else 8192 * 2))
@@ -727,7 +727,7 @@ def _malformed_chain(rng, sizes):
 
 
 def test_chain_with_unordered_or_repeated_entries_writes_nothing_in_every_mode(dws):
-    # Descending pairs (inside a tile, across tiles, across 32-tile windows)
+    # Descending pairs (inside a tile, across adjacent tiles, across distant tiles)
     # and repeated indices: every mode records DWS_ERR_BAD_DELTA and leaves
     # the snapshot exactly as it was; dws_apply, one delta at a time, skips
     # the flagged entries and applies the rest; without the malformed deltas
