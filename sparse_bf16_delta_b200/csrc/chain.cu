@@ -30,9 +30,20 @@ namespace {
 // ---------------------------------------------------------------------------
 // Tile index and validation
 // ---------------------------------------------------------------------------
+// Row g of the tile index, column k: the first entry of delta k at or past
+// the start of tile g (mod 2^32); row ntiles: the delta's entry count n.
+// With every entry valid the tiles of the entries never decrease, and
+//   rows of tensor t's tiles up to the tile of its first entry a: a,
+//   rows (tile of j-1, tile of j] for j inside t's segment: j,
+//   rows after the tile of t's last entry b-1, to t's last tile: b,
+//   all of t's rows when its segment is empty: a.
+// chain_index_ends_kernel writes the first, third and fourth kind (one
+// thread per tensor and delta), chain_index_kernel the second while it checks
+// every entry, so that no thread needs the tile of an entry of another tensor.
 constexpr int kIdxThreads = 256;
 constexpr int kIdxPerThread = 16;
-constexpr int kIdxChunk = kIdxThreads * kIdxPerThread;  // entries per block step
+constexpr int kIdxChunk = kIdxThreads * kIdxPerThread;  // entries per block
+constexpr int kEndsThreads = 256;
 
 struct IndexParams {
     WsView ws;
@@ -64,251 +75,288 @@ __device__ __forceinline__ void fill_rows(uint32_t *index, int col, long long lo
     }
 }
 
-// Tile of entry j (index i, tensor t), or -2 if i is outside the tensor.
-__device__ __forceinline__ long long entry_tile(const IndexParams &p, int t, int i) {
-    return (i >= 0 && static_cast<long long>(i) < p.ws.numel[t]) ? p.ws.first_tile[t] + (i >> kTileShift) : -2;
+__device__ __forceinline__ bool header_ok(const WsView &ws) {
+    const WsHeader *h = ws.hdr;
+    return h->magic == kWsMagic && h->fingerprint == ws.fingerprint && h->num_tiles == ws.num_tiles &&
+           h->num_tensors == ws.num_tensors;
 }
 
-// Block (x, k): entries [x * kIdxChunk, (x + 1) * kIdxChunk) of delta k,
-// 16 consecutive ones per thread.  Each thread checks its run (strictly
-// ascending, inside its tensor) and writes the index rows that start at its
-// entries: entry j starts rows (tile of entry j-1, tile of entry j], the last
-// entry also rows (its tile, ntiles] (at n).
+// Thread (t, k): the rows of tensor t's tiles before and after its segment
+// of delta k (the whole tensor if the segment is empty), and row ntiles.
+__global__ void __launch_bounds__(kEndsThreads) chain_index_ends_kernel(IndexParams p) {
+    const int lane = threadIdx.x & 31;
+    const int k = blockIdx.y;
+    const int T = p.ws.num_tensors;
+    const long long t = static_cast<long long>(blockIdx.x) * kEndsThreads + threadIdx.x;
+    if (!header_ok(p.ws) || ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) != 0u) return;  // uniform
+    const DeltaRef d = p.d[k];
+    const long long ntiles = p.ws.num_tiles;
+    if (t == 0) p.index[ntiles * kChainGroup + k] = static_cast<uint32_t>(d.offsets[T]);
+    long long lo1 = 0, hi1 = 0, lo2 = 0, hi2 = 0;  // rows (lo, hi]
+    uint32_t v1 = 0, v2 = 0;
+    if (t < T) {
+        const long long a = d.offsets[t], b = d.offsets[t + 1];
+        const long long f0 = p.ws.first_tile[t], f1 = p.ws.first_tile[t + 1];
+        if (a >= b) {
+            lo1 = f0 - 1;
+            hi1 = f1 - 1;
+            v1 = static_cast<uint32_t>(a);
+        } else {
+            // a bad index is flagged by the entry pass; here it only must
+            // not move the rows outside the tensor's own
+            long long ga = f0 + (static_cast<long long>(d.indices[a]) >> kTileShift);
+            long long gb = f0 + (static_cast<long long>(d.indices[b - 1]) >> kTileShift);
+            ga = ga < f0 - 1 ? f0 - 1 : (ga > f1 - 1 ? f1 - 1 : ga);
+            gb = gb < f0 - 1 ? f0 - 1 : (gb > f1 - 1 ? f1 - 1 : gb);
+            lo1 = f0 - 1;
+            hi1 = ga;
+            v1 = static_cast<uint32_t>(a);
+            lo2 = gb;
+            hi2 = f1 - 1;
+            v2 = static_cast<uint32_t>(b);
+        }
+    }
+    fill_rows(p.index, k, lo1, hi1, v1, lane, ntiles - 1);
+    fill_rows(p.index, k, lo2, hi2, v2, lane, ntiles - 1);
+}
+
+// Per delta, one level-by-level 32-way search over the offsets for the
+// tensor holding entry j (a non-empty one: the last t with offsets[t] <= j).
+// Lane 0 returns it with that tensor's segment [a, b), size and first tile,
+// read in the search's last level (lane c reads its candidate's).
+struct TensorMeta {
+    int t;
+    long long a, b, numel, first_tile;
+};
+__device__ __forceinline__ TensorMeta warp_tensor_meta(const WsView &ws, const long long *offsets, int T,
+                                                       long long j) {
+    const int lane = threadIdx.x & 31;
+    int lo = 0, hi = T - 1;  // the answer lies in [lo, hi]
+    while (true) {
+        const int span = hi - lo + 1;
+        const int step = (span + 31) / 32;
+        const int t = lo + lane * step;
+        const bool in = t <= hi;
+        const long long ot = in ? __ldg(offsets + t) : 0;
+        long long ob = 0, nm = 0, ft = 0;
+        if (step == 1 && in) {  // last level: the candidates' metadata too
+            ob = __ldg(offsets + t + 1);
+            nm = __ldg(ws.numel + t);
+            ft = __ldg(ws.first_tile + t);
+        }
+        const unsigned int bl = __ballot_sync(0xffffffffu, in && ot <= j);  // a prefix of lanes
+        const int c = bl ? __popc(bl) : 1;
+        if (step == 1) {
+            TensorMeta m;
+            m.t = lo + c - 1;
+            m.a = __shfl_sync(0xffffffffu, ot, c - 1);
+            m.b = __shfl_sync(0xffffffffu, ob, c - 1);
+            m.numel = __shfl_sync(0xffffffffu, nm, c - 1);
+            m.first_tile = __shfl_sync(0xffffffffu, ft, c - 1);
+            return m;
+        }
+        const int nlo = lo + (c - 1) * step;
+        const int nhi = lo + c * step - 1;
+        lo = nlo;
+        hi = nhi < hi ? nhi : hi;
+    }
+}
+
+// The rare paths of the index pass are kept out of line, so that the hot
+// one stays small in the instruction cache; they reload the thread's entries
+// (cache hits) instead of keeping them in registers.
+
+// The tensor holding entry j (a non-empty segment), searched in [lo, hi].
+__device__ __forceinline__ int tensor_in(const long long *offsets, int lo, int hi, long long j) {
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offsets[mid] <= j) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// A run across tensors, a short run, or one outside the block's first
+// tensor: every entry's tensor is walked.  Checks entries [j0, j0 + nlive),
+// writes the short gaps of rows (when `write`), sets bit q of *bigm for a
+// long one; returns the first offending entry, or -1.
+__device__ __noinline__ long long index_run_general(DeltaRef d, const long long *numel, const long long *first_tile,
+                                                    uint32_t *index, int T, int k, long long j0, int nlive,
+                                                    int t0, int t1, int write, unsigned int *bigm) {
+    int tq = tensor_in(d.offsets, t0, t1 > t0 ? t1 : t0, j0);
+    long long a = d.offsets[tq], b = d.offsets[tq + 1];
+    long long nm = numel[tq], ft = first_tile[tq];
+    int pv = j0 > 0 ? d.indices[j0 - 1] : 0;
+    for (int q = 0; q < nlive; ++q) {
+        const long long j = j0 + q;
+        while (j >= b && tq + 1 < T) {  // the next non-empty segment holding j
+            ++tq;
+            a = d.offsets[tq];
+            b = d.offsets[tq + 1];
+            nm = numel[tq];
+            ft = first_tile[tq];
+        }
+        const int i = d.indices[j];
+        const bool opens = j == a;
+        if (!(i >= 0 && i < nm && (opens || pv < i))) return j;
+        if (!opens && write) {
+            const int tp = pv >> kTileShift, tl = i >> kTileShift;
+            if (tl - tp > 32) {
+                *bigm |= 1u << q;
+            } else {
+                for (int g = tp + 1; g <= tl; ++g) index[(ft + g) * kChainGroup + k] = static_cast<uint32_t>(j);
+            }
+        }
+        pv = i;
+    }
+    return -1;
+}
+
+// The first offending entry of a run that lies in one tensor (numel nm,
+// opening its segment or not).
+__device__ __noinline__ long long index_first_bad(const int *indices, long long j0, int nm, bool opens) {
+    int pv = j0 > 0 ? indices[j0 - 1] : 0;
+    for (int q = 0; q < kIdxPerThread; ++q) {
+        const int i = indices[j0 + q];
+        if (!(i >= 0 && i < nm && ((q == 0 && opens) || pv < i))) return j0 + q;
+        pv = i;
+    }
+    return j0;
+}
+
+// Long gaps (more than 32 rows, sparse deltas): for each q, the lanes with
+// one at entry q write them together.  Every lane of the warp calls it.
+__device__ __noinline__ void index_long_gaps(DeltaRef d, const long long *first_tile, uint32_t *index, int k,
+                                             long long j0, unsigned int bigm, int t0, int t1, long long nrows) {
+    const int lane = threadIdx.x & 31;
+    for (int q = 0; q < kIdxPerThread; ++q) {
+        const bool mine = (bigm >> q) & 1u;
+        if (!__any_sync(0xffffffffu, mine)) continue;
+        long long lo = 0, hi = 0;
+        if (mine) {  // rows (tile of entry q-1, tile of entry q], both in one tensor
+            const long long j = j0 + q;
+            const long long ft = first_tile[tensor_in(d.offsets, t0, t1 > t0 ? t1 : t0, j)];
+            lo = ft + (d.indices[j - 1] >> kTileShift);
+            hi = ft + (d.indices[j] >> kTileShift);
+        }
+        fill_rows(index, k, lo, hi, static_cast<uint32_t>(j0 + q), lane, nrows);
+    }
+}
+
+// Block (x, k): entries [x * kIdxChunk, (x + 1) * kIdxChunk) of delta k, 16
+// consecutive ones per thread.  Every entry is checked (inside its tensor,
+// strictly above the entry before it in its tensor's segment) and, when the
+// index is written, entry j inside a segment writes rows (tile of j-1, tile
+// of j].  The header, the entries and the first level of the searches for
+// the tensors of the block's first and last entries are all requested at
+// once; the first tensor's metadata arrives with the search's last level.
 __global__ void __launch_bounds__(kIdxThreads, 4) chain_index_kernel(IndexParams p) {
-    __shared__ int s_t[2];
+    __shared__ TensorMeta s_m0;
+    __shared__ int s_t1;
+    __shared__ int s_ok;
+    __shared__ long long s_n;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = blockIdx.y;
     const DeltaRef d = p.d[k];
     const int T = p.ws.num_tensors;
     const long long ntiles = p.ws.num_tiles;
-    if (!ws_matches(p.ws)) return;
-    if (ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) != 0u) return;  // offsets failed: nothing else
-    const long long n = d.offsets[T];
     const long long base = static_cast<long long>(blockIdx.x) * kIdxChunk;
-    if (n == 0) {  // no entry: every row points at entry 0
-        if (p.write && blockIdx.x == 0 && warp == 0) fill_rows(p.index, k, -1, ntiles, 0u, lane, ntiles);
-        return;
-    }
-    if (base >= n) return;  // uniform
-    const long long last = (base + kIdxChunk < n ? base + kIdxChunk : n) - 1;
-    if (warp < 2) {  // tensors of the block's first and last entries
-        const int t = warp_tensor_of_entry(d.offsets, T, warp == 0 ? base : last);
-        if (lane == 0) s_t[warp] = t;
+    if (base >= d.count) return;  // uniform: past this delta's arrays
+    // the last entry the arrays hold in this block (the true last is <= it)
+    const long long last_a = (base + kIdxChunk < d.count ? base + kIdxChunk : d.count) - 1;
+
+    if (warp == 0) {
+        s_m0 = warp_tensor_meta(p.ws, d.offsets, T, base);
+    } else if (warp == 1) {
+        int lo = 0, hi = T - 1;  // tensor of last_a (an upper bound for the block's tensors)
+        while (true) {
+            const int span = hi - lo + 1;
+            const int step = (span + 31) / 32;
+            const int t = lo + lane * step;
+            const bool le = (t <= hi) && (__ldg(d.offsets + t) <= last_a);
+            const unsigned int bl = __ballot_sync(0xffffffffu, le);
+            const int c = bl ? __popc(bl) : 1;
+            if (step == 1) {
+                if (lane == 0) s_t1 = lo + c - 1;
+                break;
+            }
+            const int nlo = lo + (c - 1) * step, nhi = lo + c * step - 1;
+            lo = nlo;
+            hi = nhi < hi ? nhi : hi;
+        }
+    } else if (tid == 64) {
+        s_ok = header_ok(p.ws) && ld_relaxed_gpu_u32(&p.ws.hdr->delta_bad) == 0u;
+        s_n = d.offsets[T];
     }
     // this thread's entries and the one before them, in flight meanwhile
     const long long j0 = base + static_cast<long long>(tid) * kIdxPerThread;
-    const bool live0 = j0 <= last;
-    const int nlive = !live0 ? 0 : static_cast<int>(last - j0 + 1 < kIdxPerThread ? last - j0 + 1 : kIdxPerThread);
+    const int nload = j0 > last_a ? 0 : static_cast<int>(last_a - j0 + 1 < kIdxPerThread ? last_a - j0 + 1 : kIdxPerThread);
     int x[kIdxPerThread];
-    if (nlive == kIdxPerThread && (reinterpret_cast<uintptr_t>(d.indices) & 15u) == 0) {
+    if (nload == kIdxPerThread && (reinterpret_cast<uintptr_t>(d.indices) & 15u) == 0) {
 #pragma unroll
         for (int v = 0; v < kIdxPerThread / 4; ++v) {
-            const int4 a = __ldg(reinterpret_cast<const int4 *>(d.indices + j0) + v);
-            x[4 * v] = a.x; x[4 * v + 1] = a.y; x[4 * v + 2] = a.z; x[4 * v + 3] = a.w;
+            const int4 a4 = __ldg(reinterpret_cast<const int4 *>(d.indices + j0) + v);
+            x[4 * v] = a4.x; x[4 * v + 1] = a4.y; x[4 * v + 2] = a4.z; x[4 * v + 3] = a4.w;
         }
     } else {
 #pragma unroll
-        for (int q = 0; q < kIdxPerThread; ++q) x[q] = (q < nlive) ? __ldg(d.indices + j0 + q) : 0;
+        for (int q = 0; q < kIdxPerThread; ++q) x[q] = (q < nload) ? __ldg(d.indices + j0 + q) : 0;
     }
-    const int prev = (live0 && j0 > 0) ? __ldg(d.indices + j0 - 1) : 0;
+    const int prev = (nload > 0 && j0 > 0) ? __ldg(d.indices + j0 - 1) : 0;
     __syncthreads();
-    const int t0 = s_t[0], t1 = s_t[1];
+    if (!s_ok) {
+        if (tid == 0 && !header_ok(p.ws)) record_error(p.ws.hdr, DWS_ERR_WORKSPACE, 0);
+        return;  // uniform: a foreign workspace, or the offsets failed
+    }
+    const long long n = s_n;
+    if (base >= n) return;  // uniform
+    const TensorMeta m0 = s_m0;
+    const int t1 = s_t1;
+    const long long last = (base + kIdxChunk < n ? base + kIdxChunk : n) - 1;
+    const int nlive = j0 > last ? 0 : static_cast<int>(last - j0 + 1 < kIdxPerThread ? last - j0 + 1 : kIdxPerThread);
 
-    bool bad = false;
-    long long bad_j = 0;
-    long long glast = -2;  // tile of this thread's last entry
-    // The path is chosen per warp (both call warp-wide primitives): the fast
-    // one only if every lane's run qualifies.
-    const bool fast_lane = live0 && nlive == kIdxPerThread &&
-                           (t0 == t1 || d.offsets[t0 + 1] > j0 + kIdxPerThread - 1) && d.offsets[t0] <= j0;
-    if (__all_sync(0xffffffffu, fast_lane)) {
-        // Common case, 32-bit: the run lies in tensor t0.  It must ascend
+    long long bad_j = -1;
+    unsigned int bigm = 0;  // bit q: a long gap of rows ends at entry q
+    if (nlive == kIdxPerThread && m0.a <= j0 && j0 + kIdxPerThread - 1 < m0.b) {
+        // Common case, 32-bit: the run lies in tensor m0.t.  It must ascend
         // strictly (one compare per entry); then it is in range if its ends
-        // are.  The run's first entry may open t0's segment: no order check
-        // then, and its predecessor (another tensor's) bounds its rows.
-        const int t = t0;
-        const int nm = static_cast<int>(p.ws.numel[t]);
-        const long long ft = p.ws.first_tile[t];
-        const bool opens = d.offsets[t] == j0;
+        // are.  A run that opens the segment has no order check on its first
+        // entry and writes no rows for it (the ends kernel does).
+        const int nm = static_cast<int>(m0.numel);
+        const bool opens = m0.a == j0;
         bool viol = !opens && !(prev < x[0]);
 #pragma unroll
         for (int q = 1; q < kIdxPerThread; ++q) viol |= !(x[q - 1] < x[q]);
-        const bool ok = !viol && x[0] >= 0 && x[kIdxPerThread - 1] < nm;
-        if (!ok) {
-            // rare: the first offending entry (unrolled: x stays in registers)
-            unsigned int badm = 0;
+        if (viol || x[0] < 0 || x[kIdxPerThread - 1] >= nm) {
+            bad_j = index_first_bad(d.indices, j0, nm, opens);
+        } else if (p.write) {
+            const long long ft = m0.first_tile;
+            // any tile change in the run (or from the entry before it)?
+            int tp = opens ? (x[0] >> kTileShift) : (prev >> kTileShift);
+            if ((x[kIdxPerThread - 1] >> kTileShift) != tp) {
 #pragma unroll
-            for (int q = 0; q < kIdxPerThread; ++q) {
-                const int pv = q == 0 ? prev : x[q - 1];
-                const bool e_ok = x[q] >= 0 && x[q] < nm && ((q == 0 && opens) || pv < x[q]);
-                badm |= e_ok ? 0u : (1u << q);
-            }
-            bad = true;
-            bad_j = j0 + (badm ? __ffs(badm) - 1 : 0);
-        }
-        glast = ok ? ft + (x[kIdxPerThread - 1] >> kTileShift) : -2;
-        if (p.write) {
-            // the tile of the entry before the run: this tensor's, or, when
-            // the run opens the segment, found by a search (once per tensor)
-            long long gprev = -1;
-            if (j0 > 0) {
-                if (!opens) {
-                    gprev = ft + (prev >> kTileShift);
-                } else {
-                    int lo = 0, hi = t;  // the tensor of entry j0 - 1
-                    while (lo < hi) {
-                        const int mid = (lo + hi + 1) >> 1;
-                        if (d.offsets[mid] <= j0 - 1) lo = mid;
-                        else hi = mid - 1;
-                    }
-                    gprev = entry_tile(p, lo, prev);
-                }
-            }
-            // Rows (tile of entry q-1, tile of entry q] start at entry q, and
-            // after the delta's last entry rows (its tile, ntiles] at n.  Each
-            // lane writes its own short runs of rows (one row, usually);
-            // runs longer than 32 rows (sparse deltas) are written by the
-            // whole warp afterwards.  Bit 16 of `bigm` is the tail.
-            unsigned int bigm = 0;
-            const bool tail = ok && j0 + kIdxPerThread - 1 == n - 1;
-            if (ok && gprev >= -1) {
-                const long long g0 = ft + (x[0] >> kTileShift);
-                if (g0 > gprev) {
-                    if (g0 - gprev <= 32) {
-                        for (long long g = gprev + 1; g <= g0; ++g)
-                            p.index[g * kChainGroup + k] = static_cast<uint32_t>(j0);
-                    } else {
-                        bigm |= 1u;
-                    }
-                }
-                int tp = x[0] >> kTileShift;
-#pragma unroll
-                for (int q = 1; q < kIdxPerThread; ++q) {
+                for (int q = 0; q < kIdxPerThread; ++q) {
                     const int tl = x[q] >> kTileShift;
                     if (tl != tp) {
                         if (tl - tp <= 32) {
-                            for (long long g = ft + tp + 1; g <= ft + tl; ++g)
-                                p.index[g * kChainGroup + k] = static_cast<uint32_t>(j0 + q);
+                            for (int g = tp + 1; g <= tl; ++g)
+                                p.index[(ft + g) * kChainGroup + k] = static_cast<uint32_t>(j0 + q);
                         } else {
                             bigm |= 1u << q;
                         }
                     }
                     tp = tl;
                 }
-                if (tail) {
-                    if (ntiles - glast <= 32) {
-                        for (long long g = glast + 1; g <= ntiles; ++g)
-                            p.index[g * kChainGroup + k] = static_cast<uint32_t>(n);
-                    } else {
-                        bigm |= 1u << 16;
-                    }
-                }
-            }
-            while (__any_sync(0xffffffffu, bigm != 0u)) {
-                // one long run per lane per round, the warp writing together
-                long long lo = 0, hi = 0;
-                uint32_t v = 0;
-                if (bigm != 0u) {
-                    const int q = __ffs(bigm) - 1;
-                    bigm &= bigm - 1;
-                    if (q == 16) {
-                        lo = glast;
-                        hi = ntiles;
-                        v = static_cast<uint32_t>(n);
-                    } else {
-                        int xi = 0, xp = 0;
-#pragma unroll
-                        for (int r = 0; r < kIdxPerThread; ++r) {
-                            if (r == q) xi = x[r];
-                            if (r == q - 1) xp = x[r];
-                        }
-                        hi = ft + (xi >> kTileShift);
-                        lo = (q == 0) ? gprev : ft + (xp >> kTileShift);
-                        v = static_cast<uint32_t>(j0 + q);
-                    }
-                }
-                fill_rows(p.index, k, lo, hi, v, lane, ntiles);
             }
         }
-    } else {
-        // General case (a run across tensors, a short run, or a block that
-        // the search placed oddly): every entry's tensor is walked.
-        long long g[kIdxPerThread];
-        unsigned int okm = 0;  // bit q: entry q in range and ordered
-        long long gprev0 = -1;  // tile of the entry before the run
-        int tq = t0;
-        if (live0) {
-            int lo = t0, hi = t1;  // the tensor of entry j0
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (d.offsets[mid] <= j0) lo = mid;
-                else hi = mid - 1;
-            }
-            tq = lo;
-            if (j0 > 0) {
-                int tp = tq;
-                if (d.offsets[tq] > j0 - 1 || d.offsets[tq] == j0) {
-                    int a = 0, b = tq;  // the tensor of entry j0 - 1
-                    while (a < b) {
-                        const int mid = (a + b + 1) >> 1;
-                        if (d.offsets[mid] <= j0 - 1) a = mid;
-                        else b = mid - 1;
-                    }
-                    tp = a;
-                }
-                gprev0 = entry_tile(p, tp, prev);
-            }
-        }
-        int pv = prev;
-#pragma unroll
-        for (int q = 0; q < kIdxPerThread; ++q) {
-            const long long j = j0 + q;
-            g[q] = -2;
-            if (q < nlive) {
-                while (d.offsets[tq + 1] <= j) ++tq;  // empty tensors are skipped too
-                const int i = x[q];
-                const bool ord = j == d.offsets[tq] || pv < i;
-                g[q] = entry_tile(p, tq, i);
-                okm |= (g[q] >= 0 && ord) ? (1u << q) : 0u;
-            }
-            pv = x[q];
-        }
-        const unsigned int livem = (1u << nlive) - 1u;
-        const unsigned int badm = livem & ~okm;
-        if (badm != 0u) {
-            bad = true;
-            bad_j = j0 + (__ffs(badm) - 1);
-        }
-#pragma unroll
-        for (int r = 0; r < kIdxPerThread; ++r)
-            if (r == nlive - 1) glast = g[r];
-        if (p.write) {
-            unsigned int bnd = 0;
-            long long gp = gprev0;
-#pragma unroll
-            for (int q = 0; q < kIdxPerThread; ++q) {
-                if (((livem >> q) & 1u) && g[q] >= 0 && gp >= -1 && g[q] > gp) bnd |= 1u << q;
-                if ((livem >> q) & 1u) gp = g[q];
-            }
-            const bool tail = nlive > 0 && j0 + nlive - 1 == n - 1 && glast >= 0;
-            unsigned int any_q = __reduce_or_sync(0xffffffffu, bnd);
-            while (any_q != 0u) {
-                const int q = __ffs(any_q) - 1;
-                any_q &= any_q - 1;
-                long long lo = gprev0, gq = 0;
-#pragma unroll
-                for (int r = 0; r < kIdxPerThread; ++r) {
-                    if (r < q && ((livem >> r) & 1u)) lo = g[r];
-                    if (r == q) gq = g[r];
-                }
-                const bool mine = (bnd >> q) & 1u;
-                fill_rows(p.index, k, mine ? lo : 0, mine ? gq : 0, static_cast<uint32_t>(j0 + q), lane, ntiles);
-            }
-            if (__any_sync(0xffffffffu, tail))
-                fill_rows(p.index, k, tail ? glast : 0, tail ? ntiles : 0, static_cast<uint32_t>(n), lane, ntiles);
-        }
+    } else if (nlive > 0) {
+        bad_j = index_run_general(d, p.ws.numel, p.ws.first_tile, p.index, T, k, j0, nlive, m0.t, t1, p.write,
+                                  &bigm);
     }
-    if (bad) {
+    if (bad_j >= 0) bigm = 0;
+    if (__any_sync(0xffffffffu, bigm != 0u))
+        index_long_gaps(d, p.ws.first_tile, p.index, k, j0, bigm, m0.t, t1, ntiles - 1);
+    if (bad_j >= 0) {
         atomicOr(&p.ws.hdr->delta_bad, 1u);
         record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, bad_j);
     }
@@ -340,8 +388,8 @@ struct TileShared {
     const uint16_t *vp[kChainGroup];
     int lo[kChainGroup];
     int hi[kChainGroup];
-    long long lim[kChainGroup];
-    int vec[kChainGroup];                       // 16-byte loads allowed (aligned arrays)
+    int vlim[kChainGroup];                      // 16-byte loads at offsets below this (aligned
+                                                // arrays, 4 entries inside them)
     int C[kChainGroup + 1];                     // items of the deltas before k
     uint16_t *dst;                              // tile start in the snapshot (null: skip)
     int local;                                  // tile start within its tensor
@@ -379,11 +427,14 @@ __device__ __forceinline__ void tile_load_round(const TileShared &sm, int K, int
             kq[q] = k;
             const int o = (i - sm.C[k]) * kItemEntries + 4 * lane;
             const int lo = sm.lo[k], hi = sm.hi[k];
-            unsigned int m = 0u;
+            unsigned int m = 0xfu;
+            if (o < lo || o + 4 > hi) {  // an item's ends only
+                m = 0u;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) m |= (o + e >= lo && o + e < hi) ? (1u << e) : 0u;
+                for (int e = 0; e < 4; ++e) m |= (o + e >= lo && o + e < hi) ? (1u << e) : 0u;
+            }
             vm[q] = m;
-            if (m == 0xfu && sm.vec[k] && o + 3 < sm.lim[k]) {
+            if (o < sm.vlim[k]) {  // entries outside [lo, hi) are loaded and not used
                 ix[q] = __ldg(reinterpret_cast<const int4 *>(sm.ip[k] + o));
                 vx[q] = __ldg(reinterpret_cast<const uint2 *>(sm.vp[k] + o));
             } else if (m != 0u) {
@@ -463,9 +514,10 @@ __global__ void __launch_bounds__(kTileThreads, kTileMinBlocks) chain_tile_kerne
             sm.vp[lane] = d.values + base;
             sm.lo[lane] = static_cast<int>(s - base);
             sm.hi[lane] = static_cast<int>(s - base) + n;
-            sm.lim[lane] = d.count - base;
-            sm.vec[lane] = ((reinterpret_cast<uintptr_t>(d.indices) & 15u) == 0 &&
-                            (reinterpret_cast<uintptr_t>(d.values) & 7u) == 0) ? 1 : 0;
+            const bool vec = (reinterpret_cast<uintptr_t>(d.indices) & 15u) == 0 &&
+                             (reinterpret_cast<uintptr_t>(d.values) & 7u) == 0;
+            const long long room = d.count - base - 3;  // offsets o with o + 3 inside the arrays
+            sm.vlim[lane] = !vec ? 0 : static_cast<int>(room < (1LL << 30) ? (room > 0 ? room : 0) : (1LL << 30));
         }
         // items of delta k: ceil(hi / 128), none if it has no entry here
         int pre = n > 0 ? (static_cast<int>(s & 3LL) + n + kItemEntries - 1) / kItemEntries : 0;
@@ -527,22 +579,25 @@ __global__ void __launch_bounds__(kTileThreads, kTileMinBlocks) chain_tile_kerne
         }
     }
     __syncthreads();  // tags initialised
+    bool outside = false;  // an entry outside the tile: never, for checked entries
     for (int r = 0; r < rounds; ++r) {
         if (r > 0) tile_load_round(sm, K, r, ix, vx, kq, vm);
 #pragma unroll
         for (int q = 0; q < kTileItems; ++q) {
+            if (kq[q] < 0) continue;  // warp-uniform
             const uint32_t ver = static_cast<uint32_t>(kq[q] + 1) << 16;
+            const unsigned int m = vm[q];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                if ((vm[q] >> e) & 1u) {
-                    // position within the tile; checked entries never fall outside
-                    const uint32_t pos = static_cast<uint32_t>(int4_at(ix[q], e) - local);
-                    if (pos < static_cast<uint32_t>(count)) atomicMax(&s_tag[pos], ver | u16x4_at(vx[q], e));
-                    else record_error(p.ws.hdr, DWS_ERR_WORKSPACE, g);
-                }
+                const uint32_t pos = static_cast<uint32_t>(int4_at(ix[q], e) - local);
+                const bool use = (m == 0xfu) || ((m >> e) & 1u);
+                const bool in = pos < static_cast<uint32_t>(count);
+                if (use && in) atomicMax(&s_tag[pos], ver | u16x4_at(vx[q], e));
+                outside |= use && !in;
             }
         }
     }
+    if (outside) record_error(p.ws.hdr, DWS_ERR_WORKSPACE, g);
     __syncthreads();
     if constexpr (kMerge) {
         if (vec) {
@@ -614,6 +669,10 @@ cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs, con
         const long long gx = index_grid(deltas + k0, kg, ip);
         if (gx > 0x7fffffffLL) return cudaErrorInvalidValue;
         chain_index_kernel<<<dim3(static_cast<unsigned int>(gx), kg), kIdxThreads, 0, s>>>(ip);
+        e = launched();
+        if (e != cudaSuccess) return e;
+        const long long ex = (static_cast<long long>(ws.num_tensors) + kEndsThreads - 1) / kEndsThreads;
+        chain_index_ends_kernel<<<dim3(static_cast<unsigned int>(ex), kg), kEndsThreads, 0, s>>>(ip);
         e = launched();
         if (e != cudaSuccess) return e;
         TileParams tp;
