@@ -407,13 +407,22 @@ def touched_sectors(offsets, indices):
     return n
 
 
-def sector_model(nnz, sectors, ms, peak):
-    """The apply's DRAM traffic model: 6 bytes read per entry, and every
-    touched 32-byte sector read and written back whole by L2 (HBM has no
-    byte-masked writes): 6 nnz + 64 S bytes."""
-    b = 6 * nnz + 64 * sectors
-    return {"sectors": sectors, "sector_model_bytes": b,
-            "sector_model_GBps": round(b / ms / 1e6, 1), "sector_model_frac": round(b / ms / 1e6 / peak, 4)}
+def clean_bytes(nnz, dev):
+    """What dws_apply reads before its scatter: the delta arrays' first bytes,
+    twice the L2 size at most (indices, then values)."""
+    import torch
+    budget = 2 * torch.cuda.get_device_properties(dev).L2_cache_size
+    ib = min(4 * nnz, budget)
+    return ib + min(2 * nnz, budget - ib)
+
+
+def sector_model(nnz, sectors, ms, peak, pre=0):
+    """The apply's DRAM traffic model: 6 bytes read per entry, every touched
+    32-byte sector read and written back whole by L2 (HBM has no byte-masked
+    writes), and the `pre` bytes read before the scatter: 6 nnz + 64 S + pre."""
+    b = 6 * nnz + 64 * sectors + pre
+    return {"sectors": sectors, "traffic_model_bytes": b, "traffic_model_pre_read_bytes": pre,
+            "traffic_model_GBps": round(b / ms / 1e6, 1), "traffic_model_frac": round(b / ms / 1e6 / peak, 4)}
 
 
 def row(name, ms, alg_bytes, weight_bytes, peak, extra=None, elems=None):
@@ -989,7 +998,7 @@ def run_ours(args):
                       "weight_GBps": round(weight_bytes / app_ms / 1e6, 1),
                       "elems_per_s": round(N / app_ms * 1e3, 1),
                       "entries_per_s": round(nnz / app_ms * 1e3, 1),
-                      **sector_model(nnz, app_sectors, app_ms, peak)},
+                      **sector_model(nnz, app_sectors, app_ms, peak, clean_bytes(nnz, dev))},
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -1118,7 +1127,7 @@ def run_ours(args):
                          {"min_ms": round(mn_e, 4), "nnz": nnz2, "sparsity": round(1 - nnz2 / N, 6)})])
         rows.update([row("apply_llama3_8b_lr1e-5", ms_a, 8 * nnz2, weight_bytes, peak,
                          {"min_ms": round(mn_a, 4), "exact": ok, "entries_per_s": round(nnz2 / ms_a * 1e3, 1),
-                          **sector_model(nnz2, touched_sectors(offs2, idx2), ms_a, peak)})])
+                          **sector_model(nnz2, touched_sectors(offs2, idx2), ms_a, peak, clean_bytes(nnz2, dev))})])
         # wire form of the same delta: positions block (2 or 4 bytes each) and checksum
         pcap = 4 * nnz2
         positions = torch.empty(max(2, pcap), dtype=torch.uint8, device=dev)

@@ -290,7 +290,11 @@ DWS_API dws_status_t dws_encode_noalloc(const int64_t *numels, int32_t num_tenso
  *   snapshots, modified in place.
  * offsets, indices, values: one delta in the dws_encode layout (device).
  * count: number of entries the index/value arrays hold (host value, usually
- *   nnz).  Entries j >= min(count, offsets[T]) are never read.
+ *   nnz).  Entries j >= min(count, offsets[T]) are never applied.  Before the
+ *   scatter the arrays' first bytes (twice the L2 size at most, within count
+ *   entries) are read once, which writes back the dirty lines an earlier
+ *   kernel or copy left in L2 (scattered partial writes run slower among
+ *   them).
  * Every index is range-checked against its tensor's numel and required to be
  * ascending within its tensor; a violating entry is skipped and
  * DWS_ERR_BAD_DELTA recorded (detail = entry number).  offsets must start at

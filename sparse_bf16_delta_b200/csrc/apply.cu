@@ -11,6 +11,11 @@
 //   the touched 32-byte sectors (read-modify-write in L2) plus 6 bytes per
 //   entry, which is less than streaming the snapshot through at the
 //   densities the workloads have.
+//   Before the scatter, l2_clean_kernel reads the first 2 x L2-size bytes of
+//   the delta's own arrays: that writes back the dirty lines an earlier
+//   kernel or copy left in L2.  Partial-sector writes landing in an L2 full
+//   of dirty lines ran 15% slower (3.2 -> 3.7 ms for 283 M entries after any
+//   write of 64 MB or more, even 10 ms later); the read costs about 0.07 ms.
 //
 // The replay of a chain of deltas is in chain.cu.
 #include <cuda_runtime.h>
@@ -136,6 +141,37 @@ __global__ void __launch_bounds__(kApplyThreads) apply_kernel(ApplyParams p) {
     }
 }
 
+// Reads [a, a + abytes) and [b, b + bbytes) once (their 16-byte aligned
+// interiors): lines read in evict the dirty lines L2 holds.  The loaded words
+// are folded into a value that decides a store (taken with probability
+// 2^-32, and harmless), so that the loads are not dropped as dead.
+constexpr int kCleanThreads = 512;
+__device__ unsigned int g_clean_sink;
+__device__ __forceinline__ uint32_t fold_range(const unsigned char *a, long long bytes) {
+    uint32_t acc = 0u;
+    if (bytes <= 0) return acc;
+    const uintptr_t lo = (reinterpret_cast<uintptr_t>(a) + 15u) & ~static_cast<uintptr_t>(15u);
+    const uintptr_t hi = (reinterpret_cast<uintptr_t>(a) + static_cast<uintptr_t>(bytes)) & ~static_cast<uintptr_t>(15u);
+    if (hi <= lo) return acc;
+    const uint4 *v = reinterpret_cast<const uint4 *>(lo);
+    const long long n = static_cast<long long>((hi - lo) >> 4);
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += 4 * stride) {
+        uint4 w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) w[u] = i + u * stride < n ? v[i + u * stride] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc ^= w[u].x ^ w[u].y ^ w[u].z ^ w[u].w;
+    }
+    return acc;
+}
+__global__ void __launch_bounds__(kCleanThreads) l2_clean_kernel(const unsigned char *a, long long abytes,
+                                                                 const unsigned char *b, long long bbytes,
+                                                                 uint32_t key) {
+    const uint32_t acc = fold_range(a, abytes) ^ fold_range(b, bbytes);
+    if (acc == key) g_clean_sink = acc;  // harmless when it happens
+}
+
 }  // namespace
 
 cudaError_t launch_delta_flag_clear(const WsView &ws, cudaStream_t s) {
@@ -159,6 +195,21 @@ cudaError_t launch_apply(const WsView &ws, uint16_t *const *snap_ptrs, const Del
     cudaError_t e = launch_delta_check(ws, &d, 1, s);
     if (e != cudaSuccess) return e;
     if (d.count <= 0) return cudaSuccess;
+    DeviceInfo di;
+    e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    {  // the arrays' first 2 x L2 bytes, indices first
+        const long long budget = 2 * di.l2_bytes;
+        const long long ib = 4 * d.count < budget ? 4 * d.count : budget;
+        const long long rest = budget - ib;
+        const long long vb = 2 * d.count < rest ? 2 * d.count : rest;
+        const int grid = di.sm_count * 4;
+        l2_clean_kernel<<<grid, kCleanThreads, 0, s>>>(reinterpret_cast<const unsigned char *>(d.indices), ib,
+                                                       reinterpret_cast<const unsigned char *>(d.values), vb,
+                                                       0x9e3779b9u);
+        e = launched();
+        if (e != cudaSuccess) return e;
+    }
     ApplyParams p;
     p.ws = ws;
     p.snap_ptrs = snap_ptrs;

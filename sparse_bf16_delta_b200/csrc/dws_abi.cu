@@ -25,6 +25,9 @@ cudaError_t g_err[kMaxDevices];
 void init_device(int dev) {
     DeviceInfo di{};
     cudaError_t e = cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    int l2 = 0;
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev);
+    di.l2_bytes = l2;
     if (e == cudaSuccess) e = encode_set_attributes();
     if (e == cudaSuccess) e = encode_occupancy(&di.encode_ctas_per_sm);
     if (e == cudaSuccess) {

@@ -446,6 +446,7 @@ __device__ __forceinline__ unsigned long long pos_bytes_xor(uint32_t pos, int wi
 struct DeviceInfo {
     int sm_count;
     int encode_ctas_per_sm;
+    long long l2_bytes;
 };
 
 // Per-device constants and one-time kernel attribute setup (thread-safe).
