@@ -224,6 +224,28 @@ __device__ __noinline__ long long index_first_bad(const int *indices, long long 
     return j0;
 }
 
+// The rows a checked run inside one tensor starts (it crosses a tile, or
+// follows an entry in another tile): short gaps written here, long ones
+// marked in the returned mask.  Out of line: about one run in twenty
+// crosses a tile at the densities of the workloads.
+__device__ __noinline__ unsigned int index_run_rows(const int *indices, uint32_t *index, int k, long long j0,
+                                                    long long ft, bool opens) {
+    unsigned int bigm = 0;
+    int tp = (opens ? indices[j0] : indices[j0 - 1]) >> kTileShift;
+    for (int q = 0; q < kIdxPerThread; ++q) {
+        const int tl = indices[j0 + q] >> kTileShift;
+        if (tl != tp) {
+            if (tl - tp <= 32) {
+                for (int g = tp + 1; g <= tl; ++g) index[(ft + g) * kChainGroup + k] = static_cast<uint32_t>(j0 + q);
+            } else {
+                bigm |= 1u << q;
+            }
+        }
+        tp = tl;
+    }
+    return bigm;
+}
+
 // Long gaps (more than 32 rows, sparse deltas): for each q, the lanes with
 // one at entry q write them together.  Every lane of the warp calls it.
 __device__ __noinline__ void index_long_gaps(DeltaRef d, const long long *first_tile, uint32_t *index, int k,
@@ -250,7 +272,7 @@ __device__ __noinline__ void index_long_gaps(DeltaRef d, const long long *first_
 // of j].  The header, the entries and the first level of the searches for
 // the tensors of the block's first and last entries are all requested at
 // once; the first tensor's metadata arrives with the search's last level.
-__global__ void __launch_bounds__(kIdxThreads, 4) chain_index_kernel(IndexParams p) {
+__global__ void __launch_bounds__(kIdxThreads, 6) chain_index_kernel(IndexParams p) {
     __shared__ TensorMeta s_m0;
     __shared__ int s_t1;
     __shared__ int s_ok;
@@ -330,24 +352,10 @@ __global__ void __launch_bounds__(kIdxThreads, 4) chain_index_kernel(IndexParams
         if (viol || x[0] < 0 || x[kIdxPerThread - 1] >= nm) {
             bad_j = index_first_bad(d.indices, j0, nm, opens);
         } else if (p.write) {
-            const long long ft = m0.first_tile;
             // any tile change in the run (or from the entry before it)?
-            int tp = opens ? (x[0] >> kTileShift) : (prev >> kTileShift);
-            if ((x[kIdxPerThread - 1] >> kTileShift) != tp) {
-#pragma unroll
-                for (int q = 0; q < kIdxPerThread; ++q) {
-                    const int tl = x[q] >> kTileShift;
-                    if (tl != tp) {
-                        if (tl - tp <= 32) {
-                            for (int g = tp + 1; g <= tl; ++g)
-                                p.index[(ft + g) * kChainGroup + k] = static_cast<uint32_t>(j0 + q);
-                        } else {
-                            bigm |= 1u << q;
-                        }
-                    }
-                    tp = tl;
-                }
-            }
+            const int tp = opens ? (x[0] >> kTileShift) : (prev >> kTileShift);
+            if ((x[kIdxPerThread - 1] >> kTileShift) != tp)
+                bigm = index_run_rows(d.indices, p.index, k, j0, m0.first_tile, opens);
         }
     } else if (nlive > 0) {
         bad_j = index_run_general(d, p.ws.numel, p.ws.first_tile, p.index, T, k, j0, nlive, m0.t, t1, p.write,
