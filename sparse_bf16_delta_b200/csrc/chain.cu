@@ -376,8 +376,7 @@ __global__ void __launch_bounds__(kIdxThreads, 6) chain_index_kernel(IndexParams
 constexpr int kTileThreads = 256;
 constexpr int kTileWarps = kTileThreads / 32;
 constexpr int kItemEntries = 128;                         // 4 consecutive entries per lane
-constexpr int kTileItems = 3;                             // items per warp per round
-constexpr int kTileRoundItems = kTileWarps * kTileItems;  // items per round
+constexpr int kTileItems = 2;                             // items per warp per round
 constexpr int kTileMinBlocks = 6;
 
 struct TileParams {
@@ -412,47 +411,66 @@ __device__ __forceinline__ uint32_t u16x4_at(const uint2 &v, int e) {
     return (e & 1) ? (w >> 16) : (w & 0xffffu);
 }
 
-// Round r of this warp's items: item i = r * kTileRoundItems + warp + q *
-// kTileWarps covers entries base + 128 c + [0, 128) of delta k (c = i -
-// C[k]); lane l takes the 4 entries from base + 128 c + 4 l.  kq[q] = k
-// (warp-uniform; -1: no such item); vm[q] bit e: entry e is the tile's.
-// Every load of the round is in flight at once.
-__device__ __forceinline__ void tile_load_round(const TileShared &sm, int K, int r, int4 (&ix)[kTileItems],
-                                                uint2 (&vx)[kTileItems], int (&kq)[kTileItems],
-                                                unsigned int (&vm)[kTileItems]) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int i0 = r * kTileRoundItems + warp;
-    const int items = sm.C[K];
-    int k = 0;
-    while (k + 1 < K && sm.C[k + 1] <= i0) ++k;
+// A warp's position in the tile's item list: item i of delta k covers
+// entries base + 128 (i - C[k]) + [0, 128); the delta's constants are kept in
+// registers and reread only when the warp moves on to the next delta.
+struct ItemCursor {
+    int k, ck, cn;  // delta, C[k], C[k + 1]
+    int lo, hi, vlim;
+    const int *ip;
+    const uint16_t *vp;
+};
+
+__device__ __forceinline__ void cursor_load(const TileShared &sm, ItemCursor &c) {
+    c.ck = sm.C[c.k];
+    c.cn = sm.C[c.k + 1];
+    c.lo = sm.lo[c.k];
+    c.hi = sm.hi[c.k];
+    c.vlim = sm.vlim[c.k];
+    c.ip = sm.ip[c.k];
+    c.vp = sm.vp[c.k];
+}
+
+// Items i0 .. i0 + kTileItems - 1 of this warp (those below iend; the warp
+// takes its items in order): lane l takes the 4 entries from base + 128 c +
+// 4 l.  kq[q] = k (warp-uniform; -1: no such item); vm[q] bit e: entry e is
+// the tile's.  Every load of the round is in flight at once.
+__device__ __forceinline__ void tile_load_round(const TileShared &sm, int K, ItemCursor &c, int i0, int iend,
+                                                int4 (&ix)[kTileItems], uint2 (&vx)[kTileItems],
+                                                int (&kq)[kTileItems], unsigned int (&vm)[kTileItems]) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int q = 0; q < kTileItems; ++q) {
-        const int i = i0 + q * kTileWarps;
+        const int i = i0 + q;
         kq[q] = -1;
         vm[q] = 0u;
-        if (i < items) {  // warp-uniform
-            while (k + 1 < K && sm.C[k + 1] <= i) ++k;
-            kq[q] = k;
-            const int o = (i - sm.C[k]) * kItemEntries + 4 * lane;
-            const int lo = sm.lo[k], hi = sm.hi[k];
+        if (i < iend) {  // warp-uniform
+            if (i >= c.cn) {  // the next delta with items (C[K] > i, so k stays below K)
+                do {
+                    ++c.k;
+                } while (c.k + 1 < K && sm.C[c.k + 1] <= i);
+                cursor_load(sm, c);
+            }
+            kq[q] = c.k;
+            const int o = (i - c.ck) * kItemEntries + 4 * lane;
             unsigned int m = 0xfu;
-            if (o < lo || o + 4 > hi) {  // an item's ends only
+            if (o < c.lo || o + 4 > c.hi) {  // an item's ends only
                 m = 0u;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) m |= (o + e >= lo && o + e < hi) ? (1u << e) : 0u;
+                for (int e = 0; e < 4; ++e) m |= (o + e >= c.lo && o + e < c.hi) ? (1u << e) : 0u;
             }
             vm[q] = m;
-            if (o < sm.vlim[k]) {  // entries outside [lo, hi) are loaded and not used
-                ix[q] = __ldg(reinterpret_cast<const int4 *>(sm.ip[k] + o));
-                vx[q] = __ldg(reinterpret_cast<const uint2 *>(sm.vp[k] + o));
+            if (o < c.vlim) {  // entries outside [lo, hi) are loaded and not used
+                ix[q] = __ldg(reinterpret_cast<const int4 *>(c.ip + o));
+                vx[q] = __ldg(reinterpret_cast<const uint2 *>(c.vp + o));
             } else if (m != 0u) {
                 int xs[4] = {0, 0, 0, 0};
                 uint32_t vs[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     if ((m >> e) & 1u) {
-                        xs[e] = __ldg(sm.ip[k] + o + e);
-                        vs[e] = __ldg(sm.vp[k] + o + e);
+                        xs[e] = __ldg(c.ip + o + e);
+                        vs[e] = __ldg(c.vp + o + e);
                     }
                 }
                 ix[q] = make_int4(xs[0], xs[1], xs[2], xs[3]);
@@ -563,12 +581,19 @@ __global__ void __launch_bounds__(kTileThreads, kTileMinBlocks) chain_tile_kerne
     const int local = sm.local, count = sm.count;
     const bool vec = count == kTileElems && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0;
 
-    const int rounds = (items + kTileRoundItems - 1) / kTileRoundItems;
+    // this warp's items: a contiguous range, in rounds of kTileItems
+    const int warp = tid >> 5;
+    const int per = (items + kTileWarps - 1) / kTileWarps;
+    const int ib = warp * per < items ? warp * per : items;
+    const int ie = ib + per < items ? ib + per : items;
+    ItemCursor cur;
+    cur.k = 0;
+    cursor_load(sm, cur);
     int4 ix[kTileItems];
     uint2 vx[kTileItems];
     int kq[kTileItems];
     unsigned int vm[kTileItems];
-    tile_load_round(sm, K, 0, ix, vx, kq, vm);
+    tile_load_round(sm, K, cur, ib, ie, ix, vx, kq, vm);
     if constexpr (kMerge) {
         // tags <- the tile's values (version 0), while the entries arrive
         if (vec) {
@@ -588,8 +613,8 @@ __global__ void __launch_bounds__(kTileThreads, kTileMinBlocks) chain_tile_kerne
     }
     __syncthreads();  // tags initialised
     bool outside = false;  // an entry outside the tile: never, for checked entries
-    for (int r = 0; r < rounds; ++r) {
-        if (r > 0) tile_load_round(sm, K, r, ix, vx, kq, vm);
+    for (int i0 = ib; i0 < ie; i0 += kTileItems) {
+        if (i0 > ib) tile_load_round(sm, K, cur, i0, ie, ix, vx, kq, vm);
 #pragma unroll
         for (int q = 0; q < kTileItems; ++q) {
             if (kq[q] < 0) continue;  // warp-uniform
