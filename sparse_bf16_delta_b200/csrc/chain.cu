@@ -224,24 +224,23 @@ __device__ __noinline__ long long index_first_bad(const int *indices, long long 
     return j0;
 }
 
-// The rows a checked run inside one tensor starts (it crosses a tile, or
-// follows an entry in another tile): short gaps written here, long ones
-// marked in the returned mask.  Out of line: about one run in twenty
-// crosses a tile at the densities of the workloads.
+// The rows a checked run inside one tensor starts: bit q of `bnd` marks an
+// entry j0 + q in a later tile than the entry before it (both in this
+// tensor).  Short gaps are written here, long ones returned as a mask.  Out
+// of line, and only the marked entries are reread: at the densities of the
+// workloads a run crosses a tile about once in twenty.
 __device__ __noinline__ unsigned int index_run_rows(const int *indices, uint32_t *index, int k, long long j0,
-                                                    long long ft, bool opens) {
+                                                    long long ft, unsigned int bnd) {
     unsigned int bigm = 0;
-    int tp = (opens ? indices[j0] : indices[j0 - 1]) >> kTileShift;
-    for (int q = 0; q < kIdxPerThread; ++q) {
-        const int tl = indices[j0 + q] >> kTileShift;
-        if (tl != tp) {
-            if (tl - tp <= 32) {
-                for (int g = tp + 1; g <= tl; ++g) index[(ft + g) * kChainGroup + k] = static_cast<uint32_t>(j0 + q);
-            } else {
-                bigm |= 1u << q;
-            }
+    while (bnd != 0u) {
+        const int q = __ffs(bnd) - 1;
+        bnd &= bnd - 1;
+        const int tp = indices[j0 + q - 1] >> kTileShift, tl = indices[j0 + q] >> kTileShift;
+        if (tl - tp <= 32) {
+            for (int g = tp + 1; g <= tl; ++g) index[(ft + g) * kChainGroup + k] = static_cast<uint32_t>(j0 + q);
+        } else {
+            bigm |= 1u << q;
         }
-        tp = tl;
     }
     return bigm;
 }
@@ -354,8 +353,13 @@ __global__ void __launch_bounds__(kIdxThreads, 6) chain_index_kernel(IndexParams
         } else if (p.write) {
             // any tile change in the run (or from the entry before it)?
             const int tp = opens ? (x[0] >> kTileShift) : (prev >> kTileShift);
-            if ((x[kIdxPerThread - 1] >> kTileShift) != tp)
-                bigm = index_run_rows(d.indices, p.index, k, j0, m0.first_tile, opens);
+            if ((x[kIdxPerThread - 1] >> kTileShift) != tp) {
+                unsigned int bnd = (x[0] >> kTileShift) != tp ? 1u : 0u;
+#pragma unroll
+                for (int q = 1; q < kIdxPerThread; ++q)
+                    bnd |= ((x[q] >> kTileShift) != (x[q - 1] >> kTileShift)) ? (1u << q) : 0u;
+                bigm = index_run_rows(d.indices, p.index, k, j0, m0.first_tile, bnd);
+            }
         }
     } else if (nlive > 0) {
         bad_j = index_run_general(d, p.ws.numel, p.ws.first_tile, p.index, T, k, j0, nlive, m0.t, t1, p.write,
