@@ -116,19 +116,28 @@ __global__ void __launch_bounds__(kPackThreads) pack_positions_kernel(PackParams
     if (!s_go) return;
     const long long end = s_end;
     const int t0 = s_t[0], t1 = s_t[1];
+    // the block's first tensor, read once (a block inside one tensor, the
+    // common case, needs nothing else)
+    const long long n0 = p.ws.numel[t0], pb0 = p.pos_offsets[t0], ob0 = p.d.offsets[t0];
 #pragma unroll
     for (int r = 0; r < kPackPerThread; ++r) {
         const long long j = base + tid + r * kPackThreads;
         if (j >= end) continue;
-        const int t = (t0 == t1) ? t0 : tensor_of_entry(p.d.offsets, t0, t1, j);
-        const long long n = p.ws.numel[t];
+        int t = t0;
+        long long n = n0, pb = pb0, ob = ob0;
+        if (t0 != t1) {
+            t = tensor_of_entry(p.d.offsets, t0, t1, j);
+            n = p.ws.numel[t];
+            pb = p.pos_offsets[t];
+            ob = p.d.offsets[t];
+        }
         const int i = idx[r];
         if (i < 0 || static_cast<long long>(i) >= n) {
             record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, j);
             continue;
         }
         const int w = pos_width_of(n);
-        const long long at = p.pos_offsets[t] + (j - p.d.offsets[t]) * w;
+        const long long at = pb + (j - ob) * w;
         if (at + w > p.pos_capacity) continue;  // recorded by the offsets pass
         uint8_t *dst = p.positions + at;  // even
         if (w == 4 && (reinterpret_cast<uintptr_t>(dst) & 3u) == 0) {
@@ -164,9 +173,15 @@ __global__ void __launch_bounds__(kSumThreads) checksum_kernel(const uint8_t *po
     if (gid < head) hp ^= pos[gid];
     const uint4 *pv = reinterpret_cast<const uint4 *>(pos + head);
     unsigned long long words = 0;
-    for (long long k = gid; k < nvec; k += stride) {
-        const uint4 w = ld_stream_v4(pv + k);
-        words ^= (static_cast<unsigned long long>(w.y) << 32 | w.x) ^ (static_cast<unsigned long long>(w.w) << 32 | w.z);
+    for (long long k = gid; k < nvec; k += 4 * stride) {  // four loads in flight
+        uint4 w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            w[u] = k + u * stride < nvec ? ld_stream_v4(pv + k + u * stride) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            words ^= (static_cast<unsigned long long>(w[u].y) << 32 | w[u].x) ^
+                     (static_cast<unsigned long long>(w[u].w) << 32 | w[u].z);
     }
     hp ^= fold_bytes(words);
     for (long long k = head + (nvec << 4) + gid; k < nbytes; k += stride) hp ^= pos[k];
@@ -177,12 +192,17 @@ __global__ void __launch_bounds__(kSumThreads) checksum_kernel(const uint8_t *po
     const long long vvec = (nval - vhead) >> 3;
     if (gid < vhead) hv ^= bf16_to_f64_bits(val[gid]);
     const uint4 *vv = reinterpret_cast<const uint4 *>(val + vhead);
-    for (long long k = gid; k < vvec; k += stride) {
-        const uint4 w = ld_stream_v4(vv + k);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    for (long long k = gid; k < vvec; k += 4 * stride) {  // four loads in flight
+        uint4 w[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            hv ^= bf16_to_f64_bits(ws[q] & 0xffffu) ^ bf16_to_f64_bits(ws[q] >> 16);
+        for (int u = 0; u < 4; ++u) w[u] = k + u * stride < vvec ? ld_stream_v4(vv + k + u * stride) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {  // a zero word past the end is +0.0: double bits 0
+            const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                hv ^= bf16_to_f64_bits(ws[q] & 0xffffu) ^ bf16_to_f64_bits(ws[q] >> 16);
+        }
     }
     for (long long k = vhead + (vvec << 3) + gid; k < nval; k += stride) hv ^= bf16_to_f64_bits(val[k]);
     // CTA reduction, one atomic per output per CTA
