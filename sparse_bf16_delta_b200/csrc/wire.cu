@@ -192,6 +192,12 @@ __global__ void __launch_bounds__(kSumThreads) checksum_kernel(const uint8_t *po
     const long long vvec = (nval - vhead) >> 3;
     if (gid < vhead) hv ^= bf16_to_f64_bits(val[gid]);
     const uint4 *vv = reinterpret_cast<const uint4 *>(val + vhead);
+    // A normal bf16 (exponent 1..254) is the double with bits sign << 63 |
+    // (e + 896) << 52 | m << 45: three disjoint fields, so their XORs over many
+    // values can be kept apart and assembled once.  sm2 folds sign and
+    // mantissa bits two values at a time (one 32-bit word); ex folds e + 896.
+    // Zeros, subnormals, infinities and NaNs take the exact conversion.
+    uint32_t sm2 = 0u, ex = 0u;
     for (long long k = gid; k < vvec; k += 4 * stride) {  // four loads in flight
         uint4 w[4];
 #pragma unroll
@@ -200,9 +206,22 @@ __global__ void __launch_bounds__(kSumThreads) checksum_kernel(const uint8_t *po
         for (int u = 0; u < 4; ++u) {  // a zero word past the end is +0.0: double bits 0
             const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                hv ^= bf16_to_f64_bits(ws[q] & 0xffffu) ^ bf16_to_f64_bits(ws[q] >> 16);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t el = (ws[q] >> 7) & 0xffu, eh = (ws[q] >> 23) & 0xffu;
+                if (el - 1u < 254u && eh - 1u < 254u) {
+                    sm2 ^= ws[q] & 0x807f807fu;
+                    ex ^= (el + 896u) ^ (eh + 896u);
+                } else {
+                    hv ^= bf16_to_f64_bits(ws[q] & 0xffffu) ^ bf16_to_f64_bits(ws[q] >> 16);
+                }
+            }
         }
+    }
+    {
+        const uint32_t sgn = ((sm2 >> 15) ^ (sm2 >> 31)) & 1u;
+        const uint32_t man = (sm2 ^ (sm2 >> 16)) & 0x7fu;
+        hv ^= (static_cast<unsigned long long>(sgn) << 63) | (static_cast<unsigned long long>(ex & 0x7ffu) << 52) |
+              (static_cast<unsigned long long>(man) << 45);
     }
     for (long long k = vhead + (vvec << 3) + gid; k < nval; k += stride) hv ^= bf16_to_f64_bits(val[k]);
     // CTA reduction, one atomic per output per CTA
