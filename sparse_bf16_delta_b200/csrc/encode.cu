@@ -568,9 +568,21 @@ __device__ void count_group(const EncodeParams &p, EncodeSmem &sm, const int g) 
 // kSum: also XOR the written entries into the wire checksum halves (the
 // bytes of each position at its tensor's pos_width, the double bits of each
 // value) kept in *hp / *hv.
+// A look-back lane's share of the wire checksum (kSum).  pos: XOR of the
+// positions it wrote; the position hash is the XOR of their bytes at their
+// tensor's width, and a 2-byte position (numel <= 65536) has zero upper
+// bytes, so folding pos's four bytes at the end gives it for both widths.
+// sm, ex: XOR of the sign and mantissa bits, and of e + 896, of the normal
+// values (the double's three disjoint fields: sign << 63 | (e + 896) << 52 |
+// m << 45); hv: the exact double bits of the other values.
+struct SumAcc {
+    uint32_t pos, sm, ex;
+    unsigned long long hv;
+};
+
 template <bool kWide, bool kSum>
 __device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const Pending &e,
-                              long long prefix, unsigned long long *hp, unsigned long long *hv) {
+                              long long prefix, SumAcc *acc) {
     const int lane = threadIdx.x & 31;
     long long lim = p.capacity - prefix;
     if (lim > e.total) lim = e.total;
@@ -578,12 +590,16 @@ __device__ void write_entries(const EncodeParams &p, const uint32_t *ring, const
     const uint32_t ls = static_cast<uint32_t>(e.local_start);
     long long gs = 0;  // global position of the tile's first element
     if (kWide) gs = p.index_base[e.tensor] + e.local_start;
-    int width = 4;
-    if (kSum) width = p.ws.numel[e.tensor] <= 65536 ? 2 : 4;
     auto sum = [&](uint32_t v) {
         if (kSum) {
-            *hp ^= pos_bytes_xor(ls + (v & 0xffffu), width);
-            *hv ^= bf16_to_f64_bits(v >> 16);
+            acc->pos ^= ls + (v & 0xffffu);
+            const uint32_t b = v >> 16, ee = (b >> 7) & 0xffu;
+            if (ee - 1u < 254u) {
+                acc->sm ^= b & 0x807fu;
+                acc->ex ^= ee + 896u;
+            } else {
+                acc->hv ^= bf16_to_f64_bits(b);
+            }
         }
     };
     auto one = [&](int k) {
@@ -634,11 +650,16 @@ template <bool kCompact, bool kWide, bool kSum>
 __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
     const int lane = threadIdx.x & 31;
     const int j = (threadIdx.x >> 5) - kCountWarps;
-    unsigned long long hp = 0, hv = 0;  // this lane's share of the checksum halves (kSum)
+    SumAcc acc{0u, 0u, 0u, 0ull};  // this lane's share of the checksum (kSum)
     // Leaves through here: the warp's checksum share goes out with one
     // atomic per half (per-tile atomics on two words would be a hot spot).
     auto leave = [&]() {
         if (kSum) {
+            const uint32_t x = acc.pos ^ (acc.pos >> 16);
+            unsigned long long hp = (x ^ (x >> 8)) & 0xffu;
+            unsigned long long hv = acc.hv ^ (static_cast<unsigned long long>((acc.sm >> 15) & 1u) << 63) ^
+                                    (static_cast<unsigned long long>(acc.ex & 0x7ffu) << 52) ^
+                                    (static_cast<unsigned long long>(acc.sm & 0x7fu) << 45);
 #pragma unroll
             for (int d = 16; d > 0; d >>= 1) {
                 hp ^= __shfl_xor_sync(0xffffffffu, hp, d);
@@ -684,7 +705,7 @@ __device__ void look_group(const EncodeParams &p, EncodeSmem &sm) {
                     if (kCompact && nnz > p.capacity) record_error(p.ws.hdr, DWS_ERR_CAPACITY, nnz);
                 }
             }
-            if (kCompact) write_entries<kWide, kSum>(p, sm.ring[e.group], e, prefix, &hp, &hv);
+            if (kCompact) write_entries<kWide, kSum>(p, sm.ring[e.group], e, prefix, &acc);
         } else if (e.ticket != p.withhold) {
             if (lane == 0) *reinterpret_cast<volatile int *>(&sm.stop) = 1;
         }
