@@ -119,6 +119,29 @@ __global__ void __launch_bounds__(kPackThreads) pack_positions_kernel(PackParams
     // the block's first tensor, read once (a block inside one tensor, the
     // common case, needs nothing else)
     const long long n0 = p.ws.numel[t0], pb0 = p.pos_offsets[t0], ob0 = p.d.offsets[t0];
+    if (t0 == t1 && pos_width_of(n0) == 4) {
+        // 4-byte positions of one tensor: the block's positions are its
+        // indices, stored contiguously from at0 (checked once for room)
+        const long long at0 = pb0 + (base - ob0) * 4;
+        uint8_t *dst0 = p.positions + at0;
+        if (at0 >= 0 && at0 + (end - base) * 4 <= p.pos_capacity && (reinterpret_cast<uintptr_t>(dst0) & 3u) == 0) {
+            uint32_t *d32 = reinterpret_cast<uint32_t *>(dst0);
+            const int m = static_cast<int>(end - base);
+            long long bad_j = -1;
+#pragma unroll
+            for (int r = 0; r < kPackPerThread; ++r) {
+                const int q = tid + r * kPackThreads;
+                if (q < m) {
+                    if (static_cast<unsigned long long>(static_cast<long long>(idx[r])) < static_cast<unsigned long long>(n0))
+                        d32[q] = static_cast<uint32_t>(idx[r]);
+                    else if (bad_j < 0)
+                        bad_j = base + q;
+                }
+            }
+            if (bad_j >= 0) record_error(p.ws.hdr, DWS_ERR_BAD_DELTA, bad_j);
+            return;
+        }
+    }
 #pragma unroll
     for (int r = 0; r < kPackPerThread; ++r) {
         const long long j = base + tid + r * kPackThreads;
