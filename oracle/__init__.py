@@ -74,6 +74,10 @@ def _load():
     lib.ref_xor_encode.argtypes = [vp, vp, vp, i64]
     lib.ref_xor_apply.restype = None
     lib.ref_xor_apply.argtypes = [vp, vp, i64]
+    lib.ref_xor_byte_delta.restype = i64
+    lib.ref_xor_byte_delta.argtypes = [i32, vp, vpp, vpp, vp, vp, vp, i64]
+    lib.ref_apply_bytes.restype = i32
+    lib.ref_apply_bytes.argtypes = [i32, vp, vpp, vp, vp, vp]
     lib.ref_bf16_rne.restype = ctypes.c_uint16
     lib.ref_bf16_rne.argtypes = [f32]
     lib.ref_bf16_to_float.restype = f32
@@ -202,6 +206,49 @@ def xor_apply(buf: np.ndarray, mask) -> None:
     if m.size != buf.size:
         raise ValueError("size mismatch")
     lib.ref_xor_apply(_ptr(buf), _ptr(m), buf.size)
+
+
+def xor_byte_delta(olds, news, capacity: int | None = None):
+    """The sparse XOR delta at byte granularity of ``news`` against ``olds``
+    (lists of uint8 arrays, one per layer): per layer the ascending int32
+    positions of the bytes that differ and the new bytes there ("humans&
+    weight sync" summary, first paragraph: the XOR mask is nonzero exactly at
+    those bytes).  Returns ``(offsets int64[T+1], positions int32[n],
+    values uint8[n])``; capacity as in ``encode``."""
+    lib = _load()
+    olds = [_c(a, np.uint8) for a in olds]
+    news = [_c(a, np.uint8) for a in news]
+    if len(olds) != len(news) or any(a.size != b.size for a, b in zip(olds, news)):
+        raise ValueError("old/new layers differ in number or size")
+    T = len(olds)
+    nbytes = np.array([a.size for a in olds] or [0], dtype=np.int64)
+    offsets = np.zeros(T + 1, dtype=np.int64)
+    if capacity is None:
+        capacity = int(sum(a.size for a in olds))
+    positions = np.empty(max(1, capacity), dtype=np.int32)
+    values = np.empty(max(1, capacity), dtype=np.uint8)
+    n = lib.ref_xor_byte_delta(T, _ptr(nbytes), _ptr_array(olds), _ptr_array(news),
+                               _ptr(offsets), _ptr(positions), _ptr(values), capacity)
+    if n < 0:
+        raise ValueError("invalid layer size (must be below 2^31 bytes)")
+    kept = min(n, capacity)
+    return offsets, positions[:kept].copy(), values[:kept].copy()
+
+
+def apply_bytes(bufs, offsets, positions, values) -> None:
+    """Scatter a byte-granular delta into ``bufs`` (uint8 arrays) in place."""
+    lib = _load()
+    for b in bufs:
+        if b.dtype != np.uint8 or not b.flags.c_contiguous:
+            raise TypeError("layers must be contiguous uint8 arrays")
+    nbytes = np.array([b.size for b in bufs] or [0], dtype=np.int64)
+    offsets = _c(offsets, np.int64)
+    positions = _c(positions, np.int32) if len(positions) else np.zeros(1, np.int32)
+    values = _c(values, np.uint8) if len(values) else np.zeros(1, np.uint8)
+    rc = lib.ref_apply_bytes(len(bufs), _ptr(nbytes), _ptr_array(bufs), _ptr(offsets),
+                             _ptr(positions), _ptr(values))
+    if rc != 0:
+        raise ValueError("bad byte delta (position out of range or offsets not monotone)")
 
 
 def bf16_rne(x) -> np.ndarray:

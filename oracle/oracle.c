@@ -97,6 +97,55 @@ void ref_xor_apply(uint8_t *buf, const uint8_t *mask, int64_t nbytes)
     for (int64_t i = 0; i < nbytes; ++i) buf[i] = (uint8_t)(buf[i] ^ mask[i]);
 }
 
+/* The sparse form of the XOR delta at byte granularity: for each layer t and
+ * byte i ascending, where old and new differ, the position i and the new
+ * byte ([XOR] first paragraph: the mask is nonzero exactly there, so a
+ * receiver that knows the positions and new bytes rebuilds new from old).
+ * Same layout as ref_encode, positions int32.  Returns the total count, or
+ * -1 on a size that does not fit int32 positions. */
+int64_t ref_xor_byte_delta(int32_t T, const int64_t *nbytes,
+                           const uint8_t *const *old_t, const uint8_t *const *new_t,
+                           int64_t *offsets, int32_t *positions, uint8_t *values,
+                           int64_t capacity)
+{
+    if (T < 0) return -1;
+    for (int32_t t = 0; t < T; ++t)
+        if (nbytes[t] < 0 || nbytes[t] > (int64_t)INT32_MAX) return -1;
+    int64_t n = 0;
+    offsets[0] = 0;
+    for (int32_t t = 0; t < T; ++t) {
+        for (int64_t i = 0; i < nbytes[t]; ++i) {
+            if (old_t[t][i] != new_t[t][i]) {
+                if (n < capacity) {
+                    positions[n] = (int32_t)i;
+                    values[n] = new_t[t][i];
+                }
+                ++n;
+            }
+        }
+        offsets[t + 1] = n;
+    }
+    return n;
+}
+
+/* Its receiver: buf_t[positions[j]] = values[j] for each layer's segment.
+ * Returns 0, or -1 at the first position outside the layer. */
+int32_t ref_apply_bytes(int32_t T, const int64_t *nbytes, uint8_t *const *buf_t,
+                        const int64_t *offsets, const int32_t *positions,
+                        const uint8_t *values)
+{
+    if (offsets[0] != 0) return -1;
+    for (int32_t t = 0; t < T; ++t) {
+        if (offsets[t + 1] < offsets[t]) return -1;
+        for (int64_t j = offsets[t]; j < offsets[t + 1]; ++j) {
+            int64_t i = positions[j];
+            if (i < 0 || i >= nbytes[t]) return -1;
+            buf_t[t][i] = values[j];
+        }
+    }
+    return 0;
+}
+
 uint16_t ref_bf16_rne(float x)
 {
     uint32_t u;

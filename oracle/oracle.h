@@ -126,6 +126,20 @@ uint64_t ref_hash_bf16(const uint16_t *v, int64_t n);
  * conversion on this host). */
 uint64_t ref_bf16_to_f64_bits(uint16_t b);
 
+/* Sparse XOR delta at byte granularity ([XOR] first paragraph): per layer,
+ * the ascending int32 positions of the bytes that differ and the new bytes
+ * (ref_encode's layout).  Returns the count or -1 (a layer of 2^31 bytes or
+ * more). */
+int64_t ref_xor_byte_delta(int32_t T, const int64_t *nbytes,
+                           const uint8_t *const *old_t, const uint8_t *const *new_t,
+                           int64_t *offsets, int32_t *positions, uint8_t *values,
+                           int64_t capacity);
+
+/* buf_t[positions[j]] = values[j]; -1 at a position outside its layer. */
+int32_t ref_apply_bytes(int32_t T, const int64_t *nbytes, uint8_t *const *buf_t,
+                        const int64_t *offsets, const int32_t *positions,
+                        const uint8_t *values);
+
 #ifdef __cplusplus
 }
 #endif

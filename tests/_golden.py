@@ -66,6 +66,14 @@ def xor_example():
     return hex8(d["old"]), hex8(d["new"]), hex8(d["mask"])
 
 
+def xor_byte_delta_example():
+    d = keyed("xor_byte_delta.txt")
+    layers = [(hex8(d[f"layer{t}_old"]), hex8(d[f"layer{t}_new"])) for t in range(4)]
+    ints = lambda k: [int(x) for x in d[k]]
+    return (layers, ints("offsets"), ints("positions"), [int(x, 16) for x in d["values"]],
+            ints("word_offsets"), ints("word_indices"))
+
+
 def rounding_cases():
     out = []
     for line in _lines("bf16_rounding.txt"):

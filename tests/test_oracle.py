@@ -597,3 +597,72 @@ def test_merge_shards_of_row_shards_equals_the_unsharded_encode(world):
     np.testing.assert_array_equal(i, wi)
     np.testing.assert_array_equal(v, wv)
     assert int(o[-1]) > 100
+
+
+# ---------------------------------------------------------------- byte-granular sparse XOR
+
+
+def test_xor_byte_delta_golden():
+    layers, offs, pos, vals, woffs, widx = G.xor_byte_delta_example()
+    o, p, v = oracle.xor_byte_delta([a for a, _ in layers], [b for _, b in layers])
+    assert o.tolist() == offs and p.tolist() == pos and v.tolist() == vals
+    bufs = [a.copy() for a, _ in layers]
+    oracle.apply_bytes(bufs, o, p, v)
+    for buf, (_, b) in zip(bufs, layers):
+        np.testing.assert_array_equal(buf, b)
+    # the word form of the same layers (the sparse encode on 16-bit words)
+    wo, wi, _ = oracle.encode([a.view(np.uint16) for a, _ in layers], [b.view(np.uint16) for _, b in layers])
+    assert wo.tolist() == woffs and wi.tolist() == widx
+
+
+def test_xor_byte_delta_closed_form_on_byte_layers():
+    # Closed form: the generator knows which bytes it changed; the byte delta
+    # lists exactly those, with the new bytes; it equals the nonzero set of
+    # the dense mask; applying it to old gives new.
+    old, new, pos = W.xor_layer(1, "cpu", nbytes=3_000_000, flips=2_500)
+    old, new, pos = old.numpy(), new.numpy(), pos.numpy()
+    o, p, v = oracle.xor_byte_delta([old], [new])
+    np.testing.assert_array_equal(p, pos)
+    np.testing.assert_array_equal(v, new[pos])
+    np.testing.assert_array_equal(p, np.flatnonzero(oracle.xor_encode(old, new)))
+    buf = old.copy()
+    oracle.apply_bytes([buf], o, p, v)
+    np.testing.assert_array_equal(buf, new)
+    assert oracle.xor_byte_delta([old], [old])[0].tolist() == [0, 0]
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_xor_byte_delta_from_the_word_delta(seed):
+    # Each word entry of the sparse encode on 16-bit words is one or two byte
+    # entries (its low byte at 2i, its high byte at 2i + 1, little-endian):
+    # mapping the word delta to bytes gives the byte delta (a dropped byte, a
+    # swapped half or a wrong order fails it).
+    rng = np.random.default_rng(700 + seed)
+    sizes = [2 * int(x) for x in rng.integers(0, 3000, 6)] + [0, 2]
+    olds = [rng.integers(0, 256, n, dtype=np.uint8) for n in sizes]
+    news = []
+    for a in olds:
+        b = a.copy()
+        m = rng.random(a.size) < 0.05
+        b[m] = (b[m].astype(np.int32) + rng.integers(1, 256, int(m.sum()))).astype(np.uint8)
+        news.append(b)
+    wo, wi, wv = oracle.encode([a.view(np.uint16) for a in olds], [b.view(np.uint16) for b in news])
+    o, p, v = oracle.xor_byte_delta(olds, news)
+    for t, (a, b) in enumerate(zip(olds, news)):
+        want_p, want_v = [], []
+        for j in range(wo[t], wo[t + 1]):
+            i = int(wi[j])
+            for h in (0, 1):
+                if a[2 * i + h] != b[2 * i + h]:
+                    want_p.append(2 * i + h)
+                    want_v.append((int(wv[j]) >> (8 * h)) & 0xFF)
+        assert p[o[t]:o[t + 1]].tolist() == want_p
+        assert v[o[t]:o[t + 1]].tolist() == want_v
+    # wire size: 5 bytes per changed byte against 6 per changed word
+    assert 5 * len(p) <= 6 * len(wi) * 2 and len(wi) <= len(p) <= 2 * len(wi)
+
+
+def test_apply_bytes_rejects_a_position_outside_its_layer():
+    buf = np.zeros(4, np.uint8)
+    with pytest.raises(ValueError):
+        oracle.apply_bytes([buf], np.array([0, 1]), np.array([4], np.int32), np.array([1], np.uint8))
