@@ -701,6 +701,42 @@ def rows_xor(args, dev, peak):
     out.update([row("encode_sparse_nvfp4_" + tag, ms_e, 2 * L * B + 6 * snnz, L * B, peak,
                     {"min_ms": round(mn_e, 4), "nnz": snnz, "delta_bytes": 6 * snnz + 8 * (L + 1)},
                     elems=L * B)])
+    # the same delta at byte granularity: one entry per changed byte (int32
+    # position + the new byte, 5 bytes) made from the word delta
+    bo, bp, bv = splan.xor_bytes_from_words(sot, sd)
+    bn = int(bo[-1].item())
+    st_ = torch.cuda.current_stream().cuda_stream
+    so_, si_, sv_, sc_ = sd.as_ref()
+
+    def to_bytes():
+        dws.dws_xor_bytes_from_words(splan.handle, sot.data_ptr(), so_, si_, sv_, sc_, bo.data_ptr(),
+                                     bp.data_ptr(), bv.data_ptr(), bp.numel(), splan.workspace.data_ptr(),
+                                     splan.workspace_bytes, st_)
+
+    ms_b, mn_b = time_reps(to_bytes, args.rows_reps)
+    splan.raise_on_error("xor bytes from words")
+    conv_bytes = 8 * snnz + 5 * bn  # word entries + the old words gathered, byte entries written
+    out.update([row("bytes_from_words_nvfp4_" + tag, ms_b, conv_bytes, L * B, peak,
+                    {"min_ms": round(mn_b, 4), "byte_entries": bn, "word_entries": snnz,
+                     "delta_bytes": 5 * bn + 8 * (L + 1), "word_delta_bytes": 6 * snnz + 8 * (L + 1)},
+                    elems=L * B)])
+
+    def enc_bytes():
+        splan.encode_into(sot, snt, sd.offsets, sd.indices, sd.values)
+        to_bytes()
+
+    ms_eb, mn_eb = time_reps(enc_bytes, args.rows_reps)
+    out.update([row("encode_sparse_bytes_nvfp4_" + tag, ms_eb, 2 * L * B + 6 * snnz + conv_bytes, L * B, peak,
+                    {"min_ms": round(mn_eb, 4), "byte_entries": bn, "delta_bytes": 5 * bn + 8 * (L + 1)},
+                    elems=L * B)])
+    bst = dws.ptr_table(olds)
+    ms_ab, mn_ab = time_reps(lambda: splan.apply_bytes(bst, bo, bp, bv, count=bn), args.rows_reps)
+    splan.raise_on_error("byte xor apply")
+    ok_b = all(torch.equal(olds[l], news[l]) for l in (0, L - 1))
+    out.update([row("apply_bytes_nvfp4_" + tag, ms_ab, 6 * bn, L * B, peak,
+                    {"min_ms": round(mn_ab, 4), "exact": ok_b,
+                     "entries_per_s": round(bn / ms_ab * 1e3, 1)}, elems=L * B)])
+    del bo, bp, bv, bst
     sst = dws.ptr_table(ow)
     ms_a, mn_a = time_reps(lambda: splan.apply(sst, sd), args.rows_reps)
     splan.raise_on_error("sparse xor apply")

@@ -510,6 +510,50 @@ DWS_API dws_status_t dws_xor_apply_layers(void *const *bufs, const void *const *
                                   void *staging0, void *staging1, int64_t staging_bytes,
                                   dws_stream_t apply_stream, dws_stream_t copy_stream);
 
+/* The sparse XOR delta at byte granularity (the humans& weight-sync summary,
+ * first paragraph: the XOR mask of old and new is nonzero exactly at the
+ * changed bytes, so shipping those bytes' positions and new values rebuilds
+ * new from old): per layer, the ascending int32 positions of the changed
+ * bytes and the new bytes there, 5 bytes per changed byte (the word form,
+ * dws_encode on the layers viewed as 16-bit words, costs 6 per changed
+ * word).  Made from that word delta of the same layers:
+ * plan: the layers as 16-bit words (numel = bytes / 2; every layer below
+ *   2^30 words, so that byte positions fit int32: else DWS_ERR_INVALID).
+ * old_ptrs: device array of the old layers (2-byte aligned).
+ * word_offsets, word_indices, word_values, word_count: the word delta
+ *   (dws_encode's layout, device).
+ * byte_offsets: device int64[T+1] (8-byte aligned), written: layer t's
+ *   entries are [byte_offsets[t], byte_offsets[t+1]).
+ * byte_positions (4-byte aligned), byte_values: device arrays of `capacity`
+ *   entries; byte entry k of a changed word i is position 2i (its low byte,
+ *   the lower address) or 2i + 1 (its high byte).
+ * Errors: host -- DWS_ERR_INVALID (null or misaligned arrays, negative
+ * sizes, a layer of 2^30 words or more), workspace errors as dws_encode;
+ * device (dws_status) -- DWS_ERR_CAPACITY (detail = entries needed) when the
+ * total exceeds capacity (offsets complete, entries past capacity not
+ * written); DWS_ERR_BAD_DELTA for a word entry outside its layer or not
+ * above the one before it (its bytes are not written, the offsets of later
+ * entries still count them as none).  Uses the workspace's per-call
+ * scratch: it must not overlap an encode on the same workspace. */
+DWS_API dws_status_t dws_xor_bytes_from_words(const dws_plan_t *plan, const void *const *old_ptrs,
+                                      const int64_t *word_offsets, const int32_t *word_indices,
+                                      const uint16_t *word_values, int64_t word_count,
+                                      int64_t *byte_offsets, int32_t *byte_positions,
+                                      uint8_t *byte_values, int64_t capacity, void *workspace,
+                                      size_t workspace_bytes, dws_stream_t stream);
+
+/* Apply a byte-granular XOR delta: for each layer t and entry j of its
+ * segment, buf_t[positions[j]] = values[j] (in place).  plan, offsets,
+ * positions (4-byte aligned), count: as dws_xor_bytes_from_words and
+ * dws_apply; buf_ptrs: device array of the layers' device pointers.  Every
+ * position is range-checked against its layer (2 x numel bytes) and required
+ * to be above the one before it in its layer; a violating entry is skipped
+ * and DWS_ERR_BAD_DELTA recorded (detail = entry number). */
+DWS_API dws_status_t dws_apply_bytes(const dws_plan_t *plan, void *const *buf_ptrs,
+                             const int64_t *offsets, const int32_t *positions,
+                             const uint8_t *values, int64_t count, void *workspace,
+                             size_t workspace_bytes, dws_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Status
  * ------------------------------------------------------------------------ */

@@ -73,6 +73,8 @@ _sig("dws_apply_chain", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _vp,
 _sig("dws_apply_chain_ex", _i32, [_vp, _vp, ctypes.POINTER(dws_delta_t), _i32, _i32, _vp, _sz, _vp])
 _sig("dws_pos_width", _i32, [_vp, _i32])
 _sig("dws_merge_shards", _i32, [_vp, _i32, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
+_sig("dws_xor_bytes_from_words", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
+_sig("dws_apply_bytes", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_encode_global", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _sz, _vp])
 _sig("dws_encode_checksum", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _vp])
 _sig("dws_pack_positions", _i32, [_vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _sz, _vp])
@@ -207,6 +209,19 @@ def dws_encode_checksum(plan, old_ptrs, new_ptrs, offsets, indices, values, capa
                         checksum, workspace, workspace_bytes, stream) -> int:
     return _lib.dws_encode_checksum(plan, old_ptrs, new_ptrs, offsets, indices, values, capacity,
                                     hashes, checksum, workspace, workspace_bytes, stream)
+
+
+def dws_xor_bytes_from_words(plan, old_ptrs, word_offsets, word_indices, word_values, word_count,
+                             byte_offsets, byte_positions, byte_values, capacity, workspace,
+                             workspace_bytes, stream):
+    return _lib.dws_xor_bytes_from_words(plan, old_ptrs, word_offsets, word_indices, word_values,
+                                         word_count, byte_offsets, byte_positions, byte_values, capacity,
+                                         workspace, workspace_bytes, stream)
+
+
+def dws_apply_bytes(plan, buf_ptrs, offsets, positions, values, count, workspace, workspace_bytes, stream):
+    return _lib.dws_apply_bytes(plan, buf_ptrs, offsets, positions, values, count, workspace,
+                                workspace_bytes, stream)
 
 
 def dws_merge_shards(plan, num_ranks, rank_offsets, rank_indices, rank_values, stride, offsets,
@@ -530,6 +545,30 @@ class DeltaPlan:
                                 _stream_handle(stream)), "dws_merge_shards")
         self.raise_on_error("dws_merge_shards", stream)
         return Delta(offsets, indices, values)
+
+    # -- byte-granular sparse XOR (the plan: packed layers as 16-bit words) --
+    def xor_bytes_from_words(self, old_table, word_delta: Delta, capacity=None, stream=None):
+        """(offsets int64[T+1], positions int32[n], values uint8[n]) of the
+        byte-granular XOR delta made from a word delta of the same layers;
+        capacity defaults to twice the word entries (every byte changed)."""
+        torch = _torch()
+        cap = 2 * word_delta.count if capacity is None else int(capacity)
+        offsets = torch.empty(self.num_tensors + 1, dtype=torch.int64, device=self.device)
+        positions = torch.empty(max(1, cap), dtype=torch.int32, device=self.device)
+        values = torch.empty(max(1, cap), dtype=torch.uint8, device=self.device)
+        o, i, v, c = word_delta.as_ref()
+        _check(dws_xor_bytes_from_words(self.handle, old_table.data_ptr(), o, i, v, c, offsets.data_ptr(),
+                                        positions.data_ptr(), values.data_ptr(), cap,
+                                        self.workspace.data_ptr(), self.workspace_bytes,
+                                        _stream_handle(stream)), "dws_xor_bytes_from_words")
+        return offsets, positions, values
+
+    def apply_bytes(self, buf_table, offsets, positions, values, count=None, stream=None):
+        n = int(offsets[-1].item()) if count is None else int(count)
+        _check(dws_apply_bytes(self.handle, buf_table.data_ptr(), offsets.data_ptr(),
+                               positions.data_ptr() if n else 0, values.data_ptr() if n else 0, n,
+                               self.workspace.data_ptr(), self.workspace_bytes, _stream_handle(stream)),
+               "dws_apply_bytes")
 
     # -- wire form --
     def pos_width(self, t: int) -> int:

@@ -366,6 +366,55 @@ dws_status_t dws_merge_shards(const dws_plan_t *plan, int32_t num_ranks,
         capacity, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// Byte positions are int32: every layer below 2^30 words (2^31 bytes).
+static bool bytes_fit_int32(const dws_plan_t *plan) {
+    const long long *numel = reinterpret_cast<const long long *>(plan->image.data() + plan->layout.numel_off);
+    for (int32_t t = 0; t < plan->T; ++t)
+        if (numel[t] >= (1LL << 30)) return false;
+    return true;
+}
+
+dws_status_t dws_xor_bytes_from_words(const dws_plan_t *plan, const void *const *old_ptrs,
+                                      const int64_t *word_offsets, const int32_t *word_indices,
+                                      const uint16_t *word_values, int64_t word_count, int64_t *byte_offsets,
+                                      int32_t *byte_positions, uint8_t *byte_values, int64_t capacity,
+                                      void *workspace, size_t workspace_bytes, dws_stream_t stream) {
+    dws_status_t st = check_ws(plan, workspace, workspace_bytes);
+    if (st != DWS_OK) return st;
+    if (old_ptrs == nullptr || word_offsets == nullptr || byte_offsets == nullptr || word_count < 0 ||
+        capacity < 0)
+        return DWS_ERR_INVALID;
+    if (word_count > 0 && (word_indices == nullptr || word_values == nullptr)) return DWS_ERR_INVALID;
+    if (capacity > 0 && (byte_positions == nullptr || byte_values == nullptr)) return DWS_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(word_indices) & 3u) || (reinterpret_cast<uintptr_t>(word_values) & 1u) ||
+        (reinterpret_cast<uintptr_t>(byte_positions) & 3u) || (reinterpret_cast<uintptr_t>(byte_offsets) & 7u) ||
+        (reinterpret_cast<uintptr_t>(word_offsets) & 7u))
+        return DWS_ERR_INVALID;
+    if (!bytes_fit_int32(plan)) return DWS_ERR_INVALID;
+    dws::DeltaRef d{reinterpret_cast<const long long *>(word_offsets), reinterpret_cast<const int *>(word_indices),
+                    word_values, word_count};
+    return from_cuda(dws::launch_xor_bytes_from_words(
+        view_of(plan, workspace), reinterpret_cast<const uint16_t *const *>(old_ptrs), d, plan->N,
+        reinterpret_cast<long long *>(byte_offsets), reinterpret_cast<int *>(byte_positions), byte_values,
+        capacity, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dws_status_t dws_apply_bytes(const dws_plan_t *plan, void *const *buf_ptrs, const int64_t *offsets,
+                             const int32_t *positions, const uint8_t *values, int64_t count, void *workspace,
+                             size_t workspace_bytes, dws_stream_t stream) {
+    dws_status_t st = check_ws(plan, workspace, workspace_bytes);
+    if (st != DWS_OK) return st;
+    if (buf_ptrs == nullptr || offsets == nullptr || count < 0) return DWS_ERR_INVALID;
+    if (count > 0 && (positions == nullptr || values == nullptr)) return DWS_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(positions) & 3u) || (reinterpret_cast<uintptr_t>(offsets) & 7u))
+        return DWS_ERR_INVALID;
+    if (!bytes_fit_int32(plan)) return DWS_ERR_INVALID;
+    return from_cuda(dws::launch_apply_bytes(view_of(plan, workspace), reinterpret_cast<uint8_t *const *>(buf_ptrs),
+                                             reinterpret_cast<const long long *>(offsets),
+                                             reinterpret_cast<const int *>(positions), values, count,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int32_t dws_pos_width(const dws_plan_t *plan, int32_t t) {
     if (plan == nullptr || t < 0 || t >= plan->T) return 0;
     const long long *numel =

@@ -487,6 +487,14 @@ cudaError_t launch_apply(const WsView &ws, uint16_t *const *snap_ptrs, const Del
 cudaError_t launch_apply_chain(const WsView &ws, uint16_t *const *snap_ptrs,
                                const DeltaRef *deltas, int K, bool merge, cudaStream_t s);
 
+// The byte-granular sparse XOR delta from a word delta of the same layers
+// (xorbytes.cu); plan_elems: the plan's total elements.
+cudaError_t launch_xor_bytes_from_words(const WsView &ws, const uint16_t *const *old_ptrs, const DeltaRef &d,
+                                        long long plan_elems, long long *byte_offsets, int *positions,
+                                        uint8_t *values, long long capacity, cudaStream_t s);
+cudaError_t launch_apply_bytes(const WsView &ws, uint8_t *const *buf_ptrs, const long long *offsets,
+                               const int *positions, const uint8_t *values, long long count, cudaStream_t s);
+
 cudaError_t launch_pack_positions(const WsView &ws, const DeltaRef &d, uint8_t *positions,
                                   long long pos_capacity, long long *pos_offsets, cudaStream_t s);
 cudaError_t launch_checksum(const uint8_t *positions, long long nbytes, const uint16_t *values,

@@ -108,6 +108,24 @@ def test_host_side_argument_errors_need_no_device():
         assert dws.dws_merge_shards(p, 1, 8, 8, 9, 1, 8, 8, 8, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_merge_shards(p, 1, 8, 8, 8, -1, 8, 8, 8, 1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_merge_shards(p, 1, 8, 8, 8, 1, 8, 8, 8, 1, 0x1000, 16, None) == dws.DWS_ERR_WORKSPACE
+        # byte-granular XOR delta: null or misaligned arrays, negative sizes
+        ws = (0x1000, 1 << 20, None)
+        assert dws.dws_xor_bytes_from_words(p, None, 8, 8, 8, 1, 8, 8, 8, 1, *ws) == dws.DWS_ERR_INVALID
+        assert dws.dws_xor_bytes_from_words(p, 8, 8, 0x1001, 8, 1, 8, 8, 8, 1, *ws) == dws.DWS_ERR_INVALID
+        assert dws.dws_xor_bytes_from_words(p, 8, 8, 8, 9, 1, 8, 8, 8, 1, *ws) == dws.DWS_ERR_INVALID
+        assert dws.dws_xor_bytes_from_words(p, 8, 8, 8, 8, -1, 8, 8, 8, 1, *ws) == dws.DWS_ERR_INVALID
+        assert dws.dws_xor_bytes_from_words(p, 8, 8, 8, 8, 1, 8, 8, 8, -1, *ws) == dws.DWS_ERR_INVALID
+        assert dws.dws_xor_bytes_from_words(p, 8, 8, 8, 8, 1, 8, 0x1002, 8, 1, *ws) == dws.DWS_ERR_INVALID
+        assert dws.dws_apply_bytes(p, None, 8, 8, 8, 1, *ws) == dws.DWS_ERR_INVALID
+        assert dws.dws_apply_bytes(p, 8, 8, 0x1002, 8, 1, *ws) == dws.DWS_ERR_INVALID
+        assert dws.dws_apply_bytes(p, 8, 8, 8, 8, -1, *ws) == dws.DWS_ERR_INVALID
+        big = dws.dws_plan_create([1 << 30])  # 2^31 bytes: byte positions would not fit int32
+        try:
+            assert dws.dws_xor_bytes_from_words(big, 8, 8, 8, 8, 1, 8, 8, 8, 1, 0x1000, 1 << 26, None) \
+                == dws.DWS_ERR_INVALID
+            assert dws.dws_apply_bytes(big, 8, 8, 8, 8, 1, 0x1000, 1 << 26, None) == dws.DWS_ERR_INVALID
+        finally:
+            dws.dws_plan_destroy(big)
         assert dws.dws_apply_chain_ex(p, 1, arr, 1, 3, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_apply_chain_ex(p, 1, arr, 1, -1, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
         assert dws.dws_apply_chain_ex(p, 1, arr, 0, 2, 0x1000, 1 << 20, None) == dws.DWS_ERR_INVALID
