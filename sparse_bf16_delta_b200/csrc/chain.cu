@@ -3,15 +3,18 @@
 // between; a new replica takes the latest anchor and replays the deltas after
 // it, the later delta winning where two touch the same element).
 //
-// Two kernels per pass over the snapshot:
+// Three kernels per pass over the snapshot (up to 16 deltas a pass):
 //
 //   chain_index_kernel  reads every entry of every delta once (coalesced
 //     16-byte loads), checks it (index inside its tensor, strictly above the
 //     entry before it in its tensor's segment) and writes the chain's tile
 //     index: for tile g and delta k, the first entry of k at or past the start
-//     of g, mod 2^32.  A failed check sets the workspace's delta flag, and the
-//     replay kernel then writes nothing: a chain with a bad entry anywhere is
-//     not applied at all.
+//     of g, mod 2^32 -- the rows inside each tensor's segment.  A failed check
+//     sets the workspace's delta flag, and the replay kernel then writes
+//     nothing: a chain with a bad entry anywhere is not applied at all.
+//
+//   chain_index_ends_kernel  one thread per tensor and delta: the index rows
+//     of the tensor's tiles before its first entry and after its last.
 //
 //   chain_tile_kernel  one CTA per tile: the tile index gives each delta's
 //     entries of the tile; every entry raises its element's tag in shared
@@ -615,7 +618,7 @@ __global__ void __launch_bounds__(kTileThreads, kTileMinBlocks) chain_tile_kerne
             for (int i = tid; i < kTileElems; i += kTileThreads) s_tag[i] = i < count ? dst[i] : 0u;
         }
     }
-    __syncthreads();  // tags initialised
+    if constexpr (kMerge) __syncthreads();  // tags initialised (the scatter's were zeroed before the first barrier)
     bool outside = false;  // an entry outside the tile: never, for checked entries
     for (int i0 = ib; i0 < ie; i0 += kTileItems) {
         if (i0 > ib) tile_load_round(sm, K, cur, i0, ie, ix, vx, kq, vm);
