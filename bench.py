@@ -34,6 +34,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -225,6 +226,109 @@ def encode_traffic_per_elem():
         return float(vals["dram bytes per element"]), float(vals["nnz fraction"])
     except (KeyError, ValueError):
         return None, None
+
+
+# ---------------------------------------------------------------------------
+# ncu DRAM figures for the rows, from the committed summaries under profiles/
+# ---------------------------------------------------------------------------
+
+def ncu_dram_GBps(profile):
+    """DRAM GB/s (read + write bytes / duration) of the launch captured in a
+    committed ncu summary, or None if the file or its figures are missing.
+    ncu serialises launches and starts them with a cold cache."""
+    path = os.path.join(ROOT, "profiles", profile)
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    dur = re.search(r"^\| duration[^|]*\| ([\d.,]+) us", txt, re.M)
+    tot = re.search(r"dram__bytes_read\.sum \+ dram__bytes_write\.sum \| [\d.]+ \+ [\d.]+ = ([\d.]+) GB", txt)
+    if tot:
+        nbytes = float(tot.group(1)) * 1e9
+    else:
+        parts = [re.search(r"^\| dram__bytes_%s\.sum \| ([\d.]+) (GB|MB)" % k, txt, re.M) for k in ("read", "write")]
+        if not all(parts):
+            return None
+        nbytes = sum(float(m.group(1)) * (1e9 if m.group(2) == "GB" else 1e6) for m in parts)
+    if not dur:
+        return None
+    us = float(dur.group(1).replace(",", ""))
+    return round(nbytes / (us * 1e-6) / 1e9, 1) if us > 0 else None
+
+
+# Per bench row (first match wins): the committed captures of the kernels
+# that carry it, with what differs between the captured case and the row,
+# or why no DRAM figure applies.
+_L2_RESIDENT = ("2 MB per snapshot stays in the 126 MB L2: a latency row, "
+                "which the DRAM counters do not measure")
+_HOST_LINK = "bound by the host link (copy engine transfers to or from pinned host memory), not by a kernel's DRAM traffic"
+NCU_ROWS = [
+    (r"^count_", [("encode_kernel_count_llama3_8b_2layers.md", "encode_kernel<0,0,0>", None)], None),
+    (r"^encode_global_int64_", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>",
+                                "the int32-position encode; the int64 form (encode_kernel<1,1,0>) has the same "
+                                "body and writes 2 more bytes per entry")], None),
+    (r"^encode_checksum_", [("encode_kernel_checksum_llama3_8b_2layers.md", "encode_kernel<1,0,1>", None)], None),
+    (r"^delta_file_", [], _HOST_LINK),
+    (r"^encode_llama3_8b", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>", "captured at lr 3e-6")], None),
+    (r"^apply_llama3_8b", [("apply_kernel_llama3_8b.md", "apply_kernel", "captured at lr 3e-6")], None),
+    (r"^pack_positions_", [("pack_positions_kernel_llama3_8b_2layers.md", "pack_positions_kernel", None)], None),
+    (r"^checksum_", [("checksum_kernel_llama3_8b_2layers.md", "checksum_kernel", None)], None),
+    (r"_single_1024x1024$", [], _L2_RESIDENT),
+    (r"^apply_chain_qwen3_0p6b_k10_tile_merge$", [("chain_index_kernel_qwen3_0p6b_k10.md", "chain_index_kernel", None),
+                                                  ("chain_tile_kernel_merge_qwen3_0p6b_k10.md", "chain_tile_kernel<merge>", None)], None),
+    (r"^apply_chain_qwen3_0p6b_k10", [("chain_index_kernel_qwen3_0p6b_k10.md", "chain_index_kernel", None),
+                                      ("chain_tile_kernel_scatter_qwen3_0p6b_k10.md", "chain_tile_kernel<scatter>", None)], None),
+    (r"^merge_shards_", [("merge_copy_kernel_qwen3_0p6b_8ranks.md", "merge_copy_kernel", None)], None),
+    (r"^encode_qwen3_0p6b", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>",
+                              "the same kernel, captured on the Llama-3-8B-shaped set")], None),
+    (r"^xor_apply_layers_pinned_host", [], _HOST_LINK),
+    (r"^xor_apply_layers_double_buffered", [("xor_vec_kernel_2x0.8GB.md", "xor_vec_kernel",
+                                            "the apply kernel; the next layer's mask copy runs beside it on a copy engine")], None),
+    (r"^xor_(encode|apply)_", [("xor_vec_kernel_2x0.8GB.md", "xor_vec_kernel", None)], None),
+    (r"^encode_sparse_bytes_", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>",
+                                 "the word encode, captured on the Llama-3-8B-shaped set"),
+                                ("bytes_write_kernel_xor_2x0.8GB.md", "bytes_write_kernel", None)], None),
+    (r"^encode_sparse_", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>",
+                           "the same kernel on the layers as 16-bit words, captured on the Llama-3-8B-shaped set")], None),
+    (r"^bytes_from_words_", [("bytes_write_kernel_xor_2x0.8GB.md", "bytes_write_kernel", None)], None),
+    (r"^apply_bytes_", [("apply_bytes_kernel_xor_2x0.8GB.md", "apply_bytes_kernel", None)], None),
+    (r"^apply_sparse_from_pinned_host", [], _HOST_LINK),
+    (r"^apply_sparse_", [("apply_kernel_llama3_8b.md", "apply_kernel",
+                          "the same kernel, captured on the Llama-3-8B-shaped set")], None),
+    (r"^apply_chain_stress_.*_tile_merge$", [("chain_index_kernel_stress_1200t_k10.md", "chain_index_kernel",
+                                              "captured on the 1200-tensor stress chain"),
+                                             ("chain_tile_kernel_merge_qwen3_0p6b_k10.md", "chain_tile_kernel<merge>",
+                                              "captured on the Qwen3-0.6B-shaped chain")], None),
+    (r"^apply_chain_stress_", [("chain_index_kernel_stress_1200t_k10.md", "chain_index_kernel",
+                                "captured on the 1200-tensor stress chain"),
+                               ("chain_tile_kernel_scatter_stress_1200t_k10.md", "chain_tile_kernel<scatter>",
+                                "captured on the 1200-tensor stress chain")], None),
+    (r"^encode_stress_", [("encode_kernel_stress_1200t.md", "encode_kernel<1,0,0>",
+                           "captured on the 1200-tensor stress set")], None),
+]
+
+
+def ncu_for_row(name):
+    """The `ncu` entry of a bench row: per captured kernel its profile, its
+    DRAM GB/s in the captured launch, and what differs from the row; or the
+    reason there is none."""
+    for pat, caps, reason in NCU_ROWS:
+        if re.search(pat, name):
+            if reason is not None:
+                return {"dram_GBps": None, "reason": reason}
+            out = []
+            for prof, kernel, note in caps:
+                e = {"kernel": kernel, "profile": "profiles/" + prof, "dram_GBps": ncu_dram_GBps(prof)}
+                if note:
+                    e["note"] = note
+                out.append(e)
+            return {"captures": out, "case": "ncu: one launch, cold cache, serialised"}
+    return {"dram_GBps": None, "reason": "no committed capture for this row"}
+
+
+def attach_ncu(rows):
+    for name, row in rows.items():
+        row["ncu"] = ncu_for_row(name)
+    return rows
 
 
 # ---------------------------------------------------------------------------
@@ -913,7 +1017,7 @@ def run_ours(args):
         rows = run_rows(args, dev, peak, groups)
         exact = all(v.get("exact", True) and v.get("exact_flip_count", True) for v in rows.values())
         if rank == 0:
-            print(json.dumps({"rows": rows, "rows_only": groups}), flush=True)
+            print(json.dumps({"rows": attach_ncu(rows), "rows_only": groups}), flush=True)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()
@@ -1028,13 +1132,15 @@ def run_ours(args):
         "kernels": {
             "encode": {"ms": round(enc_ms, 4), "alg_bytes": enc_alg,
                        "alg_GBps": round(achieved, 1), "weight_GBps": round(weight_bytes / enc_ms / 1e6, 1),
-                       "elems_per_s": round(N / enc_ms * 1e3, 1)},
+                       "elems_per_s": round(N / enc_ms * 1e3, 1),
+                       "ncu": ncu_for_row("encode_llama3_8b")},
             "apply": {"ms": round(app_ms, 4), "alg_bytes": app_alg,
                       "alg_GBps": round(app_alg / app_ms / 1e6, 1),
                       "weight_GBps": round(weight_bytes / app_ms / 1e6, 1),
                       "elems_per_s": round(N / app_ms * 1e3, 1),
                       "entries_per_s": round(nnz / app_ms * 1e3, 1),
-                      **sector_model(nnz, app_sectors, app_ms, peak, clean_bytes(nnz, dev))},
+                      **sector_model(nnz, app_sectors, app_ms, peak, clean_bytes(nnz, dev)),
+                      "ncu": ncu_for_row("apply_llama3_8b")},
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -1200,7 +1306,7 @@ def run_ours(args):
         torch.cuda.empty_cache()
         if args.layers is None:
             rows.update(run_rows(args, dev, peak))
-        line["rows"] = rows
+        line["rows"] = attach_ncu(rows)
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1) ---------
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
