@@ -70,3 +70,35 @@ def test_rows_get_the_capture_of_their_own_kernel():
     assert bench.ncu_for_row("encode_sparse_bytes_nvfp4_40x0.8GB")["captures"][1]["kernel"] == "bytes_write_kernel"
     assert "reason" in bench.ncu_for_row("xor_apply_layers_pinned_host_4x0.8GB")
     assert bench.ncu_for_row("something_new")["reason"] == "no committed capture for this row"
+
+
+def _fake_tree(tmp_path, src, sha_line):
+    (tmp_path / "profiles").mkdir()
+    csrc = tmp_path / "sparse_bf16_delta_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "encode.cu").write_bytes(src)
+    (tmp_path / "profiles" / "encode_kernel_llama3_8b.md").write_text(
+        "# encode capture\n\n"
+        f"- encode.cu sha256[:16]: `{sha_line}`\n"
+        "- dram bytes per element: 4.25\n"
+        "- nnz fraction: 0.035\n")
+
+
+def test_encode_traffic_needs_the_capture_of_the_current_source(tmp_path, monkeypatch):
+    # roofline.traffic comes from the committed capture only while the
+    # kernel source is the one that was captured; any change makes it null.
+    import hashlib
+    src = b"// some kernel source\n"
+    _fake_tree(tmp_path, src, hashlib.sha256(src).hexdigest()[:16])
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.encode_traffic_per_elem() == (4.25, 0.035)
+    (tmp_path / "sparse_bf16_delta_b200" / "csrc" / "encode.cu").write_bytes(src + b"// changed\n")
+    assert bench.encode_traffic_per_elem() == (None, None)
+    (tmp_path / "profiles" / "encode_kernel_llama3_8b.md").unlink()
+    assert bench.encode_traffic_per_elem() == (None, None)
+
+
+def test_committed_encode_capture_is_of_the_committed_kernel():
+    per_elem, frac = bench.encode_traffic_per_elem()
+    assert per_elem is not None and 4.0 < per_elem < 4.4
+    assert 0.03 < frac < 0.04
