@@ -263,9 +263,7 @@ _L2_RESIDENT = ("2 MB per snapshot stays in the 126 MB L2: a latency row, "
 _HOST_LINK = "bound by the host link (copy engine transfers to or from pinned host memory), not by a kernel's DRAM traffic"
 NCU_ROWS = [
     (r"^count_", [("encode_kernel_count_llama3_8b_2layers.md", "encode_kernel<0,0,0>", None)], None),
-    (r"^encode_global_int64_", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>",
-                                "the int32-position encode; the int64 form (encode_kernel<1,1,0>) has the same "
-                                "body and writes 2 more bytes per entry")], None),
+    (r"^encode_global_int64_", [("encode_kernel_global_llama3_8b_2layers.md", "encode_kernel<1,1,0>", None)], None),
     (r"^encode_checksum_", [("encode_kernel_checksum_llama3_8b_2layers.md", "encode_kernel<1,0,1>", None)], None),
     (r"^delta_file_", [], _HOST_LINK),
     (r"^encode_llama3_8b", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>", "captured at lr 3e-6")], None),
@@ -296,8 +294,8 @@ NCU_ROWS = [
                           "the same kernel, captured on the Llama-3-8B-shaped set")], None),
     (r"^apply_chain_stress_.*_tile_merge$", [("chain_index_kernel_stress_1200t_k10.md", "chain_index_kernel",
                                               "captured on the 1200-tensor stress chain"),
-                                             ("chain_tile_kernel_merge_qwen3_0p6b_k10.md", "chain_tile_kernel<merge>",
-                                              "captured on the Qwen3-0.6B-shaped chain")], None),
+                                             ("chain_tile_kernel_merge_stress_1200t_k10.md", "chain_tile_kernel<merge>",
+                                              "captured on the 1200-tensor stress chain")], None),
     (r"^apply_chain_stress_", [("chain_index_kernel_stress_1200t_k10.md", "chain_index_kernel",
                                 "captured on the 1200-tensor stress chain"),
                                ("chain_tile_kernel_scatter_stress_1200t_k10.md", "chain_tile_kernel<scatter>",
