@@ -282,16 +282,13 @@ NCU_ROWS = [
     (r"^xor_apply_layers_double_buffered", [("xor_vec_kernel_2x0.8GB.md", "xor_vec_kernel",
                                             "the apply kernel; the next layer's mask copy runs beside it on a copy engine")], None),
     (r"^xor_(encode|apply)_", [("xor_vec_kernel_2x0.8GB.md", "xor_vec_kernel", None)], None),
-    (r"^encode_sparse_bytes_", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>",
-                                 "the word encode, captured on the Llama-3-8B-shaped set"),
+    (r"^encode_sparse_bytes_", [("encode_kernel_words_xor_2x0.8GB.md", "encode_kernel<1,0,0>", None),
                                 ("bytes_write_kernel_xor_2x0.8GB.md", "bytes_write_kernel", None)], None),
-    (r"^encode_sparse_", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>",
-                           "the same kernel on the layers as 16-bit words, captured on the Llama-3-8B-shaped set")], None),
+    (r"^encode_sparse_", [("encode_kernel_words_xor_2x0.8GB.md", "encode_kernel<1,0,0>", None)], None),
     (r"^bytes_from_words_", [("bytes_write_kernel_xor_2x0.8GB.md", "bytes_write_kernel", None)], None),
     (r"^apply_bytes_", [("apply_bytes_kernel_xor_2x0.8GB.md", "apply_bytes_kernel", None)], None),
     (r"^apply_sparse_from_pinned_host", [], _HOST_LINK),
-    (r"^apply_sparse_", [("apply_kernel_llama3_8b.md", "apply_kernel",
-                          "the same kernel, captured on the Llama-3-8B-shaped set")], None),
+    (r"^apply_sparse_", [("apply_kernel_words_xor_2x0.8GB.md", "apply_kernel", None)], None),
     (r"^apply_chain_stress_.*_tile_merge$", [("chain_index_kernel_stress_1200t_k10.md", "chain_index_kernel",
                                               "captured on the 1200-tensor stress chain"),
                                              ("chain_tile_kernel_merge_stress_1200t_k10.md", "chain_tile_kernel<merge>",
