@@ -266,8 +266,10 @@ NCU_ROWS = [
     (r"^encode_global_int64_", [("encode_kernel_global_llama3_8b_2layers.md", "encode_kernel<1,1,0>", None)], None),
     (r"^encode_checksum_", [("encode_kernel_checksum_llama3_8b_2layers.md", "encode_kernel<1,0,1>", None)], None),
     (r"^delta_file_", [], _HOST_LINK),
-    (r"^encode_llama3_8b", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>", "captured at lr 3e-6")], None),
-    (r"^apply_llama3_8b", [("apply_kernel_llama3_8b.md", "apply_kernel", "captured at lr 3e-6")], None),
+    (r"^encode_llama3_8b_lr1e-5", [("encode_kernel_llama3_8b_2layers_lr1e-5.md", "encode_kernel<1,0,0>", None)], None),
+    (r"^apply_llama3_8b_lr1e-5", [("apply_kernel_llama3_8b_2layers_lr1e-5.md", "apply_kernel", None)], None),
+    (r"^encode_llama3_8b", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>", None)], None),
+    (r"^apply_llama3_8b", [("apply_kernel_llama3_8b.md", "apply_kernel", None)], None),
     (r"^pack_positions_", [("pack_positions_kernel_llama3_8b_2layers.md", "pack_positions_kernel", None)], None),
     (r"^checksum_", [("checksum_kernel_llama3_8b_2layers.md", "checksum_kernel", None)], None),
     (r"_single_1024x1024$", [], _L2_RESIDENT),
