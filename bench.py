@@ -278,8 +278,7 @@ NCU_ROWS = [
     (r"^apply_chain_qwen3_0p6b_k10", [("chain_index_kernel_qwen3_0p6b_k10.md", "chain_index_kernel", None),
                                       ("chain_tile_kernel_scatter_qwen3_0p6b_k10.md", "chain_tile_kernel<scatter>", None)], None),
     (r"^merge_shards_", [("merge_copy_kernel_qwen3_0p6b_8ranks.md", "merge_copy_kernel", None)], None),
-    (r"^encode_qwen3_0p6b", [("encode_kernel_llama3_8b.md", "encode_kernel<1,0,0>",
-                              "the same kernel, captured on the Llama-3-8B-shaped set")], None),
+    (r"^encode_qwen3_0p6b", [("encode_kernel_qwen3_0p6b.md", "encode_kernel<1,0,0>", None)], None),
     (r"^xor_apply_layers_pinned_host", [], _HOST_LINK),
     (r"^xor_apply_layers_double_buffered", [("xor_vec_kernel_2x0.8GB.md", "xor_vec_kernel",
                                             "the apply kernel; the next layer's mask copy runs beside it on a copy engine")], None),
